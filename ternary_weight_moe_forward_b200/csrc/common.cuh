@@ -1,0 +1,114 @@
+// Shared device helpers of the ternary MoE layer kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define MAPLE_DEVFLAG_NAN 0x1u
+#define MAPLE_DEVFLAG_BAD_INDEX 0x2u
+#define MAPLE_DEVFLAG_BAD_VALUE 0x4u
+#define MAPLE_DEVFLAG_TIMEOUT 0x8u
+
+namespace maple {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// exp(x), written out from the mathematics so that host and device give the
+// same bits: clamp to [-87, 88]; n = rint(x*log2 e); r = x - n ln2 with ln2
+// split into a 17-bit head and a tail (Cody-Waite); Taylor polynomial of
+// degree 7 in r by Horner's rule with fused multiply-adds; times 2^n built
+// from exponent bits.  Coefficients are 1/k! rounded once to binary32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float exp_ref(float x)
+{
+    const float kLog2e = 0x1.715476p+0f;   // 1/ln 2
+    const float kLn2Hi = 0x1.62e4p-1f;     // 0.693145751953125
+    const float kLn2Lo = 0x1.7f7d1cp-20f;  // ln 2 - kLn2Hi
+    x = fminf(fmaxf(x, -87.0f), 88.0f);
+    float n = rintf(__fmul_rn(x, kLog2e));
+    float r = __fmaf_rn(-n, kLn2Hi, x);
+    r = __fmaf_rn(-n, kLn2Lo, r);
+    float p = 0x1.a01a02p-13f;             // 1/7!
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);  // 1/6!
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);   // 1/5!
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);   // 1/4!
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);   // 1/3!
+    p = __fmaf_rn(p, r, 0.5f);             // 1/2!
+    p = __fmaf_rn(p, r, 1.0f);             // 1/1!
+    p = __fmaf_rn(p, r, 1.0f);             // 1/0!
+    float scale = __int_as_float(((int)n + 127) << 23);
+    return __fmul_rn(p, scale);
+}
+
+// SiLU(g) * u with every step rounded once: (g / (1 + exp(-g))) * u
+__device__ __forceinline__ float swiglu(float g, float u)
+{
+    float den = __fadd_rn(1.0f, exp_ref(-g));
+    return __fmul_rn(__fdiv_rn(g, den), u);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// round a finite float to bf16 (nearest, ties to even); returns the 16 bits
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f)
+{
+    uint32_t u = __float_as_uint(f);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+// int8 absmax code of v given inv = 127/amax: clamp(rint(v*inv), -127, 127)
+__device__ __forceinline__ int quant_code(float v, float inv)
+{
+    int q = __float2int_rn(__fmul_rn(v, inv));
+    return max(-127, min(127, q));
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_int(int v)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+
+// Pairwise tree over the 32 lanes: lane l with l^16, then 8, 4, 2, 1.  Every
+// lane ends with the same value (fp addition is commutative).
+__device__ __forceinline__ float warp_tree_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+
+// d = c + sum of the four byte products (a unsigned bytes, b signed bytes)
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c)
+{
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 16-byte streaming load that skips L1 (weights are read once per use)
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void set_flag(unsigned *flag, unsigned bits)
+{
+    if (flag) atomicOr(flag, bits);
+}
+
+}  // namespace maple

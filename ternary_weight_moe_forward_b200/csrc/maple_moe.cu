@@ -1,0 +1,487 @@
+// C ABI of the ternary-weight MoE FFN layer (see include/maple_moe.h).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/maple_moe.h"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "layout.cuh"
+#include "pack.cuh"
+#include "route.cuh"
+
+using namespace maple;
+
+namespace {
+
+constexpr uint32_t kMagic = 0x4d41504cu;  // "MAPL"
+
+struct Arena {
+    size_t size = 0;
+    size_t take(size_t bytes)
+    {
+        size_t off = size;
+        size += (bytes + 255) & ~(size_t)255;
+        return off;
+    }
+};
+
+}  // namespace
+
+struct maple_moe_s {
+    uint32_t magic;
+    int D, E, K, F, Tm, dmax;
+    uint32_t cfg_flags;
+    int num_sms;
+    int device;
+    char *base;  // one device allocation: weights + workspace
+    // weights
+    uint8_t *w_gu, *w_dn;
+    float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
+    // workspace
+    int8_t *qx;
+    float *sx;
+    int *sumx;
+    float *logits;
+    int *topk_idx;
+    float *topk_w;
+    int *counts, *offsets, *perm, *inv, *active, *n_active, *blk_cnt;
+    float *h;
+    int8_t *qh;
+    float *sh;
+    int *sumqh;
+    float *ye;
+    unsigned *tg_cnt, *glob_cnt, *exp_cnt, *comb_cnt;
+    uint16_t *xn;
+    // flag word in host-mapped memory
+    unsigned *flag_host;
+    unsigned *flag_dev;
+    // optional stage events (profiling)
+    cudaEvent_t ev[4];
+    bool use_events;
+};
+
+static void stage_event(maple_moe_s *h, int i, cudaStream_t st)
+{
+    if (h->use_events) cudaEventRecord(h->ev[i], st);
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? MAPLE_OK : MAPLE_ERR_CUDA;
+}
+
+static int grid_for(int64_t n, int block, int cap)
+{
+    int64_t g = (n + block - 1) / block;
+    if (g < 1) g = 1;
+    if (g > cap) g = cap;
+    return (int)g;
+}
+
+extern "C" const char *maple_moe_status_string(int status)
+{
+    switch (status) {
+    case MAPLE_OK: return "ok";
+    case MAPLE_ERR_INVALID_ARG: return "invalid argument";
+    case MAPLE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MAPLE_ERR_OOM: return "out of device memory";
+    case MAPLE_ERR_CUDA: return "CUDA error";
+    case MAPLE_ERR_TIMEOUT: return "device wait timed out";
+    case MAPLE_ERR_DEVICE_FLAG: return "a kernel flagged an invalid value";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int maple_moe_pack_ternary(const int8_t *values, int64_t rows, int32_t cols, uint32_t *packed,
+                                      int32_t *bad_count, maple_stream_t stream)
+{
+    if (rows < 0 || cols <= 0 || cols % 16 != 0) return MAPLE_ERR_INVALID_ARG;
+    if (rows == 0) return MAPLE_OK;
+    if (!values || !packed || !aligned16(values) || ((uintptr_t)packed & 3u)) return MAPLE_ERR_INVALID_ARG;
+    const int64_t n_words = rows * (cols / 16);
+    pack_ternary_kernel<<<grid_for(n_words, 256, 148 * 16), 256, 0, (cudaStream_t)stream>>>(values, n_words, packed,
+                                                                                          bad_count);
+    return launch_status();
+}
+
+static int check_shape(const maple_moe_config *c)
+{
+    if (c->d_model <= 0 || c->d_model % 256 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_ff <= 0 || c->d_ff % 128 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->n_experts < 8 || c->n_experts > kMaxExperts || c->n_experts % 8 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->n_experts) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->max_tokens < 1 || c->max_tokens > 65536) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->decode_max_tokens < 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_weights *w, maple_stream_t stream,
+                                maple_moe_t *out)
+{
+    if (!config || !w || !out) return MAPLE_ERR_INVALID_ARG;
+    *out = nullptr;
+    int rc = check_shape(config);
+    if (rc) return rc;
+    const void *need[] = {w->w_gate, w->w_up, w->w_down, w->alpha_gate, w->alpha_up, w->alpha_down, w->router_w};
+    for (const void *p : need)
+        if (!p || !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
+    if (w->router_bias && !aligned16(w->router_bias)) return MAPLE_ERR_INVALID_ARG;
+
+    maple_moe_s *h = new (std::nothrow) maple_moe_s();
+    if (!h) return MAPLE_ERR_OOM;
+    h->magic = kMagic;
+    h->D = config->d_model;
+    h->E = config->n_experts;
+    h->K = config->top_k;
+    h->F = config->d_ff;
+    h->Tm = config->max_tokens;
+    h->dmax = config->decode_max_tokens ? config->decode_max_tokens : 64;
+    h->cfg_flags = config->flags;
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+        delete h;
+        return MAPLE_ERR_CUDA;
+    }
+    const int64_t D = h->D, E = h->E, K = h->K, F = h->F, Tm = h->Tm;
+    const int64_t S = Tm * K;
+    const int64_t nblk = (Tm + kPermBlockTokens - 1) / kPermBlockTokens;
+    Arena ar;
+    size_t o_gu = ar.take(E * gu_bytes_per_expert(D, F)), o_dn = ar.take(E * dn_bytes_per_expert(D, F));
+    size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
+    size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
+    size_t o_qx = ar.take(Tm * D), o_sx = ar.take(Tm * 4), o_sumx = ar.take(Tm * 4);
+    size_t o_lg = ar.take(Tm * E * 4), o_ti = ar.take(S * 4), o_tw = ar.take(S * 4);
+    size_t o_cnt = ar.take(E * 4), o_off = ar.take((E + 1) * 4), o_perm = ar.take(S * 4), o_inv = ar.take(S * 4);
+    size_t o_act = ar.take(E * 4), o_nact = ar.take(4), o_blk = ar.take(nblk * E * 4);
+    size_t o_h = ar.take(S * F * 4), o_qh = ar.take(S * F), o_sh = ar.take(S * 4), o_sumqh = ar.take(S * 4);
+    size_t o_ye = ar.take(S * D * 4);
+    size_t o_ctr = ar.take(0);
+    size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4), o_ec = ar.take(E * 4);
+    size_t o_cc = ar.take(Tm * (D / 32) * 4);
+    size_t o_xn = ar.take(Tm * D * 2);
+
+    if (cudaMalloc(&h->base, ar.size) != cudaSuccess) {
+        cudaGetLastError();
+        delete h;
+        return MAPLE_ERR_OOM;
+    }
+    if (cudaHostAlloc(&h->flag_host, sizeof(unsigned), cudaHostAllocMapped) != cudaSuccess ||
+        cudaHostGetDevicePointer(&h->flag_dev, h->flag_host, 0) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(h->base);
+        delete h;
+        return MAPLE_ERR_CUDA;
+    }
+    *h->flag_host = 0;
+    char *b = h->base;
+    h->w_gu = (uint8_t *)(b + o_gu);
+    h->w_dn = (uint8_t *)(b + o_dn);
+    h->alpha_gate = (float *)(b + o_ag);
+    h->alpha_up = (float *)(b + o_au);
+    h->alpha_down = (float *)(b + o_ad);
+    h->router_w = (float *)(b + o_rw);
+    h->router_bias = w->router_bias ? (float *)(b + o_rb) : nullptr;
+    h->qx = (int8_t *)(b + o_qx);
+    h->sx = (float *)(b + o_sx);
+    h->sumx = (int *)(b + o_sumx);
+    h->logits = (float *)(b + o_lg);
+    h->topk_idx = (int *)(b + o_ti);
+    h->topk_w = (float *)(b + o_tw);
+    h->counts = (int *)(b + o_cnt);
+    h->offsets = (int *)(b + o_off);
+    h->perm = (int *)(b + o_perm);
+    h->inv = (int *)(b + o_inv);
+    h->active = (int *)(b + o_act);
+    h->n_active = (int *)(b + o_nact);
+    h->blk_cnt = (int *)(b + o_blk);
+    h->h = (float *)(b + o_h);
+    h->qh = (int8_t *)(b + o_qh);
+    h->sh = (float *)(b + o_sh);
+    h->sumqh = (int *)(b + o_sumqh);
+    h->ye = (float *)(b + o_ye);
+    h->tg_cnt = (unsigned *)(b + o_tg);
+    h->glob_cnt = (unsigned *)(b + o_gc);
+    h->exp_cnt = (unsigned *)(b + o_ec);
+    h->comb_cnt = (unsigned *)(b + o_cc);
+    h->xn = (uint16_t *)(b + o_xn);
+
+    cudaStream_t st = (cudaStream_t)stream;
+    // the whole workspace starts at zero: counters must, and every index array
+    // then holds in-range values even before its first write
+    cudaMemsetAsync(b + o_qx, 0, ar.size - o_qx, st);
+    cudaMemcpyAsync(h->alpha_gate, w->alpha_gate, E * F * 4, cudaMemcpyDeviceToDevice, st);
+    cudaMemcpyAsync(h->alpha_up, w->alpha_up, E * F * 4, cudaMemcpyDeviceToDevice, st);
+    cudaMemcpyAsync(h->alpha_down, w->alpha_down, E * D * 4, cudaMemcpyDeviceToDevice, st);
+    cudaMemcpyAsync(h->router_w, w->router_w, E * D * 4, cudaMemcpyDeviceToDevice, st);
+    if (w->router_bias) cudaMemcpyAsync(h->router_bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, st);
+    const int cap = h->num_sms * 16;
+    repack_gu_kernel<<<grid_for(E * (F / 16) * (D / 64) * 128, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E,
+                                                                                     h->D, h->F, (uint32_t *)h->w_gu);
+    repack_dn_kernel<<<grid_for(E * (D / 32) * (F / 64) * 128, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
+                                                                                    (uint32_t *)h->w_dn);
+    if (cudaGetLastError() != cudaSuccess) {
+        cudaFree(h->base);
+        cudaFreeHost(h->flag_host);
+        delete h;
+        return MAPLE_ERR_CUDA;
+    }
+    *out = h;
+    return MAPLE_OK;
+}
+
+static int check_handle(maple_moe_t h)
+{
+    if (!h || h->magic != kMagic) return MAPLE_ERR_INVALID_ARG;
+    return MAPLE_OK;
+}
+
+static int take_flag(maple_moe_t h)
+{
+    unsigned f = __atomic_exchange_n(h->flag_host, 0u, __ATOMIC_ACQ_REL);
+    return f ? MAPLE_ERR_DEVICE_FLAG : MAPLE_OK;
+}
+
+// routing stage: quantise, logits, top-k (+ the permutation)
+static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
+                     float *out_w, int32_t *out_counts, bool permute, cudaStream_t st)
+{
+    RouteArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x;
+    a.T = T;
+    a.D = h->D;
+    a.E = h->E;
+    a.K = h->K;
+    a.Wr = h->router_w;
+    a.bias = h->router_bias;
+    a.qx = h->qx;
+    a.sx = h->sx;
+    a.sumx = h->sumx;
+    a.logits = h->logits;
+    a.topk_idx = h->topk_idx;
+    a.topk_w = h->topk_w;
+    if (taps) {
+        a.tap_qx = taps->q_x;
+        a.tap_sx = taps->s_x;
+        a.tap_logits = taps->logits;
+        a.tap_offsets = taps->expert_offsets;
+        a.tap_perm = taps->perm;
+    }
+    a.out_idx = out_idx ? out_idx : (taps ? taps->topk_idx : nullptr);
+    a.out_w = out_w ? out_w : (taps ? taps->topk_w : nullptr);
+    a.out_counts = out_counts ? out_counts : (taps ? taps->expert_counts : nullptr);
+    a.tg_cnt = h->tg_cnt;
+    a.glob_cnt = h->glob_cnt;
+    a.counts = h->counts;
+    a.offsets = h->offsets;
+    a.perm = h->perm;
+    a.inv = h->inv;
+    a.active = h->active;
+    a.n_active = h->n_active;
+    a.flag = h->flag_dev;
+    const bool fused = permute && (int64_t)T * h->E <= kFusedMarkBytes;
+    a.fuse_permute = fused ? 1 : 0;
+    dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
+    if (h->E <= 256)
+        route_kernel<8><<<grid, 256, 0, st>>>(a);
+    else
+        route_kernel<32><<<grid, 256, 0, st>>>(a);
+    if (permute && !fused) {
+        PermArgs p;
+        memset(&p, 0, sizeof p);
+        p.idx = h->topk_idx;
+        p.T = T;
+        p.K = h->K;
+        p.E = h->E;
+        p.blk_cnt = h->blk_cnt;
+        p.counts = h->counts;
+        p.offsets = h->offsets;
+        p.perm = h->perm;
+        p.inv = h->inv;
+        p.active = h->active;
+        p.n_active = h->n_active;
+        p.out_counts = a.out_counts;
+        p.tap_offsets = a.tap_offsets;
+        p.tap_perm = a.tap_perm;
+        p.flag = h->flag_dev;
+        const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+        perm_count_kernel<<<nblk, 256, 0, st>>>(p);
+        perm_scan_kernel<<<1, 1024, 0, st>>>(p);
+        perm_scatter_kernel<<<nblk, 256, 0, st>>>(p);
+    }
+    return launch_status();
+}
+
+static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
+                       cudaStream_t st)
+{
+    GemvArgs g;
+    memset(&g, 0, sizeof g);
+    g.T = T;
+    g.D = h->D;
+    g.E = h->E;
+    g.K = h->K;
+    g.F = h->F;
+    g.active = h->active;
+    g.n_active = h->n_active;
+    g.counts = h->counts;
+    g.offsets = h->offsets;
+    g.perm = h->perm;
+    g.inv = h->inv;
+    g.topk_w = h->topk_w;
+    g.qx = h->qx;
+    g.sx = h->sx;
+    g.sumx = h->sumx;
+    g.w_gu = h->w_gu;
+    g.w_dn = h->w_dn;
+    g.alpha_gate = h->alpha_gate;
+    g.alpha_up = h->alpha_up;
+    g.alpha_down = h->alpha_down;
+    g.h = h->h;
+    g.qh = h->qh;
+    g.sh = h->sh;
+    g.sumqh = h->sumqh;
+    g.ye = h->ye;
+    g.y = y;
+    g.resid = resid;
+    g.exp_cnt = h->exp_cnt;
+    g.comb_cnt = h->comb_cnt;
+    if (taps) {
+        g.tap_acc_gate = taps->acc_gate;
+        g.tap_acc_up = taps->acc_up;
+        g.tap_acc_down = taps->acc_down;
+        g.tap_qh = taps->q_h;
+        g.tap_sh = taps->s_h;
+    }
+    const int64_t max_active = (int64_t)T * h->K < h->E ? (int64_t)T * h->K : h->E;
+    const int cap = h->num_sms * 4;
+    gateup_gemv_kernel<<<grid_for(max_active * (h->F / 16), kGemvWarps, cap), kGemvWarps * 32, 0, st>>>(g);
+    stage_event(h, 2, st);
+    down_gemv_kernel<<<grid_for(max_active * (h->D / 32), kGemvWarps, cap), kGemvWarps * 32, 0, st>>>(g);
+    stage_event(h, 3, st);
+    return launch_status();
+}
+
+static int check_taps(const maple_moe_taps *t)
+{
+    if (!t) return MAPLE_OK;
+    const void *ps[] = {t->q_x, t->s_x, t->logits, t->topk_idx, t->topk_w, t->acc_gate, t->acc_up, t->q_h,
+                        t->s_h, t->acc_down, t->expert_counts, t->expert_offsets, t->perm};
+    for (const void *p : ps)
+        if (p && !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int32_t *topk_idx, float *topk_w,
+                               int32_t *expert_counts, maple_stream_t stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (T < 0 || T > h->Tm) return MAPLE_ERR_INVALID_ARG;
+    if ((rc = take_flag(h))) return rc;
+    if (T == 0) return MAPLE_OK;
+    if (!x || !aligned16(x)) return MAPLE_ERR_INVALID_ARG;
+    for (const void *p : {(const void *)topk_idx, (const void *)topk_w, (const void *)expert_counts})
+        if (p && !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
+    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr,
+                     (cudaStream_t)stream);
+}
+
+static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const float *resid,
+                        const maple_moe_taps *taps, cudaStream_t st)
+{
+    stage_event(h, 0, st);
+    int rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, st);
+    if (rc) return rc;
+    stage_event(h, 1, st);
+    return run_experts(h, T, y, resid, taps, st);
+}
+
+extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const maple_moe_taps *taps,
+                                 maple_stream_t stream)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (T < 0 || T > h->Tm) return MAPLE_ERR_INVALID_ARG;
+    if ((rc = take_flag(h))) return rc;
+    if (T == 0) return MAPLE_OK;
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return MAPLE_ERR_INVALID_ARG;
+    if ((rc = check_taps(taps))) return rc;
+    return forward_impl(h, x, T, y, nullptr, taps, (cudaStream_t)stream);
+}
+
+extern "C" int maple_moe_stack_forward(const maple_moe_t *layers, int32_t n_layers, float *resid, int32_t T,
+                                       maple_stream_t stream)
+{
+    if (!layers || n_layers < 0) return MAPLE_ERR_INVALID_ARG;
+    if (n_layers == 0) return MAPLE_OK;
+    for (int l = 0; l < n_layers; l++) {
+        int rc = check_handle(layers[l]);
+        if (rc) return rc;
+        const maple_moe_s *a = layers[l], *b = layers[0];
+        if (a->D != b->D || a->E != b->E || a->K != b->K || a->F != b->F) return MAPLE_ERR_INVALID_ARG;
+        if (T < 0 || T > a->Tm) return MAPLE_ERR_INVALID_ARG;
+    }
+    for (int l = 0; l < n_layers; l++) {
+        int rc = take_flag(layers[l]);
+        if (rc) return rc;
+    }
+    if (T == 0) return MAPLE_OK;
+    if (!resid || !aligned16(resid)) return MAPLE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint16_t *xn = layers[0]->xn;
+    for (int l = 0; l < n_layers; l++) {
+        rmsnorm_bf16_kernel<<<(T + 7) / 8, 256, 0, st>>>(resid, T, layers[l]->D, xn);
+        int rc = launch_status();
+        if (rc) return rc;
+        rc = forward_impl(layers[l], xn, T, resid, resid, nullptr, st);
+        if (rc) return rc;
+    }
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_set_stage_events(maple_moe_t h, void *const *events, int32_t n_events)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!events) {
+        h->use_events = false;
+        return MAPLE_OK;
+    }
+    if (n_events != 4) return MAPLE_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; i++) {
+        if (!events[i]) return MAPLE_ERR_INVALID_ARG;
+        h->ev[i] = (cudaEvent_t)events[i];
+    }
+    h->use_events = true;
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_device_flags(maple_moe_t h, uint32_t *flags, int32_t clear)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!flags) return MAPLE_ERR_INVALID_ARG;
+    *flags = clear ? __atomic_exchange_n(h->flag_host, 0u, __ATOMIC_ACQ_REL)
+                   : __atomic_load_n(h->flag_host, __ATOMIC_ACQUIRE);
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_destroy(maple_moe_t h)
+{
+    if (!h) return MAPLE_OK;
+    int rc = check_handle(h);
+    if (rc) return rc;
+    int status = MAPLE_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) status = MAPLE_ERR_CUDA;
+    if (cudaFree(h->base) != cudaSuccess) status = MAPLE_ERR_CUDA;
+    if (cudaFreeHost(h->flag_host) != cudaSuccess) status = MAPLE_ERR_CUDA;
+    h->magic = 0;
+    delete h;
+    return status;
+}

@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA layer against the CPU oracle on the same seeded inputs.
+
+Bit-exact: int8 codes and scales, router logits, expert indices and weights,
+per-expert counts/offsets/permutation, the int32 accumulators of all three
+contractions.  fp32 layer output: max relative error <= 1e-3 (it is expected
+to be bit-exact too; the tests report it).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ternary_weight_moe_forward_b200 import synth
+from ternary_weight_moe_forward_b200.layer import Layer, bf16_from_bits
+
+from parity import Y_TOL, compare_permutation, compare_tokens, gpu_forward_with_taps, max_rel
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.CONFIGS["tiny"]["shape"]
+BIG = synth.CONFIGS["decode"]["shape"]
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    w = synth.layer_weights(TINY, seed=0)
+    return w, oracle.Layer(TINY, w), Layer(TINY, w, max_tokens=512)
+
+
+@pytest.fixture(scope="module")
+def big_weights():
+    return synth.layer_weights(BIG, seed=0)
+
+
+@pytest.fixture(scope="module")
+def big(big_weights):
+    return oracle.Layer(BIG, big_weights), Layer(BIG, big_weights, max_tokens=4096)
+
+
+def _full_check(shape, L_orc, L_gpu, x_bits):
+    g = gpu_forward_with_taps(L_gpu, x_bits)
+    tokens = np.arange(x_bits.shape[0], dtype=np.int32)
+    ref = L_orc.forward_tokens(x_bits, tokens)
+    res = compare_tokens(shape, g, ref, tokens)
+    compare_permutation(shape, g, ref["topk_idx"])
+    return g, ref, res
+
+
+def test_pack_kernel_matches_oracle_packer(tiny, big_weights):
+    w, L_orc, L_gpu = tiny
+    for k in ("gate", "up", "down"):
+        assert np.array_equal(L_gpu.packed[k].cpu().numpy().view(np.uint32), L_orc.packed[k])
+    from ternary_weight_moe_forward_b200.layer import pack_on_device
+    vals = torch.from_numpy(big_weights["gate"][:4]).cuda()
+    packed, bad = pack_on_device(vals)
+    assert int(bad.item()) == 0
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), oracle.pack_ternary(big_weights["gate"][:4]))
+
+
+def test_pack_kernel_counts_invalid_values():
+    vals = torch.zeros((2, 32), dtype=torch.int8, device="cuda")
+    vals[0, 3] = 2
+    vals[1, 31] = -5
+    from ternary_weight_moe_forward_b200.layer import pack_on_device
+    packed, bad = pack_on_device(vals)
+    assert int(bad.item()) == 2
+    assert not packed.any()
+
+
+def test_tiny_config_full_parity(tiny):
+    w, L_orc, L_gpu = tiny
+    x = synth.activations(8, TINY.d_model, seed=0)
+    _, _, res = _full_check(TINY, L_orc, L_gpu, x)
+    assert res["y_rel"] <= Y_TOL
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 64])
+def test_decode_config_full_parity(big, T):
+    L_orc, L_gpu = big
+    x = synth.activations(T, BIG.d_model, seed=0)
+    _full_check(BIG, L_orc, L_gpu, x)
+
+
+@pytest.mark.parametrize("T", [3, 65, 200])
+def test_ragged_token_counts(tiny, T):
+    w, L_orc, L_gpu = tiny
+    x = synth.activations(T, TINY.d_model, seed=T)
+    _full_check(TINY, L_orc, L_gpu, x)
+
+
+def test_zero_tokens_is_a_noop(tiny):
+    w, L_orc, L_gpu = tiny
+    x = torch.empty((0, TINY.d_model), dtype=torch.bfloat16, device="cuda")
+    y = torch.full((1, TINY.d_model), 7.0, device="cuda")
+    L_gpu.forward(x, y=y)
+    torch.cuda.synchronize()
+    assert torch.all(y == 7.0)
+
+
+def test_zero_rows_and_ties(tiny):
+    w, L_orc, L_gpu = tiny
+    # identical router rows for experts 3 and 9 and 4 and 5 -> equal logits, lower index first
+    w2 = dict(w)
+    rw = w["router_w"].copy()
+    rw[9] = rw[3]
+    rw[5] = rw[4]
+    w2["router_w"] = rw
+    Lo, Lg = oracle.Layer(TINY, w2), Layer(TINY, w2, max_tokens=64)
+    x = synth.activations(16, TINY.d_model, seed=3)
+    x[5] = 0        # an all-zero token
+    g, ref, _ = _full_check(TINY, Lo, Lg, x)
+    assert not g["y"][5].any()
+    Lg.close()
+
+
+def test_all_tokens_to_the_same_experts(tiny):
+    w, L_orc, L_gpu = tiny
+    w2 = dict(w)
+    b = np.zeros(TINY.n_experts, np.float32)
+    b[[2, 11]] = 1000.0
+    w2["router_bias"] = b
+    Lo, Lg = oracle.Layer(TINY, w2), Layer(TINY, w2, max_tokens=512)
+    for T in (8, 64, 300):
+        x = synth.activations(T, TINY.d_model, seed=T + 1)
+        g, ref, _ = _full_check(TINY, Lo, Lg, x)
+        assert g["expert_counts"][2] == T and g["expert_counts"][11] == T
+    Lg.close()
+
+
+def test_deterministic_bits(big):
+    L_orc, L_gpu = big
+    x = bf16_from_bits(synth.activations(64, BIG.d_model, seed=5), "cuda")
+    y1 = L_gpu.forward(x).clone()
+    y2 = L_gpu.forward(x).clone()
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+
+
+def test_route_entry_point(big):
+    L_orc, L_gpu = big
+    x_bits = synth.activations(64, BIG.d_model, seed=6)
+    idx, w, counts = L_gpu.route(bf16_from_bits(x_bits, "cuda"))
+    torch.cuda.synchronize()
+    _, idx_ref, w_ref = L_orc.route(x_bits)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), w_ref.view(np.uint32))
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(idx_ref.ravel(), minlength=BIG.n_experts))
+
+
+def test_nan_input_sets_the_device_flag(tiny):
+    w, L_orc, L_gpu = tiny
+    x = bf16_from_bits(synth.activations(8, TINY.d_model, seed=1), "cuda")
+    x[2, 7] = float("nan")
+    L_gpu.device_flags(clear=True)
+    L_gpu.forward(x)
+    torch.cuda.synchronize()
+    assert L_gpu.device_flags(clear=True) & 0x1
+    # a clean call afterwards succeeds
+    x[2, 7] = 0.0
+    L_gpu.forward(x)
+    torch.cuda.synchronize()
+    assert L_gpu.device_flags() == 0
+
+
+def test_prefill_config_sampled_parity(big):
+    """T=4096: routing of every token and the permutation against the oracle,
+    full per-token comparison on a sample spread over the batch."""
+    L_orc, L_gpu = big
+    T = 4096
+    x = synth.activations(T, BIG.d_model, seed=0)
+    g = gpu_forward_with_taps(L_gpu, x)
+    logits, idx, w = L_orc.route(x)
+    assert np.array_equal(g["topk_idx"], idx)
+    assert np.array_equal(g["topk_w"].view(np.uint32), w.view(np.uint32))
+    assert np.array_equal(g["logits"].view(np.uint32), logits.view(np.uint32))
+    compare_permutation(BIG, g, idx)
+    tokens = np.unique(np.concatenate([[0, 1, T - 1], np.random.default_rng(0).choice(T, 21, replace=False)]))
+    tokens = tokens.astype(np.int32)
+    ref = L_orc.forward_tokens(x, tokens)
+    compare_tokens(BIG, g, ref, tokens)

@@ -116,11 +116,12 @@ def decode_bytes(n_active: int, T: int) -> int:
     return n_active * per_expert + E * D * 4 + T * D * 2 + T * D * 4
 
 
-def gateup_bytes(n_active: int, T: int) -> int:
-    """Algorithmic bytes of the gate/up kernel: the gate and up codes and
-    scales of the experts touched plus the int8 activations."""
+def experts_bytes(n_active: int, T: int) -> int:
+    """Algorithmic bytes of the expert-stage kernel (decode_experts_kernel):
+    packed codes and scales of the experts touched (gate, up, down), the int8
+    activations in and the fp32 layer output."""
     D, F = 2048, 512
-    return n_active * (2 * F * D // 4 + 2 * F * 4) + T * D
+    return n_active * (3 * F * D // 4 + (2 * F + D) * 4) + T * D + T * D * 4
 
 
 def run_gpu(args, rank: int, world: int):
@@ -182,8 +183,8 @@ def run_gpu(args, rank: int, world: int):
 
     total_ms = sum(t[1][2] for t in timed)
     per_T = {T: [t[1] for t in timed if t[0] == T] for T in DECODE_T}
-    gateup_ms = sum(x[1] - x[0] for T in DECODE_T for x in per_T[T])
-    gateup_alg = sum(gateup_bytes(n_active[T], T) for T in DECODE_T) * args.steps
+    experts_ms = sum(x[2] - x[0] for T in DECODE_T for x in per_T[T])
+    experts_alg = sum(experts_bytes(n_active[T], T) for T in DECODE_T) * args.steps
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host, all timed
     hx = {T: xs[T].cpu().pin_memory() for T in DECODE_T}
@@ -204,13 +205,13 @@ def run_gpu(args, rank: int, world: int):
                 e2e_ms += e0.elapsed_time(e1)
 
     # ---- max over ranks
-    vals = torch.tensor([total_ms, e2e_ms, gateup_ms], dtype=torch.float64, device=dev)
+    vals = torch.tensor([total_ms, e2e_ms, experts_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, gateup_ms = vals.tolist()
+    total_ms, e2e_ms, experts_ms = vals.tolist()
     tokens = sum(DECODE_T) * args.steps * world
     hbm, peak_kind = peaks()
-    achieved = gateup_alg / (gateup_ms * 1e-3) / 1e9
+    achieved = experts_alg / (experts_ms * 1e-3) / 1e9
     layer_bytes = sum(decode_bytes(n_active[T], T) for T in DECODE_T) * args.steps
     out = {
         "metric": METRIC,
@@ -232,18 +233,17 @@ def run_gpu(args, rank: int, world: int):
         "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(x[2] for x in per_T[T]) * 1e-3),
                            "us_per_forward": 1e3 * statistics.mean(x[2] for x in per_T[T]),
                            "us_route": 1e3 * statistics.mean(x[0] for x in per_T[T]),
-                           "us_gateup": 1e3 * statistics.mean(x[1] - x[0] for x in per_T[T]),
-                           "us_down": 1e3 * statistics.mean(x[2] - x[1] for x in per_T[T]),
+                           "us_experts": 1e3 * statistics.mean(x[2] - x[0] for x in per_T[T]),
                            "layer_hbm_frac": decode_bytes(n_active[T], T) /
                            (statistics.mean(x[2] for x in per_T[T]) * 1e-3) / 1e9 / hbm}
                   for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
-        "roofline": {"kernel": "gateup_gemv_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
+        "roofline": {"kernel": "decode_experts_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": None},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(T * shape.d_model * 2 for T in DECODE_T),
                 "d2h_bytes_per_step": sum(T * shape.d_model * 4 for T in DECODE_T)},
-        "gpu_launches": 3 * len(DECODE_T) * args.steps,
+        "gpu_launches": 2 * len(DECODE_T) * args.steps,
         "clocks": clocks,
     }
     return out, layer

@@ -68,8 +68,9 @@ enum {
 #define MAPLE_CFG_FORCE_TC 0x2u       /* use the tensor-core grouped GEMM for every T > 0 */
 
 /*
- * Layer shape.  Limits: d_model % 256 == 0; d_ff % 128 == 0; n_experts % 8 == 0
- * and 8 <= n_experts <= 1024; 1 <= top_k <= min(32, n_experts);
+ * Layer shape.  Limits: d_model = 256 * 2^i (256 .. 4096); d_ff = 128 * 2^j
+ * (128 .. 1024); n_experts % 16 == 0
+ * and 16 <= n_experts <= 1024; 1 <= top_k <= min(32, n_experts);
  * 1 <= max_tokens <= 65536.  max_tokens sizes the library-owned workspace.
  * decode_max_tokens: largest T served by the weight-streaming (GEMV) path;
  * 0 selects 64.  Larger T use the tcgen05 int8 grouped GEMM.

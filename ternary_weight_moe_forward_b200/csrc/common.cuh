@@ -106,6 +106,11 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p)
     return v;
 }
 
+// GPU-scope acquire-release fence: orders this thread's earlier global writes
+// before its later ones (and earlier reads before later reads) for all CTAs;
+// used around the last-arriver counters
+__device__ __forceinline__ void fence_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ void set_flag(unsigned *flag, unsigned bits)
 {
     if (flag) atomicOr(flag, bits);

@@ -11,6 +11,7 @@
 #include "layout.cuh"
 #include "pack.cuh"
 #include "route.cuh"
+#include "tc_gemm.cuh"
 
 using namespace maple;
 
@@ -38,7 +39,12 @@ struct maple_moe_s {
     int device;
     char *base;  // one device allocation: weights + workspace
     // weights
-    uint8_t *w_gu, *w_dn;
+    uint8_t *w_gu, *w_dn;          // GEMV layout
+    uint8_t *w_tc_gu, *w_tc_dn;    // tensor-core layout
+    int4 *pieces;
+    int *n_pieces;
+    int8_t *xperm;                 // q_x rows in slot order (tensor-core path)
+    CUtensorMap map_xperm, map_qh; // TMA maps of the activation operands
     float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
     // workspace
     int8_t *qx;
@@ -54,6 +60,9 @@ struct maple_moe_s {
     int *sumqh;
     float *ye;
     unsigned *tg_cnt, *glob_cnt, *exp_cnt, *comb_cnt;
+    unsigned *ready;      // [E] epoch of each expert's published q_h (decode kernel)
+    unsigned epoch;
+    int dec_nbuf, dec_buf_bytes;
     uint16_t *xn;
     // flag word in host-mapped memory
     unsigned *flag_host;
@@ -109,11 +118,105 @@ extern "C" int maple_moe_pack_ternary(const int8_t *values, int64_t rows, int32_
     return launch_status();
 }
 
+// TMA map over an int8 row matrix [rows][cols]: boxes of 128 rows x 128
+// bytes with the 128-byte swizzle (the UMMA K-major operand layout)
+typedef CUresult (*encode_tiled_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static int make_act_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols)
+{
+    static encode_tiled_fn encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return MAPLE_ERR_CUDA;
+        encode = (encode_tiled_fn)fn;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols};
+    cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcMaxN};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MAPLE_OK : MAPLE_ERR_CUDA;
+}
+
+static void allow_max_smem(const void *fn, int device)
+{
+    cudaFuncAttributes fa;
+    int optin = 0;
+    if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+}
+
+typedef void (*route_fn)(RouteArgs);
+typedef void (*gemv_fn)(GemvArgs);
+
+template <int NPER>
+static route_fn pick_route_n(int ni)
+{
+    switch (ni) {
+    case 1: return route_kernel<1, NPER>;
+    case 2: return route_kernel<2, NPER>;
+    case 4: return route_kernel<4, NPER>;
+    case 8: return route_kernel<8, NPER>;
+    case 16: return route_kernel<16, NPER>;
+    default: return nullptr;
+    }
+}
+static route_fn pick_route(int D, int E) { return E <= 256 ? pick_route_n<8>(D / 256) : pick_route_n<32>(D / 256); }
+
+template <int NPER>
+static route_fn pick_qtopk_n(int ni)
+{
+    switch (ni) {
+    case 1: return quant_topk_kernel<1, NPER>;
+    case 2: return quant_topk_kernel<2, NPER>;
+    case 4: return quant_topk_kernel<4, NPER>;
+    case 8: return quant_topk_kernel<8, NPER>;
+    case 16: return quant_topk_kernel<16, NPER>;
+    default: return nullptr;
+    }
+}
+static route_fn pick_qtopk(int D, int E) { return E <= 256 ? pick_qtopk_n<8>(D / 256) : pick_qtopk_n<32>(D / 256); }
+
+static gemv_fn pick_gateup(int D)
+{
+    switch (D / 256) {
+    case 1: return gateup_gemv_kernel<1>;
+    case 2: return gateup_gemv_kernel<2>;
+    case 4: return gateup_gemv_kernel<4>;
+    case 8: return gateup_gemv_kernel<8>;
+    case 16: return gateup_gemv_kernel<16>;
+    default: return nullptr;
+    }
+}
+static gemv_fn pick_down(int F)
+{
+    switch (F / 128) {
+    case 1: return down_gemv_kernel<1>;
+    case 2: return down_gemv_kernel<2>;
+    case 4: return down_gemv_kernel<4>;
+    case 8: return down_gemv_kernel<8>;
+    default: return nullptr;
+    }
+}
+
+static bool pow2_upto(int v, int hi) { return v >= 1 && v <= hi && (v & (v - 1)) == 0; }
+
 static int check_shape(const maple_moe_config *c)
 {
-    if (c->d_model <= 0 || c->d_model % 256 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
-    if (c->d_ff <= 0 || c->d_ff % 128 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
-    if (c->n_experts < 8 || c->n_experts > kMaxExperts || c->n_experts % 8 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_model <= 0 || c->d_model % 256 != 0 || !pow2_upto(c->d_model / 256, 16)) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->d_ff <= 0 || c->d_ff % 128 != 0 || !pow2_upto(c->d_ff / 128, 8)) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->n_experts < 16 || c->n_experts > kMaxExperts || c->n_experts % 16 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->n_experts) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     if (c->max_tokens < 1 || c->max_tokens > 65536) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     if (c->decode_max_tokens < 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
@@ -152,6 +255,9 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     const int64_t nblk = (Tm + kPermBlockTokens - 1) / kPermBlockTokens;
     Arena ar;
     size_t o_gu = ar.take(E * gu_bytes_per_expert(D, F)), o_dn = ar.take(E * dn_bytes_per_expert(D, F));
+    size_t o_tgu = ar.take(E * F * D / 2), o_tdn = ar.take(E * D * F / 4);
+    size_t o_pc = ar.take((E + S / kPieceSlots + 1) * 16), o_npc = ar.take(4);
+    size_t o_xp = ar.take(S * D);
     size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
     size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
     size_t o_qx = ar.take(Tm * D), o_sx = ar.take(Tm * 4), o_sumx = ar.take(Tm * 4);
@@ -162,7 +268,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     size_t o_ye = ar.take(S * D * 4);
     size_t o_ctr = ar.take(0);
     size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4), o_ec = ar.take(E * 4);
-    size_t o_cc = ar.take(Tm * (D / 32) * 4);
+    size_t o_cc = ar.take(Tm * (D / 32) * 4), o_rdy = ar.take(E * 4);
     size_t o_xn = ar.take(Tm * D * 2);
 
     if (cudaMalloc(&h->base, ar.size) != cudaSuccess) {
@@ -181,6 +287,11 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     char *b = h->base;
     h->w_gu = (uint8_t *)(b + o_gu);
     h->w_dn = (uint8_t *)(b + o_dn);
+    h->w_tc_gu = (uint8_t *)(b + o_tgu);
+    h->w_tc_dn = (uint8_t *)(b + o_tdn);
+    h->pieces = (int4 *)(b + o_pc);
+    h->n_pieces = (int *)(b + o_npc);
+    h->xperm = (int8_t *)(b + o_xp);
     h->alpha_gate = (float *)(b + o_ag);
     h->alpha_up = (float *)(b + o_au);
     h->alpha_down = (float *)(b + o_ad);
@@ -208,6 +319,11 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->glob_cnt = (unsigned *)(b + o_gc);
     h->exp_cnt = (unsigned *)(b + o_ec);
     h->comb_cnt = (unsigned *)(b + o_cc);
+    h->ready = (unsigned *)(b + o_rdy);
+    h->epoch = 0;
+    h->dec_buf_bytes = (int)(16 * D > 32 * F ? 16 * D : 32 * F);
+    h->dec_nbuf = kDecRingBytes / h->dec_buf_bytes;
+    if (h->dec_nbuf > 8) h->dec_nbuf = 8;
     h->xn = (uint16_t *)(b + o_xn);
 
     cudaStream_t st = (cudaStream_t)stream;
@@ -224,6 +340,25 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
                                                                                      h->D, h->F, (uint32_t *)h->w_gu);
     repack_dn_kernel<<<grid_for(E * (D / 32) * (F / 64) * 128, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
                                                                                     (uint32_t *)h->w_dn);
+    repack_tc_gu_kernel<<<grid_for(E * F * D / 8, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E, h->D, h->F,
+                                                                          (uint32_t *)h->w_tc_gu);
+    repack_tc_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
+                                                                           (uint32_t *)h->w_tc_dn);
+    if (make_act_map(&h->map_xperm, h->xperm, S, D) || make_act_map(&h->map_qh, h->qh, S, F)) {
+        cudaFree(h->base);
+        cudaFreeHost(h->flag_host);
+        delete h;
+        return MAPLE_ERR_CUDA;
+    }
+    // allow every kernel the largest dynamic shared memory the device offers, so
+    // that handles of different shapes never cap one another's launches
+    allow_max_smem((const void *)tc_gemm_kernel<0>, h->device);
+    allow_max_smem((const void *)tc_gemm_kernel<1>, h->device);
+    allow_max_smem((const void *)pick_route(h->D, h->E), h->device);
+    allow_max_smem((const void *)pick_qtopk(h->D, h->E), h->device);
+    allow_max_smem((const void *)pick_gateup(h->D), h->device);
+    allow_max_smem((const void *)pick_down(h->F), h->device);
+    allow_max_smem((const void *)decode_experts_kernel, h->device);
     if (cudaGetLastError() != cudaSuccess) {
         cudaFree(h->base);
         cudaFreeHost(h->flag_host);
@@ -248,7 +383,7 @@ static int take_flag(maple_moe_t h)
 
 // routing stage: quantise, logits, top-k (+ the permutation)
 static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
-                     float *out_w, int32_t *out_counts, bool permute, cudaStream_t st)
+                     float *out_w, int32_t *out_counts, bool permute, bool pieces, cudaStream_t st)
 {
     RouteArgs a;
     memset(&a, 0, sizeof a);
@@ -284,13 +419,21 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     a.active = h->active;
     a.n_active = h->n_active;
     a.flag = h->flag_dev;
-    const bool fused = permute && (int64_t)T * h->E <= kFusedMarkBytes;
+    // few tokens: one latency-oriented kernel (logits, top-k by the last CTA of
+    // each token group, permutation by the last group); many tokens: a tiled
+    // router GEMM, then quantise + top-k, then the multi-CTA permutation
+    const bool small = T <= kRouteSmallT;
+    const bool fused = small && permute && !pieces && (int64_t)T * h->E <= kFusedMarkBytes;
     a.fuse_permute = fused ? 1 : 0;
-    dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
-    if (h->E <= 256)
-        route_kernel<8><<<grid, 256, 0, st>>>(a);
-    else
-        route_kernel<32><<<grid, 256, 0, st>>>(a);
+    if (small) {
+        dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
+        pick_route(h->D, h->E)<<<grid, 256, route_smem_bytes(h->D), st>>>(a);
+    } else {
+        dim3 grid((T + kRgTok - 1) / kRgTok, h->E / kRgExp);
+        router_gemm_kernel<<<grid, 256, 0, st>>>(x, T, h->D, h->E, h->router_w, h->router_bias, h->logits,
+                                                 a.tap_logits);
+        pick_qtopk(h->D, h->E)<<<(T + 7) / 8, 256, (size_t)8 * h->D * 2, st>>>(a);
+    }
     if (permute && !fused) {
         PermArgs p;
         memset(&p, 0, sizeof p);
@@ -308,6 +451,8 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
         p.out_counts = a.out_counts;
         p.tap_offsets = a.tap_offsets;
         p.tap_perm = a.tap_perm;
+        p.pieces = pieces ? h->pieces : nullptr;
+        p.n_pieces = h->n_pieces;
         p.flag = h->flag_dev;
         const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
         perm_count_kernel<<<nblk, 256, 0, st>>>(p);
@@ -358,11 +503,36 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         g.tap_qh = taps->q_h;
         g.tap_sh = taps->s_h;
     }
+    g.flag_dev = h->flag_dev;
+    if (h->dec_nbuf >= 2) {
+        // persistent, cooperative: one CTA per SM streams gate/up then down
+        DecodeArgs d;
+        d.g = g;
+        d.ready = h->ready;
+        d.epoch = ++h->epoch;
+        d.nbuf = h->dec_nbuf;
+        d.buf_bytes = h->dec_buf_bytes;
+        cudaLaunchConfig_t lc;
+        memset(&lc, 0, sizeof lc);
+        lc.gridDim = dim3(h->num_sms);
+        lc.blockDim = dim3(kDecThreads);
+        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, h->dec_buf_bytes, h->dec_nbuf);
+        lc.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&lc, decode_experts_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+        stage_event(h, 2, st);
+        stage_event(h, 3, st);
+        return launch_status();
+    }
+    // one CTA per (active expert, row block); CTAs past the active experts exit at once
     const int64_t max_active = (int64_t)T * h->K < h->E ? (int64_t)T * h->K : h->E;
-    const int cap = h->num_sms * 4;
-    gateup_gemv_kernel<<<grid_for(max_active * (h->F / 16), kGemvWarps, cap), kGemvWarps * 32, 0, st>>>(g);
+    pick_gateup(h->D)<<<(unsigned)(max_active * (h->F / 32)), kGemvWarps * 32, gemv_smem_bytes(h->D), st>>>(g);
     stage_event(h, 2, st);
-    down_gemv_kernel<<<grid_for(max_active * (h->D / 32), kGemvWarps, cap), kGemvWarps * 32, 0, st>>>(g);
+    pick_down(h->F)<<<(unsigned)(max_active * (h->D / 128)), kGemvWarps * 32, gemv_smem_bytes(h->F), st>>>(g);
     stage_event(h, 3, st);
     return launch_status();
 }
@@ -388,18 +558,66 @@ extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int3
     if (!x || !aligned16(x)) return MAPLE_ERR_INVALID_ARG;
     for (const void *p : {(const void *)topk_idx, (const void *)topk_w, (const void *)expert_counts})
         if (p && !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
-    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr,
+    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr, false,
                      (cudaStream_t)stream);
+}
+
+// tensor-core expert stage: gate/up grouped GEMM, requantise, down grouped GEMM, combine
+static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
+                          cudaStream_t st)
+{
+    const int S = T * h->K;
+    TcArgs g;
+    memset(&g, 0, sizeof g);
+    g.D = h->D;
+    g.F = h->F;
+    g.K = h->K;
+    g.pieces = h->pieces;
+    g.n_pieces = h->n_pieces;
+    g.perm = h->perm;
+    g.sx = h->sx;
+    g.sh = h->sh;
+    g.flag = h->flag_dev;
+    g.codes = h->w_tc_gu;
+    g.alpha0 = h->alpha_gate;
+    g.alpha1 = h->alpha_up;
+    g.out = h->h;
+    g.tap0 = taps ? taps->acc_gate : nullptr;
+    g.tap1 = taps ? taps->acc_up : nullptr;
+    gather_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->qx, h->perm, h->K, h->D, S, h->xperm);
+    tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_xperm, g);
+    requant_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->h, S, h->F, h->perm, h->qh, h->sh, taps ? taps->q_h : nullptr,
+                                                   taps ? taps->s_h : nullptr);
+    stage_event(h, 2, st);
+    g.codes = h->w_tc_dn;
+    g.alpha0 = h->alpha_down;
+    g.alpha1 = nullptr;
+    g.out = h->ye;
+    g.tap0 = taps ? taps->acc_down : nullptr;
+    g.tap1 = nullptr;
+    tc_gemm_kernel<1><<<h->num_sms, kTcThreads, TcSmem<1>::kTotal, st>>>(h->map_qh, g);
+    combine_kernel<<<grid_for((int64_t)T * h->D / 4, 256, h->num_sms * 8), 256, 0, st>>>(h->ye, h->inv, h->topk_w, T,
+                                                                                       h->K, h->D, y, resid);
+    stage_event(h, 3, st);
+    return launch_status();
+}
+
+static bool use_tc(maple_moe_t h, int T)
+{
+    if (h->cfg_flags & MAPLE_CFG_FORCE_GEMV) return false;
+    if (h->cfg_flags & MAPLE_CFG_FORCE_TC) return true;
+    return T > h->dmax;
 }
 
 static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const float *resid,
                         const maple_moe_taps *taps, cudaStream_t st)
 {
+    const bool tc = use_tc(h, T);
     stage_event(h, 0, st);
-    int rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, st);
+    int rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, st);
     if (rc) return rc;
     stage_event(h, 1, st);
-    return run_experts(h, T, y, resid, taps, st);
+    return tc ? run_experts_tc(h, T, y, resid, taps, st) : run_experts(h, T, y, resid, taps, st);
 }
 
 extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const maple_moe_taps *taps,

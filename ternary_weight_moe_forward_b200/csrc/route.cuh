@@ -11,6 +11,7 @@ constexpr int kRouteExperts = 8;       // experts per route CTA (one per warp)
 constexpr int kFusedMarkBytes = 16384; // T*E bytes the fused single-CTA permutation can hold
 constexpr int kPermBlockTokens = 32;   // tokens per CTA of the multi-CTA permutation
 constexpr int kMaxExperts = 1024;
+constexpr int kRouteSmallT = 64;       // up to this many tokens the latency-oriented router runs
 
 struct RouteArgs {
     const uint16_t *x;
@@ -96,16 +97,19 @@ __device__ void scan_experts(const int *s_cnt, int *s_off, int E, int *active, i
 }
 
 // ---------------------------------------------------------------------------
-// quantise one token (one warp): amax, codes, scale, sum of codes
+// quantise one token (one warp) from its bf16 row xr (shared memory): amax,
+// codes, scale, sum of codes
 // ---------------------------------------------------------------------------
-__device__ void quantize_token_warp(const RouteArgs &a, int t)
+template <int NI>
+__device__ void quantize_token_warp(const RouteArgs &a, int t, const uint16_t *xr)
 {
     const int lane = threadIdx.x & 31;
-    const uint16_t *xr = a.x + (size_t)t * a.D;
+    uint4 v[NI];
     float amax = 0.0f;
-    for (int i = 0; i < a.D / 256; i++) {
-        uint4 v = *reinterpret_cast<const uint4 *>(xr + 256 * i + 8 * lane);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < NI; i++) {
+        v[i] = *reinterpret_cast<const uint4 *>(xr + 256 * i + 8 * lane);
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
         for (int m = 0; m < 4; m++) {
             amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[m] & 0xffffu)));
@@ -115,9 +119,9 @@ __device__ void quantize_token_warp(const RouteArgs &a, int t)
     amax = warp_max(amax);
     const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     int sum = 0;
-    for (int i = 0; i < a.D / 256; i++) {
-        uint4 v = *reinterpret_cast<const uint4 *>(xr + 256 * i + 8 * lane);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < NI; i++) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
         uint32_t packed[2] = {0u, 0u};
 #pragma unroll
         for (int m = 0; m < 8; m++) {
@@ -263,57 +267,67 @@ __device__ void scatter_marks(const uint8_t *mark, int t0, int nt, int K, int E,
 // with fuse_permute the last token group to finish builds the permutation.
 // Router logit order: lane l sums j = 256*i + 8*l + m (fmaf, from 0), then the
 // 32 lane partials are added by the xor tree (distance 16, 8, 4, 2, 1).
+// Dynamic shared memory: route_smem_bytes(D) (the bf16 rows of the 8 tokens,
+// later reused for the permutation's marks).
 // ---------------------------------------------------------------------------
-template <int NPER>
+__host__ __device__ inline size_t route_smem_bytes(int D)
+{
+    const size_t xb = (size_t)kRouteTokens * D * 2;
+    return xb > (size_t)kFusedMarkBytes ? xb : (size_t)kFusedMarkBytes;
+}
+
+template <int NI, int NPER>
 __global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
 {
+    extern __shared__ __align__(16) uint8_t rsm[];
+    uint16_t *xs = (uint16_t *)rsm;   // [nt][D] bf16
     __shared__ unsigned s_last;
     __shared__ int s_warp[33];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int eb = blockIdx.x, tg = blockIdx.y;
     const int t0 = tg * kRouteTokens;
     const int nt = min(kRouteTokens, a.T - t0);
+    const int e = eb * kRouteExperts + warp;
 
-    if (eb == 0 && warp < nt) quantize_token_warp(a, t0 + warp);
+    // this lane's part of the router row, all in flight at once
+    const float *wr = a.Wr + (size_t)e * a.D;
+    float4 w0[NI], w1[NI];
+#pragma unroll
+    for (int i = 0; i < NI; i++) {
+        w0[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane));
+        w1[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane + 4));
+    }
+    // stage the token rows
+    const int row8 = a.D / 8;
+    for (int i = threadIdx.x; i < nt * row8; i += blockDim.x)
+        reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D) + i);
+    __syncthreads();
 
-    {
-        const int e = eb * kRouteExperts + warp;
-        const float *wr = a.Wr + (size_t)e * a.D;
-        float acc[kRouteTokens];
+    if (eb == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
+
+    for (int tt = 0; tt < nt; tt++) {
+        float acc = 0.0f;
 #pragma unroll
-        for (int tt = 0; tt < kRouteTokens; tt++) acc[tt] = 0.0f;
-        for (int i = 0; i < a.D / 256; i++) {
-            const float4 w0 = *reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane);
-            const float4 w1 = *reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane + 4);
-            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        for (int i = 0; i < NI; i++) {
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)tt * a.D + 256 * i + 8 * lane);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            const float wv[8] = {w0[i].x, w0[i].y, w0[i].z, w0[i].w, w1[i].x, w1[i].y, w1[i].z, w1[i].w};
 #pragma unroll
-            for (int tt = 0; tt < kRouteTokens; tt++) {
-                if (tt < nt) {
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(a.x + (size_t)(t0 + tt) * a.D + 256 * i + 8 * lane);
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                    for (int m = 0; m < 8; m++) {
-                        uint32_t bits = (m & 1) ? (xw[m >> 1] >> 16) : (xw[m >> 1] & 0xffffu);
-                        acc[tt] = __fmaf_rn(bf16_bits_to_f32(bits), wv[m], acc[tt]);
-                    }
-                }
+            for (int m = 0; m < 8; m++) {
+                uint32_t bits = (m & 1) ? (xw[m >> 1] >> 16) : (xw[m >> 1] & 0xffffu);
+                acc = __fmaf_rn(bf16_bits_to_f32(bits), wv[m], acc);
             }
         }
-#pragma unroll
-        for (int tt = 0; tt < kRouteTokens; tt++) {
-            if (tt < nt) {
-                float v = warp_tree_sum(acc[tt]);
-                if (a.bias) v = __fadd_rn(v, a.bias[e]);
-                if (lane == 0) {
-                    a.logits[(size_t)(t0 + tt) * a.E + e] = v;
-                    if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = v;
-                }
-            }
+        float v = warp_tree_sum(acc);
+        if (a.bias) v = __fadd_rn(v, a.bias[e]);
+        if (lane == 0) {
+            a.logits[(size_t)(t0 + tt) * a.E + e] = v;
+            if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = v;
         }
     }
 
     // ---- last CTA of this token group: top-k + softmax
-    __threadfence();
+    fence_gpu();
     __syncthreads();
     if (threadIdx.x == 0) {
         unsigned prev = atomicAdd(a.tg_cnt + tg, 1u);
@@ -321,13 +335,13 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
+    fence_gpu();
     if (threadIdx.x == 0) a.tg_cnt[tg] = 0;
     if (warp < nt) topk_token_warp<NPER>(a, t0 + warp);
     if (!a.fuse_permute) return;
 
     // ---- last token group: permutation of all T*K slots in one CTA
-    __threadfence();
+    fence_gpu();
     __syncthreads();
     if (threadIdx.x == 0) {
         unsigned prev = atomicAdd(a.glob_cnt, 1u);
@@ -335,29 +349,29 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
+    fence_gpu();
     if (threadIdx.x == 0) *a.glob_cnt = 0;
 
-    __shared__ __align__(16) uint8_t s_mark[kFusedMarkBytes];
+    uint8_t *s_mark = rsm;   // reuses the token rows: T*E <= kFusedMarkBytes
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_off[kMaxExperts + 1];
     build_marks(s_mark, a.topk_idx, 0, a.T, a.K, a.E, a.flag);
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) {
         int c = 0;
-        for (int t = 0; t < a.T; t++) c += s_mark[t * a.E + e] != 0;
-        s_cnt[e] = c;
+        for (int t = 0; t < a.T; t++) c += s_mark[t * a.E + ee] != 0;
+        s_cnt[ee] = c;
     }
     __syncthreads();
     scan_experts(s_cnt, s_off, a.E, a.active, a.n_active, s_warp);
-    for (int e = threadIdx.x; e <= a.E; e += blockDim.x) {
-        a.offsets[e] = s_off[e];
-        if (a.tap_offsets) a.tap_offsets[e] = s_off[e];
-        if (e < a.E) {
-            a.counts[e] = s_cnt[e];
-            if (a.out_counts) a.out_counts[e] = s_cnt[e];
+    for (int ee = threadIdx.x; ee <= a.E; ee += blockDim.x) {
+        a.offsets[ee] = s_off[ee];
+        if (a.tap_offsets) a.tap_offsets[ee] = s_off[ee];
+        if (ee < a.E) {
+            a.counts[ee] = s_cnt[ee];
+            if (a.out_counts) a.out_counts[ee] = s_cnt[ee];
         }
     }
-    scatter_marks(s_mark, 0, a.T, a.K, a.E, [&](int e) { return s_off[e]; }, a.perm, a.inv, a.tap_perm);
+    scatter_marks(s_mark, 0, a.T, a.K, a.E, [&](int ee) { return s_off[ee]; }, a.perm, a.inv, a.tap_perm);
 }
 
 // ---------------------------------------------------------------------------
@@ -370,8 +384,12 @@ struct PermArgs {
     int *blk_cnt;  // [nblk][E]: counts, then (after pass 2) global base positions
     int *counts, *offsets, *perm, *inv, *active, *n_active;
     int *out_counts, *tap_offsets, *tap_perm;
+    int4 *pieces;   // optional: expert slot ranges of at most kPieceSlots for the grouped GEMM
+    int *n_pieces;
     unsigned *flag;
 };
+
+constexpr int kPieceSlots = 128;
 
 __global__ void __launch_bounds__(256) perm_count_kernel(PermArgs a)
 {
@@ -412,6 +430,20 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a)
             for (int b = 0; b < nblk; b++) a.blk_cnt[(size_t)b * a.E + e] += s_off[e];
         }
     }
+    if (a.pieces) {
+        // split every expert's slots into ceil(count / kPieceSlots) near-equal ranges
+        const int e = threadIdx.x;
+        const int cnt = e < a.E ? s_cnt[e] : 0;
+        const int np = (cnt + kPieceSlots - 1) / kPieceSlots;
+        int total;
+        const int base = block_excl_scan(np, s_warp, &total);
+        for (int i = 0; i < np; i++) {
+            const int q = cnt / np, rem = cnt % np;
+            const int start = i * q + min(i, rem);
+            a.pieces[base + i] = make_int4(e, s_off[e] + start, q + (i < rem ? 1 : 0), 0);
+        }
+        if (threadIdx.x == 0) *a.n_pieces = total;
+    }
 }
 
 __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a)
@@ -422,6 +454,114 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a)
     build_marks(s_mark, a.idx, t0, nt, a.K, a.E, nullptr);
     const int *base = a.blk_cnt + (size_t)blockIdx.x * a.E;
     scatter_marks(s_mark, t0, nt, a.K, a.E, [&](int e) { return base[e]; }, a.perm, a.inv, a.tap_perm);
+}
+
+// ---------------------------------------------------------------------------
+// Router for many tokens (register-tiled SIMT GEMM in the same fixed order).
+// CTA = 32 tokens x 16 experts, 8 warps; warp w owns tokens 8*(w/2)..+7 and
+// experts 8*(w%2)..+7 and keeps, per lane, the 64 partial sums of that lane's
+// part of K (lane l: j = 256*i + 8*l + m).  Per K chunk of 256 the CTA stages
+// the token rows (bf16) and router rows (fp32) in shared memory.  The 32 lane
+// partials of every output are then added with the same xor tree as the
+// decode router, as a transposing reduction: at the level with distance o a
+// lane keeps half of its outputs and sends the other half to lane l^o, so lane
+// l ends with outputs 2l and 2l+1 (token 2l/8, expert 2l%8 + {0,1}).
+// ---------------------------------------------------------------------------
+constexpr int kRgTok = 32, kRgExp = 16;
+
+template <int N>
+__device__ __forceinline__ void tree_level(float (&v)[64], int off, bool upper)
+{
+#pragma unroll
+    for (int j = 0; j < N / 2; j++) {
+        const float send = upper ? v[j] : v[j + N / 2];
+        const float keep = upper ? v[j + N / 2] : v[j];
+        v[j] = __fadd_rn(keep, __shfl_xor_sync(FULL, send, off));
+    }
+}
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *x, int T, int D, int E, const float *Wr,
+                                                          const float *bias, float *logits, float *tap_logits)
+{
+    __shared__ __align__(16) uint16_t sx[kRgTok][256];
+    __shared__ __align__(16) float sw[kRgExp][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * kRgTok, e0 = blockIdx.y * kRgExp;
+    const int wt = (warp >> 1) * 8, we = (warp & 1) * 8;
+    float acc[64];
+#pragma unroll
+    for (int o = 0; o < 64; o++) acc[o] = 0.0f;
+    for (int i = 0; i < D / 256; i++) {
+        __syncthreads();
+        // stage token rows (32 x 256 bf16 = 1024 x 16 B) and router rows (16 x 256 fp32 = 1024 x 16 B)
+        for (int q = threadIdx.x; q < kRgTok * 32; q += 256) {
+            const int tt = q >> 5, c = q & 31;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (t0 + tt < T) v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * D + 256 * i) + c);
+            reinterpret_cast<uint4 *>(&sx[tt][0])[c] = v;
+        }
+        for (int q = threadIdx.x; q < kRgExp * 64; q += 256) {
+            const int ee = q >> 6, c = q & 63;
+            reinterpret_cast<float4 *>(&sw[ee][0])[c] =
+                __ldg(reinterpret_cast<const float4 *>(Wr + (size_t)(e0 + ee) * D + 256 * i) + c);
+        }
+        __syncthreads();
+        float wv[8][8];
+#pragma unroll
+        for (int b = 0; b < 8; b++) {
+            const float4 w0 = *reinterpret_cast<const float4 *>(&sw[we + b][8 * lane]);
+            const float4 w1 = *reinterpret_cast<const float4 *>(&sw[we + b][8 * lane + 4]);
+            wv[b][0] = w0.x; wv[b][1] = w0.y; wv[b][2] = w0.z; wv[b][3] = w0.w;
+            wv[b][4] = w1.x; wv[b][5] = w1.y; wv[b][6] = w1.z; wv[b][7] = w1.w;
+        }
+#pragma unroll
+        for (int a = 0; a < 8; a++) {
+            const uint4 xv = *reinterpret_cast<const uint4 *>(&sx[wt + a][8 * lane]);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            float xf[8];
+#pragma unroll
+            for (int m = 0; m < 8; m++) xf[m] = bf16_bits_to_f32((m & 1) ? (xw[m >> 1] >> 16) : (xw[m >> 1] & 0xffffu));
+#pragma unroll
+            for (int b = 0; b < 8; b++)
+#pragma unroll
+                for (int m = 0; m < 8; m++) acc[a * 8 + b] = __fmaf_rn(xf[m], wv[b][m], acc[a * 8 + b]);
+        }
+    }
+    tree_level<64>(acc, 16, lane & 16);
+    tree_level<32>(acc, 8, lane & 8);
+    tree_level<16>(acc, 4, lane & 4);
+    tree_level<8>(acc, 2, lane & 2);
+    tree_level<4>(acc, 1, lane & 1);
+#pragma unroll
+    for (int q = 0; q < 2; q++) {
+        const int o = 2 * lane + q;
+        const int t = t0 + wt + o / 8, e = e0 + we + o % 8;
+        if (t < T) {
+            float v = acc[q];
+            if (bias) v = __fadd_rn(v, bias[e]);
+            logits[(size_t)t * E + e] = v;
+            if (tap_logits) tap_logits[(size_t)t * E + e] = v;
+        }
+    }
+}
+
+// quantise + top-k/softmax for many tokens: one warp per token
+// (dynamic shared memory: 8 rows of D bf16)
+template <int NI, int NPER>
+__global__ void __launch_bounds__(256) quant_topk_kernel(RouteArgs a)
+{
+    extern __shared__ __align__(16) uint8_t qsm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint16_t *xr = (uint16_t *)qsm + (size_t)warp * NI * 256;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= a.T) return;
+#pragma unroll
+    for (int i = 0; i < NI; i++)
+        reinterpret_cast<uint4 *>(xr + 256 * i)[lane] =
+            __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t * a.D + 256 * i) + lane);
+    __syncwarp();
+    quantize_token_warp<NI>(a, t, xr);
+    topk_token_warp<NPER>(a, t);
 }
 
 }  // namespace maple

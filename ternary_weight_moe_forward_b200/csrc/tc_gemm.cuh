@@ -1,0 +1,565 @@
+// Prefill expert stage on the 5th-generation tensor cores (tcgen05, int8).
+//
+// Grouped GEMM over "pieces": a piece is up to 128 consecutive slots of one
+// expert in the permutation.  A tile is (piece, 128-row block of the weight
+// matrix).  The MMA computes D[128 weight rows][N slots] (M = 128, N = the
+// piece size rounded up to 16, K = 32 per instruction) with
+//   A = ternary weights, expanded in shared memory from 2-bit codes to int8
+//       {0, +64, -64} (64 * t: the code sits in the two top bits of the byte),
+//   B = int8 activation rows of the piece's slots, loaded by the tensor
+//       memory accelerator (TMA) from a slot-ordered copy of the rows,
+// both K-major with the 128-byte swizzle, the int32 accumulator in tensor
+// memory (two accumulator buffers, so the epilogue of one tile overlaps the
+// MMAs of the next).  The accumulator is 64x the ternary dot product; the epilogue shifts
+// it back (exact).
+//
+// Warp roles (16 warps): warp 0 issues the bulk copies of the 2-bit codes
+// and the TMA loads of the activation tiles, warp 1 issues the MMAs (and owns
+// the TMEM allocation), warps 4..7 run the epilogue (TMEM lane quarter =
+// warp % 4), warps 8..15 expand the codes into int8 tiles.  Stage hand-off uses mbarriers; every wait is
+// bounded in time and a timeout makes the whole CTA drain and return with a
+// device flag set.
+//
+// Mode 0 (gate/up): A = gate rows and up rows of one 128-row block (two MMAs
+// per K step, gate and up accumulators 128 columns apart), B = q_x rows of the
+// slots' tokens; the epilogue writes h = SiLU(g) * u (fp32, slot order).
+// Mode 1 (down): A = 128 output channels of the down matrix, B = q_h rows
+// (consecutive slot positions); the epilogue writes yE (fp32, slot order).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace maple {
+
+constexpr int kTcThreads = 512;
+constexpr int kTcMaxN = 128;
+constexpr int kTcBK = 128;  // K elements (bytes) per stage = one swizzle row
+
+// 2-bit tensor-core layout, one 16-value word per (row, 16-column chunk):
+//   gate/up [E][F/128][D/128][2][128][8] words, down [E][D/128][F/128][128][8]
+// word w of (row, stage ks) holds columns ks*128 + 16w + 4k + b at bits
+// 8b + 2k as a two's complement 2-bit code (+1 -> 01, -1 -> 11, 0 -> 00).
+__host__ __device__ inline uint32_t tc_word(uint32_t canon)
+{
+    uint32_t out = 0;
+    for (int i = 0; i < 16; i++) {
+        uint32_t c = (canon >> (2 * i)) & 3u;
+        uint32_t s = c == 1u ? 1u : (c == 2u ? 3u : 0u);
+        out |= s << (8 * (i & 3) + 2 * (i >> 2));
+    }
+    return out;
+}
+
+template <int MODE>
+struct TcCfg;
+template <>
+struct TcCfg<0> {
+    static constexpr int kStages = 4;
+    static constexpr int kABytes = 2 * 128 * kTcBK;   // gate + up blocks
+    static constexpr int kCodeBytes = 2 * 128 * 32;   // 8 words of 4 bytes per row
+};
+template <>
+struct TcCfg<1> {
+    static constexpr int kStages = 6;
+    static constexpr int kABytes = 128 * kTcBK;
+    static constexpr int kCodeBytes = 128 * 32;
+};
+
+template <int MODE>
+struct TcSmem {
+    static constexpr int kBBytes = kTcMaxN * kTcBK;
+    static constexpr int kStage = TcCfg<MODE>::kABytes + kBBytes + TcCfg<MODE>::kCodeBytes;
+    static constexpr int kA = 0, kB = TcCfg<MODE>::kABytes, kCodes = kB + kBBytes;
+    static constexpr int kBars = TcCfg<MODE>::kStages * kStage;
+    static constexpr int kTotal = kBars + 1024 + 1024;  // barriers etc. + alignment slack
+    static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+};
+
+struct TcArgs {
+    int D, F, K;
+    const int4 *pieces;      // {expert, first position, count, 0}
+    const int *n_pieces;
+    const uint8_t *codes;    // tensor-core layout
+    const int *perm;         // position -> slot
+    const float *sx, *sh;
+    const float *alpha0, *alpha1;  // mode 0: gate, up; mode 1: down, unused
+    float *out;              // mode 0: h [S][F]; mode 1: yE [S][D]
+    int *tap0, *tap1;        // mode 0: acc_gate, acc_up; mode 1: acc_down
+    unsigned *flag;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any legitimate wait
+
+// Wait for the phase of `bar` with the given parity to complete.  Gives up
+// after kWaitLimitNs, or at once when another role of the CTA has given up;
+// returns false then (and raises the CTA abort word and the device flag).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, unsigned *flag)
+{
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_test(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            *abort = 1u;
+            set_flag(flag, MAPLE_DEVFLAG_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+// 2-D tiled TMA load (box given by the tensor map) into 128B-swizzled shared memory
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t holder_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder_smem), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, int8 x int8 -> int32
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;             // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: next 8-row atom
+    d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;             // 128-byte swizzle
+    return d;
+}
+
+// instruction descriptor: kind::i8, s8 x s8 -> s32, both K-major, M = 128
+__device__ __forceinline__ uint32_t idesc_i8(int n)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// byte offset of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+// four planes of a 2-bit word as int8 {0, +64, -64}, 16 consecutive columns
+__device__ __forceinline__ uint4 expand_word(uint32_t w)
+{
+    return make_uint4((w << 6) & 0xC0C0C0C0u, (w << 4) & 0xC0C0C0C0u, (w << 2) & 0xC0C0C0C0u, w & 0xC0C0C0C0u);
+}
+
+// ---------------------------------------------------------------------------
+template <int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map, TcArgs a)
+{
+    using Cfg = TcCfg<MODE>;
+    using L = TcSmem<MODE>;
+    constexpr int S = Cfg::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t *bars = (uint64_t *)(smem + L::kBars);
+    // bars: codes_full[S], full[S], empty[S], acc_full[2], acc_empty[2], drain
+    uint32_t *tmem_holder = (uint32_t *)(bars + 3 * S + 5);
+    volatile uint32_t *abort = tmem_holder + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t b_codes_full = smem_addr(bars), b_full = b_codes_full + 8 * S, b_empty = b_full + 8 * S;
+    const uint32_t b_acc_full = b_empty + 8 * S, b_acc_empty = b_acc_full + 16, b_drain = b_acc_empty + 16;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(b_codes_full + 8 * s, 1);
+            mbar_init(b_full + 8 * s, 8);      // one arrival per producer warp
+            mbar_init(b_empty + 8 * s, 1);     // MMA commit
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(b_acc_full + 8 * b, 1);
+            mbar_init(b_acc_empty + 8 * b, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(b_drain, 1);
+        *abort = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_addr(tmem_holder), 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+
+    const int R = MODE == 0 ? a.F / 128 : a.D / 128;   // row blocks per piece
+    const int KS = MODE == 0 ? a.D / kTcBK : a.F / kTcBK;
+    const int n_tiles = __ldg(a.n_pieces) * R;
+
+    if (warp == 0) {
+        // ---------------- bulk copies of the 2-bit codes
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+                const int4 pc = a.pieces[tile / R];
+                const int rt = tile % R;
+                const uint8_t *src = a.codes + ((size_t)pc.x * R + rt) * KS * Cfg::kCodeBytes;
+                for (int ks = 0; ks < KS; ks++, it++) {
+                    const int s = it % S;
+                    if (!mbar_wait(b_empty + 8 * s, ((it / S) & 1) ^ 1, abort, a.flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(b_codes_full + 8 * s, Cfg::kCodeBytes + L::kBBytes);
+                    bulk_g2s(smem_addr(smem + s * L::kStage + L::kCodes), src + (size_t)ks * Cfg::kCodeBytes,
+                             Cfg::kCodeBytes, b_codes_full + 8 * s);
+                    tma_load_2d(smem_addr(smem + s * L::kStage + L::kB), &act_map, ks * kTcBK, pc.y,
+                                b_codes_full + 8 * s);
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies still in flight, the last S issued
+                for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; j++) {
+                    const uint64_t t0 = global_ns();
+                    while (!mbar_test(b_codes_full + 8 * (j % S), (j / S) & 1) && global_ns() - t0 < kWaitLimitNs) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issue
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, tc++) {
+                const int4 pc = a.pieces[tile / R];
+                const int npad = (pc.z + 15) & ~15;
+                const uint32_t idesc = idesc_i8(npad);
+                const uint32_t ab = tc & 1, dt = tmem + 256 * ab;
+                if (!mbar_wait(b_acc_empty + 8 * ab, ((tc >> 1) & 1) ^ 1, abort, a.flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < KS; ks++, it++) {
+                    const int s = it % S;
+                    if (!mbar_wait(b_full + 8 * s, (it / S) & 1, abort, a.flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + s * L::kStage + L::kA);
+                    const uint32_t sb = smem_addr(smem + s * L::kStage + L::kB);
+                    const uint64_t da0 = desc_sw128(sa), db = desc_sw128(sb);
+                    const uint64_t da1 = desc_sw128(sa + 128 * kTcBK);
+#pragma unroll
+                    for (int k = 0; k < kTcBK / 32; k++) {
+                        const uint32_t acc = (ks | k) != 0;
+                        mma_i8(dt, da0 + 2 * k, db + 2 * k, idesc, acc);
+                        if (MODE == 0) mma_i8(dt + 128, da1 + 2 * k, db + 2 * k, idesc, acc);
+                    }
+                    mma_commit(b_empty + 8 * s);
+                }
+                if (!ok) break;
+                mma_commit(b_acc_full + 8 * ab);
+            }
+            // make sure every issued MMA has finished before TMEM is released
+            mma_commit(b_drain);
+            const uint64_t t0 = global_ns();
+            while (!mbar_test(b_drain, 0) && global_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- epilogue: TMEM -> registers -> global
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+        uint32_t tc = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, tc++) {
+            const int4 pc = a.pieces[tile / R];
+            const int rt = tile % R;
+            const int row = rt * 128 + r;
+            const uint32_t ab = tc & 1, tb = tbase + 256 * ab;
+            if (!mbar_wait(b_acc_full + 8 * ab, (tc >> 1) & 1, abort, a.flag)) break;
+            tc_fence_after();
+            const int e = pc.x, p0 = pc.y, n = pc.z;
+            if (MODE == 0) {
+                const float ag = a.alpha0[(size_t)e * a.F + row], au = a.alpha1[(size_t)e * a.F + row];
+                for (int c0 = 0; c0 < n; c0 += 32) {
+                    int g[32], u[32];
+                    tmem_ld32(tb + c0, g);
+                    tmem_ld32(tb + 128 + c0, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int col = c0 + j;
+                        if (col < n) {
+                            const int p = p0 + col;
+                            const int slot = __ldg(a.perm + p);
+                            const float sxt = __ldg(a.sx + slot / a.K);
+                            const int gi = g[j] >> 6, ui = u[j] >> 6;
+                            const float gv = __fmul_rn((float)gi, __fmul_rn(ag, sxt));
+                            const float uv = __fmul_rn((float)ui, __fmul_rn(au, sxt));
+                            a.out[(size_t)p * a.F + row] = swiglu(gv, uv);
+                            if (a.tap0) a.tap0[(size_t)slot * a.F + row] = gi;
+                            if (a.tap1) a.tap1[(size_t)slot * a.F + row] = ui;
+                        }
+                    }
+                }
+            } else {
+                const float ad = a.alpha0[(size_t)e * a.D + row];
+                for (int c0 = 0; c0 < n; c0 += 32) {
+                    int d[32];
+                    tmem_ld32(tb + c0, d);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j++) {
+                        const int col = c0 + j;
+                        if (col < n) {
+                            const int p = p0 + col;
+                            const int di = d[j] >> 6;
+                            a.out[(size_t)p * a.D + row] = __fmul_rn((float)di, __fmul_rn(ad, __ldg(a.sh + p)));
+                            if (a.tap0) a.tap0[(size_t)__ldg(a.perm + p) * a.D + row] = di;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b_acc_empty + 8 * ab);
+        }
+    } else if (warp >= 8) {
+        // ---------------- producers: expand the 2-bit codes into int8 A tiles
+        const int pid = threadIdx.x - 256;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            for (int ks = 0; ks < KS; ks++, it++) {
+                const int s = it % S;
+                if (!mbar_wait(b_codes_full + 8 * s, (it / S) & 1, abort, a.flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *st = smem + s * L::kStage;
+                const uint4 *codes = (const uint4 *)(st + L::kCodes);
+                constexpr int kQuads = Cfg::kCodeBytes / 16;   // four words = one row's half stage
+#pragma unroll
+                for (int i = 0; i < kQuads / 256; i++) {
+                    const int qi = pid + 256 * i;
+                    const int mrow = qi >> 1, w0 = (qi & 1) * 4;  // row within gate|up (or down), first word
+                    const uint4 c4 = codes[qi];
+                    *(uint4 *)(st + L::kA + sw128(mrow, w0 + 0)) = expand_word(c4.x);
+                    *(uint4 *)(st + L::kA + sw128(mrow, w0 + 1)) = expand_word(c4.y);
+                    *(uint4 *)(st + L::kA + sw128(mrow, w0 + 2)) = expand_word(c4.z);
+                    *(uint4 *)(st + L::kA + sw128(mrow, w0 + 3)) = expand_word(c4.w);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_full + 8 * s);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// slot-ordered copy of the int8 activation rows: xperm[p] = q_x[perm[p] / K]
+// (one warp per position)
+// ---------------------------------------------------------------------------
+__global__ void gather_rows_kernel(const int8_t *qx, const int *perm, int K, int D, int S, int8_t *xperm)
+{
+    const int lane = threadIdx.x & 31;
+    const int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (p >= S) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(qx + (size_t)(perm[p] / K) * D);
+    uint4 *dst = reinterpret_cast<uint4 *>(xperm + (size_t)p * D);
+    for (int i = lane; i < D / 16; i += 32) dst[i] = __ldg(src + i);
+}
+
+// ---------------------------------------------------------------------------
+// requantise h rows (one warp per slot position) for the tensor-core path
+// ---------------------------------------------------------------------------
+__global__ void requant_rows_kernel(const float *h, int S, int F, const int *perm, int8_t *qh, float *sh,
+                                    int8_t *tap_qh, float *tap_sh)
+{
+    const int lane = threadIdx.x & 31;
+    const int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    if (p >= S) return;
+    const float4 *hr = reinterpret_cast<const float4 *>(h + (size_t)p * F);
+    float amax = 0.0f;
+    for (int i = lane; i < F / 4; i += 32) {
+        float4 v = hr[i];
+        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
+    }
+    amax = warp_max(amax);
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const int slot = perm[p];
+    for (int i = lane; i < F / 4; i += 32) {
+        float4 v = hr[i];
+        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+        if (amax > 0.0f) {
+            q0 = quant_code(v.x, inv);
+            q1 = quant_code(v.y, inv);
+            q2 = quant_code(v.z, inv);
+            q3 = quant_code(v.w, inv);
+        }
+        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+                            ((uint32_t)(q3 & 0xff) << 24);
+        reinterpret_cast<uint32_t *>(qh + (size_t)p * F)[i] = pk;
+        if (tap_qh) reinterpret_cast<uint32_t *>(tap_qh + (size_t)slot * F)[i] = pk;
+    }
+    if (lane == 0) {
+        const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+        sh[p] = s;
+        if (tap_sh) tap_sh[slot] = s;
+    }
+}
+
+// y[t][c] = (resid[t][c] +) sum_k fmaf(w[t][k], yE[inv[t*K+k]][c]) in rank order
+__global__ void combine_kernel(const float *ye, const int *inv, const float *topk_w, int T, int K, int D, float *y,
+                               const float *resid)
+{
+    const int64_t n4 = (int64_t)T * D / 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / (D / 4));
+        const int c4 = (int)(i % (D / 4));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < K; k++) {
+            const float w = topk_w[t * K + k];
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(ye + (size_t)inv[t * K + k] * D) + c4);
+            acc.x = __fmaf_rn(w, v.x, acc.x);
+            acc.y = __fmaf_rn(w, v.y, acc.y);
+            acc.z = __fmaf_rn(w, v.z, acc.z);
+            acc.w = __fmaf_rn(w, v.w, acc.w);
+        }
+        if (resid) {
+            const float4 r = reinterpret_cast<const float4 *>(resid)[i];
+            acc.x = __fadd_rn(r.x, acc.x);
+            acc.y = __fadd_rn(r.y, acc.y);
+            acc.z = __fadd_rn(r.z, acc.z);
+            acc.w = __fadd_rn(r.w, acc.w);
+        }
+        reinterpret_cast<float4 *>(y)[i] = acc;
+    }
+}
+
+// 2-bit interchange -> tensor-core layout (one thread per output word)
+__global__ void repack_tc_gu_kernel(const uint32_t *gate, const uint32_t *up, int E, int D, int F, uint32_t *out)
+{
+    const int FT = F / 128, KS = D / 128;
+    const int64_t n = (int64_t)E * FT * KS * 2 * 128 * 8;
+    for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
+        int64_t q = o;
+        const int w = q % 8; q /= 8;
+        const int row = q % 128; q /= 128;
+        const int mat = q % 2; q /= 2;
+        const int ks = q % KS; q /= KS;
+        const int ft = q % FT; q /= FT;
+        const int e = (int)q;
+        const uint32_t *src = (mat == 0 ? gate : up) + ((int64_t)e * F + ft * 128 + row) * (D / 16);
+        out[o] = tc_word(src[ks * 8 + w]);
+    }
+}
+
+__global__ void repack_tc_dn_kernel(const uint32_t *down, int E, int D, int F, uint32_t *out)
+{
+    const int CT = D / 128, KS = F / 128;
+    const int64_t n = (int64_t)E * CT * KS * 128 * 8;
+    for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
+        int64_t q = o;
+        const int w = q % 8; q /= 8;
+        const int row = q % 128; q /= 128;
+        const int ks = q % KS; q /= KS;
+        const int ct = q % CT; q /= CT;
+        const int e = (int)q;
+        const uint32_t *src = down + ((int64_t)e * D + ct * 128 + row) * (F / 16);
+        out[o] = tc_word(src[ks * 8 + w]);
+    }
+}
+
+}  // namespace maple

@@ -110,6 +110,11 @@ def layer_weights(shape: LayerShape, seed: int, layer: int = 0, zipf: float | No
     return w
 
 
+def layer_weights_from_args(args) -> dict:
+    """layer_weights(*args): a picklable entry point for process pools."""
+    return layer_weights(*args)
+
+
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round finite fp32 values to bf16 (nearest, ties to even); returns uint16 bits."""
     u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)

@@ -177,3 +177,47 @@ def test_prefill_config_sampled_parity(big):
     tokens = tokens.astype(np.int32)
     ref = L_orc.forward_tokens(x, tokens)
     compare_tokens(BIG, g, ref, tokens)
+
+
+# ---------------------------------------------------------------------------- both expert paths
+import ternary_weight_moe_forward_b200 as tw  # noqa: E402
+
+
+@pytest.mark.parametrize("T", [1, 8, 37, 300])
+def test_tensor_core_path_forced_tiny(tiny, T):
+    """The tcgen05 grouped GEMM at any T (pieces of 1..256 slots, ragged N)."""
+    w, L_orc, _ = tiny
+    Lg = Layer(TINY, w, max_tokens=512, flags=tw.MAPLE_CFG_FORCE_TC)
+    x = synth.activations(T, TINY.d_model, seed=100 + T)
+    _full_check(TINY, L_orc, Lg, x)
+    Lg.close()
+
+
+@pytest.mark.parametrize("T", [65, 300])
+def test_gemv_path_forced_large_T(tiny, T):
+    w, L_orc, _ = tiny
+    Lg = Layer(TINY, w, max_tokens=512, flags=tw.MAPLE_CFG_FORCE_GEMV)
+    x = synth.activations(T, TINY.d_model, seed=200 + T)
+    _full_check(TINY, L_orc, Lg, x)
+    Lg.close()
+
+
+def test_tensor_core_path_forced_decode_shape(big_weights, big):
+    L_orc, _ = big
+    Lg = Layer(BIG, big_weights, max_tokens=64, flags=tw.MAPLE_CFG_FORCE_TC)
+    for T in (1, 64):
+        x = synth.activations(T, BIG.d_model, seed=300 + T)
+        _full_check(BIG, L_orc, Lg, x)
+    Lg.close()
+
+
+def test_paths_agree_bitwise(big_weights, big):
+    """GEMV and tensor-core paths give identical bits on the same input."""
+    Lt = Layer(BIG, big_weights, max_tokens=128, flags=tw.MAPLE_CFG_FORCE_TC)
+    Lv = Layer(BIG, big_weights, max_tokens=128, flags=tw.MAPLE_CFG_FORCE_GEMV)
+    x = bf16_from_bits(synth.activations(128, BIG.d_model, seed=7), "cuda")
+    yt, yv = Lt.forward(x), Lv.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(yt.view(torch.int32), yv.view(torch.int32))
+    Lt.close()
+    Lv.close()

@@ -178,6 +178,35 @@ int maple_moe_stack_forward(const maple_moe_t *layers, int32_t n_layers, float *
  */
 int maple_moe_set_stage_events(maple_moe_t layer, void *const *events, int32_t n_events);
 
+/*
+ * Routing without any device allocation.  The source pages have no counterpart
+ * of this entry point; it exists for callers that cannot let a library call
+ * cudaMalloc: processes whose device memory belongs to their own pool
+ * allocator (an allocation behind the pool's back fragments it and may
+ * synchronise the device) and serving loops that forbid allocation once
+ * running.  No handle is needed: the router weights are read from the
+ * caller's buffers and the scratch (logits, int8 codes, counters,
+ * permutation) lives in a fixed 1 MiB device array inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ * Computes exactly what maple_moe_route computes: topk_idx [T][K] int32,
+ * topk_w [T][K] fp32 and expert_counts [E] int32 (may be NULL).
+ * x: DEVICE [T][D] bf16; router_w: DEVICE [E][D] fp32; router_bias: DEVICE [E]
+ * or NULL; all 16-byte aligned.
+ * Limits (else MAPLE_ERR_INVALID_ARG / MAPLE_ERR_UNSUPPORTED_SHAPE):
+ * 0 <= T <= 64, T * n_experts <= 16384, and the shape limits of
+ * maple_moe_config for d_model, n_experts and top_k.
+ * The first call on a device looks up the array's device address and raises
+ * the routing kernel's shared-memory limit for that device; make that first
+ * call before any stream capture.  Every call uses the same array and it keeps
+ * the previous call's contents (the counters that must start at zero are
+ * cleared by each call on its stream), so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race: order them on one stream.
+ * A NaN logit is ranked last; this entry point has no flag word to report it.
+ */
+int maple_moe_route_noalloc(const uint16_t *x, int32_t T, int32_t d_model, int32_t n_experts, int32_t top_k,
+                            const float *router_w, const float *router_bias, int32_t *topk_idx, float *topk_w,
+                            int32_t *expert_counts, maple_stream_t stream);
+
 /* Read (and optionally clear) the device flag word; no synchronisation. */
 int maple_moe_device_flags(maple_moe_t layer, uint32_t *flags, int32_t clear);
 

@@ -31,7 +31,7 @@ MAPLE_CFG_FORCE_TC = 0x2
 
 EXPORTED = ("maple_moe_status_string", "maple_moe_pack_ternary", "maple_moe_create", "maple_moe_route",
             "maple_moe_forward", "maple_moe_stack_forward", "maple_moe_set_stage_events", "maple_moe_device_flags",
-            "maple_moe_destroy")
+            "maple_moe_destroy", "maple_moe_route_noalloc")
 
 
 class MapleError(RuntimeError):
@@ -80,6 +80,7 @@ def lib():
         L.maple_moe_set_stage_events.argtypes = [P, C.POINTER(C.c_void_p), I32]
         L.maple_moe_device_flags.argtypes = [P, C.POINTER(C.c_uint32), I32]
         L.maple_moe_destroy.argtypes = [P]
+        L.maple_moe_route_noalloc.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P, P]
         for name in EXPORTED:
             if name != "maple_moe_status_string":
                 getattr(L, name).restype = C.c_int
@@ -147,6 +148,14 @@ def maple_moe_device_flags(handle, clear: bool = False) -> int:
     f = C.c_uint32()
     _check(lib().maple_moe_device_flags(handle, C.byref(f), 1 if clear else 0), "maple_moe_device_flags")
     return f.value
+
+
+def maple_moe_route_noalloc(x, T: int, d_model: int, n_experts: int, top_k: int, router_w, router_bias,
+                            topk_idx, topk_w, expert_counts=None, stream=None) -> None:
+    """Routing with no device allocation (scratch in a fixed array of the library)."""
+    _check(lib().maple_moe_route_noalloc(_p(x), T, d_model, n_experts, top_k, _p(router_w), _p(router_bias),
+                                         _p(topk_idx), _p(topk_w), _p(expert_counts), _p(stream)),
+           "maple_moe_route_noalloc")
 
 
 def maple_moe_destroy(handle) -> None:

@@ -3,6 +3,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "../../include/maple_moe.h"
@@ -702,4 +703,125 @@ extern "C" int maple_moe_destroy(maple_moe_t h)
     h->magic = 0;
     delete h;
     return status;
+}
+
+// ===========================================================================
+// Routing that allocates nothing.
+//
+// Some callers cannot let a library call cudaMalloc: processes whose device
+// memory is handed out by their own pool allocator (a cudaMalloc behind the
+// pool's back fragments it and can synchronise the whole device), and serving
+// loops that forbid any allocation once they are running.  For them,
+// maple_moe_route_noalloc runs the routing kernel with its scratch (logits,
+// int8 codes, counters, permutation) in the fixed array below instead of a
+// handle's workspace.  The array is a file-scope device variable: every GPU
+// that loads this library holds its kNoallocScratchBytes until the process
+// exits.
+// ===========================================================================
+namespace {
+
+constexpr size_t kNoallocScratchBytes = (size_t)1 << 20;   // 1 MiB
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_route_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kNoallocMaxDevices];   // device address of g_route_scratch on each device
+
+// Once per device, with that device current: look up the device address of
+// the scratch array (in host code its name is only a host-side stand-in) and
+// raise the routing kernels' dynamic shared-memory limit.
+int noalloc_scratch(void **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+        cudaGetLastError();
+        return MAPLE_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return MAPLE_ERR_CUDA;
+        }
+        for (int ni = 1; ni <= 16; ni *= 2) {
+            allow_max_smem((const void *)pick_route(ni * 256, 16), dev);
+            allow_max_smem((const void *)pick_route(ni * 256, 1024), dev);
+        }
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return MAPLE_OK;
+}
+
+}  // namespace
+
+extern "C" int maple_moe_route_noalloc(const uint16_t *x, int32_t T, int32_t d_model, int32_t n_experts,
+                                       int32_t top_k, const float *router_w, const float *router_bias,
+                                       int32_t *topk_idx, float *topk_w, int32_t *expert_counts,
+                                       maple_stream_t stream)
+{
+    maple_moe_config c;
+    memset(&c, 0, sizeof c);
+    c.d_model = d_model;
+    c.n_experts = n_experts;
+    c.top_k = top_k;
+    c.d_ff = 128;
+    c.max_tokens = 1;
+    int rc = check_shape(&c);
+    if (rc) return rc;
+    if (T < 0 || T > kRouteSmallT || (int64_t)T * n_experts > kFusedMarkBytes) return MAPLE_ERR_INVALID_ARG;
+    if (T == 0) return MAPLE_OK;
+    if (!x || !router_w || !topk_idx || !topk_w || !aligned16(x) || !aligned16(router_w) || !aligned16(topk_idx) ||
+        !aligned16(topk_w) || (router_bias && !aligned16(router_bias)) || (expert_counts && !aligned16(expert_counts)))
+        return MAPLE_ERR_INVALID_ARG;
+
+    const int64_t D = d_model, E = n_experts, K = top_k, S = (int64_t)T * top_k;
+    Arena ar;
+    const size_t o_lg = ar.take(T * E * 4), o_qx = ar.take(T * D), o_sx = ar.take(T * 4), o_sumx = ar.take(T * 4);
+    const size_t o_ti = ar.take(S * 4), o_tw = ar.take(S * 4), o_cnt = ar.take(E * 4), o_off = ar.take((E + 1) * 4);
+    const size_t o_perm = ar.take(S * 4), o_inv = ar.take(S * 4), o_act = ar.take(E * 4), o_nact = ar.take(4);
+    const size_t o_ctr = ar.take(((kRouteSmallT + kRouteTokens - 1) / kRouteTokens + 1) * 4);
+    if (ar.size > kNoallocScratchBytes) return MAPLE_ERR_INVALID_ARG;
+
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    char *b = (char *)scratch;
+    cudaStream_t st = (cudaStream_t)stream;
+    // the last-arriver counters must start at zero; the array keeps whatever the last call left
+    const int n_tg = (T + kRouteTokens - 1) / kRouteTokens;
+    if (cudaMemsetAsync(b + o_ctr, 0, (size_t)(n_tg + 1) * 4, st) != cudaSuccess) return MAPLE_ERR_CUDA;
+
+    RouteArgs a;
+    memset(&a, 0, sizeof a);
+    a.x = x;
+    a.T = T;
+    a.D = d_model;
+    a.E = n_experts;
+    a.K = top_k;
+    a.Wr = router_w;
+    a.bias = router_bias;
+    a.qx = (int8_t *)(b + o_qx);
+    a.sx = (float *)(b + o_sx);
+    a.sumx = (int *)(b + o_sumx);
+    a.logits = (float *)(b + o_lg);
+    a.topk_idx = (int *)(b + o_ti);
+    a.topk_w = (float *)(b + o_tw);
+    a.out_idx = topk_idx;
+    a.out_w = topk_w;
+    a.out_counts = expert_counts;
+    a.tg_cnt = (unsigned *)(b + o_ctr);
+    a.glob_cnt = (unsigned *)(b + o_ctr) + n_tg;
+    a.fuse_permute = 1;
+    a.counts = (int *)(b + o_cnt);
+    a.offsets = (int *)(b + o_off);
+    a.perm = (int *)(b + o_perm);
+    a.inv = (int *)(b + o_inv);
+    a.active = (int *)(b + o_act);
+    a.n_active = (int *)(b + o_nact);
+    a.flag = nullptr;
+    dim3 grid(n_experts / kRouteExperts, n_tg);
+    pick_route(d_model, n_experts)<<<grid, 256, route_smem_bytes(d_model), st>>>(a);
+    return launch_status();
 }

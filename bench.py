@@ -7,8 +7,9 @@ ternary 2-bit weights, seed 0) run on the four decode batches T = 1, 8, 32
 and 64 (105 tokens).  A step is one forward pass of the whole layer (routing,
 permutation, gate/up, down, combine) for each of the four batches.  Before
 every forward pass L2 is flushed (a 256 MB write, outside the timed events),
-so the weights come from HBM.  Each forward is timed with CUDA events on its
-stream; the step time is their sum.  value = tokens per second over all ranks.
+so the weights come from HBM.  Each forward is a replay of a CUDA graph of the
+library call, timed with CUDA events on its stream (the library records
+per-stage events inside the graph); the step time is their sum.  value = tokens per second over all ranks.
 
 The JSON line adds: roofline (dominant kernel vs measured HBM bandwidth),
 cpu_baseline (the CPU oracle timed on a sample), e2e (host buffers with the
@@ -107,6 +108,22 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+# ---------------------------------------------------------------------------- ranks
+def reduce_max_over_ranks(values, device=None):
+    """Max over ranks of per-rank device timings (identity on one process)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- GPU arm
 def decode_bytes(n_active: int, T: int) -> int:
     """Algorithmic HBM bytes of one decode forward: packed codes and scales of
@@ -147,21 +164,48 @@ def run_gpu(args, rank: int, world: int):
         n_active[T] = int((counts > 0).sum().item())
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
+    # One CUDA graph per batch size: the forward (routing kernel, permutation
+    # and expert kernel) replays without host launch gaps.  The library's
+    # per-stage events are captured with it, so the stages are timed on the
+    # device as well.
     ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(4)] for T in DECODE_T}
     for T in DECODE_T:
         for e in ev[T]:
             e.record(stream)
     torch.cuda.synchronize(dev)
+    graphs = {}
+    for T in DECODE_T:
+        tw.maple_moe_set_stage_events(layer.handle, ev[T])
+        layer.forward(xs[T], y=ys[T])          # warm the path before capture
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer.forward(xs[T], y=ys[T])
+        graphs[T] = g
+    tw.maple_moe_set_stage_events(layer.handle, None)
+    torch.cuda.synchronize(dev)
+
+    e_beg = {T: torch.cuda.Event(enable_timing=True) for T in DECODE_T}
+    e_end = {T: torch.cuda.Event(enable_timing=True) for T in DECODE_T}
+    stages_in_graph = True
 
     def one_step(timed: list | None):
+        nonlocal stages_in_graph
         for T in DECODE_T:
             flush.fill_(1.0)
-            tw.maple_moe_set_stage_events(layer.handle, ev[T])
-            layer.forward(xs[T], y=ys[T])
+            e_beg[T].record(stream)
+            graphs[T].replay()
+            e_end[T].record(stream)
             if timed is not None:
-                timed.append((T, [e for e in ev[T]]))
                 torch.cuda.synchronize(dev)
-                timed[-1] = (T, [ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)])
+                total = e_beg[T].elapsed_time(e_end[T])
+                st = None
+                if stages_in_graph:
+                    try:
+                        st = [ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)]
+                    except Exception:
+                        stages_in_graph = False
+                timed.append((T, total, st))
 
     for _ in range(args.warmup):
         one_step(None)
@@ -179,10 +223,27 @@ def run_gpu(args, rank: int, world: int):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks = clk.stop()
-    tw.maple_moe_set_stage_events(layer.handle, None)
 
-    total_ms = sum(t[1][2] for t in timed)
-    per_T = {T: [t[1] for t in timed if t[0] == T] for T in DECODE_T}
+    if not stages_in_graph or any(t[2] is None for t in timed):
+        # stage split from host-launched forwards instead (same kernels, stage events on the stream)
+        stage_src = "host-launched forwards"
+        split = {T: [] for T in DECODE_T}
+        tw.maple_moe_set_stage_events(layer.handle, None)
+        for _ in range(args.steps):
+            for T in DECODE_T:
+                flush.fill_(1.0)
+                tw.maple_moe_set_stage_events(layer.handle, ev[T])
+                layer.forward(xs[T], y=ys[T])
+                torch.cuda.synchronize(dev)
+                split[T].append([ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)])
+        tw.maple_moe_set_stage_events(layer.handle, None)
+        timed = [(T, tot, split[T][n % len(split[T])]) for n, (T, tot, _) in enumerate(timed)]
+    else:
+        stage_src = "events inside the graph"
+
+    total_ms = sum(t[1] for t in timed)
+    per_T = {T: [t[2] for t in timed if t[0] == T] for T in DECODE_T}
+    fwd_T = {T: [t[1] for t in timed if t[0] == T] for T in DECODE_T}
     experts_ms = sum(x[2] - x[0] for T in DECODE_T for x in per_T[T])
     experts_alg = sum(experts_bytes(n_active[T], T) for T in DECODE_T) * args.steps
 
@@ -205,17 +266,14 @@ def run_gpu(args, rank: int, world: int):
                 e2e_ms += e0.elapsed_time(e1)
 
     # ---- max over ranks
-    vals = torch.tensor([total_ms, e2e_ms, experts_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, experts_ms = vals.tolist()
-    tokens = sum(DECODE_T) * args.steps * world
+    total_ms, e2e_ms, experts_ms = reduce_max_over_ranks([total_ms, e2e_ms, experts_ms], device=dev)
+    tokens_rank = sum(DECODE_T) * args.steps
     hbm, peak_kind = peaks()
     achieved = experts_alg / (experts_ms * 1e-3) / 1e9
     layer_bytes = sum(decode_bytes(n_active[T], T) for T in DECODE_T) * args.steps
     out = {
         "metric": METRIC,
-        "value": tokens / (total_ms * 1e-3),
+        "value": whole_job_rate(tokens_rank, world, total_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -230,20 +288,22 @@ def run_gpu(args, rank: int, world: int):
                    "experts_touched": {str(T): n_active[T] for T in DECODE_T},
                    "l2": "flushed before every timed forward (256 MB write, outside the events)",
                    "parallelism": f"replicas x{world}"},
-        "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(x[2] for x in per_T[T]) * 1e-3),
-                           "us_per_forward": 1e3 * statistics.mean(x[2] for x in per_T[T]),
+        "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(fwd_T[T]) * 1e-3),
+                           "us_per_forward": 1e3 * statistics.mean(fwd_T[T]),
                            "us_route": 1e3 * statistics.mean(x[0] for x in per_T[T]),
                            "us_experts": 1e3 * statistics.mean(x[2] - x[0] for x in per_T[T]),
                            "layer_hbm_frac": decode_bytes(n_active[T], T) /
-                           (statistics.mean(x[2] for x in per_T[T]) * 1e-3) / 1e9 / hbm}
+                           (statistics.mean(fwd_T[T]) * 1e-3) / 1e9 / hbm}
                   for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
         "roofline": {"kernel": "decode_experts_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": None},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(tokens_rank, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(T * shape.d_model * 2 for T in DECODE_T),
                 "d2h_bytes_per_step": sum(T * shape.d_model * 4 for T in DECODE_T)},
         "gpu_launches": 2 * len(DECODE_T) * args.steps,
+        "cuda_graphs": True,
+        "stage_split_from": stage_src,
         "clocks": clocks,
     }
     return out, layer

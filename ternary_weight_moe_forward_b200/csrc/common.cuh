@@ -13,6 +13,11 @@ namespace maple {
 
 constexpr unsigned FULL = 0xffffffffu;
 
+// upper bound (ns) a thread may stay suspended in one mbarrier.try_wait; the
+// hardware wakes it as soon as the phase completes, so waiting threads take no
+// issue slots from the ones doing work
+constexpr uint32_t kSuspendHintNs = 200000;
+
 // ---------------------------------------------------------------------------
 // exp(x), written out from the mathematics so that host and device give the
 // same bits: clamp to [-87, 88]; n = rint(x*log2 e); r = x - n ln2 with ln2

@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "layout.cuh"
+#include "route.cuh"
 
 namespace maple {
 
@@ -88,6 +89,57 @@ __device__ __forceinline__ void chunk_tokens(const uint4 wv, const int8_t *xs, i
                 acc[j] = dp4a_us(pw[4 * w + 1], xv.y, acc[j]);
                 acc[j] = dp4a_us(pw[4 * w + 2], xv.z, acc[j]);
                 acc[j] = dp4a_us(pw[4 * w + 3], xv.w, acc[j]);
+            }
+        }
+    }
+}
+
+// Same as chunk_tokens with four partial sums per token (one per byte plane),
+// so the dp4a chains of a single token run four wide; acc4[j][k] are summed
+// by the caller (int32, exact in any order).
+__device__ __forceinline__ void chunk_tokens4(const uint4 wv, const int8_t *xs, int ld, int off, int nb,
+                                              int (&acc4)[kGemvTokens][4])
+{
+    const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int j = 0; j < kGemvTokens; j++) {
+        if (j < nb) {
+            const uint4 *x4 = reinterpret_cast<const uint4 *>(xs + (size_t)j * ld + off);
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 xv = x4[w];
+                acc4[j][0] = dp4a_us(plane(w4[w], 0), xv.x, acc4[j][0]);
+                acc4[j][1] = dp4a_us(plane(w4[w], 1), xv.y, acc4[j][1]);
+                acc4[j][2] = dp4a_us(plane(w4[w], 2), xv.z, acc4[j][2]);
+                acc4[j][3] = dp4a_us(plane(w4[w], 3), xv.w, acc4[j][3]);
+            }
+        }
+    }
+}
+
+// acc[j][0..1] += the 64 values of one chunk (this lane's row) against token j's
+// 64 activations (16-byte rows x4[j*ld16 .. +3]), j < nb.  The byte planes are
+// taken once per chunk and serve every token; two partial sums per token keep
+// the dp4a chains short (int32, exact in any order).
+__device__ __forceinline__ void chunk_dot(const uint4 wv, const uint4 *x4, int ld16, int nb,
+                                          int (&acc)[kGemvTokens][2])
+{
+    const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+    uint32_t pw[16];
+#pragma unroll
+    for (int w = 0; w < 4; w++)
+#pragma unroll
+        for (int k = 0; k < 4; k++) pw[4 * w + k] = plane(w4[w], k);
+#pragma unroll
+    for (int j = 0; j < kGemvTokens; j++) {
+        if (j < nb) {
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 xv = x4[j * ld16 + w];
+                acc[j][w & 1] = dp4a_us(pw[4 * w + 0], xv.x, acc[j][w & 1]);
+                acc[j][w & 1] = dp4a_us(pw[4 * w + 1], xv.y, acc[j][w & 1]);
+                acc[j][w & 1] = dp4a_us(pw[4 * w + 2], xv.z, acc[j][w & 1]);
+                acc[j][w & 1] = dp4a_us(pw[4 * w + 3], xv.w, acc[j][w & 1]);
             }
         }
     }
@@ -309,33 +361,89 @@ __global__ void __launch_bounds__(kGemvWarps * 32, MAPLE_GEMV_MINB) down_gemv_ke
 // ---------------------------------------------------------------------------
 // Persistent weight-streaming kernel for the whole expert stage (decode).
 //
-// Grid = one CTA per SM, launched cooperatively (all CTAs resident).  Work
-// items: gate/up items (active expert, 32 gate + 32 up rows = two row groups)
-// then down items (active expert, 128 output channels).  Every CTA takes an
-// equal contiguous range of the gate/up items and of the down items.  One
-// producer thread streams the 2-bit codes of its items with bulk copies into
-// a ring of shared-memory buffers (the copies do not depend on any result, so
-// they run ahead into the down items while gate/up is computed); eight
-// compute warps consume them.  The last CTA to finish an expert's gate/up
-// items requantises that expert's slots and publishes ready[e] = epoch; a
-// down item waits (bounded) for that before reading q_h.
+// Grid = one CTA per SM, launched cooperatively (all CTAs resident).  Every
+// CTA first builds the permutation of all T*K slots for itself from the
+// router's top-k (in shared memory), so no routing step needs a grid-wide
+// hand-off.  Work items: gate/up items (active expert, 32 gate + 32 up rows)
+// then down items (active expert, 128 output channels); every CTA takes an
+// equal contiguous range of each kind.  Warp roles:
+//   warp 0      streams the 2-bit codes and row scales of its items, in order,
+//               with bulk copies into a ring of weight slots;
+//   warps 1, 2  stage the activations of compute group 0 / 1 (double
+//               buffered): for gate/up the int8 rows of the item's tokens, for
+//               down the fp32 SwiGLU rows h of the item's slots once every
+//               gate/up item of that expert has finished;
+//   warps 3, 4  publish the results of group 0 / 1: make a finished gate/up
+//               item visible (GPU fence, arrival counter of its expert), and for
+//               a down item count each token's arrival on its channel block,
+//               the last of the K arrivals combining that token's 128 channels;
+//   warps 5..20 two compute groups of eight warps; group g takes items g, g+2,
+//               ... of the CTA.
+// Compute groups never wait on global memory: fences, atomics and the
+// combine run on the publishing warps.  Down items requantise h locally (the
+// same per-slot absmax int8 rule).  Every wait is bounded (2 s) and raises the
+// device flag on expiry.
 // ---------------------------------------------------------------------------
-constexpr int kDecThreads = (kGemvWarps + 1) * 32;   // + one producer warp
-constexpr int kDecRingBytes = 160 * 1024;
+constexpr int kDecWSlots = 4;
+constexpr int kDecGroups = 2;
+constexpr int kDecGroupWarps = 8;
+constexpr int kDecGroupThreads = kDecGroupWarps * 32;
+constexpr int kDecRec = 4;   // completion records per group
+constexpr int kDecFirstCompute = 1 + 2 * kDecGroups;
+constexpr int kDecThreads = (kDecFirstCompute + kDecGroups * kDecGroupWarps) * 32;   // 672
+
+struct DecActMeta {
+    int nb, b0, base, e;
+    int slot[kGemvTokens];
+    float s[kGemvTokens];     // gate/up: s_x of the token
+    int sum[kGemvTokens];     // gate/up: sum of the token's int8 codes
+};
+struct DecWMeta {
+    int e, sub, kind, cnt, base;
+};
+struct DecRecord {            // one finished batch of a compute group
+    int kind, e, sub, nb, base, last;
+    int slot[kGemvTokens];
+};
 
 struct DecodeArgs {
     GemvArgs g;
-    unsigned *ready;     // [E]: epoch of the last requantisation
-    unsigned epoch;
-    int nbuf;            // ring buffers
-    int buf_bytes;       // bytes per ring buffer
+    unsigned *arrive;     // [E] finished gate/up items per expert, zero at launch
+    int wslot_bytes;      // codes + scales of one item
+    int aslot_bytes;      // activation rows of one batch
+    int nw;               // weight ring slots (2..kDecWSlots)
+    const int *topk_idx;  // [T][K] the router's choices (distinct per token)
+    const float *topk_w;  // [T][K] their softmax weights
+    // outputs of the permutation, written by CTA 0 (may be null)
+    int *tap_counts, *tap_offsets, *tap_perm;
 };
 
-__host__ __device__ inline size_t decode_smem_bytes(int D, int F, int buf_bytes, int nbuf)
+__host__ __device__ inline int dec_wslot_bytes(int D, int F)
 {
-    const int row = D > F ? D : F;
-    return (size_t)nbuf * buf_bytes + (size_t)kGemvTokens * row + (size_t)kGemvWarps * kGemvTokens * 32 * 4 +
-           (size_t)2 * 8 * nbuf + 1024;
+    const int g = 16 * D + 256, d = 32 * F + 512;
+    return ((g > d ? g : d) + 127) & ~127;
+}
+__host__ __device__ inline int dec_aslot_bytes(int D, int F)
+{
+    const int g = kGemvTokens * D, d = kGemvTokens * F * 4;
+    return ((g > d ? g : d) + 127) & ~127;
+}
+// routing tables every CTA builds for itself in shared memory
+__host__ __device__ inline size_t dec_table_bytes(int T, int K, int E)
+{
+    return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E;
+}
+__host__ __device__ inline size_t dec_group_scratch_bytes(int F)
+{
+    return (size_t)kDecGroupWarps * kGemvTokens * 32 * 4 + (size_t)kGemvTokens * F + 2 * kGemvTokens * 4;
+}
+constexpr int kDecBars = 2 * kDecWSlots + 4 * kDecGroups + 2 * kDecRec * kDecGroups;
+__host__ __device__ inline size_t decode_smem_bytes(int D, int F, int T, int K, int E, int nw)
+{
+    return (size_t)nw * dec_wslot_bytes(D, F) + (size_t)kDecGroups * 2 * dec_aslot_bytes(D, F) +
+           kDecGroups * dec_group_scratch_bytes(F) + kDecGroups * 2 * sizeof(DecActMeta) +
+           kDecWSlots * sizeof(DecWMeta) + kDecGroups * kDecRec * sizeof(DecRecord) + 8 * kDecBars + 64 +
+           dec_table_bytes(T, K, E);
 }
 
 // bounded wait on an mbarrier phase (2 s); false on timeout
@@ -346,254 +454,497 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity)
     while (true) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
             : "memory");
         if (ok) return true;
         if (global_timer_ns() - t0 > 2000000000ull) return false;
     }
 }
+__device__ __forceinline__ void dec_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void dec_expect(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void dec_bulk(void *dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    for (uint32_t off = 0; off < bytes; off += 8192) {
+        const uint32_t n = bytes - off < 8192 ? bytes - off : 8192;
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         d + off),
+                     "l"((const uint8_t *)src + off), "r"(n), "r"(bar)
+                     : "memory");
+    }
+}
 
 __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeArgs d)
 {
-    const GemvArgs &a = d.g;
+    GemvArgs a = d.g;
+    const int nw = d.nw;
     extern __shared__ __align__(1024) uint8_t dsm[];
-    uint8_t *ring = dsm;
-    const int rowmax = a.D > a.F ? a.D : a.F;
-    int8_t *xs = (int8_t *)(dsm + (size_t)d.nbuf * d.buf_bytes);
-    int *red = (int *)(xs + (size_t)kGemvTokens * rowmax);
-    uint64_t *bars = (uint64_t *)(red + kGemvWarps * kGemvTokens * 32);   // full[nbuf], empty[nbuf]
-    __shared__ int s_slot[kGemvTokens];
-    __shared__ int s_done[kGemvTokens];
-    __shared__ unsigned s_flag;
+    uint8_t *wring = dsm;
+    uint8_t *aring = wring + (size_t)nw * d.wslot_bytes;                          // [group][2][aslot]
+    uint8_t *gscr = aring + (size_t)kDecGroups * 2 * d.aslot_bytes;               // [group] scratch
+    const size_t gscr_bytes = dec_group_scratch_bytes(a.F);
+    DecActMeta *ameta = (DecActMeta *)(gscr + kDecGroups * gscr_bytes);           // [group][2]
+    DecWMeta *wmeta = (DecWMeta *)(ameta + kDecGroups * 2);                       // [kDecWSlots]
+    DecRecord *recs = (DecRecord *)(wmeta + kDecWSlots);                          // [group][kDecRec]
+    uint64_t *bars = (uint64_t *)(((uintptr_t)(recs + kDecGroups * kDecRec) + 7) & ~(uintptr_t)7);
+    // bars: wfull[W], wempty[W], afull[G][2], aempty[G][2], rfull[G][R], rempty[G][R]
+    const uint32_t b_wfull = (uint32_t)__cvta_generic_to_shared(bars), b_wempty = b_wfull + 8 * kDecWSlots;
+    const uint32_t b_afull = b_wempty + 8 * kDecWSlots, b_aempty = b_afull + 8 * 2 * kDecGroups;
+    const uint32_t b_rfull = b_aempty + 8 * 2 * kDecGroups, b_rempty = b_rfull + 8 * kDecRec * kDecGroups;
+    // routing tables
+    const int T = a.T, K = a.K, E = a.E, S = a.T * a.K;
+    int *t_idx = (int *)(bars + kDecBars);
+    float *t_w = (float *)(t_idx + S);
+    int *t_perm = (int *)(t_w + S);
+    int *t_inv = t_perm + S;
+    int *t_cnt = t_inv + S;
+    int *t_off = t_cnt + E;
+    int *t_act = t_off + E + 1;
+    float *t_sx = (float *)(t_act + E);
+    int *t_sumx = (int *)(t_sx + T);
+    int *t_misc = t_sumx + T;   // [0] n_active, [8..40] scan scratch
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t b_full = (uint32_t)__cvta_generic_to_shared(bars), b_empty = b_full + 8 * d.nbuf;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < d.nbuf; i++) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b_full + 8 * i), "r"(1) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b_empty + 8 * i), "r"(1) : "memory");
-        }
+        for (int i = 0; i < kDecBars; i++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b_wfull + 8 * i), "r"(1) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    __syncthreads();
 
-    const int n_active = __ldg(a.n_active);
+    // ---------------- prologue: the permutation of the T*K slots (T <= 64), from the
+    // router's choices: a token bitmask per expert gives the counts, and a slot's
+    // rank within its expert is the number of earlier tokens in that mask
+    unsigned long long *tmask = (unsigned long long *)(((uintptr_t)(t_misc + 48) + 7) & ~(uintptr_t)7);
+    const bool writer = blockIdx.x == 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) tmask[e] = 0ull;
+    for (int q = threadIdx.x; q < S; q += blockDim.x) {
+        t_idx[q] = __ldcg(d.topk_idx + q);
+        t_w[q] = __ldcg(d.topk_w + q);
+    }
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        t_sx[t] = __ldcg(a.sx + t);
+        t_sumx[t] = __ldcg(a.sumx + t);
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < S; q += blockDim.x) {
+        const int e = t_idx[q];
+        if (e >= 0 && e < E)
+            atomicOr(tmask + e, 1ull << (q / K));
+        else if (writer)
+            set_flag(a.flag_dev, MAPLE_DEVFLAG_BAD_INDEX);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int per = (E + 31) / 32, e0 = lane * per;
+        int csum = 0, asum = 0;
+        for (int i = 0; i < per; i++) {
+            const int e = e0 + i;
+            if (e < E) {
+                const int c = __popcll(tmask[e]);
+                csum += c;
+                asum += c > 0;
+            }
+        }
+        int cs = csum, as = asum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL, cs, o), w = __shfl_up_sync(FULL, as, o);
+            if (lane >= o) {
+                cs += v;
+                as += w;
+            }
+        }
+        int coff = cs - csum, aoff = as - asum;
+        for (int i = 0; i < per; i++) {
+            const int e = e0 + i;
+            if (e < E) {
+                const int c = __popcll(tmask[e]);
+                t_cnt[e] = c;
+                t_off[e] = coff;
+                if (writer && d.tap_counts) d.tap_counts[e] = c;
+                if (writer && d.tap_offsets) d.tap_offsets[e] = coff;
+                coff += c;
+                if (c) t_act[aoff++] = e;
+            }
+        }
+        if (lane == 31) {
+            t_off[E] = cs;
+            t_misc[0] = as;
+            if (writer && d.tap_offsets) d.tap_offsets[E] = cs;
+        }
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < S; q += blockDim.x) {
+        const int e = t_idx[q];
+        if (e < 0 || e >= E) continue;
+        const int t = q / K;
+        const int p = t_off[e] + __popcll(tmask[e] & ((1ull << t) - 1ull));
+        t_perm[p] = q;
+        t_inv[q] = p;
+        if (writer && d.tap_perm) d.tap_perm[p] = q;
+    }
+    __syncthreads();
+    a.active = t_act;
+    a.n_active = t_misc;
+    a.counts = t_cnt;
+    a.offsets = t_off;
+    a.perm = t_perm;
+    a.inv = t_inv;
+    a.topk_w = t_w;
+    a.sx = t_sx;
+    a.sumx = t_sumx;
+
+    const int n_active = t_misc[0];
     const int pairs = a.F / 32, blocks = a.D / 128;
     const int n_g = n_active * pairs, n_d = n_active * blocks;
     const int g0 = (int)((int64_t)n_g * blockIdx.x / gridDim.x), g1 = (int)((int64_t)n_g * (blockIdx.x + 1) / gridDim.x);
     const int d0 = (int)((int64_t)n_d * blockIdx.x / gridDim.x), d1 = (int)((int64_t)n_d * (blockIdx.x + 1) / gridDim.x);
-    const int n_mine = (g1 - g0) + (d1 - d0);
+    const int nG = g1 - g0, n_items = nG + (d1 - d0);
     const int Cg = a.D / 64, Cd = a.F / 64;
-    const uint32_t g_bytes = (uint32_t)(2 * Cg * 512), d_bytes = (uint32_t)(4 * Cd * 512);
+    // item i of this CTA -> kind (0 gate/up, 1 down), active index, sub-block
+    auto item_of = [&](int i, int &kind, int &ai, int &sub) {
+        if (i < nG) {
+            kind = 0;
+            ai = (g0 + i) / pairs;
+            sub = (g0 + i) % pairs;
+        } else {
+            kind = 1;
+            ai = (d0 + i - nG) / blocks;
+            sub = (d0 + i - nG) % blocks;
+        }
+    };
 
-    if (warp == kGemvWarps) {
-        // ---------------- producer: bulk copies of the codes, in item order
+    if (warp == 0) {
+        // ---------------- codes and scales of every item, in order
         if (lane == 0) {
-            for (int i = 0; i < n_mine; i++) {
-                const int buf = i % d.nbuf;
-                if (!dec_wait(b_empty + 8 * buf, ((i / d.nbuf) & 1) ^ 1)) {
+            int issued = 0;
+            for (int i = 0; i < n_items; i++) {
+                const int ws = i % nw;
+                if (!dec_wait(b_wempty + 8 * ws, ((i / nw) & 1) ^ 1)) {
                     set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
                     break;
                 }
-                const uint8_t *src;
-                uint32_t bytes;
-                if (i < g1 - g0) {
-                    const int it = g0 + i, e = a.active[it / pairs], pr = it % pairs;
-                    src = a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)(2 * pr) * Cg * 512;
-                    bytes = g_bytes;
+                issued = i + 1;
+                int kind, ai, sub;
+                item_of(i, kind, ai, sub);
+                const int e = a.active[ai];
+                DecWMeta *m = wmeta + ws;
+                m->e = e;
+                m->sub = sub;
+                m->kind = kind;
+                m->cnt = a.counts[e];
+                m->base = a.offsets[e];
+                uint8_t *dst = wring + (size_t)ws * d.wslot_bytes;
+                const uint32_t bar = b_wfull + 8 * ws;
+                if (kind == 0) {
+                    const uint32_t cb = (uint32_t)(2 * Cg * 512);
+                    dec_expect(bar, cb + 256);
+                    dec_bulk(dst, a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)(2 * sub) * Cg * 512, cb, bar);
+                    dec_bulk(dst + cb, a.alpha_gate + (size_t)e * a.F + 32 * sub, 128, bar);
+                    dec_bulk(dst + cb + 128, a.alpha_up + (size_t)e * a.F + 32 * sub, 128, bar);
                 } else {
-                    const int it = d0 + (i - (g1 - g0)), e = a.active[it / blocks], blk = it % blocks;
-                    src = a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)(4 * blk) * Cd * 512;
-                    bytes = d_bytes;
-                }
-                const uint32_t dst = (uint32_t)__cvta_generic_to_shared(ring + (size_t)buf * d.buf_bytes);
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b_full + 8 * buf),
-                             "r"(bytes)
-                             : "memory");
-                for (uint32_t off = 0; off < bytes; off += 8192) {
-                    const uint32_t n = bytes - off < 8192 ? bytes - off : 8192;
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                            dst + off),
-                        "l"(src + off), "r"(n), "r"(b_full + 8 * buf)
-                        : "memory");
+                    const uint32_t cb = (uint32_t)(4 * Cd * 512);
+                    dec_expect(bar, cb + 512);
+                    dec_bulk(dst, a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)(4 * sub) * Cd * 512, cb, bar);
+                    dec_bulk(dst + cb, a.alpha_down + (size_t)e * a.D + 128 * sub, 512, bar);
                 }
             }
+            // no copy may still be landing when the CTA exits
+            for (int j = issued > nw ? issued - nw : 0; j < issued; j++)
+                (void)dec_wait(b_wfull + 8 * (j % nw), (j / nw) & 1);
         }
-        return;   // the producer warp takes no part in the compute barriers below
+        return;
     }
 
-    // ---------------- compute warps (named barrier 1, kGemvWarps*32 threads)
-    auto csync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kGemvWarps * 32) : "memory"); };
-    bool ok = true;
-    int staged_e = -1, staged_b0 = -1, staged_kind = -1;
-    for (int i = 0; i < n_mine && ok; i++) {
-        const int buf = i % d.nbuf;
-        const bool is_down = i >= g1 - g0;
-        const int it = is_down ? d0 + (i - (g1 - g0)) : g0 + i;
-        const int ai = is_down ? it / blocks : it / pairs;
-        const int e = a.active[ai];
-        const int cnt = a.counts[e], base = a.offsets[e];
-        if (is_down && staged_kind != 1 + e) {
-            // wait until expert e's q_h is published
-            if (threadIdx.x == 0) {
-                const uint64_t t0 = global_timer_ns();
-                unsigned v;
-                s_flag = 1;
-                while (true) {
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(d.ready + e) : "memory");
-                    if (v == d.epoch) break;
-                    if (global_timer_ns() - t0 > 2000000000ull) {
+    if (warp <= kDecGroups) {
+        // ---------------- activation staging for compute group g
+        const int g = warp - 1;
+        if (lane == 0) {
+            int k = 0;
+            bool ok = true;
+            int staged = 0;   // units whose copies were issued
+            for (int i = g; i < n_items && ok; i += kDecGroups) {
+                int kind, ai, sub;
+                item_of(i, kind, ai, sub);
+                const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
+                if (kind == 1) {
+                    // every gate/up item of expert e must be done before its h rows are read
+                    const uint64_t t0 = global_timer_ns();
+                    unsigned v = 0;
+                    while (true) {
+                        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(d.arrive + e) : "memory");
+                        if (v >= (unsigned)pairs) break;
+                        __nanosleep(128);
+                        if (global_timer_ns() - t0 > 2000000000ull) {
+                            set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                }
+                for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++) {
+                    const int buf = k & 1;
+                    if (!dec_wait(b_aempty + 8 * (2 * g + buf), ((k >> 1) & 1) ^ 1)) {
                         set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
-                        s_flag = 0;
+                        ok = false;
                         break;
                     }
+                    const int nb = min(kGemvTokens, cnt - b0);
+                    DecActMeta *m = ameta + 2 * g + buf;
+                    m->nb = nb;
+                    m->b0 = b0;
+                    m->base = base;
+                    m->e = e;
+                    uint8_t *dst = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
+                    const uint32_t bar = b_afull + 8 * (2 * g + buf);
+                    if (kind == 0) {
+                        for (int j = 0; j < nb; j++) {
+                            const int slot = a.perm[base + b0 + j], t = slot / a.K;
+                            m->slot[j] = slot;
+                            m->s[j] = a.sx[t];
+                            m->sum[j] = a.sumx[t];
+                        }
+                        dec_expect(bar, (uint32_t)(nb * a.D));
+                        for (int j = 0; j < nb; j++)
+                            dec_bulk(dst + (size_t)j * a.D, a.qx + (size_t)(m->slot[j] / a.K) * a.D, (uint32_t)a.D, bar);
+                    } else {
+                        for (int j = 0; j < nb; j++) m->slot[j] = a.perm[base + b0 + j];
+                        dec_expect(bar, (uint32_t)(nb * a.F * 4));
+                        dec_bulk(dst, a.h + (size_t)(base + b0) * a.F, (uint32_t)(nb * a.F * 4), bar);
+                    }
+                    staged = k + 1;
                 }
             }
-            csync();
-            if (!s_flag) break;
+            for (int j = staged > 2 ? staged - 2 : 0; j < staged; j++)
+                (void)dec_wait(b_afull + 8 * (2 * g + (j & 1)), (j >> 1) & 1);
         }
-        if (!dec_wait(b_full + 8 * buf, (i / d.nbuf) & 1)) {
-            if (threadIdx.x == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+        return;
+    }
+
+    if (warp < kDecFirstCompute) {
+        // ---------------- publishing warp of group g
+        const int g = warp - 1 - kDecGroups;
+        int r = 0;
+        for (int i = g; i < n_items; i += kDecGroups) {
+            int kind, ai, sub;
+            item_of(i, kind, ai, sub);
+            const int cnt = a.counts[a.active[ai]];
+            bool ok = true;
+            for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, r++) {
+                const int rs = r % kDecRec;
+                if (!dec_wait(b_rfull + 8 * (kDecRec * g + rs), (r / kDecRec) & 1)) {
+                    if (lane == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                const DecRecord rec = recs[kDecRec * g + rs];
+                fence_gpu();   // the group's h / yE stores, seen through the barrier chain, before what follows
+                if (rec.kind == 0) {
+                    if (rec.last && lane == 0)
+                        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(d.arrive + rec.e) : "memory");
+                } else {
+                    unsigned prev = 0;
+                    int t = 0;
+                    if (lane < rec.nb) {
+                        t = rec.slot[lane] / a.K;
+                        prev = atomicAdd(a.comb_cnt + (size_t)t * blocks + rec.sub, 1u);
+                    }
+                    unsigned done = __ballot_sync(FULL, lane < rec.nb && prev == (unsigned)(a.K - 1));
+                    if (done) fence_gpu();
+                    while (done) {
+                        const int j = __ffs(done) - 1;
+                        done &= done - 1;
+                        const int tt = __shfl_sync(FULL, t, j);
+                        // channels rec.sub*128 + 4*lane .. +3 of token tt, in rank order
+                        const int cc = rec.sub * 128 + 4 * lane;
+                        float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int kk = 0; kk < a.K; kk++) {
+                            const int sl = tt * a.K + kk;
+                            const float wk = a.topk_w[sl];
+                            const float4 ev = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)a.inv[sl] * a.D + cc));
+                            yv.x = __fmaf_rn(wk, ev.x, yv.x);
+                            yv.y = __fmaf_rn(wk, ev.y, yv.y);
+                            yv.z = __fmaf_rn(wk, ev.z, yv.z);
+                            yv.w = __fmaf_rn(wk, ev.w, yv.w);
+                        }
+                        const size_t o = (size_t)tt * a.D + cc;
+                        if (a.resid) {
+                            const float4 rv = *reinterpret_cast<const float4 *>(a.resid + o);
+                            yv.x = __fadd_rn(rv.x, yv.x);
+                            yv.y = __fadd_rn(rv.y, yv.y);
+                            yv.z = __fadd_rn(rv.z, yv.z);
+                            yv.w = __fadd_rn(rv.w, yv.w);
+                        }
+                        *reinterpret_cast<float4 *>(a.y + o) = yv;
+                        if (lane == j) a.comb_cnt[(size_t)tt * blocks + rec.sub] = 0;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) dec_arrive(b_rempty + 8 * (kDecRec * g + rs));
+            }
+            if (!ok) break;
+        }
+        return;
+    }
+
+    // ---------------- compute group g: eight warps
+    const int g = (warp - kDecFirstCompute) / kDecGroupWarps, gw = (warp - kDecFirstCompute) % kDecGroupWarps;
+    const int gtid = gw * 32 + lane;
+    const int bar_id = 1 + g;
+    auto gsync = [&] { asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kDecGroupThreads) : "memory"); };
+    uint8_t *scr = gscr + (size_t)g * gscr_bytes;
+    int *red = (int *)scr;                                            // [8 warps][kGemvTokens][32]
+    int8_t *qh = (int8_t *)(red + kDecGroupWarps * kGemvTokens * 32);  // [kGemvTokens][F]
+    float *shs = (float *)(qh + (size_t)kGemvTokens * a.F);          // [kGemvTokens]
+    int *sumqh = (int *)(shs + kGemvTokens);                         // [kGemvTokens]
+
+    int k = 0, r = 0;
+    for (int i = g; i < n_items; i += kDecGroups) {
+        const int ws = i % nw;
+        if (!dec_wait(b_wfull + 8 * ws, (i / nw) & 1)) {
+            if (gtid == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
             break;
         }
-        const uint8_t *wb = ring + (size_t)buf * d.buf_bytes;
-        if (!is_down) {
-            const int pr = it % pairs;
-            const int gl = warp >> 2, kq = warp & 3, NI = Cg / 4;
-            for (int b0 = 0; b0 < cnt; b0 += kGemvTokens) {
-                const int nb = min(kGemvTokens, cnt - b0);
-                if (!(staged_kind == 0 && staged_e == e && staged_b0 == b0)) {
-                    if (threadIdx.x < nb) s_slot[threadIdx.x] = a.perm[base + b0 + threadIdx.x];
-                    csync();
-                    const int row16 = a.D / 16;
-                    for (int q = threadIdx.x; q < nb * row16; q += kGemvWarps * 32) {
-                        const int j = q / row16, c16 = q - j * row16;
-                        reinterpret_cast<uint4 *>(xs + (size_t)j * a.D)[c16] =
-                            __ldg(reinterpret_cast<const uint4 *>(a.qx + (size_t)(s_slot[j] / a.K) * a.D) + c16);
-                    }
-                    staged_kind = 0;
-                    staged_e = e;
-                    staged_b0 = b0;
-                }
-                csync();
-                int acc[kGemvTokens];
+        const DecWMeta wm = wmeta[ws];
+        const uint8_t *wb = wring + (size_t)ws * d.wslot_bytes;
+        const int cnt = wm.cnt, base = wm.base;
+        bool ok = true;
+        for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++, r++) {
+            const int buf = k & 1;
+            if (!dec_wait(b_afull + 8 * (2 * g + buf), (k >> 1) & 1)) {
+                if (gtid == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                ok = false;
+                break;
+            }
+            const DecActMeta &am = ameta[2 * g + buf];
+            const uint8_t *ab = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
+            const int nb = am.nb;
+            int acc2[kGemvTokens][2];
 #pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) acc[j] = 0;
-                const uint8_t *wl = wb + (size_t)gl * Cg * 512 + lane * 16;
-                for (int u = 0; u < NI; u++) {
-                    const int c = kq * NI + u;
-                    chunk_tokens(*reinterpret_cast<const uint4 *>(wl + (size_t)c * 512), xs, a.D, 64 * c, nb, acc);
+            for (int j = 0; j < kGemvTokens; j++) acc2[j][0] = acc2[j][1] = 0;
+            if (wm.kind == 0) {
+                // ---- gate/up: warp gw = row group gw/4 (of the pair), K quarter gw%4
+                const int rg = gw >> 2, kq = gw & 3, quarter = Cg / 4;
+                const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)rg * Cg * 512) + lane;
+                const uint4 *xl = reinterpret_cast<const uint4 *>(ab);
+#pragma unroll 1
+                for (int u = 0; u < quarter; u++) {
+                    const int c = kq * quarter + u;
+                    chunk_dot(wl[32 * c], xl + 4 * c, a.D / 16, nb, acc2);
                 }
 #pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) red[(warp * kGemvTokens + j) * 32 + lane] = acc[j];
-                csync();
-                if (warp < 2) {
-                    const int rr = (2 * pr + warp) * 16 + (lane & 15);
+                for (int j = 0; j < kGemvTokens; j++) red[(gw * kGemvTokens + j) * 32 + lane] = acc2[j][0] + acc2[j][1];
+                gsync();
+                if (kq == 0) {
                     const bool is_up = lane >= 16;
-                    const float al = is_up ? a.alpha_up[(size_t)e * a.F + rr] : a.alpha_gate[(size_t)e * a.F + rr];
+                    const int rr = (2 * wm.sub + rg) * 16 + (lane & 15);
+                    const float al = ((const float *)(wb + 2 * Cg * 512))[(is_up ? 32 : 0) + 16 * rg + (lane & 15)];
                     for (int j = 0; j < nb; j++) {
                         int sum = 0;
 #pragma unroll
-                        for (int q = 0; q < 4; q++) sum += red[((warp * 4 + q) * kGemvTokens + j) * 32 + lane];
-                        const int slot = s_slot[j], t = slot / a.K;
-                        const int av = sum - a.sumx[t];
-                        const float v = __fmul_rn((float)av, __fmul_rn(al, a.sx[t]));
+                        for (int q = 0; q < 4; q++) sum += red[((gw + q) * kGemvTokens + j) * 32 + lane];
+                        const int av = sum - am.sum[j];
+                        const float v = __fmul_rn((float)av, __fmul_rn(al, am.s[j]));
                         const float uu = __shfl_down_sync(FULL, v, 16);
-                        if (!is_up) a.h[(size_t)(base + b0 + j) * a.F + rr] = swiglu(v, uu);
+                        if (!is_up) a.h[(size_t)(base + am.b0 + j) * a.F + rr] = swiglu(v, uu);
                         int *tap = is_up ? a.tap_acc_up : a.tap_acc_gate;
-                        if (tap) tap[(size_t)slot * a.F + rr] = av;
+                        if (tap) tap[(size_t)am.slot[j] * a.F + rr] = av;
                     }
                 }
-                csync();
-            }
-            if (threadIdx.x == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b_empty + 8 * buf) : "memory");
-            // the last item of expert e to finish requantises e's slots and publishes them
-            if (warp < 2) fence_gpu();
-            csync();
-            if (threadIdx.x == 0) s_flag = atomicAdd(a.exp_cnt + e, 1u) == (unsigned)(pairs - 1);
-            csync();
-            if (s_flag) {
-                fence_gpu();
-                if (threadIdx.x == 0) a.exp_cnt[e] = 0;
-                requant_slots_warps(a, base, cnt, kGemvWarps);
-                fence_gpu();
-                csync();
-                if (threadIdx.x == 0) asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(d.ready + e), "r"(d.epoch) : "memory");
-            }
-        } else {
-            const int blk = it % blocks;
-            const int gl = warp >> 1, kh = warp & 1, NH = Cd / 2;
-            for (int b0 = 0; b0 < cnt; b0 += kGemvTokens) {
-                const int nb = min(kGemvTokens, cnt - b0);
-                if (!(staged_kind == 1 + e && staged_b0 == b0)) {
-                    if (threadIdx.x < nb) s_slot[threadIdx.x] = a.perm[base + b0 + threadIdx.x];
-                    const int n16 = nb * a.F / 16;
-                    for (int q = threadIdx.x; q < n16; q += kGemvWarps * 32)
-                        reinterpret_cast<uint4 *>(xs)[q] =
-                            __ldcg(reinterpret_cast<const uint4 *>(a.qh + (size_t)(base + b0) * a.F) + q);
-                    staged_kind = 1 + e;
-                    staged_b0 = b0;
-                }
-                csync();
-                int acc[kGemvTokens];
-#pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) acc[j] = 0;
-                const uint8_t *wl = wb + (size_t)gl * Cd * 512 + lane * 16;
-                for (int u = 0; u < NH; u++) {
-                    const int c = kh * NH + u;
-                    chunk_tokens(*reinterpret_cast<const uint4 *>(wl + (size_t)c * 512), xs, a.F, 64 * c, nb, acc);
-                }
-#pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) red[(warp * kGemvTokens + j) * 32 + lane] = acc[j];
-                csync();
-                if (warp < 4) {
-                    const int cg = (blk * 4 + warp) * 32 + lane;
-                    const float al = a.alpha_down[(size_t)e * a.D + cg];
-                    for (int j = 0; j < nb; j++) {
-                        const int p = base + b0 + j;
-                        const int sum = red[((2 * warp) * kGemvTokens + j) * 32 + lane] +
-                                        red[((2 * warp + 1) * kGemvTokens + j) * 32 + lane];
-                        const int av = sum - __ldcg(a.sumqh + p);
-                        a.ye[(size_t)p * a.D + cg] = __fmul_rn((float)av, __fmul_rn(al, __ldcg(a.sh + p)));
-                        if (a.tap_acc_down) a.tap_acc_down[(size_t)s_slot[j] * a.D + cg] = av;
+            } else {
+                // ---- down: requantise the batch's h rows (one slot per warp), then warp gw =
+                //      channel group 4*blk + gw/2, K half gw%2
+                const float *hr = (const float *)ab;
+                for (int j = gw; j < nb; j += kDecGroupWarps) {
+                    const float4 *h4 = reinterpret_cast<const float4 *>(hr + (size_t)j * a.F);
+                    float amax = 0.0f;
+                    for (int q = lane; q < a.F / 4; q += 32) {
+                        const float4 v = h4[q];
+                        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
                     }
-                    fence_gpu();
-                }
-                csync();
-                if (threadIdx.x < nb) {
-                    const int t = s_slot[threadIdx.x] / a.K;
-                    const unsigned prev = atomicAdd(a.comb_cnt + (size_t)t * blocks + blk, 1u);
-                    s_done[threadIdx.x] = prev == (unsigned)(a.K - 1);
-                }
-                csync();
-                for (int j = 0; j < nb; j++) {
-                    if (!s_done[j]) continue;
-                    fence_gpu();
-                    const int t = s_slot[j] / a.K;
-                    if (threadIdx.x < 128) {
-                        const int cc = blk * 128 + threadIdx.x;
-                        float yv = 0.0f;
-                        for (int k = 0; k < a.K; k++) {
-                            const int s = t * a.K + k;
-                            yv = __fmaf_rn(a.topk_w[s], __ldcg(a.ye + (size_t)a.inv[s] * a.D + cc), yv);
+                    amax = warp_max(amax);
+                    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+                    int sum = 0;
+                    for (int q = lane; q < a.F / 4; q += 32) {
+                        const float4 v = h4[q];
+                        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+                        if (amax > 0.0f) {
+                            q0 = quant_code(v.x, inv);
+                            q1 = quant_code(v.y, inv);
+                            q2 = quant_code(v.z, inv);
+                            q3 = quant_code(v.w, inv);
                         }
-                        const size_t o = (size_t)t * a.D + cc;
-                        a.y[o] = a.resid ? __fadd_rn(a.resid[o], yv) : yv;
+                        sum += q0 + q1 + q2 + q3;
+                        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                                            ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+                        reinterpret_cast<uint32_t *>(qh + (size_t)j * a.F)[q] = pk;
+                        if (wm.sub == 0 && a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)am.slot[j] * a.F)[q] = pk;
                     }
-                    if (threadIdx.x == 0) a.comb_cnt[(size_t)t * blocks + blk] = 0;
+                    sum = warp_sum_int(sum);
+                    if (lane == 0) {
+                        const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+                        shs[j] = sv;
+                        sumqh[j] = sum;
+                        if (wm.sub == 0 && a.tap_sh) a.tap_sh[am.slot[j]] = sv;
+                    }
                 }
-                csync();
+                gsync();
+                const int cgl = gw >> 1, kh = gw & 1, half = Cd / 2;
+                const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)cgl * Cd * 512) + lane;
+                const uint4 *xl = reinterpret_cast<const uint4 *>(qh);
+#pragma unroll 1
+                for (int u = 0; u < half; u++) {
+                    const int c = kh * half + u;
+                    chunk_dot(wl[32 * c], xl + 4 * c, a.F / 16, nb, acc2);
+                }
+#pragma unroll
+                for (int j = 0; j < kGemvTokens; j++) red[(gw * kGemvTokens + j) * 32 + lane] = acc2[j][0] + acc2[j][1];
+                gsync();
+                if (kh == 0) {
+                    const int cg = (wm.sub * 4 + cgl) * 32 + lane;
+                    const float al = ((const float *)(wb + 4 * Cd * 512))[cgl * 32 + lane];
+                    for (int j = 0; j < nb; j++) {
+                        const int p = base + am.b0 + j;
+                        const int av = red[(gw * kGemvTokens + j) * 32 + lane] +
+                                       red[((gw + 1) * kGemvTokens + j) * 32 + lane] - sumqh[j];
+                        a.ye[(size_t)p * a.D + cg] = __fmul_rn((float)av, __fmul_rn(al, shs[j]));
+                        if (a.tap_acc_down) a.tap_acc_down[(size_t)am.slot[j] * a.D + cg] = av;
+                    }
+                }
             }
-            if (threadIdx.x == 0)
-                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b_empty + 8 * buf) : "memory");
+            gsync();
+            if (gtid == 0) {
+                // hand the batch to the publishing warp, free the activation slot
+                const int rs = r % kDecRec;
+                if (!dec_wait(b_rempty + 8 * (kDecRec * g + rs), ((r / kDecRec) & 1) ^ 1))
+                    set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                DecRecord *rec = recs + kDecRec * g + rs;
+                rec->kind = wm.kind;
+                rec->e = wm.e;
+                rec->sub = wm.sub;
+                rec->nb = nb;
+                rec->base = base;
+                rec->last = b0 + kGemvTokens >= cnt;
+                for (int j = 0; j < nb; j++) rec->slot[j] = am.slot[j];
+                dec_arrive(b_rfull + 8 * (kDecRec * g + rs));
+                dec_arrive(b_aempty + 8 * (2 * g + buf));
+            }
         }
+        if (!ok) break;
+        gsync();
+        if (gtid == 0) dec_arrive(b_wempty + 8 * ws);
     }
-    (void)ok;
 }
 
 }  // namespace maple

@@ -45,6 +45,7 @@ struct maple_moe_s {
     int4 *pieces;
     int *n_pieces;
     int8_t *xperm;                 // q_x rows in slot order (tensor-core path)
+    float *pscale;                 // s_x of each position's token (tensor-core path)
     CUtensorMap map_xperm, map_qh; // TMA maps of the activation operands
     float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
     // workspace
@@ -61,9 +62,9 @@ struct maple_moe_s {
     int *sumqh;
     float *ye;
     unsigned *tg_cnt, *glob_cnt, *exp_cnt, *comb_cnt;
-    unsigned *ready;      // [E] epoch of each expert's published q_h (decode kernel)
-    unsigned epoch;
-    int dec_nbuf, dec_buf_bytes;
+    unsigned *arrive;     // [E] finished gate/up items per expert (decode kernel)
+    bool dec_persistent;  // the persistent decode kernel fits this shape
+    int dec_optin;        // shared memory a block may opt in to
     uint16_t *xn;
     // flag word in host-mapped memory
     unsigned *flag_host;
@@ -73,9 +74,17 @@ struct maple_moe_s {
     bool use_events;
 };
 
+// Stage events are recorded as external event nodes when the stream is being
+// captured into a CUDA graph, so that they can still be timed after replay.
 static void stage_event(maple_moe_s *h, int i, cudaStream_t st)
 {
-    if (h->use_events) cudaEventRecord(h->ev[i], st);
+    if (!h->use_events) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(h->ev[i], st, cudaEventRecordExternal);
+    else
+        cudaEventRecord(h->ev[i], st);
 }
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
@@ -258,7 +267,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     size_t o_gu = ar.take(E * gu_bytes_per_expert(D, F)), o_dn = ar.take(E * dn_bytes_per_expert(D, F));
     size_t o_tgu = ar.take(E * F * D / 2), o_tdn = ar.take(E * D * F / 4);
     size_t o_pc = ar.take((E + S / kPieceSlots + 1) * 16), o_npc = ar.take(4);
-    size_t o_xp = ar.take(S * D);
+    size_t o_xp = ar.take(S * D), o_ps = ar.take(S * 4 + 512);
     size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
     size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
     size_t o_qx = ar.take(Tm * D), o_sx = ar.take(Tm * 4), o_sumx = ar.take(Tm * 4);
@@ -293,6 +302,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->pieces = (int4 *)(b + o_pc);
     h->n_pieces = (int *)(b + o_npc);
     h->xperm = (int8_t *)(b + o_xp);
+    h->pscale = (float *)(b + o_ps);
     h->alpha_gate = (float *)(b + o_ag);
     h->alpha_up = (float *)(b + o_au);
     h->alpha_down = (float *)(b + o_ad);
@@ -320,11 +330,13 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->glob_cnt = (unsigned *)(b + o_gc);
     h->exp_cnt = (unsigned *)(b + o_ec);
     h->comb_cnt = (unsigned *)(b + o_cc);
-    h->ready = (unsigned *)(b + o_rdy);
-    h->epoch = 0;
-    h->dec_buf_bytes = (int)(16 * D > 32 * F ? 16 * D : 32 * F);
-    h->dec_nbuf = kDecRingBytes / h->dec_buf_bytes;
-    if (h->dec_nbuf > 8) h->dec_nbuf = 8;
+    h->arrive = (unsigned *)(b + o_rdy);
+    {
+        int optin = 0;
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+        h->dec_optin = optin;
+        h->dec_persistent = decode_smem_bytes(h->D, h->F, 1, h->K, h->E, 2) <= (size_t)optin;
+    }
     h->xn = (uint16_t *)(b + o_xn);
 
     cudaStream_t st = (cudaStream_t)stream;
@@ -357,6 +369,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     allow_max_smem((const void *)tc_gemm_kernel<1>, h->device);
     allow_max_smem((const void *)pick_route(h->D, h->E), h->device);
     allow_max_smem((const void *)pick_qtopk(h->D, h->E), h->device);
+    allow_max_smem((const void *)router_gemm_kernel, h->device);
     allow_max_smem((const void *)pick_gateup(h->D), h->device);
     allow_max_smem((const void *)pick_down(h->F), h->device);
     allow_max_smem((const void *)decode_experts_kernel, h->device);
@@ -384,7 +397,8 @@ static int take_flag(maple_moe_t h)
 
 // routing stage: quantise, logits, top-k (+ the permutation)
 static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
-                     float *out_w, int32_t *out_counts, bool permute, bool pieces, cudaStream_t st)
+                     float *out_w, int32_t *out_counts, bool permute, bool pieces, bool logits_only,
+                     cudaStream_t st, unsigned *clear = nullptr, int n_clear = 0)
 {
     RouteArgs a;
     memset(&a, 0, sizeof a);
@@ -426,13 +440,25 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     const bool small = T <= kRouteSmallT;
     const bool fused = small && permute && !pieces && (int64_t)T * h->E <= kFusedMarkBytes;
     a.fuse_permute = fused ? 1 : 0;
+    a.logits_only = logits_only ? 1 : 0;
+    if (clear && !small) {
+        if (cudaMemsetAsync(clear, 0, (size_t)n_clear * 4, st) != cudaSuccess) return MAPLE_ERR_CUDA;
+    } else {
+        a.clear = clear;
+        a.n_clear = n_clear;
+    }
+    if (logits_only) {
+        dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
+        pick_route(h->D, h->E)<<<grid, 256, route_smem_bytes(h->D), st>>>(a);
+        return launch_status();
+    }
     if (small) {
         dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
         pick_route(h->D, h->E)<<<grid, 256, route_smem_bytes(h->D), st>>>(a);
     } else {
         dim3 grid((T + kRgTok - 1) / kRgTok, h->E / kRgExp);
-        router_gemm_kernel<<<grid, 256, 0, st>>>(x, T, h->D, h->E, h->router_w, h->router_bias, h->logits,
-                                                 a.tap_logits);
+        router_gemm_kernel<<<grid, 256, 2 * kRgStage, st>>>(x, T, h->D, h->E, h->router_w, h->router_bias,
+                                                           h->logits, a.tap_logits);
         pick_qtopk(h->D, h->E)<<<(T + 7) / 8, 256, (size_t)8 * h->D * 2, st>>>(a);
     }
     if (permute && !fused) {
@@ -463,8 +489,17 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     return launch_status();
 }
 
+// smallest ring of weight slots (2..4) whose decode kernel fits, 0 if none
+static int decode_ring_slots(maple_moe_t h, int T)
+{
+    if (!h->dec_persistent || T > kRouteSmallT || (int64_t)T * h->E > kFusedMarkBytes) return 0;
+    for (int nw = kDecWSlots; nw >= 2; nw--)
+        if (decode_smem_bytes(h->D, h->F, T, h->K, h->E, nw) <= (size_t)h->dec_optin) return nw;
+    return 0;
+}
+
 static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
-                       cudaStream_t st)
+                       int nw, cudaStream_t st)
 {
     GemvArgs g;
     memset(&g, 0, sizeof g);
@@ -505,19 +540,29 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         g.tap_sh = taps->s_h;
     }
     g.flag_dev = h->flag_dev;
-    if (h->dec_nbuf >= 2) {
-        // persistent, cooperative: one CTA per SM streams gate/up then down
+    if (nw) {
+        // persistent, cooperative: one CTA per SM builds the permutation from
+        // the router's top-k, then streams gate/up and down
         DecodeArgs d;
+        memset(&d, 0, sizeof d);
         d.g = g;
-        d.ready = h->ready;
-        d.epoch = ++h->epoch;
-        d.nbuf = h->dec_nbuf;
-        d.buf_bytes = h->dec_buf_bytes;
+        d.arrive = h->arrive;
+        d.wslot_bytes = dec_wslot_bytes(h->D, h->F);
+        d.aslot_bytes = dec_aslot_bytes(h->D, h->F);
+        d.nw = nw;
+        d.topk_idx = h->topk_idx;
+        d.topk_w = h->topk_w;
+        if (taps) {
+            d.tap_counts = taps->expert_counts;
+            d.tap_offsets = taps->expert_offsets;
+            d.tap_perm = taps->perm;
+        }
+        // h->arrive was zeroed by the routing kernel
         cudaLaunchConfig_t lc;
         memset(&lc, 0, sizeof lc);
         lc.gridDim = dim3(h->num_sms);
         lc.blockDim = dim3(kDecThreads);
-        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, h->dec_buf_bytes, h->dec_nbuf);
+        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E, nw);
         lc.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;
@@ -559,7 +604,7 @@ extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int3
     if (!x || !aligned16(x)) return MAPLE_ERR_INVALID_ARG;
     for (const void *p : {(const void *)topk_idx, (const void *)topk_w, (const void *)expert_counts})
         if (p && !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
-    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr, false,
+    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr, false, false,
                      (cudaStream_t)stream);
 }
 
@@ -578,6 +623,7 @@ static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, co
     g.perm = h->perm;
     g.sx = h->sx;
     g.sh = h->sh;
+    g.pscale = h->pscale;
     g.flag = h->flag_dev;
     g.codes = h->w_tc_gu;
     g.alpha0 = h->alpha_gate;
@@ -585,7 +631,7 @@ static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, co
     g.out = h->h;
     g.tap0 = taps ? taps->acc_gate : nullptr;
     g.tap1 = taps ? taps->acc_up : nullptr;
-    gather_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->qx, h->perm, h->K, h->D, S, h->xperm);
+    gather_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->qx, h->sx, h->perm, h->K, h->D, S, h->xperm, h->pscale);
     tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_xperm, g);
     requant_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->h, S, h->F, h->perm, h->qh, h->sh, taps ? taps->q_h : nullptr,
                                                    taps ? taps->s_h : nullptr);
@@ -614,11 +660,15 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
                         const maple_moe_taps *taps, cudaStream_t st)
 {
     const bool tc = use_tc(h, T);
+    const int nw = tc ? 0 : decode_ring_slots(h, T);
     stage_event(h, 0, st);
-    int rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, st);
+    // the persistent decode kernel builds its own permutation from the top-k; the
+    // routing kernel zeroes its arrival counters
+    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, false, st, h->arrive, h->E)
+                : run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, false, st);
     if (rc) return rc;
     stage_event(h, 1, st);
-    return tc ? run_experts_tc(h, T, y, resid, taps, st) : run_experts(h, T, y, resid, taps, st);
+    return tc ? run_experts_tc(h, T, y, resid, taps, st) : run_experts(h, T, y, resid, taps, nw, st);
 }
 
 extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const maple_moe_taps *taps,

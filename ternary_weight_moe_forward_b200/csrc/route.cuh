@@ -33,6 +33,9 @@ struct RouteArgs {
     unsigned *tg_cnt, *glob_cnt;
     // permutation (filled by the last CTA when fuse_permute)
     int fuse_permute;
+    int logits_only;   // stop after the logits and the int8 codes (top-k is done by the consumer)
+    unsigned *clear;   // [n_clear] counters of the next kernel, zeroed by CTA (0, 0) (may be null)
+    int n_clear;
     int *counts, *offsets, *perm, *inv, *active, *n_active;
     int *out_counts, *tap_offsets, *tap_perm;
     unsigned *flag;
@@ -153,8 +156,11 @@ __device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be)
     return v > bv || (v == bv && e < be);
 }
 
+// Top-k of one row of E logits (one warp); lane k < K ends with the k-th
+// choice (my_e) and its softmax weight (my_w).  A NaN logit ranks last and
+// raises the flag.
 template <int NPER>
-__device__ void topk_token_warp(const RouteArgs &a, int t)
+__device__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
 {
     const int lane = threadIdx.x & 31;
     float lv[NPER];
@@ -163,8 +169,8 @@ __device__ void topk_token_warp(const RouteArgs &a, int t)
     for (int j = 0; j < NPER; j++) {
         int e = lane + 32 * j;
         float v = -INFINITY;
-        if (e < a.E) {
-            v = __ldcg(a.logits + (size_t)t * a.E + e);
+        if (e < E) {
+            v = __ldcg(row + e);
             if (isnan(v)) {
                 nan_seen = true;
                 v = -INFINITY;
@@ -172,17 +178,17 @@ __device__ void topk_token_warp(const RouteArgs &a, int t)
         }
         lv[j] = v;
     }
-    if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(a.flag, MAPLE_DEVFLAG_NAN);
+    if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
     uint32_t taken = 0;
     float my_v = 0.0f;
-    int my_e = 0;
-    for (int k = 0; k < a.K; k++) {
+    my_e = 0;
+    for (int k = 0; k < K; k++) {
         float bv = -INFINITY;
         int be = 0x7fffffff;
 #pragma unroll
         for (int j = 0; j < NPER; j++) {
             int e = lane + 32 * j;
-            if (e < a.E && !((taken >> j) & 1u) && ranks_before(lv[j], e, bv, be)) {
+            if (e < E && !((taken >> j) & 1u) && ranks_before(lv[j], e, bv, be)) {
                 bv = lv[j];
                 be = e;
             }
@@ -206,14 +212,105 @@ __device__ void topk_token_warp(const RouteArgs &a, int t)
     const float l0 = __shfl_sync(FULL, my_v, 0);
     const float ek = exp_ref(__fsub_rn(my_v, l0));
     float S = 0.0f;
-    for (int k = 0; k < a.K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
+    for (int k = 0; k < K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
+    my_w = __fdiv_rn(ek, S);
+}
+
+// Top-k of NT rows at once in one warp (the rows' chains interleave, which
+// hides the shuffle latency); row r < nrows at rows[r].  Lane k < K ends with
+// row r's k-th choice in my_e[r] and its softmax weight in my_w[r].  Same
+// ranking, tie rule and softmax as topk_row_warp.
+template <int NPER, int NT>
+__device__ void topk_rows_warp(const float *const (&rows)[NT], int nrows, int E, int K, unsigned *flag,
+                               int (&my_e)[NT], float (&my_w)[NT])
+{
+    const int lane = threadIdx.x & 31;
+    float lv[NT][NPER];
+    bool nan_seen = false;
+#pragma unroll
+    for (int r = 0; r < NT; r++)
+#pragma unroll
+        for (int j = 0; j < NPER; j++) {
+            const int e = lane + 32 * j;
+            float v = -INFINITY;
+            if (r < nrows && e < E) {
+                v = __ldcg(rows[r] + e);
+                if (isnan(v)) {
+                    nan_seen = true;
+                    v = -INFINITY;
+                }
+            }
+            lv[r][j] = v;
+        }
+    if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
+    uint32_t taken[NT];
+    float my_v[NT];
+#pragma unroll
+    for (int r = 0; r < NT; r++) {
+        taken[r] = 0;
+        my_v[r] = 0.0f;
+        my_e[r] = 0;
+    }
+    for (int k = 0; k < K; k++) {
+        float bv[NT];
+        int be[NT];
+#pragma unroll
+        for (int r = 0; r < NT; r++) {
+            bv[r] = -INFINITY;
+            be[r] = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < NPER; j++) {
+                const int e = lane + 32 * j;
+                if (e < E && !((taken[r] >> j) & 1u) && ranks_before(lv[r][j], e, bv[r], be[r])) {
+                    bv[r] = lv[r][j];
+                    be[r] = e;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+            for (int r = 0; r < NT; r++) {
+                const float ov = __shfl_xor_sync(FULL, bv[r], o);
+                const int oe = __shfl_xor_sync(FULL, be[r], o);
+                if (ranks_before(ov, oe, bv[r], be[r])) {
+                    bv[r] = ov;
+                    be[r] = oe;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < NT; r++) {
+            if ((be[r] & 31) == lane) taken[r] |= 1u << (be[r] >> 5);
+            if (lane == k) {
+                my_v[r] = bv[r];
+                my_e[r] = be[r];
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < NT; r++) {
+        const float l0 = __shfl_sync(FULL, my_v[r], 0);
+        const float ek = exp_ref(__fsub_rn(my_v[r], l0));
+        float S = 0.0f;
+        for (int k = 0; k < K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
+        my_w[r] = __fdiv_rn(ek, S);
+    }
+}
+
+template <int NPER>
+__device__ void topk_token_warp(const RouteArgs &a, int t)
+{
+    const int lane = threadIdx.x & 31;
+    int my_e;
+    float my_w;
+    topk_row_warp<NPER>(a.logits + (size_t)t * a.E, a.E, a.K, a.flag, my_e, my_w);
     if (lane < a.K) {
-        const float w = __fdiv_rn(ek, S);
         const size_t o = (size_t)t * a.K + lane;
         a.topk_idx[o] = my_e;
-        a.topk_w[o] = w;
+        a.topk_w[o] = my_w;
         if (a.out_idx) a.out_idx[o] = my_e;
-        if (a.out_w) a.out_w[o] = w;
+        if (a.out_w) a.out_w[o] = my_w;
     }
 }
 
@@ -277,7 +374,7 @@ __host__ __device__ inline size_t route_smem_bytes(int D)
 }
 
 template <int NI, int NPER>
-__global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
+__global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
 {
     extern __shared__ __align__(16) uint8_t rsm[];
     uint16_t *xs = (uint16_t *)rsm;   // [nt][D] bf16
@@ -288,6 +385,8 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
     const int t0 = tg * kRouteTokens;
     const int nt = min(kRouteTokens, a.T - t0);
     const int e = eb * kRouteExperts + warp;
+    if (a.clear && eb == 0 && tg == 0)
+        for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
 
     // this lane's part of the router row, all in flight at once
     const float *wr = a.Wr + (size_t)e * a.D;
@@ -325,6 +424,8 @@ __global__ void __launch_bounds__(256) route_kernel(RouteArgs a)
             if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = v;
         }
     }
+
+    if (a.logits_only) return;
 
     // ---- last CTA of this token group: top-k + softmax
     fence_gpu();
@@ -409,13 +510,16 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a)
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_off[kMaxExperts + 1];
     __shared__ int s_warp[33];
+    constexpr int kB = 16;   // per-block counts loaded 16 at a time (independent loads in flight)
     const int nblk = (a.T + kPermBlockTokens - 1) / kPermBlockTokens;
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
         int run = 0;
-        for (int b = 0; b < nblk; b++) {
-            int c = a.blk_cnt[(size_t)b * a.E + e];
-            a.blk_cnt[(size_t)b * a.E + e] = run;
-            run += c;
+        for (int b0 = 0; b0 < nblk; b0 += kB) {
+            int c[kB];
+#pragma unroll
+            for (int j = 0; j < kB; j++) c[j] = b0 + j < nblk ? a.blk_cnt[(size_t)(b0 + j) * a.E + e] : 0;
+#pragma unroll
+            for (int j = 0; j < kB; j++) run += c[j];
         }
         s_cnt[e] = run;
     }
@@ -427,7 +531,19 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a)
         if (e < a.E) {
             a.counts[e] = s_cnt[e];
             if (a.out_counts) a.out_counts[e] = s_cnt[e];
-            for (int b = 0; b < nblk; b++) a.blk_cnt[(size_t)b * a.E + e] += s_off[e];
+            // first position of expert e's slots in each token block
+            int run = s_off[e];
+            for (int b0 = 0; b0 < nblk; b0 += kB) {
+                int c[kB];
+#pragma unroll
+                for (int j = 0; j < kB; j++) c[j] = b0 + j < nblk ? a.blk_cnt[(size_t)(b0 + j) * a.E + e] : 0;
+#pragma unroll
+                for (int j = 0; j < kB; j++)
+                    if (b0 + j < nblk) {
+                        a.blk_cnt[(size_t)(b0 + j) * a.E + e] = run;
+                        run += c[j];
+                    }
+            }
         }
     }
     if (a.pieces) {
@@ -480,52 +596,75 @@ __device__ __forceinline__ void tree_level(float (&v)[64], int off, bool upper)
     }
 }
 
-__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t *x, int T, int D, int E, const float *Wr,
-                                                          const float *bias, float *logits, float *tap_logits)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred)
 {
-    __shared__ __align__(16) uint16_t sx[kRgTok][256];
-    __shared__ __align__(16) float sw[kRgExp][256];
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
+    const int n = pred ? 16 : 0;   // zero-fill when out of range
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// dynamic shared memory: two stages of (32 token rows x 256 bf16, 16 router rows x 256 fp32)
+constexpr int kRgStage = kRgTok * 256 * 2 + kRgExp * 256 * 4;
+
+__global__ void __launch_bounds__(256, 2) router_gemm_kernel(const uint16_t *x, int T, int D, int E, const float *Wr,
+                                                             const float *bias, float *logits, float *tap_logits)
+{
+    extern __shared__ __align__(16) uint8_t rg_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * kRgTok, e0 = blockIdx.y * kRgExp;
     const int wt = (warp >> 1) * 8, we = (warp & 1) * 8;
-    float acc[64];
-#pragma unroll
-    for (int o = 0; o < 64; o++) acc[o] = 0.0f;
-    for (int i = 0; i < D / 256; i++) {
-        __syncthreads();
-        // stage token rows (32 x 256 bf16 = 1024 x 16 B) and router rows (16 x 256 fp32 = 1024 x 16 B)
+    const int NI = D / 256;
+    auto stage = [&](int i, int buf) {
+        uint16_t *sx = (uint16_t *)(rg_smem + buf * kRgStage);
+        float *sw = (float *)(rg_smem + buf * kRgStage + kRgTok * 256 * 2);
         for (int q = threadIdx.x; q < kRgTok * 32; q += 256) {
             const int tt = q >> 5, c = q & 31;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (t0 + tt < T) v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * D + 256 * i) + c);
-            reinterpret_cast<uint4 *>(&sx[tt][0])[c] = v;
+            const bool ok = t0 + tt < T;
+            cp_async16(sx + tt * 256 + c * 8, x + (size_t)(ok ? t0 + tt : 0) * D + 256 * i + c * 8, ok);
         }
         for (int q = threadIdx.x; q < kRgExp * 64; q += 256) {
             const int ee = q >> 6, c = q & 63;
-            reinterpret_cast<float4 *>(&sw[ee][0])[c] =
-                __ldg(reinterpret_cast<const float4 *>(Wr + (size_t)(e0 + ee) * D + 256 * i) + c);
+            cp_async16(sw + ee * 256 + c * 4, Wr + (size_t)(e0 + ee) * D + 256 * i + c * 4, true);
+        }
+        cp_async_commit();
+    };
+    float acc[64];
+#pragma unroll
+    for (int o = 0; o < 64; o++) acc[o] = 0.0f;
+    stage(0, 0);
+    for (int i = 0; i < NI; i++) {
+        if (i + 1 < NI) {
+            stage(i + 1, (i + 1) & 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
         __syncthreads();
-        float wv[8][8];
+        const uint16_t *sx = (const uint16_t *)(rg_smem + (i & 1) * kRgStage);
+        const float *sw = (const float *)(rg_smem + (i & 1) * kRgStage + kRgTok * 256 * 2);
 #pragma unroll
-        for (int b = 0; b < 8; b++) {
-            const float4 w0 = *reinterpret_cast<const float4 *>(&sw[we + b][8 * lane]);
-            const float4 w1 = *reinterpret_cast<const float4 *>(&sw[we + b][8 * lane + 4]);
-            wv[b][0] = w0.x; wv[b][1] = w0.y; wv[b][2] = w0.z; wv[b][3] = w0.w;
-            wv[b][4] = w1.x; wv[b][5] = w1.y; wv[b][6] = w1.z; wv[b][7] = w1.w;
+        for (int h = 0; h < 2; h++) {   // lane's 8 elements of the chunk, 4 at a time (m = 4h .. 4h+3)
+            float wv[8][4];
+#pragma unroll
+            for (int b = 0; b < 8; b++) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(sw + (we + b) * 256 + 8 * lane + 4 * h);
+                wv[b][0] = w4.x; wv[b][1] = w4.y; wv[b][2] = w4.z; wv[b][3] = w4.w;
+            }
+#pragma unroll
+            for (int aa = 0; aa < 8; aa++) {
+                const uint2 xv = *reinterpret_cast<const uint2 *>(sx + (wt + aa) * 256 + 8 * lane + 4 * h);
+                const float xf[4] = {bf16_bits_to_f32(xv.x & 0xffffu), bf16_bits_to_f32(xv.x >> 16),
+                                     bf16_bits_to_f32(xv.y & 0xffffu), bf16_bits_to_f32(xv.y >> 16)};
+#pragma unroll
+                for (int b = 0; b < 8; b++)
+#pragma unroll
+                    for (int m = 0; m < 4; m++) acc[aa * 8 + b] = __fmaf_rn(xf[m], wv[b][m], acc[aa * 8 + b]);
+            }
         }
-#pragma unroll
-        for (int a = 0; a < 8; a++) {
-            const uint4 xv = *reinterpret_cast<const uint4 *>(&sx[wt + a][8 * lane]);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-            float xf[8];
-#pragma unroll
-            for (int m = 0; m < 8; m++) xf[m] = bf16_bits_to_f32((m & 1) ? (xw[m >> 1] >> 16) : (xw[m >> 1] & 0xffffu));
-#pragma unroll
-            for (int b = 0; b < 8; b++)
-#pragma unroll
-                for (int m = 0; m < 8; m++) acc[a * 8 + b] = __fmaf_rn(xf[m], wv[b][m], acc[a * 8 + b]);
-        }
+        __syncthreads();
     }
     tree_level<64>(acc, 16, lane & 16);
     tree_level<32>(acc, 8, lane & 8);

@@ -72,8 +72,9 @@ struct TcSmem {
     static constexpr int kBBytes = kTcMaxN * kTcBK;
     static constexpr int kStage = TcCfg<MODE>::kABytes + kBBytes + TcCfg<MODE>::kCodeBytes;
     static constexpr int kA = 0, kB = TcCfg<MODE>::kABytes, kCodes = kB + kBBytes;
-    static constexpr int kBars = TcCfg<MODE>::kStages * kStage;
-    static constexpr int kTotal = kBars + 1024 + 1024;  // barriers etc. + alignment slack
+    static constexpr int kBars = TcCfg<MODE>::kStages * kStage;   // barriers, TMEM holder, abort word: 256 B
+    static constexpr int kMeta = kBars + 256;                       // epilogue column metadata [2][2][128]
+    static constexpr int kTotal = kMeta + 2 * 2 * kTcMaxN * 4;
     static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
 };
 
@@ -84,6 +85,7 @@ struct TcArgs {
     const uint8_t *codes;    // tensor-core layout
     const int *perm;         // position -> slot
     const float *sx, *sh;
+    const float *pscale;     // mode 0: s_x of each position's token
     const float *alpha0, *alpha1;  // mode 0: gate, up; mode 1: down, unused
     float *out;              // mode 0: h [S][F]; mode 1: yE [S][D]
     int *tap0, *tap1;        // mode 0: acc_gate, acc_up; mode 1: acc_down
@@ -112,10 +114,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -158,6 +160,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
     asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
                  ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
                  : "memory");
+}
+__device__ __forceinline__ void cp_async4_tc(void *smem, const void *gmem)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(d), "l"(gmem) : "memory");
 }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_barrier_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
@@ -239,8 +246,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     using Cfg = TcCfg<MODE>;
     using L = TcSmem<MODE>;
     constexpr int S = Cfg::kStages;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
+    if (smem_addr(smem) & 1023u) {   // the 128-byte-swizzled tiles need 1024-byte alignment
+        if (threadIdx.x == 0) set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
+        return;
+    }
+    int *meta_slot = (int *)(smem + L::kMeta);                      // [2][kTcMaxN]
+    float *meta_scale = (float *)(smem + L::kMeta + 2 * kTcMaxN * 4);
     uint64_t *bars = (uint64_t *)(smem + L::kBars);
     // bars: codes_full[S], full[S], empty[S], acc_full[2], acc_empty[2], drain
     uint32_t *tmem_holder = (uint32_t *)(bars + 3 * S + 5);
@@ -279,8 +292,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
             uint32_t it = 0;
             bool ok = true;
+            int4 npc = blockIdx.x < n_tiles ? a.pieces[blockIdx.x / R] : make_int4(0, 0, 0, 0);
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                const int4 pc = a.pieces[tile / R];
+                const int4 pc = npc;   // fetched one tile ahead
+                if (tile + (int)gridDim.x < n_tiles) npc = a.pieces[(tile + gridDim.x) / R];
                 const int rt = tile % R;
                 const uint8_t *src = a.codes + ((size_t)pc.x * R + rt) * KS * Cfg::kCodeBytes;
                 for (int ks = 0; ks < KS; ks++, it++) {
@@ -310,8 +325,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         if (lane == 0) {
             uint32_t it = 0, tc = 0;
             bool ok = true;
+            int4 npc = blockIdx.x < n_tiles ? a.pieces[blockIdx.x / R] : make_int4(0, 0, 0, 0);
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, tc++) {
-                const int4 pc = a.pieces[tile / R];
+                const int4 pc = npc;   // fetched one tile ahead
+                if (tile + (int)gridDim.x < n_tiles) npc = a.pieces[(tile + gridDim.x) / R];
                 const int npad = (pc.z + 15) & ~15;
                 const uint32_t idesc = idesc_i8(npad);
                 const uint32_t ab = tc & 1, dt = tmem + 256 * ab;
@@ -350,20 +367,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue: TMEM -> registers -> global
+        // The next tile's per-column metadata (slot ids and token / slot
+        // scales, both contiguous per piece) is copied with cp.async and its
+        // row scales loaded into registers while this tile is processed, so
+        // no global latency sits between the MMAs and the stores.
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+        const int ldo = MODE == 0 ? a.F : a.D;
+        const float *scale_src = MODE == 0 ? a.pscale : a.sh;
+        auto fetch = [&](int tile, int buf, const int4 &pc, float &al0, float &al1) {
+            const int row = (tile % R) * 128 + r;
+            al0 = a.alpha0[(size_t)pc.x * ldo + row];
+            al1 = MODE == 0 ? a.alpha1[(size_t)pc.x * ldo + row] : 0.0f;
+            if (r < pc.z) {   // one slot id and one scale per column (4-byte copies: any alignment of p0)
+                cp_async4_tc(meta_slot + buf * kTcMaxN + r, a.perm + pc.y + r);
+                cp_async4_tc(meta_scale + buf * kTcMaxN + r, scale_src + pc.y + r);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
         uint32_t tc = 0;
+        bool dead = false;   // after a failed wait: keep the loop (and its named barrier) in step, do nothing
+        int4 npc = make_int4(0, 0, 0, 0), nnpc = make_int4(0, 0, 0, 0);
+        float nal0 = 0.0f, nal1 = 0.0f;
+        if (blockIdx.x < n_tiles) {
+            npc = a.pieces[blockIdx.x / R];
+            fetch(blockIdx.x, 0, npc, nal0, nal1);
+        }
+        if (blockIdx.x + (int)gridDim.x < n_tiles) nnpc = a.pieces[(blockIdx.x + gridDim.x) / R];
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, tc++) {
-            const int4 pc = a.pieces[tile / R];
+            const int4 pc = npc;
+            const float al0 = nal0, al1 = nal1;
             const int rt = tile % R;
             const int row = rt * 128 + r;
             const uint32_t ab = tc & 1, tb = tbase + 256 * ab;
-            if (!mbar_wait(b_acc_full + 8 * ab, (tc >> 1) & 1, abort, a.flag)) break;
+            const int p0 = pc.y, n = pc.z;
+            const int *ms = meta_slot + ab * kTcMaxN;
+            const float *mf = meta_scale + ab * kTcMaxN;
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            asm volatile("bar.sync 2, 128;" ::: "memory");   // this tile's metadata is in place
+            if (tile + (int)gridDim.x < n_tiles) {
+                npc = nnpc;
+                fetch(tile + gridDim.x, ab ^ 1, npc, nal0, nal1);
+                if (tile + 2 * (int)gridDim.x < n_tiles) nnpc = a.pieces[(tile + 2 * gridDim.x) / R];
+            }
+            if (!dead && !mbar_wait(b_acc_full + 8 * ab, (tc >> 1) & 1, abort, a.flag)) dead = true;
+            if (dead) continue;
             tc_fence_after();
-            const int e = pc.x, p0 = pc.y, n = pc.z;
             if (MODE == 0) {
-                const float ag = a.alpha0[(size_t)e * a.F + row], au = a.alpha1[(size_t)e * a.F + row];
                 for (int c0 = 0; c0 < n; c0 += 32) {
                     int g[32], u[32];
                     tmem_ld32(tb + c0, g);
@@ -374,11 +425,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         const int col = c0 + j;
                         if (col < n) {
                             const int p = p0 + col;
-                            const int slot = __ldg(a.perm + p);
-                            const float sxt = __ldg(a.sx + slot / a.K);
+                            const int slot = ms[col];
+                            const float sxt = mf[col];
                             const int gi = g[j] >> 6, ui = u[j] >> 6;
-                            const float gv = __fmul_rn((float)gi, __fmul_rn(ag, sxt));
-                            const float uv = __fmul_rn((float)ui, __fmul_rn(au, sxt));
+                            const float gv = __fmul_rn((float)gi, __fmul_rn(al0, sxt));
+                            const float uv = __fmul_rn((float)ui, __fmul_rn(al1, sxt));
                             a.out[(size_t)p * a.F + row] = swiglu(gv, uv);
                             if (a.tap0) a.tap0[(size_t)slot * a.F + row] = gi;
                             if (a.tap1) a.tap1[(size_t)slot * a.F + row] = ui;
@@ -386,19 +437,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     }
                 }
             } else {
-                const float ad = a.alpha0[(size_t)e * a.D + row];
                 for (int c0 = 0; c0 < n; c0 += 32) {
-                    int d[32];
-                    tmem_ld32(tb + c0, d);
+                    int dd[32];
+                    tmem_ld32(tb + c0, dd);
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; j++) {
                         const int col = c0 + j;
                         if (col < n) {
                             const int p = p0 + col;
-                            const int di = d[j] >> 6;
-                            a.out[(size_t)p * a.D + row] = __fmul_rn((float)di, __fmul_rn(ad, __ldg(a.sh + p)));
-                            if (a.tap0) a.tap0[(size_t)__ldg(a.perm + p) * a.D + row] = di;
+                            const int di = dd[j] >> 6;
+                            a.out[(size_t)p * a.D + row] = __fmul_rn((float)di, __fmul_rn(al0, mf[col]));
+                            if (a.tap0) a.tap0[(size_t)ms[col] * a.D + row] = di;
                         }
                     }
                 }
@@ -451,12 +501,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 // slot-ordered copy of the int8 activation rows: xperm[p] = q_x[perm[p] / K]
 // (one warp per position)
 // ---------------------------------------------------------------------------
-__global__ void gather_rows_kernel(const int8_t *qx, const int *perm, int K, int D, int S, int8_t *xperm)
+__global__ void gather_rows_kernel(const int8_t *qx, const float *sx, const int *perm, int K, int D, int S,
+                                   int8_t *xperm, float *pscale)
 {
     const int lane = threadIdx.x & 31;
     const int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (p >= S) return;
-    const uint4 *src = reinterpret_cast<const uint4 *>(qx + (size_t)(perm[p] / K) * D);
+    const int t = perm[p] / K;
+    if (lane == 0) pscale[p] = sx[t];
+    const uint4 *src = reinterpret_cast<const uint4 *>(qx + (size_t)t * D);
     uint4 *dst = reinterpret_cast<uint4 *>(xperm + (size_t)p * D);
     for (int i = lane; i < D / 16; i += 32) dst[i] = __ldg(src + i);
 }

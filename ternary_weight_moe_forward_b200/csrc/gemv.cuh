@@ -94,54 +94,62 @@ __device__ __forceinline__ void chunk_tokens(const uint4 wv, const int8_t *xs, i
     }
 }
 
-// Same as chunk_tokens with four partial sums per token (one per byte plane),
-// so the dp4a chains of a single token run four wide; acc4[j][k] are summed
-// by the caller (int32, exact in any order).
-__device__ __forceinline__ void chunk_tokens4(const uint4 wv, const int8_t *xs, int ld, int off, int nb,
-                                              int (&acc4)[kGemvTokens][4])
+// Padded token count of a decode batch: the dot kernels below exist for 1, 2
+// and 4 tokens (8 = two passes of 4); rows nb..nbp-1 of the batch hold zeros.
+__device__ __forceinline__ int dec_pad_tokens(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
+
+// Sum over chunks [c0, c0+nch) of this lane's row against NB token rows (16-byte
+// units x[j*ld16 + 4c + w]).  Byte plane k is taken as w & (0x03030303 << 2k),
+// i.e. 4^k times the offset codes, one logic op per plane, and gets its own
+// accumulator; acc_k is then an exact multiple of 4^k and the row total is
+// acc_0 + acc_1/4 + acc_2/16 + acc_3/64 (int32, exact).  Token j's total goes
+// to out[32 j].
+template <int NB>
+__device__ __forceinline__ void dot_rows(const uint4 *wl, const uint4 *x, int ld16, int c0, int nch, int *out)
 {
-    const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+    int acc[NB][4];
 #pragma unroll
-    for (int j = 0; j < kGemvTokens; j++) {
-        if (j < nb) {
-            const uint4 *x4 = reinterpret_cast<const uint4 *>(xs + (size_t)j * ld + off);
+    for (int j = 0; j < NB; j++)
+#pragma unroll
+        for (int k = 0; k < 4; k++) acc[j][k] = 0;
+    const uint4 *wr = wl + 32 * c0;
+    const uint4 *xr = x + 4 * c0;
+#pragma unroll 1
+    for (int u = 0; u < nch; u++) {
+        const uint4 wv = wr[32 * u];
+        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t pw[16];
+#pragma unroll
+        for (int w = 0; w < 4; w++)
+#pragma unroll
+            for (int k = 0; k < 4; k++) pw[4 * w + k] = w4[w] & (0x03030303u << (2 * k));
+#pragma unroll
+        for (int j = 0; j < NB; j++) {
 #pragma unroll
             for (int w = 0; w < 4; w++) {
-                const uint4 xv = x4[w];
-                acc4[j][0] = dp4a_us(plane(w4[w], 0), xv.x, acc4[j][0]);
-                acc4[j][1] = dp4a_us(plane(w4[w], 1), xv.y, acc4[j][1]);
-                acc4[j][2] = dp4a_us(plane(w4[w], 2), xv.z, acc4[j][2]);
-                acc4[j][3] = dp4a_us(plane(w4[w], 3), xv.w, acc4[j][3]);
+                const uint4 xv = xr[j * ld16 + 4 * u + w];
+                acc[j][0] = dp4a_us(pw[4 * w + 0], xv.x, acc[j][0]);
+                acc[j][1] = dp4a_us(pw[4 * w + 1], xv.y, acc[j][1]);
+                acc[j][2] = dp4a_us(pw[4 * w + 2], xv.z, acc[j][2]);
+                acc[j][3] = dp4a_us(pw[4 * w + 3], xv.w, acc[j][3]);
             }
         }
     }
+#pragma unroll
+    for (int j = 0; j < NB; j++) out[32 * j] = acc[j][0] + (acc[j][1] >> 2) + (acc[j][2] >> 4) + (acc[j][3] >> 6);
 }
 
-// acc[j][0..1] += the 64 values of one chunk (this lane's row) against token j's
-// 64 activations (16-byte rows x4[j*ld16 .. +3]), j < nb.  The byte planes are
-// taken once per chunk and serve every token; two partial sums per token keep
-// the dp4a chains short (int32, exact in any order).
-__device__ __forceinline__ void chunk_dot(const uint4 wv, const uint4 *x4, int ld16, int nb,
-                                          int (&acc)[kGemvTokens][2])
+__device__ __forceinline__ void dot_rows_any(int nbp, const uint4 *wl, const uint4 *x, int ld16, int c0, int nch,
+                                             int *out)
 {
-    const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
-    uint32_t pw[16];
-#pragma unroll
-    for (int w = 0; w < 4; w++)
-#pragma unroll
-        for (int k = 0; k < 4; k++) pw[4 * w + k] = plane(w4[w], k);
-#pragma unroll
-    for (int j = 0; j < kGemvTokens; j++) {
-        if (j < nb) {
-#pragma unroll
-            for (int w = 0; w < 4; w++) {
-                const uint4 xv = x4[j * ld16 + w];
-                acc[j][w & 1] = dp4a_us(pw[4 * w + 0], xv.x, acc[j][w & 1]);
-                acc[j][w & 1] = dp4a_us(pw[4 * w + 1], xv.y, acc[j][w & 1]);
-                acc[j][w & 1] = dp4a_us(pw[4 * w + 2], xv.z, acc[j][w & 1]);
-                acc[j][w & 1] = dp4a_us(pw[4 * w + 3], xv.w, acc[j][w & 1]);
-            }
-        }
+    switch (nbp) {
+    case 1: dot_rows<1>(wl, x, ld16, c0, nch, out); break;
+    case 2: dot_rows<2>(wl, x, ld16, c0, nch, out); break;
+    case 4: dot_rows<4>(wl, x, ld16, c0, nch, out); break;
+    default:   // two passes of four tokens keep the accumulators in registers
+        dot_rows<4>(wl, x, ld16, c0, nch, out);
+        dot_rows<4>(wl, x + 4 * ld16, ld16, c0, nch, out + 4 * 32);
+        break;
     }
 }
 
@@ -365,8 +373,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, MAPLE_GEMV_MINB) down_gemv_ke
 // CTA first builds the permutation of all T*K slots for itself from the
 // router's top-k (in shared memory), so no routing step needs a grid-wide
 // hand-off.  Work items: gate/up items (active expert, 32 gate + 32 up rows)
-// then down items (active expert, 128 output channels); every CTA takes an
-// equal contiguous range of each kind.  Warp roles:
+// then down items (active expert, 128 output channels); every CTA takes a
+// contiguous range of each kind holding an equal share of its estimated cost
+// (the cost of an item grows with its expert's token count).  Warp roles:
 //   warp 0      streams the 2-bit codes and row scales of its items, in order,
 //               with bulk copies into a ring of weight slots;
 //   warps 1, 2  stage the activations of compute group 0 / 1 (double
@@ -412,6 +421,7 @@ struct DecodeArgs {
     int wslot_bytes;      // codes + scales of one item
     int aslot_bytes;      // activation rows of one batch
     int nw;               // weight ring slots (2..kDecWSlots)
+    const int8_t *zrow;   // D zero bytes (padding rows of a gate/up batch)
     const int *topk_idx;  // [T][K] the router's choices (distinct per token)
     const float *topk_w;  // [T][K] their softmax weights
     // outputs of the permutation, written by CTA 0 (may be null)
@@ -431,7 +441,8 @@ __host__ __device__ inline int dec_aslot_bytes(int D, int F)
 // routing tables every CTA builds for itself in shared memory
 __host__ __device__ inline size_t dec_table_bytes(int T, int K, int E)
 {
-    return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E;
+    return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E +
+           (size_t)2 * (E + 1) * 4;
 }
 __host__ __device__ inline size_t dec_group_scratch_bytes(int F)
 {
@@ -481,6 +492,35 @@ __device__ __forceinline__ void dec_bulk(void *dst, const void *src, uint32_t by
                      "l"((const uint8_t *)src + off), "r"(n), "r"(bar)
                      : "memory");
     }
+}
+
+// Relative cost of one work item of an expert with c tokens (kind 0 gate/up, 1
+// down): per batch of up to 8 tokens a fixed part (waits, barriers, epilogue)
+// plus a part per padded token (the dot), in units of about 0.1 us measured on
+// the decode-shape layer.  Only the split of the items over CTAs depends on it.
+__device__ __forceinline__ int dec_item_cost(int c, int kind)
+{
+    int cost = 0;
+    for (int b0 = 0; b0 < c; b0 += kGemvTokens) {
+        const int nbp = dec_pad_tokens(min(kGemvTokens, c - b0));
+        cost += kind == 0 ? 23 + 5 * nbp : 18 + 7 * nbp;
+    }
+    return cost;
+}
+
+// First item whose cumulative cost start is >= target; pref[ai] is the cost of
+// the items of active experts before ai (per_exp items of equal cost each).
+__device__ __forceinline__ int dec_item_at(const int *pref, int n_active, int per_exp, int64_t target)
+{
+    if (target >= pref[n_active]) return n_active * per_exp;
+    int lo = 0, hi = n_active - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] <= target) lo = mid;
+        else hi = mid - 1;
+    }
+    const int w = (pref[lo + 1] - pref[lo]) / per_exp;
+    return lo * per_exp + (int)((target - pref[lo] + w - 1) / w);
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeArgs d)
@@ -605,9 +645,46 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
 
     const int n_active = t_misc[0];
     const int pairs = a.F / 32, blocks = a.D / 128;
-    const int n_g = n_active * pairs, n_d = n_active * blocks;
-    const int g0 = (int)((int64_t)n_g * blockIdx.x / gridDim.x), g1 = (int)((int64_t)n_g * (blockIdx.x + 1) / gridDim.x);
-    const int d0 = (int)((int64_t)n_d * blockIdx.x / gridDim.x), d1 = (int)((int64_t)n_d * (blockIdx.x + 1) / gridDim.x);
+    // split each kind of item over the CTAs in equal shares of estimated cost
+    int *t_pg = (int *)(tmask + E), *t_pd = t_pg + E + 1;
+    if (warp == 0) {
+        const int per = (n_active + 31) / 32, a0 = lane * per;
+        int sg = 0, sd = 0;
+        for (int i = 0; i < per; i++)
+            if (a0 + i < n_active) {
+                const int c = t_cnt[t_act[a0 + i]];
+                sg += pairs * dec_item_cost(c, 0);
+                sd += blocks * dec_item_cost(c, 1);
+            }
+        int cg = sg, cd = sd;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(FULL, cg, o), w = __shfl_up_sync(FULL, cd, o);
+            if (lane >= o) {
+                cg += v;
+                cd += w;
+            }
+        }
+        int og = cg - sg, od = cd - sd;
+        for (int i = 0; i < per; i++)
+            if (a0 + i < n_active) {
+                const int c = t_cnt[t_act[a0 + i]];
+                t_pg[a0 + i] = og;
+                t_pd[a0 + i] = od;
+                og += pairs * dec_item_cost(c, 0);
+                od += blocks * dec_item_cost(c, 1);
+            }
+        if (lane == 31) {
+            t_pg[n_active] = cg;
+            t_pd[n_active] = cd;
+        }
+    }
+    __syncthreads();
+    const int64_t WG = t_pg[n_active], WD = t_pd[n_active];
+    const int g0 = dec_item_at(t_pg, n_active, pairs, WG * blockIdx.x / gridDim.x);
+    const int g1 = dec_item_at(t_pg, n_active, pairs, WG * (blockIdx.x + 1) / gridDim.x);
+    const int d0 = dec_item_at(t_pd, n_active, blocks, WD * blockIdx.x / gridDim.x);
+    const int d1 = dec_item_at(t_pd, n_active, blocks, WD * (blockIdx.x + 1) / gridDim.x);
     const int nG = g1 - g0, n_items = nG + (d1 - d0);
     const int Cg = a.D / 64, Cd = a.F / 64;
     // item i of this CTA -> kind (0 gate/up, 1 down), active index, sub-block
@@ -715,9 +792,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                             m->s[j] = a.sx[t];
                             m->sum[j] = a.sumx[t];
                         }
-                        dec_expect(bar, (uint32_t)(nb * a.D));
-                        for (int j = 0; j < nb; j++)
-                            dec_bulk(dst + (size_t)j * a.D, a.qx + (size_t)(m->slot[j] / a.K) * a.D, (uint32_t)a.D, bar);
+                        const int nbp = dec_pad_tokens(nb);
+                        dec_expect(bar, (uint32_t)(nbp * a.D));
+                        for (int j = 0; j < nbp; j++)
+                            dec_bulk(dst + (size_t)j * a.D,
+                                     j < nb ? a.qx + (size_t)(m->slot[j] / a.K) * a.D : d.zrow, (uint32_t)a.D, bar);
                     } else {
                         for (int j = 0; j < nb; j++) m->slot[j] = a.perm[base + b0 + j];
                         dec_expect(bar, (uint32_t)(nb * a.F * 4));
@@ -830,21 +909,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
             const DecActMeta &am = ameta[2 * g + buf];
             const uint8_t *ab = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
             const int nb = am.nb;
-            int acc2[kGemvTokens][2];
-#pragma unroll
-            for (int j = 0; j < kGemvTokens; j++) acc2[j][0] = acc2[j][1] = 0;
+            const int nbp = dec_pad_tokens(nb);
+            int *red_w = red + gw * kGemvTokens * 32 + lane;
             if (wm.kind == 0) {
                 // ---- gate/up: warp gw = row group gw/4 (of the pair), K quarter gw%4
                 const int rg = gw >> 2, kq = gw & 3, quarter = Cg / 4;
                 const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)rg * Cg * 512) + lane;
-                const uint4 *xl = reinterpret_cast<const uint4 *>(ab);
-#pragma unroll 1
-                for (int u = 0; u < quarter; u++) {
-                    const int c = kq * quarter + u;
-                    chunk_dot(wl[32 * c], xl + 4 * c, a.D / 16, nb, acc2);
-                }
-#pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) red[(gw * kGemvTokens + j) * 32 + lane] = acc2[j][0] + acc2[j][1];
+                dot_rows_any(nbp, wl, reinterpret_cast<const uint4 *>(ab), a.D / 16, kq * quarter, quarter, red_w);
                 gsync();
                 if (kq == 0) {
                     const bool is_up = lane >= 16;
@@ -866,6 +937,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                 // ---- down: requantise the batch's h rows (one slot per warp), then warp gw =
                 //      channel group 4*blk + gw/2, K half gw%2
                 const float *hr = (const float *)ab;
+                for (int j = nb + gw; j < nbp; j += kDecGroupWarps)
+                    for (int q = lane; q < a.F / 16; q += 32)
+                        reinterpret_cast<uint4 *>(qh + (size_t)j * a.F)[q] = make_uint4(0u, 0u, 0u, 0u);
                 for (int j = gw; j < nb; j += kDecGroupWarps) {
                     const float4 *h4 = reinterpret_cast<const float4 *>(hr + (size_t)j * a.F);
                     float amax = 0.0f;
@@ -902,14 +976,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                 gsync();
                 const int cgl = gw >> 1, kh = gw & 1, half = Cd / 2;
                 const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)cgl * Cd * 512) + lane;
-                const uint4 *xl = reinterpret_cast<const uint4 *>(qh);
-#pragma unroll 1
-                for (int u = 0; u < half; u++) {
-                    const int c = kh * half + u;
-                    chunk_dot(wl[32 * c], xl + 4 * c, a.F / 16, nb, acc2);
-                }
-#pragma unroll
-                for (int j = 0; j < kGemvTokens; j++) red[(gw * kGemvTokens + j) * 32 + lane] = acc2[j][0] + acc2[j][1];
+                dot_rows_any(nbp, wl, reinterpret_cast<const uint4 *>(qh), a.F / 16, kh * half, half, red_w);
                 gsync();
                 if (kh == 0) {
                     const int cg = (wm.sub * 4 + cgl) * 32 + lane;

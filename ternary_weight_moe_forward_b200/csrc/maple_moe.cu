@@ -50,6 +50,7 @@ struct maple_moe_s {
     float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
     // workspace
     int8_t *qx;
+    const int8_t *zrow;   // zeros, never written after create
     float *sx;
     int *sumx;
     float *logits;
@@ -280,6 +281,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4), o_ec = ar.take(E * 4);
     size_t o_cc = ar.take(Tm * (D / 32) * 4), o_rdy = ar.take(E * 4);
     size_t o_xn = ar.take(Tm * D * 2);
+    size_t o_zr = ar.take(D > F * 4 ? D : F * 4);   // a row of zeros (padding rows of the decode kernel)
 
     if (cudaMalloc(&h->base, ar.size) != cudaSuccess) {
         cudaGetLastError();
@@ -338,6 +340,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
         h->dec_persistent = decode_smem_bytes(h->D, h->F, 1, h->K, h->E, 2) <= (size_t)optin;
     }
     h->xn = (uint16_t *)(b + o_xn);
+    h->zrow = (const int8_t *)(b + o_zr);
 
     cudaStream_t st = (cudaStream_t)stream;
     // the whole workspace starts at zero: counters must, and every index array
@@ -550,6 +553,7 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         d.wslot_bytes = dec_wslot_bytes(h->D, h->F);
         d.aslot_bytes = dec_aslot_bytes(h->D, h->F);
         d.nw = nw;
+        d.zrow = h->zrow;
         d.topk_idx = h->topk_idx;
         d.topk_w = h->topk_w;
         if (taps) {

@@ -124,6 +124,37 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms * 1e-3)
 
 
+# ---------------------------------------------------------------------------- measured traffic
+PROFILE_T64 = os.path.join(ROOT, "profiles", "decode_experts_kernel__decode_T64.md")
+
+
+def csrc_digest() -> str:
+    """sha256 over the CUDA sources (file names and contents, sorted)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "ternary_weight_moe_forward_b200", "csrc", "*"))):
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """DRAM bytes (read + write) of one T=64 launch of decode_experts_kernel from
+    the committed ncu summary, or None when the sources changed since."""
+    try:
+        with open(PROFILE_T64) as f:
+            txt = f.read()
+        fields = dict(line.split(": ", 1) for line in txt.splitlines()
+                      if line.startswith(("csrc_sha256: ", "traffic_bytes: ")))
+        if fields.get("csrc_sha256", "").strip() != csrc_digest():
+            return None
+        return int(fields["traffic_bytes"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ---------------------------------------------------------------------------- GPU arm
 def decode_bytes(n_active: int, T: int) -> int:
     """Algorithmic HBM bytes of one decode forward: packed codes and scales of
@@ -297,7 +328,9 @@ def run_gpu(args, rank: int, world: int):
                   for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
         "roofline": {"kernel": "decode_experts_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": None},
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": measured_traffic(), "traffic_launch": "T=64 (ncu, profiles/)",
+                     "algorithmic_bytes_T64": experts_bytes(n_active[64], 64)},
         "e2e": {"value": whole_job_rate(tokens_rank, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(T * shape.d_model * 2 for T in DECODE_T),
                 "d2h_bytes_per_step": sum(T * shape.d_model * 4 for T in DECODE_T)},

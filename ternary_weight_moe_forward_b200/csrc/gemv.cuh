@@ -94,65 +94,6 @@ __device__ __forceinline__ void chunk_tokens(const uint4 wv, const int8_t *xs, i
     }
 }
 
-// Padded token count of a decode batch: the dot kernels below exist for 1, 2
-// and 4 tokens (8 = two passes of 4); rows nb..nbp-1 of the batch hold zeros.
-__device__ __forceinline__ int dec_pad_tokens(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
-
-// Sum over chunks [c0, c0+nch) of this lane's row against NB token rows (16-byte
-// units x[j*ld16 + 4c + w]).  Byte plane k is taken as w & (0x03030303 << 2k),
-// i.e. 4^k times the offset codes, one logic op per plane, and gets its own
-// accumulator; acc_k is then an exact multiple of 4^k and the row total is
-// acc_0 + acc_1/4 + acc_2/16 + acc_3/64 (int32, exact).  Token j's total goes
-// to out[32 j].
-template <int NB>
-__device__ __forceinline__ void dot_rows(const uint4 *wl, const uint4 *x, int ld16, int c0, int nch, int *out)
-{
-    int acc[NB][4];
-#pragma unroll
-    for (int j = 0; j < NB; j++)
-#pragma unroll
-        for (int k = 0; k < 4; k++) acc[j][k] = 0;
-    const uint4 *wr = wl + 32 * c0;
-    const uint4 *xr = x + 4 * c0;
-#pragma unroll 1
-    for (int u = 0; u < nch; u++) {
-        const uint4 wv = wr[32 * u];
-        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
-        uint32_t pw[16];
-#pragma unroll
-        for (int w = 0; w < 4; w++)
-#pragma unroll
-            for (int k = 0; k < 4; k++) pw[4 * w + k] = w4[w] & (0x03030303u << (2 * k));
-#pragma unroll
-        for (int j = 0; j < NB; j++) {
-#pragma unroll
-            for (int w = 0; w < 4; w++) {
-                const uint4 xv = xr[j * ld16 + 4 * u + w];
-                acc[j][0] = dp4a_us(pw[4 * w + 0], xv.x, acc[j][0]);
-                acc[j][1] = dp4a_us(pw[4 * w + 1], xv.y, acc[j][1]);
-                acc[j][2] = dp4a_us(pw[4 * w + 2], xv.z, acc[j][2]);
-                acc[j][3] = dp4a_us(pw[4 * w + 3], xv.w, acc[j][3]);
-            }
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < NB; j++) out[32 * j] = acc[j][0] + (acc[j][1] >> 2) + (acc[j][2] >> 4) + (acc[j][3] >> 6);
-}
-
-__device__ __forceinline__ void dot_rows_any(int nbp, const uint4 *wl, const uint4 *x, int ld16, int c0, int nch,
-                                             int *out)
-{
-    switch (nbp) {
-    case 1: dot_rows<1>(wl, x, ld16, c0, nch, out); break;
-    case 2: dot_rows<2>(wl, x, ld16, c0, nch, out); break;
-    case 4: dot_rows<4>(wl, x, ld16, c0, nch, out); break;
-    default:   // two passes of four tokens keep the accumulators in registers
-        dot_rows<4>(wl, x, ld16, c0, nch, out);
-        dot_rows<4>(wl, x + 4 * ld16, ld16, c0, nch, out + 4 * 32);
-        break;
-    }
-}
-
 // requantise every slot of an expert (positions [base, base+cnt)) from h; the
 // first nw warps of the CTA take one slot each
 __device__ void requant_slots_warps(const GemvArgs &a, int base, int cnt, int nw)
@@ -367,48 +308,48 @@ __global__ void __launch_bounds__(kGemvWarps * 32, MAPLE_GEMV_MINB) down_gemv_ke
 }
 
 // ---------------------------------------------------------------------------
-// Persistent weight-streaming kernel for the whole expert stage (decode).
+// Persistent expert-stage kernel for decode batches (T <= 64).
 //
 // Grid = one CTA per SM, launched cooperatively (all CTAs resident).  Every
 // CTA first builds the permutation of all T*K slots for itself from the
 // router's top-k (in shared memory), so no routing step needs a grid-wide
-// hand-off.  Work items: gate/up items (active expert, 32 gate + 32 up rows)
-// then down items (active expert, 128 output channels); every CTA takes a
-// contiguous range of each kind holding an equal share of its estimated cost
-// (the cost of an item grows with its expert's token count).  Warp roles:
-//   warp 0      streams the 2-bit codes and row scales of its items, in order,
-//               with bulk copies into a ring of weight slots;
-//   warps 1, 2  stage the activations of compute group 0 / 1 (double
-//               buffered): for gate/up the int8 rows of the item's tokens, for
-//               down the fp32 SwiGLU rows h of the item's slots once every
-//               gate/up item of that expert has finished;
-//   warps 3, 4  publish the results of group 0 / 1: make a finished gate/up
+// hand-off.  Work items: gate/up items (active expert, 8 groups of 16 gate +
+// 16 up rows) then down items (active expert, 8 groups of 32 output
+// channels); every CTA takes a contiguous range of each kind holding an equal
+// share of its estimated cost (an item's cost grows with its token count).
+// Warp roles:
+//   warps 0, 1  stage the activations of compute group 0 / 1 (double
+//               buffered): for gate/up the int8 rows of the item's tokens; for
+//               down, once every gate/up item of the expert has finished, the
+//               fp32 SwiGLU rows h of the item's slots, which the warp then
+//               requantises (per-slot absmax int8) into the buffer;
+//   warps 2, 3  publish the results of group 0 / 1: make a finished gate/up
 //               item visible (GPU fence, arrival counter of its expert), and for
-//               a down item count each token's arrival on its channel block,
-//               the last of the K arrivals combining that token's 128 channels;
-//   warps 5..20 two compute groups of eight warps; group g takes items g, g+2,
-//               ... of the CTA.
-// Compute groups never wait on global memory: fences, atomics and the
-// combine run on the publishing warps.  Down items requantise h locally (the
-// same per-slot absmax int8 rule).  Every wait is bounded (2 s) and raises the
-// device flag on expiry.
+//               a down item count each token's arrival on its 256-channel block,
+//               the last of the K arrivals combining that token's channels;
+//   warps 4..19 two compute groups of eight warps; group g takes items g, g+2,
+//               ... of the CTA.  Warp w of a group owns row group w of the
+//               item over all of K: it streams its own 2-bit codes (512
+//               contiguous bytes per 64 columns, one 16-byte cp.async per lane,
+//               kDecStages chunks in flight) and runs them against the staged
+//               activations, then its own epilogue.  The last warp of a batch
+//               to finish hands it on and frees the activation buffer; no
+//               barrier spans the group.
+// Every wait is bounded (2 s) and raises the device flag on expiry.
 // ---------------------------------------------------------------------------
-constexpr int kDecWSlots = 4;
 constexpr int kDecGroups = 2;
 constexpr int kDecGroupWarps = 8;
-constexpr int kDecGroupThreads = kDecGroupWarps * 32;
 constexpr int kDecRec = 4;   // completion records per group
-constexpr int kDecFirstCompute = 1 + 2 * kDecGroups;
-constexpr int kDecThreads = (kDecFirstCompute + kDecGroups * kDecGroupWarps) * 32;   // 672
+constexpr int kDecFirstCompute = 2 * kDecGroups;
+constexpr int kDecThreads = (kDecFirstCompute + kDecGroups * kDecGroupWarps) * 32;   // 640
+constexpr int kDecStages = 12;   // 512-byte weight chunks in flight per compute warp
 
 struct DecActMeta {
     int nb, b0, base, e;
     int slot[kGemvTokens];
-    float s[kGemvTokens];     // gate/up: s_x of the token
-    int sum[kGemvTokens];     // gate/up: sum of the token's int8 codes
-};
-struct DecWMeta {
-    int e, sub, kind, cnt, base;
+    float s[kGemvTokens];     // gate/up: s_x of the token; down: s_h of the slot
+    int sum[kGemvTokens];     // sum of the row's int8 codes (q_x or q_h)
+    unsigned done;            // warps finished with the batch
 };
 struct DecRecord {            // one finished batch of a compute group
     int kind, e, sub, nb, base, last;
@@ -418,9 +359,7 @@ struct DecRecord {            // one finished batch of a compute group
 struct DecodeArgs {
     GemvArgs g;
     unsigned *arrive;     // [E] finished gate/up items per expert, zero at launch
-    int wslot_bytes;      // codes + scales of one item
-    int aslot_bytes;      // activation rows of one batch
-    int nw;               // weight ring slots (2..kDecWSlots)
+    int aslot_bytes;      // one activation buffer
     const int8_t *zrow;   // D zero bytes (padding rows of a gate/up batch)
     const int *topk_idx;  // [T][K] the router's choices (distinct per token)
     const float *topk_w;  // [T][K] their softmax weights
@@ -428,33 +367,25 @@ struct DecodeArgs {
     int *tap_counts, *tap_offsets, *tap_perm;
 };
 
-__host__ __device__ inline int dec_wslot_bytes(int D, int F)
-{
-    const int g = 16 * D + 256, d = 32 * F + 512;
-    return ((g > d ? g : d) + 127) & ~127;
-}
-__host__ __device__ inline int dec_aslot_bytes(int D, int F)
+// activation buffer: [x rows int8 | h rows fp32] [q_h rows int8]
+__host__ __device__ inline int dec_qh_off(int D, int F)
 {
     const int g = kGemvTokens * D, d = kGemvTokens * F * 4;
     return ((g > d ? g : d) + 127) & ~127;
 }
+__host__ __device__ inline int dec_aslot_bytes(int D, int F) { return dec_qh_off(D, F) + ((kGemvTokens * F + 127) & ~127); }
 // routing tables every CTA builds for itself in shared memory
 __host__ __device__ inline size_t dec_table_bytes(int T, int K, int E)
 {
     return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E +
            (size_t)2 * (E + 1) * 4;
 }
-__host__ __device__ inline size_t dec_group_scratch_bytes(int F)
+constexpr int kDecBars = 6 * kDecGroups + 2 * kDecRec * kDecGroups;
+constexpr int kDecRingBytes = kDecGroups * kDecGroupWarps * kDecStages * 512;
+__host__ __device__ inline size_t decode_smem_bytes(int D, int F, int T, int K, int E)
 {
-    return (size_t)kDecGroupWarps * kGemvTokens * 32 * 4 + (size_t)kGemvTokens * F + 2 * kGemvTokens * 4;
-}
-constexpr int kDecBars = 2 * kDecWSlots + 4 * kDecGroups + 2 * kDecRec * kDecGroups;
-__host__ __device__ inline size_t decode_smem_bytes(int D, int F, int T, int K, int E, int nw)
-{
-    return (size_t)nw * dec_wslot_bytes(D, F) + (size_t)kDecGroups * 2 * dec_aslot_bytes(D, F) +
-           kDecGroups * dec_group_scratch_bytes(F) + kDecGroups * 2 * sizeof(DecActMeta) +
-           kDecWSlots * sizeof(DecWMeta) + kDecGroups * kDecRec * sizeof(DecRecord) + 8 * kDecBars + 64 +
-           dec_table_bytes(T, K, E);
+    return (size_t)kDecRingBytes + (size_t)kDecGroups * 2 * dec_aslot_bytes(D, F) + kDecGroups * 2 * sizeof(DecActMeta) +
+           kDecGroups * kDecRec * sizeof(DecRecord) + 8 * kDecBars + 64 + dec_table_bytes(T, K, E);
 }
 
 // bounded wait on an mbarrier phase (2 s); false on timeout
@@ -494,16 +425,94 @@ __device__ __forceinline__ void dec_bulk(void *dst, const void *src, uint32_t by
     }
 }
 
-// Relative cost of one work item of an expert with c tokens (kind 0 gate/up, 1
-// down): per batch of up to 8 tokens a fixed part (waits, barriers, epilogue)
-// plus a part per padded token (the dot), in units of about 0.1 us measured on
-// the decode-shape layer.  Only the split of the items over CTAs depends on it.
-__device__ __forceinline__ int dec_item_cost(int c, int kind)
+// Padded token count of a decode batch: the dot below exists for 1, 2, 4 and 8
+// tokens; rows nb..nbp-1 of a batch hold zeros.
+__device__ __forceinline__ int dec_pad_tokens(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
+
+// Issue the first kDecStages-1 chunks of a warp's weight stream (this lane's
+// 16 bytes of each 512-byte chunk) into its ring, one commit group each.
+__device__ __forceinline__ void dec_stream_start(uint8_t *ring, const uint8_t *src, int nch)
+{
+#pragma unroll
+    for (int s = 0; s < kDecStages - 1; s++) {
+        if (s < nch) cp_async16(ring + s * 512, src + (size_t)s * 512, true);
+        cp_async_commit();
+    }
+}
+
+// This lane's row against NB token rows over nch chunks of 64 columns; the
+// codes stream through the ring (each lane reads back only the bytes it
+// copied, so no barrier is needed), chunk c + kDecStages - 1 being issued while
+// chunk c is used.  Byte plane k is taken as w & (0x03030303 << 2k), i.e. 4^k
+// times the offset codes, one logic op per plane, into its own accumulator;
+// acc_k is an exact multiple of 4^k and the row total is acc_0 + acc_1/4 +
+// acc_2/16 + acc_3/64 (int32, exact).  Activations: 16-byte units
+// x[j*ld16 + 4c + w], read as broadcasts.
+template <int NB>
+__device__ __forceinline__ void dec_stream_dot(uint8_t *ring, const uint8_t *src, int nch, const uint4 *x, int ld16,
+                                               int (&tot)[kGemvTokens])
+{
+    int acc[NB][4];
+#pragma unroll
+    for (int j = 0; j < NB; j++)
+#pragma unroll
+        for (int k = 0; k < 4; k++) acc[j][k] = 0;
+    int st = 0;   // ring stage of chunk c
+#pragma unroll 1
+    for (int c = 0; c < nch; c++) {
+        cp_async_wait<kDecStages - 2>();
+        const uint4 wv = *reinterpret_cast<const uint4 *>(ring + st * 512);
+        const int cn = c + kDecStages - 1;
+        const int sn = st == 0 ? kDecStages - 1 : st - 1;   // stage of chunk c-1, now free
+        if (cn < nch) cp_async16(ring + sn * 512, src + (size_t)cn * 512, true);
+        cp_async_commit();
+        st = st == kDecStages - 1 ? 0 : st + 1;
+        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+        uint32_t pw[16];
+#pragma unroll
+        for (int w = 0; w < 4; w++)
+#pragma unroll
+            for (int k = 0; k < 4; k++) pw[4 * w + k] = w4[w] & (0x03030303u << (2 * k));
+#pragma unroll
+        for (int j = 0; j < NB; j++) {
+#pragma unroll
+            for (int w = 0; w < 4; w++) {
+                const uint4 xv = x[j * ld16 + 4 * c + w];
+                acc[j][0] = dp4a_us(pw[4 * w + 0], xv.x, acc[j][0]);
+                acc[j][1] = dp4a_us(pw[4 * w + 1], xv.y, acc[j][1]);
+                acc[j][2] = dp4a_us(pw[4 * w + 2], xv.z, acc[j][2]);
+                acc[j][3] = dp4a_us(pw[4 * w + 3], xv.w, acc[j][3]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kGemvTokens; j++)
+        tot[j] = j < NB ? acc[j < NB ? j : 0][0] + (acc[j < NB ? j : 0][1] >> 2) + (acc[j < NB ? j : 0][2] >> 4) +
+                              (acc[j < NB ? j : 0][3] >> 6)
+                        : 0;
+}
+
+__device__ __forceinline__ void dec_stream_dot_any(int nbp, uint8_t *ring, const uint8_t *src, int nch, const uint4 *x,
+                                                   int ld16, int (&tot)[kGemvTokens])
+{
+    switch (nbp) {
+    case 1: dec_stream_dot<1>(ring, src, nch, x, ld16, tot); break;
+    case 2: dec_stream_dot<2>(ring, src, nch, x, ld16, tot); break;
+    case 4: dec_stream_dot<4>(ring, src, nch, x, ld16, tot); break;
+    default: dec_stream_dot<8>(ring, src, nch, x, ld16, tot); break;
+    }
+}
+
+// Relative cost of one work item of an expert with c tokens: per batch of up to
+// 8 tokens, the item's chunks per warp times the instructions per chunk (a
+// fixed part and one per padded token), plus a fixed part per batch.  Only the
+// split of the items over the CTAs depends on it.
+__device__ __forceinline__ int dec_item_cost(int c, int nch)
 {
     int cost = 0;
     for (int b0 = 0; b0 < c; b0 += kGemvTokens) {
         const int nbp = dec_pad_tokens(min(kGemvTokens, c - b0));
-        cost += kind == 0 ? 23 + 5 * nbp : 18 + 7 * nbp;
+        cost += nch * (6 + 20 * nbp) + 400;
     }
     return cost;
 }
@@ -526,20 +535,17 @@ __device__ __forceinline__ int dec_item_at(const int *pref, int n_active, int pe
 __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeArgs d)
 {
     GemvArgs a = d.g;
-    const int nw = d.nw;
     extern __shared__ __align__(1024) uint8_t dsm[];
-    uint8_t *wring = dsm;
-    uint8_t *aring = wring + (size_t)nw * d.wslot_bytes;                          // [group][2][aslot]
-    uint8_t *gscr = aring + (size_t)kDecGroups * 2 * d.aslot_bytes;               // [group] scratch
-    const size_t gscr_bytes = dec_group_scratch_bytes(a.F);
-    DecActMeta *ameta = (DecActMeta *)(gscr + kDecGroups * gscr_bytes);           // [group][2]
-    DecWMeta *wmeta = (DecWMeta *)(ameta + kDecGroups * 2);                       // [kDecWSlots]
-    DecRecord *recs = (DecRecord *)(wmeta + kDecWSlots);                          // [group][kDecRec]
+    uint8_t *wring = dsm;                                                         // [group][warp][stage][512]
+    uint8_t *aring = wring + kDecRingBytes;                                       // [group][2][aslot]
+    DecActMeta *ameta = (DecActMeta *)(aring + (size_t)kDecGroups * 2 * d.aslot_bytes);   // [group][2]
+    DecRecord *recs = (DecRecord *)(ameta + kDecGroups * 2);                      // [group][kDecRec]
     uint64_t *bars = (uint64_t *)(((uintptr_t)(recs + kDecGroups * kDecRec) + 7) & ~(uintptr_t)7);
-    // bars: wfull[W], wempty[W], afull[G][2], aempty[G][2], rfull[G][R], rempty[G][R]
-    const uint32_t b_wfull = (uint32_t)__cvta_generic_to_shared(bars), b_wempty = b_wfull + 8 * kDecWSlots;
-    const uint32_t b_afull = b_wempty + 8 * kDecWSlots, b_aempty = b_afull + 8 * 2 * kDecGroups;
-    const uint32_t b_rfull = b_aempty + 8 * 2 * kDecGroups, b_rempty = b_rfull + 8 * kDecRec * kDecGroups;
+    // bars: afull[G][2], aempty[G][2], hfull[G][2], rfull[G][R], rempty[G][R]
+    const uint32_t b_afull = (uint32_t)__cvta_generic_to_shared(bars), b_aempty = b_afull + 8 * 2 * kDecGroups;
+    const uint32_t b_hfull = b_aempty + 8 * 2 * kDecGroups, b_rfull = b_hfull + 8 * 2 * kDecGroups;
+    const uint32_t b_rempty = b_rfull + 8 * kDecRec * kDecGroups;
+    const int qh_off = dec_qh_off(a.D, a.F);
     // routing tables
     const int T = a.T, K = a.K, E = a.E, S = a.T * a.K;
     int *t_idx = (int *)(bars + kDecBars);
@@ -551,19 +557,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     int *t_act = t_off + E + 1;
     float *t_sx = (float *)(t_act + E);
     int *t_sumx = (int *)(t_sx + T);
-    int *t_misc = t_sumx + T;   // [0] n_active, [8..40] scan scratch
+    int *t_misc = t_sumx + T;   // [0] n_active
+    unsigned long long *tmask = (unsigned long long *)(((uintptr_t)(t_misc + 48) + 7) & ~(uintptr_t)7);
+    int *t_pg = (int *)(tmask + E), *t_pd = t_pg + E + 1;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecBars; i++)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b_wfull + 8 * i), "r"(1) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b_afull + 8 * i), "r"(1) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (threadIdx.x < kDecGroups * 2) ameta[threadIdx.x].done = 0u;
 
     // ---------------- prologue: the permutation of the T*K slots (T <= 64), from the
     // router's choices: a token bitmask per expert gives the counts, and a slot's
     // rank within its expert is the number of earlier tokens in that mask
-    unsigned long long *tmask = (unsigned long long *)(((uintptr_t)(t_misc + 48) + 7) & ~(uintptr_t)7);
     const bool writer = blockIdx.x == 0;
     for (int e = threadIdx.x; e < E; e += blockDim.x) tmask[e] = 0ull;
     for (int q = threadIdx.x; q < S; q += blockDim.x) {
@@ -632,7 +640,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
         t_inv[q] = p;
         if (writer && d.tap_perm) d.tap_perm[p] = q;
     }
-    __syncthreads();
     a.active = t_act;
     a.n_active = t_misc;
     a.counts = t_cnt;
@@ -644,17 +651,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     a.sumx = t_sumx;
 
     const int n_active = t_misc[0];
-    const int pairs = a.F / 32, blocks = a.D / 128;
+    const int Cg = a.D / 64, Cd = a.F / 64;
+    const int gitems = a.F / 128, ditems = a.D / 256;   // items per expert (8 row groups each)
     // split each kind of item over the CTAs in equal shares of estimated cost
-    int *t_pg = (int *)(tmask + E), *t_pd = t_pg + E + 1;
     if (warp == 0) {
         const int per = (n_active + 31) / 32, a0 = lane * per;
         int sg = 0, sd = 0;
         for (int i = 0; i < per; i++)
             if (a0 + i < n_active) {
                 const int c = t_cnt[t_act[a0 + i]];
-                sg += pairs * dec_item_cost(c, 0);
-                sd += blocks * dec_item_cost(c, 1);
+                sg += gitems * dec_item_cost(c, Cg);
+                sd += ditems * dec_item_cost(c, Cd);
             }
         int cg = sg, cd = sd;
 #pragma unroll
@@ -671,8 +678,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                 const int c = t_cnt[t_act[a0 + i]];
                 t_pg[a0 + i] = og;
                 t_pd[a0 + i] = od;
-                og += pairs * dec_item_cost(c, 0);
-                od += blocks * dec_item_cost(c, 1);
+                og += gitems * dec_item_cost(c, Cg);
+                od += ditems * dec_item_cost(c, Cd);
             }
         if (lane == 31) {
             t_pg[n_active] = cg;
@@ -681,85 +688,41 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     }
     __syncthreads();
     const int64_t WG = t_pg[n_active], WD = t_pd[n_active];
-    const int g0 = dec_item_at(t_pg, n_active, pairs, WG * blockIdx.x / gridDim.x);
-    const int g1 = dec_item_at(t_pg, n_active, pairs, WG * (blockIdx.x + 1) / gridDim.x);
-    const int d0 = dec_item_at(t_pd, n_active, blocks, WD * blockIdx.x / gridDim.x);
-    const int d1 = dec_item_at(t_pd, n_active, blocks, WD * (blockIdx.x + 1) / gridDim.x);
+    const int g0 = dec_item_at(t_pg, n_active, gitems, WG * blockIdx.x / gridDim.x);
+    const int g1 = dec_item_at(t_pg, n_active, gitems, WG * (blockIdx.x + 1) / gridDim.x);
+    const int d0 = dec_item_at(t_pd, n_active, ditems, WD * blockIdx.x / gridDim.x);
+    const int d1 = dec_item_at(t_pd, n_active, ditems, WD * (blockIdx.x + 1) / gridDim.x);
     const int nG = g1 - g0, n_items = nG + (d1 - d0);
-    const int Cg = a.D / 64, Cd = a.F / 64;
-    // item i of this CTA -> kind (0 gate/up, 1 down), active index, sub-block
+    // item i of this CTA -> kind (0 gate/up, 1 down), active index, sub-item
     auto item_of = [&](int i, int &kind, int &ai, int &sub) {
         if (i < nG) {
             kind = 0;
-            ai = (g0 + i) / pairs;
-            sub = (g0 + i) % pairs;
+            ai = (g0 + i) / gitems;
+            sub = (g0 + i) % gitems;
         } else {
             kind = 1;
-            ai = (d0 + i - nG) / blocks;
-            sub = (d0 + i - nG) % blocks;
+            ai = (d0 + i - nG) / ditems;
+            sub = (d0 + i - nG) % ditems;
         }
     };
 
-    if (warp == 0) {
-        // ---------------- codes and scales of every item, in order
-        if (lane == 0) {
-            int issued = 0;
-            for (int i = 0; i < n_items; i++) {
-                const int ws = i % nw;
-                if (!dec_wait(b_wempty + 8 * ws, ((i / nw) & 1) ^ 1)) {
-                    set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
-                    break;
-                }
-                issued = i + 1;
-                int kind, ai, sub;
-                item_of(i, kind, ai, sub);
-                const int e = a.active[ai];
-                DecWMeta *m = wmeta + ws;
-                m->e = e;
-                m->sub = sub;
-                m->kind = kind;
-                m->cnt = a.counts[e];
-                m->base = a.offsets[e];
-                uint8_t *dst = wring + (size_t)ws * d.wslot_bytes;
-                const uint32_t bar = b_wfull + 8 * ws;
-                if (kind == 0) {
-                    const uint32_t cb = (uint32_t)(2 * Cg * 512);
-                    dec_expect(bar, cb + 256);
-                    dec_bulk(dst, a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)(2 * sub) * Cg * 512, cb, bar);
-                    dec_bulk(dst + cb, a.alpha_gate + (size_t)e * a.F + 32 * sub, 128, bar);
-                    dec_bulk(dst + cb + 128, a.alpha_up + (size_t)e * a.F + 32 * sub, 128, bar);
-                } else {
-                    const uint32_t cb = (uint32_t)(4 * Cd * 512);
-                    dec_expect(bar, cb + 512);
-                    dec_bulk(dst, a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)(4 * sub) * Cd * 512, cb, bar);
-                    dec_bulk(dst + cb, a.alpha_down + (size_t)e * a.D + 128 * sub, 512, bar);
-                }
-            }
-            // no copy may still be landing when the CTA exits
-            for (int j = issued > nw ? issued - nw : 0; j < issued; j++)
-                (void)dec_wait(b_wfull + 8 * (j % nw), (j / nw) & 1);
-        }
-        return;
-    }
-
-    if (warp <= kDecGroups) {
-        // ---------------- activation staging for compute group g
-        const int g = warp - 1;
-        if (lane == 0) {
-            int k = 0;
-            bool ok = true;
-            int staged = 0;   // units whose copies were issued
-            for (int i = g; i < n_items && ok; i += kDecGroups) {
-                int kind, ai, sub;
-                item_of(i, kind, ai, sub);
-                const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
-                if (kind == 1) {
-                    // every gate/up item of expert e must be done before its h rows are read
+    if (warp < kDecGroups) {
+        // ---------------- activation staging for compute group g (whole warp)
+        const int g = warp;
+        int k = 0, kh0 = 0, kh1 = 0;   // batches staged; down batches staged per buffer
+        bool ok = true;
+        for (int i = g; i < n_items && ok; i += kDecGroups) {
+            int kind, ai, sub;
+            item_of(i, kind, ai, sub);
+            const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
+            if (kind == 1) {
+                // every gate/up item of expert e must be done before its h rows are read
+                if (lane == 0) {
                     const uint64_t t0 = global_timer_ns();
                     unsigned v = 0;
                     while (true) {
                         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(d.arrive + e) : "memory");
-                        if (v >= (unsigned)pairs) break;
+                        if (v >= (unsigned)gitems) break;
                         __nanosleep(128);
                         if (global_timer_ns() - t0 > 2000000000ull) {
                             set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
@@ -767,53 +730,109 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                             break;
                         }
                     }
-                    if (!ok) break;
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                 }
-                for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++) {
-                    const int buf = k & 1;
-                    if (!dec_wait(b_aempty + 8 * (2 * g + buf), ((k >> 1) & 1) ^ 1)) {
-                        set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
-                        ok = false;
-                        break;
+                ok = __shfl_sync(FULL, ok, 0);
+                if (!ok) break;
+            }
+            for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++) {
+                const int buf = k & 1;
+                if (!dec_wait(b_aempty + 8 * (2 * g + buf), ((k >> 1) & 1) ^ 1)) {
+                    if (lane == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                const int nb = min(kGemvTokens, cnt - b0), nbp = dec_pad_tokens(nb);
+                DecActMeta *m = ameta + 2 * g + buf;
+                uint8_t *dst = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
+                if (lane < nb) {
+                    const int slot = a.perm[base + b0 + lane];
+                    m->slot[lane] = slot;
+                    if (kind == 0) {
+                        m->s[lane] = a.sx[slot / a.K];
+                        m->sum[lane] = a.sumx[slot / a.K];
                     }
-                    const int nb = min(kGemvTokens, cnt - b0);
-                    DecActMeta *m = ameta + 2 * g + buf;
+                }
+                if (lane == 0) {
                     m->nb = nb;
                     m->b0 = b0;
                     m->base = base;
                     m->e = e;
-                    uint8_t *dst = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
-                    const uint32_t bar = b_afull + 8 * (2 * g + buf);
-                    if (kind == 0) {
-                        for (int j = 0; j < nb; j++) {
-                            const int slot = a.perm[base + b0 + j], t = slot / a.K;
-                            m->slot[j] = slot;
-                            m->s[j] = a.sx[t];
-                            m->sum[j] = a.sumx[t];
-                        }
-                        const int nbp = dec_pad_tokens(nb);
+                }
+                __syncwarp();
+                if (kind == 0) {
+                    if (lane == 0) {
+                        const uint32_t bar = b_afull + 8 * (2 * g + buf);
                         dec_expect(bar, (uint32_t)(nbp * a.D));
                         for (int j = 0; j < nbp; j++)
                             dec_bulk(dst + (size_t)j * a.D,
                                      j < nb ? a.qx + (size_t)(m->slot[j] / a.K) * a.D : d.zrow, (uint32_t)a.D, bar);
-                    } else {
-                        for (int j = 0; j < nb; j++) m->slot[j] = a.perm[base + b0 + j];
-                        dec_expect(bar, (uint32_t)(nb * a.F * 4));
-                        dec_bulk(dst, a.h + (size_t)(base + b0) * a.F, (uint32_t)(nb * a.F * 4), bar);
                     }
-                    staged = k + 1;
+                    continue;
                 }
+                // down: bring the h rows in, requantise them per slot into the buffer
+                const uint32_t hb = b_hfull + 8 * (2 * g + buf);
+                if (lane == 0) {
+                    dec_expect(hb, (uint32_t)(nb * a.F * 4));
+                    dec_bulk(dst, a.h + (size_t)(base + b0) * a.F, (uint32_t)(nb * a.F * 4), hb);
+                }
+                const int kh = buf ? kh1++ : kh0++;
+                if (!dec_wait(hb, kh & 1)) {
+                    if (lane == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                int8_t *qh = (int8_t *)(dst + qh_off);
+                for (int j = 0; j < nb; j++) {
+                    const float4 *h4 = reinterpret_cast<const float4 *>(dst + (size_t)j * a.F * 4);
+                    float amax = 0.0f;
+                    for (int q = lane; q < a.F / 4; q += 32) {
+                        const float4 v = h4[q];
+                        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
+                    }
+                    amax = warp_max(amax);
+                    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+                    int sum = 0;
+                    for (int q = lane; q < a.F / 4; q += 32) {
+                        const float4 v = h4[q];
+                        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+                        if (amax > 0.0f) {
+                            q0 = quant_code(v.x, inv);
+                            q1 = quant_code(v.y, inv);
+                            q2 = quant_code(v.z, inv);
+                            q3 = quant_code(v.w, inv);
+                        }
+                        sum += q0 + q1 + q2 + q3;
+                        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                                            ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+                        reinterpret_cast<uint32_t *>(qh + (size_t)j * a.F)[q] = pk;
+                        if (sub == 0 && a.tap_qh)
+                            reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)m->slot[j] * a.F)[q] = pk;
+                    }
+                    sum = warp_sum_int(sum);
+                    if (lane == 0) {
+                        const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+                        m->s[j] = sv;
+                        m->sum[j] = sum;
+                        if (sub == 0 && a.tap_sh) a.tap_sh[m->slot[j]] = sv;
+                    }
+                }
+                for (int j = nb; j < nbp; j++)
+                    for (int q = lane; q < a.F / 16; q += 32)
+                        reinterpret_cast<uint4 *>(qh + (size_t)j * a.F)[q] = make_uint4(0u, 0u, 0u, 0u);
+                __syncwarp();
+                if (lane == 0) dec_arrive(b_afull + 8 * (2 * g + buf));
             }
-            for (int j = staged > 2 ? staged - 2 : 0; j < staged; j++)
-                (void)dec_wait(b_afull + 8 * (2 * g + (j & 1)), (j >> 1) & 1);
         }
+        // no copy may still be landing when the CTA exits
+        for (int j = k > 2 ? k - 2 : 0; j < k; j++) (void)dec_wait(b_afull + 8 * (2 * g + (j & 1)), (j >> 1) & 1);
         return;
     }
 
     if (warp < kDecFirstCompute) {
         // ---------------- publishing warp of group g
-        const int g = warp - 1 - kDecGroups;
+        const int g = warp - kDecGroups;
+        const int nblk = a.D / 256;
         int r = 0;
         for (int i = g; i < n_items; i += kDecGroups) {
             int kind, ai, sub;
@@ -837,7 +856,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                     int t = 0;
                     if (lane < rec.nb) {
                         t = rec.slot[lane] / a.K;
-                        prev = atomicAdd(a.comb_cnt + (size_t)t * blocks + rec.sub, 1u);
+                        prev = atomicAdd(a.comb_cnt + (size_t)t * nblk + rec.sub, 1u);
                     }
                     unsigned done = __ballot_sync(FULL, lane < rec.nb && prev == (unsigned)(a.K - 1));
                     if (done) fence_gpu();
@@ -845,28 +864,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
                         const int j = __ffs(done) - 1;
                         done &= done - 1;
                         const int tt = __shfl_sync(FULL, t, j);
-                        // channels rec.sub*128 + 4*lane .. +3 of token tt, in rank order
-                        const int cc = rec.sub * 128 + 4 * lane;
-                        float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int kk = 0; kk < a.K; kk++) {
-                            const int sl = tt * a.K + kk;
-                            const float wk = a.topk_w[sl];
-                            const float4 ev = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)a.inv[sl] * a.D + cc));
-                            yv.x = __fmaf_rn(wk, ev.x, yv.x);
-                            yv.y = __fmaf_rn(wk, ev.y, yv.y);
-                            yv.z = __fmaf_rn(wk, ev.z, yv.z);
-                            yv.w = __fmaf_rn(wk, ev.w, yv.w);
+                        // channels rec.sub*256 + 4*lane .. +3 and +128 of token tt, in rank order
+#pragma unroll
+                        for (int hlf = 0; hlf < 2; hlf++) {
+                            const int cc = rec.sub * 256 + 128 * hlf + 4 * lane;
+                            float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int kk = 0; kk < a.K; kk++) {
+                                const int sl = tt * a.K + kk;
+                                const float wk = a.topk_w[sl];
+                                const float4 ev =
+                                    __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)a.inv[sl] * a.D + cc));
+                                yv.x = __fmaf_rn(wk, ev.x, yv.x);
+                                yv.y = __fmaf_rn(wk, ev.y, yv.y);
+                                yv.z = __fmaf_rn(wk, ev.z, yv.z);
+                                yv.w = __fmaf_rn(wk, ev.w, yv.w);
+                            }
+                            const size_t o = (size_t)tt * a.D + cc;
+                            if (a.resid) {
+                                const float4 rv = *reinterpret_cast<const float4 *>(a.resid + o);
+                                yv.x = __fadd_rn(rv.x, yv.x);
+                                yv.y = __fadd_rn(rv.y, yv.y);
+                                yv.z = __fadd_rn(rv.z, yv.z);
+                                yv.w = __fadd_rn(rv.w, yv.w);
+                            }
+                            *reinterpret_cast<float4 *>(a.y + o) = yv;
                         }
-                        const size_t o = (size_t)tt * a.D + cc;
-                        if (a.resid) {
-                            const float4 rv = *reinterpret_cast<const float4 *>(a.resid + o);
-                            yv.x = __fadd_rn(rv.x, yv.x);
-                            yv.y = __fadd_rn(rv.y, yv.y);
-                            yv.z = __fadd_rn(rv.z, yv.z);
-                            yv.w = __fadd_rn(rv.w, yv.w);
-                        }
-                        *reinterpret_cast<float4 *>(a.y + o) = yv;
-                        if (lane == j) a.comb_cnt[(size_t)tt * blocks + rec.sub] = 0;
+                        if (lane == j) a.comb_cnt[(size_t)tt * nblk + rec.sub] = 0;
                     }
                 }
                 __syncwarp();
@@ -877,140 +900,93 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
         return;
     }
 
-    // ---------------- compute group g: eight warps
+    // ---------------- compute warp gw of group g: row group gw of every item of the group
     const int g = (warp - kDecFirstCompute) / kDecGroupWarps, gw = (warp - kDecFirstCompute) % kDecGroupWarps;
-    const int gtid = gw * 32 + lane;
-    const int bar_id = 1 + g;
-    auto gsync = [&] { asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kDecGroupThreads) : "memory"); };
-    uint8_t *scr = gscr + (size_t)g * gscr_bytes;
-    int *red = (int *)scr;                                            // [8 warps][kGemvTokens][32]
-    int8_t *qh = (int8_t *)(red + kDecGroupWarps * kGemvTokens * 32);  // [kGemvTokens][F]
-    float *shs = (float *)(qh + (size_t)kGemvTokens * a.F);          // [kGemvTokens]
-    int *sumqh = (int *)(shs + kGemvTokens);                         // [kGemvTokens]
-
-    int k = 0, r = 0;
+    uint8_t *ring = wring + (size_t)((g * kDecGroupWarps + gw) * kDecStages) * 512 + lane * 16;
+    int k = 0;   // batches of this group (= completion record index)
     for (int i = g; i < n_items; i += kDecGroups) {
-        const int ws = i % nw;
-        if (!dec_wait(b_wfull + 8 * ws, (i / nw) & 1)) {
-            if (gtid == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
-            break;
-        }
-        const DecWMeta wm = wmeta[ws];
-        const uint8_t *wb = wring + (size_t)ws * d.wslot_bytes;
-        const int cnt = wm.cnt, base = wm.base;
-        bool ok = true;
-        for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++, r++) {
+        int kind, ai, sub;
+        item_of(i, kind, ai, sub);
+        const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
+        const int grp = sub * kDecGroupWarps + gw;   // row group (32 rows) within the expert
+        const int nch = kind == 0 ? Cg : Cd;
+        const uint8_t *src = kind == 0
+                                 ? a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)grp * Cg * 512 + lane * 16
+                                 : a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)grp * Cd * 512 + lane * 16;
+        // the row scale: gate/up lanes 0..15 gate rows grp*16+l, lanes 16..31 the up rows of
+        // the same outputs; down lane l channel grp*32+l
+        const float al = kind == 0 ? __ldg((lane < 16 ? a.alpha_gate : a.alpha_up) + (size_t)e * a.F + grp * 16 + (lane & 15))
+                                   : __ldg(a.alpha_down + (size_t)e * a.D + grp * 32 + lane);
+        for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++) {
             const int buf = k & 1;
+            dec_stream_start(ring, src, nch);   // the codes stream in while the activations are awaited
             if (!dec_wait(b_afull + 8 * (2 * g + buf), (k >> 1) & 1)) {
-                if (gtid == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
-                ok = false;
-                break;
+                if (lane == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
+                cp_async_wait<0>();
+                return;
             }
-            const DecActMeta &am = ameta[2 * g + buf];
+            DecActMeta *am = ameta + 2 * g + buf;
             const uint8_t *ab = aring + (size_t)(2 * g + buf) * d.aslot_bytes;
-            const int nb = am.nb;
-            const int nbp = dec_pad_tokens(nb);
-            int *red_w = red + gw * kGemvTokens * 32 + lane;
-            if (wm.kind == 0) {
-                // ---- gate/up: warp gw = row group gw/4 (of the pair), K quarter gw%4
-                const int rg = gw >> 2, kq = gw & 3, quarter = Cg / 4;
-                const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)rg * Cg * 512) + lane;
-                dot_rows_any(nbp, wl, reinterpret_cast<const uint4 *>(ab), a.D / 16, kq * quarter, quarter, red_w);
-                gsync();
-                if (kq == 0) {
-                    const bool is_up = lane >= 16;
-                    const int rr = (2 * wm.sub + rg) * 16 + (lane & 15);
-                    const float al = ((const float *)(wb + 2 * Cg * 512))[(is_up ? 32 : 0) + 16 * rg + (lane & 15)];
-                    for (int j = 0; j < nb; j++) {
-                        int sum = 0;
+            const int nb = am->nb;
+            int tot[kGemvTokens];
+            if (kind == 0)
+                dec_stream_dot_any(dec_pad_tokens(nb), ring, src, nch, reinterpret_cast<const uint4 *>(ab), a.D / 16,
+                                   tot);
+            else
+                dec_stream_dot_any(dec_pad_tokens(nb), ring, src, nch, reinterpret_cast<const uint4 *>(ab + qh_off),
+                                   a.F / 16, tot);
+            if (kind == 0) {
+                const bool is_up = lane >= 16;
+                const int rr = grp * 16 + (lane & 15);
+                int *tap = is_up ? a.tap_acc_up : a.tap_acc_gate;
 #pragma unroll
-                        for (int q = 0; q < 4; q++) sum += red[((gw + q) * kGemvTokens + j) * 32 + lane];
-                        const int av = sum - am.sum[j];
-                        const float v = __fmul_rn((float)av, __fmul_rn(al, am.s[j]));
+                for (int j = 0; j < kGemvTokens; j++) {
+                    if (j < nb) {
+                        const int av = tot[j] - am->sum[j];
+                        const float v = __fmul_rn((float)av, __fmul_rn(al, am->s[j]));
                         const float uu = __shfl_down_sync(FULL, v, 16);
-                        if (!is_up) a.h[(size_t)(base + am.b0 + j) * a.F + rr] = swiglu(v, uu);
-                        int *tap = is_up ? a.tap_acc_up : a.tap_acc_gate;
-                        if (tap) tap[(size_t)am.slot[j] * a.F + rr] = av;
+                        if (!is_up) a.h[(size_t)(base + b0 + j) * a.F + rr] = swiglu(v, uu);
+                        if (tap) tap[(size_t)am->slot[j] * a.F + rr] = av;
                     }
                 }
             } else {
-                // ---- down: requantise the batch's h rows (one slot per warp), then warp gw =
-                //      channel group 4*blk + gw/2, K half gw%2
-                const float *hr = (const float *)ab;
-                for (int j = nb + gw; j < nbp; j += kDecGroupWarps)
-                    for (int q = lane; q < a.F / 16; q += 32)
-                        reinterpret_cast<uint4 *>(qh + (size_t)j * a.F)[q] = make_uint4(0u, 0u, 0u, 0u);
-                for (int j = gw; j < nb; j += kDecGroupWarps) {
-                    const float4 *h4 = reinterpret_cast<const float4 *>(hr + (size_t)j * a.F);
-                    float amax = 0.0f;
-                    for (int q = lane; q < a.F / 4; q += 32) {
-                        const float4 v = h4[q];
-                        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
-                    }
-                    amax = warp_max(amax);
-                    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                    int sum = 0;
-                    for (int q = lane; q < a.F / 4; q += 32) {
-                        const float4 v = h4[q];
-                        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-                        if (amax > 0.0f) {
-                            q0 = quant_code(v.x, inv);
-                            q1 = quant_code(v.y, inv);
-                            q2 = quant_code(v.z, inv);
-                            q3 = quant_code(v.w, inv);
-                        }
-                        sum += q0 + q1 + q2 + q3;
-                        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
-                                            ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
-                        reinterpret_cast<uint32_t *>(qh + (size_t)j * a.F)[q] = pk;
-                        if (wm.sub == 0 && a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)am.slot[j] * a.F)[q] = pk;
-                    }
-                    sum = warp_sum_int(sum);
-                    if (lane == 0) {
-                        const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-                        shs[j] = sv;
-                        sumqh[j] = sum;
-                        if (wm.sub == 0 && a.tap_sh) a.tap_sh[am.slot[j]] = sv;
-                    }
-                }
-                gsync();
-                const int cgl = gw >> 1, kh = gw & 1, half = Cd / 2;
-                const uint4 *wl = reinterpret_cast<const uint4 *>(wb + (size_t)cgl * Cd * 512) + lane;
-                dot_rows_any(nbp, wl, reinterpret_cast<const uint4 *>(qh), a.F / 16, kh * half, half, red_w);
-                gsync();
-                if (kh == 0) {
-                    const int cg = (wm.sub * 4 + cgl) * 32 + lane;
-                    const float al = ((const float *)(wb + 4 * Cd * 512))[cgl * 32 + lane];
-                    for (int j = 0; j < nb; j++) {
-                        const int p = base + am.b0 + j;
-                        const int av = red[(gw * kGemvTokens + j) * 32 + lane] +
-                                       red[((gw + 1) * kGemvTokens + j) * 32 + lane] - sumqh[j];
-                        a.ye[(size_t)p * a.D + cg] = __fmul_rn((float)av, __fmul_rn(al, shs[j]));
-                        if (a.tap_acc_down) a.tap_acc_down[(size_t)am.slot[j] * a.D + cg] = av;
+                const int cg = grp * 32 + lane;
+#pragma unroll
+                for (int j = 0; j < kGemvTokens; j++) {
+                    if (j < nb) {
+                        const int av = tot[j] - am->sum[j];
+                        a.ye[(size_t)(base + b0 + j) * a.D + cg] = __fmul_rn((float)av, __fmul_rn(al, am->s[j]));
+                        if (a.tap_acc_down) a.tap_acc_down[(size_t)am->slot[j] * a.D + cg] = av;
                     }
                 }
             }
-            gsync();
-            if (gtid == 0) {
-                // hand the batch to the publishing warp, free the activation slot
-                const int rs = r % kDecRec;
-                if (!dec_wait(b_rempty + 8 * (kDecRec * g + rs), ((r / kDecRec) & 1) ^ 1))
+            // the last warp of the batch hands it to the publishing warp and frees the buffer
+            __syncwarp();
+            unsigned prev = 0;
+            if (lane == 0) {
+                __threadfence_block();
+                prev = atomicAdd(&am->done, 1u);
+                __threadfence_block();
+            }
+            prev = __shfl_sync(FULL, prev, 0);
+            if (prev != (unsigned)(kDecGroupWarps - 1)) continue;
+            if (lane == 0) {
+                am->done = 0u;
+                const int rs = k % kDecRec;
+                if (!dec_wait(b_rempty + 8 * (kDecRec * g + rs), ((k / kDecRec) & 1) ^ 1))
                     set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
                 DecRecord *rec = recs + kDecRec * g + rs;
-                rec->kind = wm.kind;
-                rec->e = wm.e;
-                rec->sub = wm.sub;
+                rec->kind = kind;
+                rec->e = e;
+                rec->sub = sub;
                 rec->nb = nb;
                 rec->base = base;
                 rec->last = b0 + kGemvTokens >= cnt;
-                for (int j = 0; j < nb; j++) rec->slot[j] = am.slot[j];
+                for (int j = 0; j < nb; j++) rec->slot[j] = am->slot[j];
                 dec_arrive(b_rfull + 8 * (kDecRec * g + rs));
                 dec_arrive(b_aempty + 8 * (2 * g + buf));
             }
         }
-        if (!ok) break;
-        gsync();
-        if (gtid == 0) dec_arrive(b_wempty + 8 * ws);
     }
 }
 

@@ -337,7 +337,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
         h->dec_optin = optin;
-        h->dec_persistent = decode_smem_bytes(h->D, h->F, 1, h->K, h->E, 2) <= (size_t)optin;
+        h->dec_persistent = decode_smem_bytes(h->D, h->F, 1, h->K, h->E) <= (size_t)optin;
     }
     h->xn = (uint16_t *)(b + o_xn);
     h->zrow = (const int8_t *)(b + o_zr);
@@ -492,13 +492,11 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     return launch_status();
 }
 
-// smallest ring of weight slots (2..4) whose decode kernel fits, 0 if none
+// 1 when the persistent decode kernel runs this batch (it fits the shape and T), else 0
 static int decode_ring_slots(maple_moe_t h, int T)
 {
     if (!h->dec_persistent || T > kRouteSmallT || (int64_t)T * h->E > kFusedMarkBytes) return 0;
-    for (int nw = kDecWSlots; nw >= 2; nw--)
-        if (decode_smem_bytes(h->D, h->F, T, h->K, h->E, nw) <= (size_t)h->dec_optin) return nw;
-    return 0;
+    return decode_smem_bytes(h->D, h->F, T, h->K, h->E) <= (size_t)h->dec_optin ? 1 : 0;
 }
 
 static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
@@ -550,9 +548,7 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         memset(&d, 0, sizeof d);
         d.g = g;
         d.arrive = h->arrive;
-        d.wslot_bytes = dec_wslot_bytes(h->D, h->F);
         d.aslot_bytes = dec_aslot_bytes(h->D, h->F);
-        d.nw = nw;
         d.zrow = h->zrow;
         d.topk_idx = h->topk_idx;
         d.topk_w = h->topk_w;
@@ -566,7 +562,7 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         memset(&lc, 0, sizeof lc);
         lc.gridDim = dim3(h->num_sms);
         lc.blockDim = dim3(kDecThreads);
-        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E, nw);
+        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E);
         lc.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;

@@ -315,8 +315,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32, MAPLE_GEMV_MINB) down_gemv_ke
 // router's top-k (in shared memory), so no routing step needs a grid-wide
 // hand-off.  Work items: gate/up items (active expert, 8 groups of 16 gate +
 // 16 up rows) then down items (active expert, 8 groups of 32 output
-// channels); every CTA takes a contiguous range of each kind holding an equal
-// share of its estimated cost (an item's cost grows with its token count).
+// channels).  Items are handed out dynamically: compute group 0 or 1 of
+// any CTA claims the next one from a global counter (gate/up items first, so
+// no down item can wait on an unclaimed gate/up item), which balances the
+// load whatever the tokens per expert; a small queue in shared memory passes a
+// group's claims to its warps.
 // Warp roles:
 //   warps 0, 1  stage the activations of compute group 0 / 1 (double
 //               buffered): for gate/up the int8 rows of the item's tokens; for
@@ -351,6 +354,11 @@ struct DecActMeta {
     int sum[kGemvTokens];     // sum of the row's int8 codes (q_x or q_h)
     unsigned done;            // warps finished with the batch
 };
+constexpr int kDecQueue = 16;   // claimed items a group's queue holds
+struct DecQueue {               // the items a compute group has claimed, in order
+    int item[kDecQueue];        // global item id (>= total: no more work)
+    int n;                      // items claimed so far
+};
 struct DecRecord {            // one finished batch of a compute group
     int kind, e, sub, nb, base, last;
     int slot[kGemvTokens];
@@ -361,6 +369,7 @@ struct DecodeArgs {
     unsigned *arrive;     // [E] finished gate/up items per expert, zero at launch
     int aslot_bytes;      // one activation buffer
     const int8_t *zrow;   // D zero bytes (padding rows of a gate/up batch)
+    int *item_ctr;        // work items claimed so far, zero at launch
     const int *topk_idx;  // [T][K] the router's choices (distinct per token)
     const float *topk_w;  // [T][K] their softmax weights
     // outputs of the permutation, written by CTA 0 (may be null)
@@ -377,15 +386,15 @@ __host__ __device__ inline int dec_aslot_bytes(int D, int F) { return dec_qh_off
 // routing tables every CTA builds for itself in shared memory
 __host__ __device__ inline size_t dec_table_bytes(int T, int K, int E)
 {
-    return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E +
-           (size_t)2 * (E + 1) * 4;
+    return (size_t)4 * T * K * 4 + (size_t)(3 * E + 1) * 4 + (size_t)2 * T * 4 + 48 * 4 + 8 + (size_t)8 * E;
 }
 constexpr int kDecBars = 6 * kDecGroups + 2 * kDecRec * kDecGroups;
 constexpr int kDecRingBytes = kDecGroups * kDecGroupWarps * kDecStages * 512;
 __host__ __device__ inline size_t decode_smem_bytes(int D, int F, int T, int K, int E)
 {
     return (size_t)kDecRingBytes + (size_t)kDecGroups * 2 * dec_aslot_bytes(D, F) + kDecGroups * 2 * sizeof(DecActMeta) +
-           kDecGroups * kDecRec * sizeof(DecRecord) + 8 * kDecBars + 64 + dec_table_bytes(T, K, E);
+           kDecGroups * sizeof(DecQueue) + kDecGroups * kDecRec * sizeof(DecRecord) + 8 * kDecBars + 64 +
+           dec_table_bytes(T, K, E);
 }
 
 // bounded wait on an mbarrier phase (2 s); false on timeout
@@ -429,27 +438,37 @@ __device__ __forceinline__ void dec_bulk(void *dst, const void *src, uint32_t by
 // tokens; rows nb..nbp-1 of a batch hold zeros.
 __device__ __forceinline__ int dec_pad_tokens(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
 
-// Issue the first kDecStages-1 chunks of a warp's weight stream (this lane's
-// 16 bytes of each 512-byte chunk) into its ring, one commit group each.
-__device__ __forceinline__ void dec_stream_start(uint8_t *ring, const uint8_t *src, int nch)
-{
-#pragma unroll
-    for (int s = 0; s < kDecStages - 1; s++) {
-        if (s < nch) cp_async16(ring + s * 512, src + (size_t)s * 512, true);
-        cp_async_commit();
-    }
-}
+// The weight stream of one compute warp: for every batch of every item the
+// warp takes (items g, g+2, ... of the CTA; a batch is up to 8 tokens of the
+// item's expert), the nch chunks of its row group, 512 contiguous bytes per 64
+// columns, this lane's 16 bytes of each copied with one cp.async into a ring of
+// kDecStages chunks.  The issue cursor runs kDecStages-1 chunks ahead of the
+// chunk in use, across batch and item boundaries, so the pipeline never drains
+// between items.  Each lane reads back only the bytes it copied itself, so no
+// barrier is needed.
+struct DecStream {
+    uint8_t *ring;          // this lane's 16 bytes of stage 0
+    const uint8_t *src;     // this lane's 16 bytes of chunk 0 of the current segment
+    int nch, c, left;       // chunks in the segment, next chunk, batches left in the item
+    int item, st;           // queue ordinal of the issue cursor's item, ring stage to fill next
 
-// This lane's row against NB token rows over nch chunks of 64 columns; the
-// codes stream through the ring (each lane reads back only the bytes it
-// copied, so no barrier is needed), chunk c + kDecStages - 1 being issued while
-// chunk c is used.  Byte plane k is taken as w & (0x03030303 << 2k), i.e. 4^k
-// times the offset codes, one logic op per plane, into its own accumulator;
-// acc_k is an exact multiple of 4^k and the row total is acc_0 + acc_1/4 +
-// acc_2/16 + acc_3/64 (int32, exact).  Activations: 16-byte units
-// x[j*ld16 + 4c + w], read as broadcasts.
-template <int NB>
-__device__ __forceinline__ void dec_stream_dot(uint8_t *ring, const uint8_t *src, int nch, const uint4 *x, int ld16,
+    __device__ __forceinline__ void issue()
+    {
+        if (left > 0) cp_async16(ring + st * 512, src + (size_t)c * 512, true);
+        cp_async_commit();
+        st = st == kDecStages - 1 ? 0 : st + 1;
+    }
+};
+
+// This lane's row against NB token rows over the nch chunks of the current
+// batch; for every chunk used one more is issued (advance() moves the issue
+// cursor).  Byte plane k is taken as w & (0x03030303 << 2k), i.e. 4^k times the
+// offset codes, one logic op per plane, into its own accumulator; acc_k is an
+// exact multiple of 4^k and the row total is acc_0 + acc_1/4 + acc_2/16 +
+// acc_3/64 (int32, exact).  Activations: 16-byte units x[j*ld16 + 4c + w], read
+// as broadcasts.
+template <int NB, class Adv>
+__device__ __forceinline__ void dec_stream_dot(DecStream &ws, int &cst, int nch, const uint4 *x, int ld16, Adv &advance,
                                                int (&tot)[kGemvTokens])
 {
     int acc[NB][4];
@@ -457,16 +476,13 @@ __device__ __forceinline__ void dec_stream_dot(uint8_t *ring, const uint8_t *src
     for (int j = 0; j < NB; j++)
 #pragma unroll
         for (int k = 0; k < 4; k++) acc[j][k] = 0;
-    int st = 0;   // ring stage of chunk c
 #pragma unroll 1
     for (int c = 0; c < nch; c++) {
         cp_async_wait<kDecStages - 2>();
-        const uint4 wv = *reinterpret_cast<const uint4 *>(ring + st * 512);
-        const int cn = c + kDecStages - 1;
-        const int sn = st == 0 ? kDecStages - 1 : st - 1;   // stage of chunk c-1, now free
-        if (cn < nch) cp_async16(ring + sn * 512, src + (size_t)cn * 512, true);
-        cp_async_commit();
-        st = st == kDecStages - 1 ? 0 : st + 1;
+        const uint4 wv = *reinterpret_cast<const uint4 *>(ws.ring + cst * 512);
+        cst = cst == kDecStages - 1 ? 0 : cst + 1;
+        ws.issue();
+        advance();
         const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
         uint32_t pw[16];
 #pragma unroll
@@ -492,44 +508,82 @@ __device__ __forceinline__ void dec_stream_dot(uint8_t *ring, const uint8_t *src
                         : 0;
 }
 
-__device__ __forceinline__ void dec_stream_dot_any(int nbp, uint8_t *ring, const uint8_t *src, int nch, const uint4 *x,
-                                                   int ld16, int (&tot)[kGemvTokens])
+// Eight tokens: byte planes by shift and mask (two ops for k > 0) into a single
+// accumulator per token, which keeps the eight accumulators in registers.
+template <class Adv>
+__device__ __forceinline__ void dec_stream_dot8(DecStream &ws, int &cst, int nch, const uint4 *x, int ld16, Adv &advance,
+                                                int (&tot)[kGemvTokens])
+{
+#pragma unroll
+    for (int j = 0; j < kGemvTokens; j++) tot[j] = 0;
+#pragma unroll 1
+    for (int c = 0; c < nch; c++) {
+        cp_async_wait<kDecStages - 2>();
+        const uint4 wv = *reinterpret_cast<const uint4 *>(ws.ring + cst * 512);
+        cst = cst == kDecStages - 1 ? 0 : cst + 1;
+        ws.issue();
+        advance();
+        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int w = 0; w < 4; w++) {
+            uint32_t pw[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) pw[k] = plane(w4[w], k);
+#pragma unroll
+            for (int j = 0; j < kGemvTokens; j++) {
+                const uint4 xv = x[j * ld16 + 4 * c + w];
+                tot[j] = dp4a_us(pw[0], xv.x, tot[j]);
+                tot[j] = dp4a_us(pw[1], xv.y, tot[j]);
+                tot[j] = dp4a_us(pw[2], xv.z, tot[j]);
+                tot[j] = dp4a_us(pw[3], xv.w, tot[j]);
+            }
+        }
+    }
+}
+
+template <class Adv>
+__device__ __forceinline__ void dec_stream_dot_any(int nbp, DecStream &ws, int &cst, int nch, const uint4 *x, int ld16,
+                                                   Adv &advance, int (&tot)[kGemvTokens])
 {
     switch (nbp) {
-    case 1: dec_stream_dot<1>(ring, src, nch, x, ld16, tot); break;
-    case 2: dec_stream_dot<2>(ring, src, nch, x, ld16, tot); break;
-    case 4: dec_stream_dot<4>(ring, src, nch, x, ld16, tot); break;
-    default: dec_stream_dot<8>(ring, src, nch, x, ld16, tot); break;
+    case 1: dec_stream_dot<1>(ws, cst, nch, x, ld16, advance, tot); break;
+    case 2: dec_stream_dot<2>(ws, cst, nch, x, ld16, advance, tot); break;
+    case 4: dec_stream_dot<4>(ws, cst, nch, x, ld16, advance, tot); break;
+    default: dec_stream_dot8(ws, cst, nch, x, ld16, advance, tot); break;
     }
 }
 
-// Relative cost of one work item of an expert with c tokens: per batch of up to
-// 8 tokens, the item's chunks per warp times the instructions per chunk (a
-// fixed part and one per padded token), plus a fixed part per batch.  Only the
-// split of the items over the CTAs depends on it.
-__device__ __forceinline__ int dec_item_cost(int c, int nch)
+// Item m of a compute group's queue (all 32 lanes of a warp call it).  With
+// claim, the warp takes the next global item (lane 0, atomically; n_tot once
+// all are taken) and appends it; otherwise it waits (bounded, 2 s; n_tot and
+// the device flag on expiry) until the claiming warp has appended item m.
+// Out of line: it runs once per item, and keeps the dot loop's registers free.
+__device__ __noinline__ int dec_queue_item(DecQueue *qp, int m, bool claim, int n_tot, int *ctr, unsigned *flag)
 {
-    int cost = 0;
-    for (int b0 = 0; b0 < c; b0 += kGemvTokens) {
-        const int nbp = dec_pad_tokens(min(kGemvTokens, c - b0));
-        cost += nch * (6 + 20 * nbp) + 400;
+    volatile DecQueue *q = qp;
+    const int lane = threadIdx.x & 31;
+    if (claim) {
+        int x = 0;
+        if (lane == 0) {
+            x = min(atomicAdd(ctr, 1), n_tot);
+            q->item[m & (kDecQueue - 1)] = x;
+            __threadfence_block();
+            q->n = m + 1;
+        }
+        return __shfl_sync(FULL, x, 0);
     }
-    return cost;
-}
-
-// First item whose cumulative cost start is >= target; pref[ai] is the cost of
-// the items of active experts before ai (per_exp items of equal cost each).
-__device__ __forceinline__ int dec_item_at(const int *pref, int n_active, int per_exp, int64_t target)
-{
-    if (target >= pref[n_active]) return n_active * per_exp;
-    int lo = 0, hi = n_active - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pref[mid] <= target) lo = mid;
-        else hi = mid - 1;
+    if (q->n <= m) {
+        const uint64_t t0 = global_timer_ns();
+        while (q->n <= m) {
+            __nanosleep(64);
+            if (global_timer_ns() - t0 > 2000000000ull) {
+                if (lane == 0) set_flag(flag, MAPLE_DEVFLAG_TIMEOUT);
+                return n_tot;
+            }
+        }
     }
-    const int w = (pref[lo + 1] - pref[lo]) / per_exp;
-    return lo * per_exp + (int)((target - pref[lo] + w - 1) / w);
+    __threadfence_block();
+    return q->item[m & (kDecQueue - 1)];
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeArgs d)
@@ -539,7 +593,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     uint8_t *wring = dsm;                                                         // [group][warp][stage][512]
     uint8_t *aring = wring + kDecRingBytes;                                       // [group][2][aslot]
     DecActMeta *ameta = (DecActMeta *)(aring + (size_t)kDecGroups * 2 * d.aslot_bytes);   // [group][2]
-    DecRecord *recs = (DecRecord *)(ameta + kDecGroups * 2);                      // [group][kDecRec]
+    DecQueue *queue = (DecQueue *)(ameta + kDecGroups * 2);                       // [group]
+    DecRecord *recs = (DecRecord *)(queue + kDecGroups);                          // [group][kDecRec]
     uint64_t *bars = (uint64_t *)(((uintptr_t)(recs + kDecGroups * kDecRec) + 7) & ~(uintptr_t)7);
     // bars: afull[G][2], aempty[G][2], hfull[G][2], rfull[G][R], rempty[G][R]
     const uint32_t b_afull = (uint32_t)__cvta_generic_to_shared(bars), b_aempty = b_afull + 8 * 2 * kDecGroups;
@@ -559,7 +614,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     int *t_sumx = (int *)(t_sx + T);
     int *t_misc = t_sumx + T;   // [0] n_active
     unsigned long long *tmask = (unsigned long long *)(((uintptr_t)(t_misc + 48) + 7) & ~(uintptr_t)7);
-    int *t_pg = (int *)(tmask + E), *t_pd = t_pg + E + 1;
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) {
@@ -568,6 +622,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (threadIdx.x < kDecGroups * 2) ameta[threadIdx.x].done = 0u;
+    if (threadIdx.x < kDecGroups) queue[threadIdx.x].n = 0;
 
     // ---------------- prologue: the permutation of the T*K slots (T <= 64), from the
     // router's choices: a token bitmask per expert gives the counts, and a slot's
@@ -653,57 +708,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     const int n_active = t_misc[0];
     const int Cg = a.D / 64, Cd = a.F / 64;
     const int gitems = a.F / 128, ditems = a.D / 256;   // items per expert (8 row groups each)
-    // split each kind of item over the CTAs in equal shares of estimated cost
-    if (warp == 0) {
-        const int per = (n_active + 31) / 32, a0 = lane * per;
-        int sg = 0, sd = 0;
-        for (int i = 0; i < per; i++)
-            if (a0 + i < n_active) {
-                const int c = t_cnt[t_act[a0 + i]];
-                sg += gitems * dec_item_cost(c, Cg);
-                sd += ditems * dec_item_cost(c, Cd);
-            }
-        int cg = sg, cd = sd;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(FULL, cg, o), w = __shfl_up_sync(FULL, cd, o);
-            if (lane >= o) {
-                cg += v;
-                cd += w;
-            }
-        }
-        int og = cg - sg, od = cd - sd;
-        for (int i = 0; i < per; i++)
-            if (a0 + i < n_active) {
-                const int c = t_cnt[t_act[a0 + i]];
-                t_pg[a0 + i] = og;
-                t_pd[a0 + i] = od;
-                og += gitems * dec_item_cost(c, Cg);
-                od += ditems * dec_item_cost(c, Cd);
-            }
-        if (lane == 31) {
-            t_pg[n_active] = cg;
-            t_pd[n_active] = cd;
-        }
-    }
     __syncthreads();
-    const int64_t WG = t_pg[n_active], WD = t_pd[n_active];
-    const int g0 = dec_item_at(t_pg, n_active, gitems, WG * blockIdx.x / gridDim.x);
-    const int g1 = dec_item_at(t_pg, n_active, gitems, WG * (blockIdx.x + 1) / gridDim.x);
-    const int d0 = dec_item_at(t_pd, n_active, ditems, WD * blockIdx.x / gridDim.x);
-    const int d1 = dec_item_at(t_pd, n_active, ditems, WD * (blockIdx.x + 1) / gridDim.x);
-    const int nG = g1 - g0, n_items = nG + (d1 - d0);
-    // item i of this CTA -> kind (0 gate/up, 1 down), active index, sub-item
-    auto item_of = [&](int i, int &kind, int &ai, int &sub) {
-        if (i < nG) {
+    const int n_g = n_active * gitems, n_tot = n_g + n_active * ditems;
+    // global item id x -> kind (0 gate/up, 1 down), active index, sub-item
+    auto item_of = [&](int x, int &kind, int &ai, int &sub) {
+        if (x < n_g) {
             kind = 0;
-            ai = (g0 + i) / gitems;
-            sub = (g0 + i) % gitems;
+            ai = x / gitems;
+            sub = x % gitems;
         } else {
             kind = 1;
-            ai = (d0 + i - nG) / ditems;
-            sub = (d0 + i - nG) % ditems;
+            ai = (x - n_g) / ditems;
+            sub = (x - n_g) % ditems;
         }
+    };
+    auto q_get = [&](int g, int m) -> int {
+        return dec_queue_item(queue + g, m, false, n_tot, d.item_ctr, a.flag_dev);
     };
 
     if (warp < kDecGroups) {
@@ -711,9 +731,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
         const int g = warp;
         int k = 0, kh0 = 0, kh1 = 0;   // batches staged; down batches staged per buffer
         bool ok = true;
-        for (int i = g; i < n_items && ok; i += kDecGroups) {
+        for (int m = 0; ok; m++) {
+            const int x = q_get(g, m);
+            if (x >= n_tot) break;
             int kind, ai, sub;
-            item_of(i, kind, ai, sub);
+            item_of(x, kind, ai, sub);
             const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
             if (kind == 1) {
                 // every gate/up item of expert e must be done before its h rows are read
@@ -834,9 +856,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
         const int g = warp - kDecGroups;
         const int nblk = a.D / 256;
         int r = 0;
-        for (int i = g; i < n_items; i += kDecGroups) {
+        for (int m = 0;; m++) {
+            const int x = q_get(g, m);
+            if (x >= n_tot) break;
             int kind, ai, sub;
-            item_of(i, kind, ai, sub);
+            item_of(x, kind, ai, sub);
             const int cnt = a.counts[a.active[ai]];
             bool ok = true;
             for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, r++) {
@@ -902,24 +926,60 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
 
     // ---------------- compute warp gw of group g: row group gw of every item of the group
     const int g = (warp - kDecFirstCompute) / kDecGroupWarps, gw = (warp - kDecFirstCompute) % kDecGroupWarps;
-    uint8_t *ring = wring + (size_t)((g * kDecGroupWarps + gw) * kDecStages) * 512 + lane * 16;
-    int k = 0;   // batches of this group (= completion record index)
-    for (int i = g; i < n_items; i += kDecGroups) {
+    // the issue cursor: item ws.item, batches left ws.left, chunk ws.c of its row group
+    DecStream ws;
+    ws.ring = wring + (size_t)((g * kDecGroupWarps + gw) * kDecStages) * 512 + lane * 16;
+    ws.st = 0;
+    ws.c = 0;
+    auto seg_of = [&](int x, const uint8_t *&src, int &nch, int &nbat) {
         int kind, ai, sub;
-        item_of(i, kind, ai, sub);
+        item_of(x, kind, ai, sub);
+        const int e = a.active[ai], grp = sub * kDecGroupWarps + gw;
+        nch = kind == 0 ? Cg : Cd;
+        nbat = (a.counts[e] + kGemvTokens - 1) / kGemvTokens;
+        src = (kind == 0 ? a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)grp * Cg * 512
+                         : a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)grp * Cd * 512) +
+              lane * 16;
+    };
+    // warp 0 of the group claims the items as its issue cursor reaches them; the
+    // other warps take them from the queue
+    auto next_item = [&](int m) -> int {
+        return dec_queue_item(queue + g, m, gw == 0, n_tot, d.item_ctr, a.flag_dev);
+    };
+    ws.item = 0;   // ordinal of the issue cursor's item in the group's queue
+    ws.left = 0;
+    {
+        const int x = next_item(0);
+        if (x < n_tot) seg_of(x, ws.src, ws.nch, ws.left);
+    }
+    auto advance = [&]() {
+        if (ws.left <= 0) return;
+        if (++ws.c < ws.nch) return;
+        ws.c = 0;
+        if (--ws.left > 0) return;   // next batch of the same item: the same chunks again
+        const int x = next_item(++ws.item);
+        if (x < n_tot) seg_of(x, ws.src, ws.nch, ws.left);
+    };
+    for (int s = 0; s < kDecStages - 1; s++) {
+        ws.issue();
+        advance();
+    }
+    int cst = 0;   // ring stage of the next chunk to use
+    int k = 0;     // batches of this group (= completion record index)
+    for (int m = 0;; m++) {
+        const int x = q_get(g, m);   // already claimed: this warp's issue cursor is past it
+        if (x >= n_tot) break;
+        int kind, ai, sub;
+        item_of(x, kind, ai, sub);
         const int e = a.active[ai], cnt = a.counts[e], base = a.offsets[e];
         const int grp = sub * kDecGroupWarps + gw;   // row group (32 rows) within the expert
         const int nch = kind == 0 ? Cg : Cd;
-        const uint8_t *src = kind == 0
-                                 ? a.w_gu + (size_t)e * gu_bytes_per_expert(a.D, a.F) + (size_t)grp * Cg * 512 + lane * 16
-                                 : a.w_dn + (size_t)e * dn_bytes_per_expert(a.D, a.F) + (size_t)grp * Cd * 512 + lane * 16;
         // the row scale: gate/up lanes 0..15 gate rows grp*16+l, lanes 16..31 the up rows of
         // the same outputs; down lane l channel grp*32+l
         const float al = kind == 0 ? __ldg((lane < 16 ? a.alpha_gate : a.alpha_up) + (size_t)e * a.F + grp * 16 + (lane & 15))
                                    : __ldg(a.alpha_down + (size_t)e * a.D + grp * 32 + lane);
         for (int b0 = 0; b0 < cnt; b0 += kGemvTokens, k++) {
             const int buf = k & 1;
-            dec_stream_start(ring, src, nch);   // the codes stream in while the activations are awaited
             if (!dec_wait(b_afull + 8 * (2 * g + buf), (k >> 1) & 1)) {
                 if (lane == 0) set_flag(a.flag_dev, MAPLE_DEVFLAG_TIMEOUT);
                 cp_async_wait<0>();
@@ -930,11 +990,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
             const int nb = am->nb;
             int tot[kGemvTokens];
             if (kind == 0)
-                dec_stream_dot_any(dec_pad_tokens(nb), ring, src, nch, reinterpret_cast<const uint4 *>(ab), a.D / 16,
-                                   tot);
+                dec_stream_dot_any(dec_pad_tokens(nb), ws, cst, nch, reinterpret_cast<const uint4 *>(ab), a.D / 16,
+                                   advance, tot);
             else
-                dec_stream_dot_any(dec_pad_tokens(nb), ring, src, nch, reinterpret_cast<const uint4 *>(ab + qh_off),
-                                   a.F / 16, tot);
+                dec_stream_dot_any(dec_pad_tokens(nb), ws, cst, nch, reinterpret_cast<const uint4 *>(ab + qh_off),
+                                   a.F / 16, advance, tot);
             if (kind == 0) {
                 const bool is_up = lane >= 16;
                 const int rr = grp * 16 + (lane & 15);
@@ -988,6 +1048,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
             }
         }
     }
+    cp_async_wait<0>();
 }
 
 }  // namespace maple

@@ -279,7 +279,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     size_t o_ye = ar.take(S * D * 4);
     size_t o_ctr = ar.take(0);
     size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4), o_ec = ar.take(E * 4);
-    size_t o_cc = ar.take(Tm * (D / 32) * 4), o_rdy = ar.take(E * 4);
+    size_t o_cc = ar.take(Tm * (D / 32) * 4), o_rdy = ar.take((E + 1) * 4);
     size_t o_xn = ar.take(Tm * D * 2);
     size_t o_zr = ar.take(D > F * 4 ? D : F * 4);   // a row of zeros (padding rows of the decode kernel)
 
@@ -550,6 +550,7 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         d.arrive = h->arrive;
         d.aslot_bytes = dec_aslot_bytes(h->D, h->F);
         d.zrow = h->zrow;
+        d.item_ctr = (int *)(h->arrive + h->E);
         d.topk_idx = h->topk_idx;
         d.topk_w = h->topk_w;
         if (taps) {
@@ -663,8 +664,8 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
     const int nw = tc ? 0 : decode_ring_slots(h, T);
     stage_event(h, 0, st);
     // the persistent decode kernel builds its own permutation from the top-k; the
-    // routing kernel zeroes its arrival counters
-    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, false, st, h->arrive, h->E)
+    // routing kernel zeroes its arrival counters and its work-item counter
+    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, false, st, h->arrive, h->E + 1)
                 : run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, false, st);
     if (rc) return rc;
     stage_event(h, 1, st);

@@ -41,6 +41,16 @@ struct RouteArgs {
     unsigned *flag;
 };
 
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
+    const int n = pred ? 16 : 0;   // zero-fill when out of range
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // ---------------------------------------------------------------------------
 // block-wide exclusive scan of one int per thread (blockDim multiple of 32)
 // ---------------------------------------------------------------------------
@@ -396,10 +406,19 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
         w0[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane));
         w1[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane + 4));
     }
-    // stage the token rows
-    const int row8 = a.D / 8;
-    for (int i = threadIdx.x; i < nt * row8; i += blockDim.x)
-        reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D) + i);
+    // stage the token rows (nt * D/8 16-byte units, at most NI per thread) with
+    // asynchronous copies, all in flight at once
+    {
+        const int n16 = nt * (a.D / 8);
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D);
+#pragma unroll
+        for (int i = 0; i < NI; i++) {
+            const int idx = threadIdx.x + 256 * i;
+            if (idx < n16) cp_async16(reinterpret_cast<uint4 *>(xs) + idx, src + idx, true);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+    }
     __syncthreads();
 
     if (eb == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
@@ -596,15 +615,6 @@ __device__ __forceinline__ void tree_level(float (&v)[64], int off, bool upper)
     }
 }
 
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred)
-{
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem);
-    const int n = pred ? 16 : 0;   // zero-fill when out of range
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // dynamic shared memory: two stages of (32 token rows x 256 bf16, 16 router rows x 256 fp32)
 constexpr int kRgStage = kRgTok * 256 * 2 + kRgExp * 256 * 4;

@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, MAPLE_GEMV_MINB) down_gemv_ke
 // ---------------------------------------------------------------------------
 // Persistent expert-stage kernel for decode batches (T <= 64).
 //
-// Grid = one CTA per SM, launched cooperatively (all CTAs resident).  Every
+// Grid = one CTA per SM (a plain launch: no CTA waits on work of a CTA that
+// has not started, so residency of the whole grid is not needed).  Every
 // CTA first builds the permutation of all T*K slots for itself from the
 // router's top-k (in shared memory), so no routing step needs a grid-wide
 // hand-off.  Work items: gate/up items (active expert, 8 groups of 16 gate +

@@ -542,7 +542,7 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
     }
     g.flag_dev = h->flag_dev;
     if (nw) {
-        // persistent, cooperative: one CTA per SM builds the permutation from
+        // persistent: one CTA per SM builds the permutation from
         // the router's top-k, then streams gate/up and down
         DecodeArgs d;
         memset(&d, 0, sizeof d);
@@ -558,19 +558,11 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
             d.tap_offsets = taps->expert_offsets;
             d.tap_perm = taps->perm;
         }
-        // h->arrive was zeroed by the routing kernel
-        cudaLaunchConfig_t lc;
-        memset(&lc, 0, sizeof lc);
-        lc.gridDim = dim3(h->num_sms);
-        lc.blockDim = dim3(kDecThreads);
-        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E);
-        lc.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        lc.attrs = attr;
-        lc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&lc, decode_experts_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+        // h->arrive and the item counter were zeroed by the routing kernel.  A plain
+        // launch: the kernel needs no co-residency, since a CTA only ever waits on
+        // items that running CTAs have already claimed (gate/up items, all claimed
+        // before any down item, wait on nothing of other CTAs).
+        decode_experts_kernel<<<h->num_sms, kDecThreads, decode_smem_bytes(h->D, h->F, T, h->K, h->E), st>>>(d);
         stage_event(h, 2, st);
         stage_event(h, 3, st);
         return launch_status();

@@ -400,8 +400,8 @@ static int take_flag(maple_moe_t h)
 
 // routing stage: quantise, logits, top-k (+ the permutation)
 static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
-                     float *out_w, int32_t *out_counts, bool permute, bool pieces, bool logits_only,
-                     cudaStream_t st, unsigned *clear = nullptr, int n_clear = 0)
+                     float *out_w, int32_t *out_counts, bool permute, bool pieces, cudaStream_t st,
+                     unsigned *clear = nullptr, int n_clear = 0)
 {
     RouteArgs a;
     memset(&a, 0, sizeof a);
@@ -443,17 +443,11 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     const bool small = T <= kRouteSmallT;
     const bool fused = small && permute && !pieces && (int64_t)T * h->E <= kFusedMarkBytes;
     a.fuse_permute = fused ? 1 : 0;
-    a.logits_only = logits_only ? 1 : 0;
     if (clear && !small) {
         if (cudaMemsetAsync(clear, 0, (size_t)n_clear * 4, st) != cudaSuccess) return MAPLE_ERR_CUDA;
     } else {
         a.clear = clear;
         a.n_clear = n_clear;
-    }
-    if (logits_only) {
-        dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
-        pick_route(h->D, h->E)<<<grid, 256, route_smem_bytes(h->D), st>>>(a);
-        return launch_status();
     }
     if (small) {
         dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
@@ -597,7 +591,7 @@ extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int3
     if (!x || !aligned16(x)) return MAPLE_ERR_INVALID_ARG;
     for (const void *p : {(const void *)topk_idx, (const void *)topk_w, (const void *)expert_counts})
         if (p && !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
-    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr, false, false,
+    return run_route(h, x, T, nullptr, topk_idx, topk_w, expert_counts, expert_counts != nullptr, false,
                      (cudaStream_t)stream);
 }
 
@@ -657,8 +651,8 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
     stage_event(h, 0, st);
     // the persistent decode kernel builds its own permutation from the top-k; the
     // routing kernel zeroes its arrival counters and its work-item counter
-    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, false, st, h->arrive, h->E + 1)
-                : run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, false, st);
+    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, st, h->arrive, h->E + 1)
+                : run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, st);
     if (rc) return rc;
     stage_event(h, 1, st);
     return tc ? run_experts_tc(h, T, y, resid, taps, st) : run_experts(h, T, y, resid, taps, nw, st);
@@ -820,7 +814,7 @@ extern "C" int maple_moe_route_noalloc(const uint16_t *x, int32_t T, int32_t d_m
         !aligned16(topk_w) || (router_bias && !aligned16(router_bias)) || (expert_counts && !aligned16(expert_counts)))
         return MAPLE_ERR_INVALID_ARG;
 
-    const int64_t D = d_model, E = n_experts, K = top_k, S = (int64_t)T * top_k;
+    const int64_t D = d_model, E = n_experts, S = (int64_t)T * top_k;
     Arena ar;
     const size_t o_lg = ar.take(T * E * 4), o_qx = ar.take(T * D), o_sx = ar.take(T * 4), o_sumx = ar.take(T * 4);
     const size_t o_ti = ar.take(S * 4), o_tw = ar.take(S * 4), o_cnt = ar.take(E * 4), o_off = ar.take((E + 1) * 4);

@@ -33,7 +33,6 @@ struct RouteArgs {
     unsigned *tg_cnt, *glob_cnt;
     // permutation (filled by the last CTA when fuse_permute)
     int fuse_permute;
-    int logits_only;   // stop after the logits and the int8 codes (top-k is done by the consumer)
     unsigned *clear;   // [n_clear] counters of the next kernel, zeroed by CTA (0, 0) (may be null)
     int n_clear;
     int *counts, *offsets, *perm, *inv, *active, *n_active;
@@ -226,88 +225,6 @@ __device__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, in
     my_w = __fdiv_rn(ek, S);
 }
 
-// Top-k of NT rows at once in one warp (the rows' chains interleave, which
-// hides the shuffle latency); row r < nrows at rows[r].  Lane k < K ends with
-// row r's k-th choice in my_e[r] and its softmax weight in my_w[r].  Same
-// ranking, tie rule and softmax as topk_row_warp.
-template <int NPER, int NT>
-__device__ void topk_rows_warp(const float *const (&rows)[NT], int nrows, int E, int K, unsigned *flag,
-                               int (&my_e)[NT], float (&my_w)[NT])
-{
-    const int lane = threadIdx.x & 31;
-    float lv[NT][NPER];
-    bool nan_seen = false;
-#pragma unroll
-    for (int r = 0; r < NT; r++)
-#pragma unroll
-        for (int j = 0; j < NPER; j++) {
-            const int e = lane + 32 * j;
-            float v = -INFINITY;
-            if (r < nrows && e < E) {
-                v = __ldcg(rows[r] + e);
-                if (isnan(v)) {
-                    nan_seen = true;
-                    v = -INFINITY;
-                }
-            }
-            lv[r][j] = v;
-        }
-    if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
-    uint32_t taken[NT];
-    float my_v[NT];
-#pragma unroll
-    for (int r = 0; r < NT; r++) {
-        taken[r] = 0;
-        my_v[r] = 0.0f;
-        my_e[r] = 0;
-    }
-    for (int k = 0; k < K; k++) {
-        float bv[NT];
-        int be[NT];
-#pragma unroll
-        for (int r = 0; r < NT; r++) {
-            bv[r] = -INFINITY;
-            be[r] = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < NPER; j++) {
-                const int e = lane + 32 * j;
-                if (e < E && !((taken[r] >> j) & 1u) && ranks_before(lv[r][j], e, bv[r], be[r])) {
-                    bv[r] = lv[r][j];
-                    be[r] = e;
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-#pragma unroll
-            for (int r = 0; r < NT; r++) {
-                const float ov = __shfl_xor_sync(FULL, bv[r], o);
-                const int oe = __shfl_xor_sync(FULL, be[r], o);
-                if (ranks_before(ov, oe, bv[r], be[r])) {
-                    bv[r] = ov;
-                    be[r] = oe;
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < NT; r++) {
-            if ((be[r] & 31) == lane) taken[r] |= 1u << (be[r] >> 5);
-            if (lane == k) {
-                my_v[r] = bv[r];
-                my_e[r] = be[r];
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < NT; r++) {
-        const float l0 = __shfl_sync(FULL, my_v[r], 0);
-        const float ek = exp_ref(__fsub_rn(my_v[r], l0));
-        float S = 0.0f;
-        for (int k = 0; k < K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
-        my_w[r] = __fdiv_rn(ek, S);
-    }
-}
-
 template <int NPER>
 __device__ void topk_token_warp(const RouteArgs &a, int t)
 {
@@ -443,8 +360,6 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
             if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = v;
         }
     }
-
-    if (a.logits_only) return;
 
     // ---- last CTA of this token group: top-k + softmax
     fence_gpu();

@@ -8,8 +8,10 @@ and 64 (105 tokens).  A step is one forward pass of the whole layer (routing,
 permutation, gate/up, down, combine) for each of the four batches.  Before
 every forward pass L2 is flushed (a 256 MB write, outside the timed events),
 so the weights come from HBM.  Each forward is a replay of a CUDA graph of the
-library call, timed with CUDA events on its stream (the library records
-per-stage events inside the graph); the step time is their sum.  value = tokens per second over all ranks.
+library call (its two kernels), timed with CUDA events on its stream; the step
+time is their sum.  value = tokens per second over all ranks.  The per-stage
+split (routing / experts) comes from a second set of graphs that also record
+the library's stage events, replayed after the timed region.
 
 The JSON line adds: roofline (dominant kernel vs measured HBM bandwidth),
 cpu_baseline (the CPU oracle timed on a sample), e2e (host buffers with the
@@ -204,16 +206,24 @@ def run_gpu(args, rank: int, world: int):
         for e in ev[T]:
             e.record(stream)
     torch.cuda.synchronize(dev)
-    graphs = {}
+    # Two graphs per batch size: the timed one holds only the library's kernels;
+    # the second also records the per-stage events (an event between the routing
+    # and the expert kernel would keep them from overlapping their launch) and
+    # gives the stage split after the timed region.
+    graphs, split_graphs = {}, {}
     for T in DECODE_T:
-        tw.maple_moe_set_stage_events(layer.handle, ev[T])
         layer.forward(xs[T], y=ys[T])          # warm the path before capture
         torch.cuda.synchronize(dev)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             layer.forward(xs[T], y=ys[T])
         graphs[T] = g
-    tw.maple_moe_set_stage_events(layer.handle, None)
+        tw.maple_moe_set_stage_events(layer.handle, ev[T])
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer.forward(xs[T], y=ys[T])
+        split_graphs[T] = g
+        tw.maple_moe_set_stage_events(layer.handle, None)
     torch.cuda.synchronize(dev)
 
     e_beg = {T: torch.cuda.Event(enable_timing=True) for T in DECODE_T}
@@ -221,7 +231,6 @@ def run_gpu(args, rank: int, world: int):
     stages_in_graph = True
 
     def one_step(timed: list | None):
-        nonlocal stages_in_graph
         for T in DECODE_T:
             flush.fill_(1.0)
             e_beg[T].record(stream)
@@ -229,14 +238,22 @@ def run_gpu(args, rank: int, world: int):
             e_end[T].record(stream)
             if timed is not None:
                 torch.cuda.synchronize(dev)
-                total = e_beg[T].elapsed_time(e_end[T])
-                st = None
-                if stages_in_graph:
-                    try:
-                        st = [ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)]
-                    except Exception:
-                        stages_in_graph = False
-                timed.append((T, total, st))
+                timed.append((T, e_beg[T].elapsed_time(e_end[T]), None))
+
+    def split_step():
+        """Stage times (route, gate/up, experts end) from the graphs with events."""
+        nonlocal stages_in_graph
+        out = {}
+        for T in DECODE_T:
+            flush.fill_(1.0)
+            split_graphs[T].replay()
+            torch.cuda.synchronize(dev)
+            try:
+                out[T] = [ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)]
+            except Exception:
+                stages_in_graph = False
+                return None
+        return out
 
     for _ in range(args.warmup):
         one_step(None)
@@ -255,7 +272,19 @@ def run_gpu(args, rank: int, world: int):
     torch.cuda.synchronize(dev)
     clocks = clk.stop()
 
-    if not stages_in_graph or any(t[2] is None for t in timed):
+    # stage split: the same number of forwards again, from the graphs with events
+    split = {T: [] for T in DECODE_T}
+    for _ in range(args.steps):
+        sp = split_step()
+        if sp is None:
+            break
+        for T in DECODE_T:
+            split[T].append(sp[T])
+    if stages_in_graph:
+        stage_src = "events inside a second set of graphs (untimed replays)"
+        timed = [(T, tot, split[T][n % len(split[T])]) for n, (T, tot, _) in enumerate(timed)]
+
+    if not stages_in_graph:
         # stage split from host-launched forwards instead (same kernels, stage events on the stream)
         stage_src = "host-launched forwards"
         split = {T: [] for T in DECODE_T}
@@ -269,8 +298,6 @@ def run_gpu(args, rank: int, world: int):
                 split[T].append([ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)])
         tw.maple_moe_set_stage_events(layer.handle, None)
         timed = [(T, tot, split[T][n % len(split[T])]) for n, (T, tot, _) in enumerate(timed)]
-    else:
-        stage_src = "events inside the graph"
 
     total_ms = sum(t[1] for t in timed)
     per_T = {T: [t[2] for t in timed if t[0] == T] for T in DECODE_T}

@@ -624,6 +624,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_experts_kernel(DecodeAr
     }
     if (threadIdx.x < kDecGroups * 2) ameta[threadIdx.x].done = 0u;
     if (threadIdx.x < kDecGroups) queue[threadIdx.x].n = 0;
+    // The kernel may be launched while the routing kernel still runs (programmatic
+    // dependent launch): nothing it writes is read before this point.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // ---------------- prologue: the permutation of the T*K slots (T <= 64), from the
     // router's choices: a token bitmask per expert gives the counts, and a slot's

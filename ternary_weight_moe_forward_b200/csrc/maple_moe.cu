@@ -556,7 +556,21 @@ static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const
         // launch: the kernel needs no co-residency, since a CTA only ever waits on
         // items that running CTAs have already claimed (gate/up items, all claimed
         // before any down item, wait on nothing of other CTAs).
-        decode_experts_kernel<<<h->num_sms, kDecThreads, decode_smem_bytes(h->D, h->F, T, h->K, h->E), st>>>(d);
+        // Launched as a programmatic dependent of the routing kernel before it: its
+        // launch and set-up overlap the router's tail, and griddepcontrol.wait in
+        // the kernel orders every read of the routing outputs after that grid.
+        cudaLaunchConfig_t lc;
+        memset(&lc, 0, sizeof lc);
+        lc.gridDim = dim3(h->num_sms);
+        lc.blockDim = dim3(kDecThreads);
+        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E);
+        lc.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        if (cudaLaunchKernelEx(&lc, decode_experts_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
         stage_event(h, 2, st);
         stage_event(h, 3, st);
         return launch_status();

@@ -312,6 +312,9 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
     const int t0 = tg * kRouteTokens;
     const int nt = min(kRouteTokens, a.T - t0);
     const int e = eb * kRouteExperts + warp;
+    // let a kernel launched after this one as a programmatic dependent start its
+    // set-up now (it waits for this grid's completion before reading any output)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (a.clear && eb == 0 && tg == 0)
         for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
 

@@ -12,12 +12,12 @@
  *  - Ternary linear layers: every weight is one of {-alpha, 0, +alpha} with one
  *    alpha per output row, so a product becomes add (+alpha), subtract
  *    (-alpha) or skip (0).  ("linlog.top/article/1232", section
- *    三值权重：把乘法变成加法; the model table in section 架构设计 gives
- *    "2-bit ternary, one alpha per row".)  Here the accumulation over the input
+ *    三值权重; its model table in section 架构设计 lists the weights as
+ *    2-bit ternary with one alpha per row.)  Here the accumulation over the input
  *    dimension is done in int32 on int8 activation codes and the scales are
  *    applied afterwards.
  *  - Routing: every token scores all experts and keeps the top-8 of 256
- *    (same page, 架构设计 table: "Top-K 路由 Top-8", 256 experts).
+ *    (same page, 架构设计 table: top-8 routing over 256 experts).
  *  - Everything the pages leave open (SwiGLU expert MLP, the per-token int8
  *    absmax quantiser, fp32 router, rounding and summation orders, exp, the
  *    2-bit code map) follows one fixed reading, stated at each function.

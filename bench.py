@@ -14,9 +14,13 @@ split (routing / experts) comes from a second set of graphs that also record
 the library's stage events, replayed after the timed region.
 
 The JSON line adds: roofline (dominant kernel vs measured HBM bandwidth),
-cpu_baseline (the CPU oracle timed on a sample), e2e (host buffers with the
-copies inside the timed region), clocks sampled during the timed region, and
-gpu_launches.
+cpu_baseline (the CPU oracle timed on a sample, pinned to one host core),
+e2e (host buffers with the copies inside the timed region), clocks sampled
+during the timed region, gpu_launches, and per_config: the other workloads
+of the layer, each timed the same way (CUDA graph replays, L2 flushed before
+each, CUDA events on the stream): prefill T = 4096 (tensor-core path, with
+its grouped GEMMs against the int8 tensor peak), the skewed-routing layer at
+T = 16384, the 24-layer stack at T = 1 and 32, and the tiny layer.
 
 With N > 1 every rank runs its own replica on its own tokens (the layer
 shards by tokens with no exchange): scaling is weak, timing is the max over
@@ -49,6 +53,17 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def int8_peak_tops():
+    """Dense int8 tensor peak, TOPS: the measured bf16 burst GEMM rate times the
+    nominal int8 : bf16 ratio of the part (4.5 : 2.25 PFLOP/s = 2)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return 2.0 * float(p["bf16_tflops"]), "2 x measured bf16 burst (nominal int8:bf16 = 2)"
+    except Exception:
+        return 2.0 * 1590.0, "2 x fallback bf16 1590 TFLOP/s (nominal int8:bf16 = 2)"
 
 
 # ---------------------------------------------------------------------------- clocks
@@ -174,6 +189,194 @@ def experts_bytes(n_active: int, T: int) -> int:
     return n_active * (3 * F * D // 4 + (2 * F + D) * 4) + T * D + T * D * 4
 
 
+
+def expected_experts(T: int, E: int = 256, K: int = 8) -> float:
+    """Expected number of distinct experts a batch of T tokens touches under
+    uniform routing."""
+    return E * (1.0 - ((E - K) / E) ** T)
+
+
+def prefill_ops(S: int, D: int = 2048, F: int = 512) -> tuple[int, int]:
+    """int8 operations (2 per multiply-add) of the two grouped GEMMs for S slots."""
+    return 2 * S * (2 * F) * D, 2 * S * D * F
+
+
+class GraphTimer:
+    """One library call captured as a CUDA graph (plus a second capture that
+    also records the library's stage events), replayed after an L2 flush and
+    timed with CUDA events on the stream."""
+
+    def __init__(self, fn, stream, flush, set_events=None, n_events: int = 4):
+        import torch
+        self.torch, self.stream, self.flush = torch, stream, flush
+        fn()
+        torch.cuda.synchronize()
+        # captured on torch's capture stream (fn reads torch's current stream),
+        # replayed on `stream`
+        self.g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g):
+            fn()
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_events)]
+        self.gs = None
+        if set_events is not None:
+            for e in self.ev:
+                e.record(stream)
+            torch.cuda.synchronize()
+            set_events(self.ev)
+            self.gs = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.gs):
+                fn()
+            set_events(None)
+        self.e0 = torch.cuda.Event(enable_timing=True)
+        self.e1 = torch.cuda.Event(enable_timing=True)
+
+    def replay_ms(self) -> float:
+        self.flush.fill_(1.0)
+        self.e0.record(self.stream)
+        self.g.replay()
+        self.e1.record(self.stream)
+        self.torch.cuda.synchronize()
+        return self.e0.elapsed_time(self.e1)
+
+    def stages_ms(self):
+        """Stage boundaries (ms after the first event), from the graph with events."""
+        if self.gs is None:
+            return None
+        self.flush.fill_(1.0)
+        self.gs.replay()
+        self.torch.cuda.synchronize()
+        return [self.ev[0].elapsed_time(e) for e in self.ev[1:]]
+
+    def run(self, steps: int, warmup: int):
+        for _ in range(warmup):
+            self.replay_ms()
+        t = [self.replay_ms() for _ in range(steps)]
+        st = [self.stages_ms() for _ in range(steps)] if self.gs is not None else None
+        return t, st
+
+
+def _mean_stage(st, i):
+    return statistics.mean(x[i] - (x[i - 1] if i > 0 else 0.0) for x in st)
+
+
+def bench_prefill(args, dev, stream, flush, hbm, name, T, zipf, seed_x):
+    """One prefill-shape layer at T tokens on the tensor-core path."""
+    import torch
+
+    import ternary_weight_moe_forward_b200 as tw
+    from ternary_weight_moe_forward_b200 import synth
+    from ternary_weight_moe_forward_b200.layer import Layer, bf16_from_bits
+    shape = synth.CONFIGS["decode"]["shape"]
+    w = synth.layer_weights_device(shape, seed=0, zipf=zipf, device=dev)
+    layer = Layer(shape, w, max_tokens=T, device=dev)
+    del w
+    x = bf16_from_bits(synth.activations(T, shape.d_model, seed=seed_x), dev)
+    y = torch.empty((T, shape.d_model), dtype=torch.float32, device=dev)
+    _, _, counts = layer.route(x)
+    counts = counts.cpu().numpy()
+    gt = GraphTimer(lambda: layer.forward(x, y=y), stream, flush,
+                    lambda ev: tw.maple_moe_set_stage_events(layer.handle, ev))
+    t, st = gt.run(args.steps, args.warmup)
+    fwd = statistics.mean(t)
+    S = T * shape.top_k
+    ops_gu, ops_dn = prefill_ops(S)
+    peak, peak_kind = int8_peak_tops()
+    us = {"route_and_permute": 1e3 * _mean_stage(st, 0), "gate_up_stage": 1e3 * _mean_stage(st, 1),
+          "down_stage": 1e3 * _mean_stage(st, 2)}
+    gemm_us = us["gate_up_stage"] + us["down_stage"]
+
+    def roof(kernel, ops, u):
+        a = ops / (u * 1e-6) / 1e12
+        return {"kernel": kernel, "bound": "tensor", "dtype": "int8", "achieved": a, "peak": peak,
+                "peak_kind": peak_kind, "unit": "TOPS", "frac": a / peak, "ops": ops}
+
+    # end to end: pinned host x in, forward, y out, all inside the events
+    hx = x.cpu().pin_memory()
+    hy = torch.empty((T, shape.d_model), dtype=torch.float32).pin_memory()
+    dx = torch.empty_like(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e = []
+    for it in range(args.warmup + args.steps):
+        flush.fill_(1.0)
+        e0.record(stream)
+        dx.copy_(hx, non_blocking=True)
+        layer.forward(dx, y=y)
+        hy.copy_(y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            e2e.append(e0.elapsed_time(e1))
+    layer.close()
+    out = {
+        "workload": f"{name}: d_model=2048, 256 experts, top-8, d_ff=512, T={T}"
+                    + (", Zipf(1.1) router bias" if zipf else ""),
+        "tokens_per_s": T / (fwd * 1e-3), "us_per_forward": 1e3 * fwd, "us_stages": us,
+        "experts_touched": int((counts > 0).sum()), "max_tokens_per_expert": int(counts.max()),
+        "roofline_gemms": roof("gate/up + down stages (grouped GEMMs with their epilogue kernels)",
+                               ops_gu + ops_dn, gemm_us),
+        "roofline_gate_up": roof("gate/up stage", ops_gu, us["gate_up_stage"]),
+        "roofline_down": roof("down stage (incl. combine)", ops_dn, us["down_stage"]),
+        "e2e": {"value": T / (statistics.mean(e2e) * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * shape.d_model * 2, "d2h_bytes_per_step": T * shape.d_model * 4},
+    }
+    return out
+
+
+def bench_stack(args, dev, stream, flush, hbm):
+    """The 24-layer stack (RMSNorm + layer, residual) at T = 1 and 32, one graph."""
+    import torch
+
+    import ternary_weight_moe_forward_b200 as tw
+    from ternary_weight_moe_forward_b200 import synth
+    from ternary_weight_moe_forward_b200.layer import Layer
+    cfg = synth.CONFIGS["stack"]
+    shape = cfg["shape"]
+    layers = []
+    for l in range(cfg["layers"]):
+        w = synth.layer_weights_device(shape, seed=1000, layer=l, device=dev)
+        layers.append(Layer(shape, w, max_tokens=max(cfg["tokens"]), device=dev, flags=tw.MAPLE_CFG_DECODE_ONLY))
+        del w
+    torch.cuda.synchronize()
+    handles = [L.handle for L in layers]
+    out = {}
+    for T in cfg["tokens"]:
+        r0 = torch.from_numpy(synth.residual(T, shape.d_model, seed=T)).to(dev)
+        resid = r0.clone()
+
+        def step():
+            resid.copy_(r0)
+            tw.maple_moe_stack_forward(handles, resid, T, torch.cuda.current_stream(dev).cuda_stream)
+
+        gt = GraphTimer(step, stream, flush)
+        t, _ = gt.run(args.steps, args.warmup)
+        ms = statistics.mean(t)
+        n_exp = expected_experts(T)
+        byts = cfg["layers"] * decode_bytes(int(round(n_exp)), T)
+        out[str(T)] = {"tokens_per_s": T / (ms * 1e-3), "us_per_step": 1e3 * ms,
+                       "hbm_frac": byts / (ms * 1e-3) / 1e9 / hbm,
+                       "bytes_note": f"expected distinct experts per layer {n_exp:.1f} (uniform routing)"}
+    for L in layers:
+        L.close()
+    return {"workload": "24-layer MoE-FFN stack (pre-norm RMSNorm + residual), d_model=2048, 256 experts, "
+                        "top-8, d_ff=512, independent layers", "per_T": out}
+
+
+def bench_tiny(args, dev, stream, flush):
+    import torch
+
+    from ternary_weight_moe_forward_b200 import synth
+    from ternary_weight_moe_forward_b200.layer import Layer, bf16_from_bits
+    shape = synth.CONFIGS["tiny"]["shape"]
+    layer = Layer(shape, synth.layer_weights(shape, seed=0), max_tokens=8, device=dev)
+    x = bf16_from_bits(synth.activations(8, shape.d_model, seed=0), dev)
+    y = torch.empty((8, shape.d_model), dtype=torch.float32, device=dev)
+    gt = GraphTimer(lambda: layer.forward(x, y=y), stream, flush)
+    t, _ = gt.run(args.steps, args.warmup)
+    layer.close()
+    return {"workload": "tiny: d_model=256, 16 experts, top-2, d_ff=128, T=8", "us_per_forward": 1e3 * statistics.mean(t),
+            "tokens_per_s": 8 / (statistics.mean(t) * 1e-3), "bound": "latency"}
+
+
 def run_gpu(args, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -197,63 +400,19 @@ def run_gpu(args, rank: int, world: int):
         n_active[T] = int((counts > 0).sum().item())
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
-    # One CUDA graph per batch size: the forward (routing kernel, permutation
-    # and expert kernel) replays without host launch gaps.  The library's
-    # per-stage events are captured with it, so the stages are timed on the
-    # device as well.
-    ev = {T: [torch.cuda.Event(enable_timing=True) for _ in range(4)] for T in DECODE_T}
-    for T in DECODE_T:
-        for e in ev[T]:
-            e.record(stream)
-    torch.cuda.synchronize(dev)
-    # Two graphs per batch size: the timed one holds only the library's kernels;
-    # the second also records the per-stage events (an event between the routing
-    # and the expert kernel would keep them from overlapping their launch) and
-    # gives the stage split after the timed region.
-    graphs, split_graphs = {}, {}
-    for T in DECODE_T:
-        layer.forward(xs[T], y=ys[T])          # warm the path before capture
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            layer.forward(xs[T], y=ys[T])
-        graphs[T] = g
-        tw.maple_moe_set_stage_events(layer.handle, ev[T])
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            layer.forward(xs[T], y=ys[T])
-        split_graphs[T] = g
-        tw.maple_moe_set_stage_events(layer.handle, None)
-    torch.cuda.synchronize(dev)
-
-    e_beg = {T: torch.cuda.Event(enable_timing=True) for T in DECODE_T}
-    e_end = {T: torch.cuda.Event(enable_timing=True) for T in DECODE_T}
-    stages_in_graph = True
+    # One CUDA graph per batch size: the forward (routing kernel and expert
+    # kernel) replays without host launch gaps.  A second graph per batch size
+    # also records the library's per-stage events (an event between the routing
+    # and the expert kernel keeps them from overlapping their launch), replayed
+    # after the timed region for the stage split.
+    timers = {T: GraphTimer(lambda T=T: layer.forward(xs[T], y=ys[T]), stream, flush,
+                            lambda ev: tw.maple_moe_set_stage_events(layer.handle, ev)) for T in DECODE_T}
 
     def one_step(timed: list | None):
         for T in DECODE_T:
-            flush.fill_(1.0)
-            e_beg[T].record(stream)
-            graphs[T].replay()
-            e_end[T].record(stream)
+            ms = timers[T].replay_ms()
             if timed is not None:
-                torch.cuda.synchronize(dev)
-                timed.append((T, e_beg[T].elapsed_time(e_end[T]), None))
-
-    def split_step():
-        """Stage times (route, gate/up, experts end) from the graphs with events."""
-        nonlocal stages_in_graph
-        out = {}
-        for T in DECODE_T:
-            flush.fill_(1.0)
-            split_graphs[T].replay()
-            torch.cuda.synchronize(dev)
-            try:
-                out[T] = [ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)]
-            except Exception:
-                stages_in_graph = False
-                return None
-        return out
+                timed.append((T, ms))
 
     for _ in range(args.warmup):
         one_step(None)
@@ -273,36 +432,12 @@ def run_gpu(args, rank: int, world: int):
     clocks = clk.stop()
 
     # stage split: the same number of forwards again, from the graphs with events
-    split = {T: [] for T in DECODE_T}
-    for _ in range(args.steps):
-        sp = split_step()
-        if sp is None:
-            break
-        for T in DECODE_T:
-            split[T].append(sp[T])
-    if stages_in_graph:
-        stage_src = "events inside a second set of graphs (untimed replays)"
-        timed = [(T, tot, split[T][n % len(split[T])]) for n, (T, tot, _) in enumerate(timed)]
-
-    if not stages_in_graph:
-        # stage split from host-launched forwards instead (same kernels, stage events on the stream)
-        stage_src = "host-launched forwards"
-        split = {T: [] for T in DECODE_T}
-        tw.maple_moe_set_stage_events(layer.handle, None)
-        for _ in range(args.steps):
-            for T in DECODE_T:
-                flush.fill_(1.0)
-                tw.maple_moe_set_stage_events(layer.handle, ev[T])
-                layer.forward(xs[T], y=ys[T])
-                torch.cuda.synchronize(dev)
-                split[T].append([ev[T][0].elapsed_time(ev[T][i]) for i in range(1, 4)])
-        tw.maple_moe_set_stage_events(layer.handle, None)
-        timed = [(T, tot, split[T][n % len(split[T])]) for n, (T, tot, _) in enumerate(timed)]
+    split = {T: [timers[T].stages_ms() for _ in range(args.steps)] for T in DECODE_T}
+    stage_src = "events inside a second set of graphs (untimed replays)"
 
     total_ms = sum(t[1] for t in timed)
-    per_T = {T: [t[2] for t in timed if t[0] == T] for T in DECODE_T}
     fwd_T = {T: [t[1] for t in timed if t[0] == T] for T in DECODE_T}
-    experts_ms = sum(x[2] - x[0] for T in DECODE_T for x in per_T[T])
+    experts_ms = sum(x[2] - x[0] for T in DECODE_T for x in split[T])
     experts_alg = sum(experts_bytes(n_active[T], T) for T in DECODE_T) * args.steps
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host, all timed
@@ -322,6 +457,8 @@ def run_gpu(args, rank: int, world: int):
             torch.cuda.synchronize(dev)
             if it >= args.warmup:
                 e2e_ms += e0.elapsed_time(e1)
+    del timers
+    layer.close()
 
     # ---- max over ranks
     total_ms, e2e_ms, experts_ms = reduce_max_over_ranks([total_ms, e2e_ms, experts_ms], device=dev)
@@ -342,19 +479,20 @@ def run_gpu(args, rank: int, world: int):
         "vs_baseline": None,
         "dtype": "int8",
         "data": "synthetic (seeded ternary weights P=.3/.4/.3, lognormal alpha, N(0,1) bf16 x)",
-        "config": {"workload": WORKLOAD, "tokens_per_step": sum(DECODE_T), "layers": 1,
-                   "experts_touched": {str(T): n_active[T] for T in DECODE_T},
-                   "l2": "flushed before every timed forward (256 MB write, outside the events)",
-                   "parallelism": f"replicas x{world}"},
+        "config": config_of(world),
+        "experts_touched": {str(T): n_active[T] for T in DECODE_T},
+        "l2": "flushed before every timed forward (256 MB write, outside the events)",
         "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(fwd_T[T]) * 1e-3),
                            "us_per_forward": 1e3 * statistics.mean(fwd_T[T]),
-                           "us_route": 1e3 * statistics.mean(x[0] for x in per_T[T]),
-                           "us_experts": 1e3 * statistics.mean(x[2] - x[0] for x in per_T[T]),
+                           "us_route": 1e3 * statistics.mean(x[0] for x in split[T]),
+                           "us_experts": 1e3 * statistics.mean(x[2] - x[0] for x in split[T]),
                            "layer_hbm_frac": decode_bytes(n_active[T], T) /
-                           (statistics.mean(fwd_T[T]) * 1e-3) / 1e9 / hbm}
+                           (statistics.mean(fwd_T[T]) * 1e-3) / 1e9 / hbm,
+                           "experts_hbm_frac": experts_bytes(n_active[T], T) /
+                           (statistics.mean(x[2] - x[0] for x in split[T]) * 1e-3) / 1e9 / hbm}
                   for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
-        "roofline": {"kernel": "decode_experts_kernel", "bound": "hbm", "achieved": achieved, "peak": hbm,
+        "roofline": {"kernel": "decode expert stage", "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": measured_traffic(), "traffic_launch": "T=64 (ncu, profiles/)",
                      "algorithmic_bytes_T64": experts_bytes(n_active[64], 64)},
@@ -366,51 +504,103 @@ def run_gpu(args, rank: int, world: int):
         "stage_split_from": stage_src,
         "clocks": clocks,
     }
-    return out, layer
+    if not args.decode_only:
+        # the other workloads, each on its own (timed after the headline's region)
+        per = {}
+        per["prefill"] = bench_prefill(args, dev, stream, flush, hbm, "prefill", 4096, None, 0)
+        per["skewed"] = bench_prefill(args, dev, stream, flush, hbm, "skewed routing", 16384, 1.1, 5)
+        per["stack"] = bench_stack(args, dev, stream, flush, hbm)
+        per["tiny"] = bench_tiny(args, dev, stream, flush)
+        out["per_config"] = per
+        out["roofline_prefill"] = per["prefill"]["roofline_gemms"]
+    return out
 
 
-def cpu_baseline(seconds_cap: float = 20.0) -> dict:
-    """Time the CPU oracle (single thread) on a sample of the same workload:
-    up to 8 tokens of each decode batch (25 tokens), the router over all
-    experts and the expert FFNs of every kept expert."""
-    import oracle
+def config_of(world: int) -> dict:
+    return {"workload": WORKLOAD, "tokens_per_step": sum(DECODE_T), "layers": 1,
+            "parallelism": f"replicas x{world}"}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class pinned_to_one_core:
+    """Run the enclosed block on a single host core (the first one this
+    process may use); restores the affinity afterwards."""
+
+    def __enter__(self):
+        self.old = os.sched_getaffinity(0)
+        self.core = min(self.old)
+        os.sched_setaffinity(0, {self.core})
+        return self
+
+    def __exit__(self, *a):
+        os.sched_setaffinity(0, self.old)
+
+
+def _oracle_sample():
+    """The oracle's sample of the workload: the first <= 8 tokens of each decode
+    batch (T = 1, 8, 32, 64: 25 tokens) and 16 tokens of the T = 4096 prefill
+    batch, all through the full layer (router over every expert, the kept
+    experts' FFNs, combine)."""
     from ternary_weight_moe_forward_b200 import synth
     shape = synth.CONFIGS["decode"]["shape"]
+    xs = [synth.activations(T, shape.d_model, seed=0)[:min(T, 8)] for T in DECODE_T]
+    xs.append(synth.activations(4096, shape.d_model, seed=0)[:16])
+    return shape, xs
+
+
+def cpu_baseline() -> dict:
+    """Time the CPU oracle, single-threaded and pinned to one core, on its sample."""
+    import oracle
+    from ternary_weight_moe_forward_b200 import synth
+    shape, xs = _oracle_sample()
     L = oracle.Layer(shape, synth.layer_weights(shape, seed=0))
-    n_tok = 0
-    t0 = time.perf_counter()
-    for T in DECODE_T:
-        x = synth.activations(T, shape.d_model, seed=0)
-        n = min(T, 8)
-        L.forward_tokens(x[:n], taps=False)
-        n_tok += n
-    dt = time.perf_counter() - t0
-    return {"value": n_tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n_tok} tokens (first <=8 of each decode batch T=1,8,32,64), single-threaded C oracle, {dt:.1f} s"}
+    n_tok = sum(x.shape[0] for x in xs)
+    with pinned_to_one_core() as pin:
+        t0 = time.perf_counter()
+        for x in xs:
+            L.forward_tokens(x, taps=False)
+        dt = time.perf_counter() - t0
+    return {"value": n_tok / dt, "unit": "tokens/s", "cores": 1, "cores_total": os.cpu_count(),
+            "cpu_model": cpu_model(), "pinned_core": pin.core, "kind": "oracle",
+            "sample": f"{n_tok} tokens: first <=8 of each decode batch T=1,8,32,64 and 16 of the T=4096 prefill "
+                      f"batch; single-threaded C oracle on 1 of {os.cpu_count()} cores, {dt:.1f} s"}
 
 
 def run_reference(args):
-    """The CPU oracle as the reference arm: each step = the 25-token sample."""
+    """The CPU oracle as the reference arm: each step = the oracle's sample
+    (tokens are independent, so its tokens/s is that of the whole workload)."""
     import oracle
     from ternary_weight_moe_forward_b200 import synth
-    shape = synth.CONFIGS["decode"]["shape"]
+    shape, xs = _oracle_sample()
     L = oracle.Layer(shape, synth.layer_weights(shape, seed=0))
-    xs = {T: synth.activations(T, shape.d_model, seed=0)[:min(T, 8)] for T in DECODE_T}
-    per_step = sum(x.shape[0] for x in xs.values())
-    for _ in range(args.warmup):
-        for x in xs.values():
-            L.forward_tokens(x, taps=False)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        for x in xs.values():
-            L.forward_tokens(x, taps=False)
-    dt = time.perf_counter() - t0
+    per_step = sum(x.shape[0] for x in xs)
+    with pinned_to_one_core() as pin:
+        for _ in range(args.warmup):
+            for x in xs:
+                L.forward_tokens(x, taps=False)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            for x in xs:
+                L.forward_tokens(x, taps=False)
+        dt = time.perf_counter() - t0
     v = per_step * args.steps / dt
-    sample = f"{per_step} tokens per step (first <=8 of each decode batch T=1,8,32,64), single-threaded C oracle"
+    sample = (f"{per_step} tokens per step (first <=8 of each decode batch T=1,8,32,64 and 16 of the T=4096 "
+              f"prefill batch), single-threaded C oracle on 1 of {os.cpu_count()} cores")
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": {"workload": WORKLOAD},
-            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": config_of(1),
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "cores_total": os.cpu_count(),
+                             "cpu_model": cpu_model(), "pinned_core": pin.core, "kind": "oracle", "sample": sample},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -421,6 +611,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="skip the per_config workloads")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -437,8 +628,7 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    out, layer = run_gpu(args, rank, world)
-    layer.close()
+    out = run_gpu(args, rank, world)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline()

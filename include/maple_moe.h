@@ -32,6 +32,15 @@
  *    router logit, an out-of-range expert id) sets a flag in host-mapped
  *    memory; the next call on the same handle returns MAPLE_ERR_DEVICE_FLAG
  *    (and clears it), and maple_moe_device_flags reads it on demand.
+ *  - Every wait inside a kernel (on another warp, another CTA or a copy in
+ *    flight) is bounded in time (2 s unless maple_moe_set_debug sets another
+ *    limit).  A wait that gives up sets MAPLE_FLAG_TIMEOUT; the kernel drains
+ *    its copies in flight and returns, and the outputs of that call are not
+ *    valid.  The next call on the handle that sees the flag returns
+ *    MAPLE_ERR_TIMEOUT, after resetting the handle's internal counters on its
+ *    stream, so that the call after it runs normally.  Calls enqueued before
+ *    the flag became visible to the host may be wrong as well; synchronise
+ *    and check maple_moe_device_flags when that matters.
  *  - A handle may be used from one stream at a time.
  */
 #ifndef MAPLE_MOE_H
@@ -54,7 +63,7 @@ enum {
     MAPLE_ERR_UNSUPPORTED_SHAPE = -2, /* shape outside the limits listed at maple_moe_config */
     MAPLE_ERR_OOM = -3,               /* device allocation failed in create */
     MAPLE_ERR_CUDA = -4,              /* a CUDA runtime call or a kernel launch failed */
-    MAPLE_ERR_TIMEOUT = -5,           /* a bounded device wait gave up (reported via the flag word) */
+    MAPLE_ERR_TIMEOUT = -5,           /* an earlier call's bounded device wait gave up (MAPLE_FLAG_TIMEOUT) */
     MAPLE_ERR_DEVICE_FLAG = -6,       /* an earlier kernel on this handle flagged an invalid value */
 };
 
@@ -62,18 +71,27 @@ enum {
 #define MAPLE_FLAG_NAN_LOGIT 0x1u     /* a router logit was NaN; it was ranked last */
 #define MAPLE_FLAG_BAD_INDEX 0x2u     /* an expert id outside [0, E) reached the permutation */
 #define MAPLE_FLAG_BAD_VALUE 0x4u     /* maple_moe_pack_ternary met a value outside {-1, 0, +1} */
+#define MAPLE_FLAG_TIMEOUT 0x8u       /* a bounded wait inside a kernel gave up (reported as MAPLE_ERR_TIMEOUT) */
 
-/* config.flags: path selection (default 0 = automatic) */
-#define MAPLE_CFG_FORCE_GEMV 0x1u     /* never use the tensor-core grouped GEMM */
-#define MAPLE_CFG_FORCE_TC 0x2u       /* use the tensor-core grouped GEMM for every T > 0 */
+/* config.flags: path selection and weight layouts (default 0 = automatic, both layouts) */
+#define MAPLE_CFG_FORCE_GEMV 0x1u     /* never use the tensor-core grouped GEMM: T <= 64 on the decode
+                                         kernel whatever decode_max_tokens says, larger T rejected
+                                         (MAPLE_ERR_UNSUPPORTED_SHAPE); only the decode layout is built */
+#define MAPLE_CFG_FORCE_TC 0x2u       /* the tensor-core grouped GEMM for every T > 0; only its layout is
+                                         built (may not be combined with the other flags) */
+#define MAPLE_CFG_DECODE_ONLY 0x4u    /* build only the decode layout (half the weight memory);
+                                         T > decode_max_tokens is rejected (MAPLE_ERR_UNSUPPORTED_SHAPE) */
 
 /*
  * Layer shape.  Limits: d_model = 256 * 2^i (256 .. 4096); d_ff = 128 * 2^j
  * (128 .. 1024); n_experts % 16 == 0
  * and 16 <= n_experts <= 1024; 1 <= top_k <= min(32, n_experts);
  * 1 <= max_tokens <= 65536.  max_tokens sizes the library-owned workspace.
- * decode_max_tokens: largest T served by the weight-streaming (GEMV) path;
- * 0 selects 64.  Larger T use the tcgen05 int8 grouped GEMM.
+ * decode_max_tokens (0 .. 64, 0 selects 64): largest T served by the decode
+ * kernel (weight streaming on warp-level int8 MMA); larger T use the tcgen05
+ * int8 grouped GEMM.  The decode kernel needs d_ff <= d_model and its
+ * shared memory to fit; shapes outside that run every T on the tensor cores
+ * (and then reject MAPLE_CFG_FORCE_GEMV and MAPLE_CFG_DECODE_ONLY).
  */
 typedef struct {
     int32_t d_model, n_experts, top_k, d_ff, max_tokens;
@@ -135,10 +153,11 @@ int maple_moe_pack_ternary(const int8_t *values, int64_t rows, int32_t cols, uin
 
 /*
  * Create a layer: validate the shape, allocate the library-owned weight copies
- * (re-laid out for the decode GEMV and for the tcgen05 GEMM) and a workspace
- * for max_tokens tokens, and launch the re-layout on `stream`.  *out receives
- * the handle.  Errors: INVALID_ARG, UNSUPPORTED_SHAPE, OOM, CUDA; on error
- * nothing stays allocated.
+ * (re-laid out for the decode kernel and/or the tcgen05 GEMM, as config.flags
+ * say) and a workspace for max_tokens tokens, and launch the re-layout on
+ * `stream`.  *out receives the handle.  Errors: INVALID_ARG (also for unknown
+ * or conflicting flags), UNSUPPORTED_SHAPE, OOM, CUDA; on error nothing stays
+ * allocated.
  */
 int maple_moe_create(const maple_moe_config *config, const maple_moe_weights *weights, maple_stream_t stream,
                      maple_moe_t *out);
@@ -197,7 +216,8 @@ int maple_moe_set_stage_events(maple_moe_t layer, void *const *events, int32_t n
  * maple_moe_config for d_model, n_experts and top_k.
  * The first call on a device looks up the array's device address and raises
  * the routing kernel's shared-memory limit for that device; make that first
- * call before any stream capture.  Every call uses the same array and it keeps
+ * call before any stream capture.  Both are kept for the life of the process:
+ * after a cudaDeviceReset of a device, do not call this entry point on it.  Every call uses the same array and it keeps
  * the previous call's contents (the counters that must start at zero are
  * cleared by each call on its stream), so calls whose work overlaps on the GPU
  * (other streams, other host threads) race: order them on one stream.
@@ -207,8 +227,22 @@ int maple_moe_route_noalloc(const uint16_t *x, int32_t T, int32_t d_model, int32
                             const float *router_w, const float *router_bias, int32_t *topk_idx, float *topk_w,
                             int32_t *expert_counts, maple_stream_t stream);
 
-/* Read (and optionally clear) the device flag word; no synchronisation. */
+/* Read (and optionally clear) the device flag word; no synchronisation.
+ * Clearing a MAPLE_FLAG_TIMEOUT here still makes the next call reset the
+ * handle's internal counters (that call then returns normally). */
 int maple_moe_device_flags(maple_moe_t layer, uint32_t *flags, int32_t clear);
+
+/* maple_moe_set_debug flags (testing the failure handling only) */
+#define MAPLE_DEBUG_STALL_DOWN 0x1u   /* the decode expert kernel's down stage waits for an arrival
+                                         count that is never reached, so that its bounded wait expires */
+
+/*
+ * Failure-handling knobs of a handle, for tests.  wait_limit_us: the limit of
+ * every bounded device wait of later calls, in microseconds (0 = the default
+ * 2 s; at most 60 s).  debug_flags: MAPLE_DEBUG_* bits (0 in normal use).
+ * Takes effect for calls made after it returns.  Errors: INVALID_ARG.
+ */
+int maple_moe_set_debug(maple_moe_t layer, int32_t wait_limit_us, uint32_t debug_flags);
 
 /* Synchronise all work of the layer and free everything it owns.  NULL is a no-op. */
 int maple_moe_destroy(maple_moe_t layer);

@@ -25,13 +25,17 @@ MAPLE_ERR_DEVICE_FLAG = -6
 MAPLE_FLAG_NAN_LOGIT = 0x1
 MAPLE_FLAG_BAD_INDEX = 0x2
 MAPLE_FLAG_BAD_VALUE = 0x4
+MAPLE_FLAG_TIMEOUT = 0x8
 
 MAPLE_CFG_FORCE_GEMV = 0x1
 MAPLE_CFG_FORCE_TC = 0x2
+MAPLE_CFG_DECODE_ONLY = 0x4
+
+MAPLE_DEBUG_STALL_DOWN = 0x1
 
 EXPORTED = ("maple_moe_status_string", "maple_moe_pack_ternary", "maple_moe_create", "maple_moe_route",
             "maple_moe_forward", "maple_moe_stack_forward", "maple_moe_set_stage_events", "maple_moe_device_flags",
-            "maple_moe_destroy", "maple_moe_route_noalloc")
+            "maple_moe_destroy", "maple_moe_route_noalloc", "maple_moe_set_debug")
 
 
 class MapleError(RuntimeError):
@@ -81,6 +85,7 @@ def lib():
         L.maple_moe_device_flags.argtypes = [P, C.POINTER(C.c_uint32), I32]
         L.maple_moe_destroy.argtypes = [P]
         L.maple_moe_route_noalloc.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P, P]
+        L.maple_moe_set_debug.argtypes = [P, I32, C.c_uint32]
         for name in EXPORTED:
             if name != "maple_moe_status_string":
                 getattr(L, name).restype = C.c_int
@@ -156,6 +161,11 @@ def maple_moe_route_noalloc(x, T: int, d_model: int, n_experts: int, top_k: int,
     _check(lib().maple_moe_route_noalloc(_p(x), T, d_model, n_experts, top_k, _p(router_w), _p(router_bias),
                                          _p(topk_idx), _p(topk_w), _p(expert_counts), _p(stream)),
            "maple_moe_route_noalloc")
+
+
+def maple_moe_set_debug(handle, wait_limit_us: int = 0, debug_flags: int = 0) -> None:
+    """Wait limit of the handle's bounded device waits (0 = 2 s) and test hooks."""
+    _check(lib().maple_moe_set_debug(handle, wait_limit_us, debug_flags), "maple_moe_set_debug")
 
 
 def maple_moe_destroy(handle) -> None:

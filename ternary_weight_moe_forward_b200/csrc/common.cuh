@@ -18,6 +18,17 @@ constexpr unsigned FULL = 0xffffffffu;
 // issue slots from the ones doing work
 constexpr uint32_t kSuspendHintNs = 200000;
 
+// default limit of every bounded wait in the kernels (2 s, far above any
+// legitimate wait); a handle may set another one
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 // ---------------------------------------------------------------------------
 // exp(x), written out from the mathematics so that host and device give the
 // same bits: clamp to [-87, 88]; n = rint(x*log2 e); r = x - n ln2 with ln2

@@ -4,20 +4,27 @@
 // uint32 words, value j in word j/16 at bits 2*(j%16)..+1, code 0 = 0,
 // 1 = +1, 2 = -1 (3 reads as 0).
 //
-// GEMV layout (weight streaming, T <= decode_max_tokens).  The codes of 32
-// rows are interleaved in 16-byte chunks so that one warp-wide 128-bit load
-// fetches chunk c of 32 different rows (512 contiguous bytes, lane l = row l):
-//   gate/up  [E][F/16 groups][D/64 chunks][32 lanes][4 words]
-//            lane l < 16: gate row 16*g + l;  lane l >= 16: up row 16*g + l - 16
-//   down     [E][D/32 groups][F/64 chunks][32 lanes][4 words], lane l: row 32*g + l
-// Word w of chunk c holds values j = 64*c + 16*w + 4*k + b (k, b = 0..3) as
-// offset codes t + 1 in {0, 1, 2} at bits 8*b + 2*k.  Then (word >> 2k) &
-// 0x03030303 is four bytes, one per value j = 64c+16w+4k+0..3, and dp4a with
-// the four int8 activations x_j gives sum (t_j + 1) x_j; subtracting the
-// token's sum of codes sum_j x_j leaves the exact ternary dot product.
-//
 // GEMM layout (tcgen05 int8 grouped GEMM, T > decode_max_tokens): see
 // tc_gemm.cuh.
+//
+// MMA-tile layout (the persistent decode kernel, warp-level int8 MMA
+// m16n8k32 with the weights as the 16 x 32 A operand).  A tile is 16 rows
+// over the whole K, stored as K/128 blocks of 512 bytes (32 lanes x 4 words):
+//   gate/up  [E][F/8 tiles][D/128][32][4]  rows 0..7 = gate rows 8t..8t+7,
+//                                          rows 8..15 = the up rows of the same outputs
+//   down     [E][D/16 tiles][F/128][32][4] row r = channel 16t + r
+// Lane l (g = l/4, c = l%4), word i, byte j, plane q (bits 8j + 2q) holds the
+// offset code t + 1 of row g + 8*(i%2), column 128*kb + 32q + 16*(i/2) + 4c + j.
+// So w_i & (0x03030303 << 2q) is A-fragment register i of the MMA over
+// columns 128kb + 32q .. +31, with every value scaled by 4^q: one logic
+// operation per register, one accumulator per plane, combined exactly as
+// acc_0 + acc_1/4 + acc_2/16 + acc_3/64 (each acc_q a multiple of 4^q).
+//
+// The matching B operand (activations, 8 tokens per MMA) wants, from token
+// g's 128 columns of block kb, the four bytes at 32q + 16h + 4c (h = 0, 1)
+// in lane 4g + c.  frag_word_pos(w) is where 4-byte word w (columns 4w ..
+// 4w+3) of a 128-column block goes so that lane c of a token reads its eight
+// words (q = 0..3, h = 0..1) as 32 contiguous bytes at 32c.
 #pragma once
 
 #include <stdint.h>
@@ -33,15 +40,28 @@ __host__ __device__ inline uint32_t offset_code(uint32_t code)
     return code == 1u ? 2u : (code == 2u ? 0u : 1u);
 }
 
-// re-order the 16 codes of one interchange word into the GEMV word
-__host__ __device__ inline uint32_t gemv_word(uint32_t canon)
+// word position of 4-byte word w (0..31) of a 128-column block in the fragment order
+__host__ __device__ inline int frag_word_pos(int w)
 {
+    const int q = w >> 3, h = (w >> 2) & 1, c = w & 3;
+    return c * 8 + q * 2 + h;
+}
+
+// tile row (0..15) whose codes sit in word i of lane `lane`
+__host__ __device__ inline int mma_word_row(int lane, int i) { return (lane >> 2) + 8 * (i & 1); }
+
+// the MMA-tile word (lane, word i) of k-block kb from the interchange words of
+// its row (src = that row's words, mma_word_row(lane, i) of the tile)
+__host__ __device__ inline uint32_t mma_word(const uint32_t *src, int lane, int i, int kb)
+{
+    const int c = lane & 3;
     uint32_t out = 0;
-#pragma unroll
-    for (int i = 0; i < 16; i++) {
-        uint32_t oc = offset_code((canon >> (2 * i)) & 3u);
-        int k = i >> 2, b = i & 3;
-        out |= oc << (8 * b + 2 * k);
+    for (int q = 0; q < 4; q++) {
+        // columns 128kb + 32q + 16(i/2) + 4c + j (j = 0..3): one interchange word,
+        // positions 4c + j
+        const uint32_t w = src[kb * 8 + q * 2 + (i >> 1)];
+        for (int j = 0; j < 4; j++)
+            out |= offset_code((w >> (2 * (4 * c + j))) & 3u) << (8 * j + 2 * q);
     }
     return out;
 }

@@ -8,7 +8,7 @@
 
 #include "../../include/maple_moe.h"
 #include "common.cuh"
-#include "gemv.cuh"
+#include "decode.cuh"
 #include "layout.cuh"
 #include "pack.cuh"
 #include "route.cuh"
@@ -38,38 +38,47 @@ struct maple_moe_s {
     uint32_t cfg_flags;
     int num_sms;
     int device;
-    char *base;  // one device allocation: weights + workspace
+    int optin;                     // shared memory a block may opt in to
+    char *base;                    // one device allocation: weights + workspace
     // weights
-    uint8_t *w_gu, *w_dn;          // GEMV layout
-    uint8_t *w_tc_gu, *w_tc_dn;    // tensor-core layout
-    int4 *pieces;
-    int *n_pieces;
-    int8_t *xperm;                 // q_x rows in slot order (tensor-core path)
-    float *pscale;                 // s_x of each position's token (tensor-core path)
-    CUtensorMap map_xperm, map_qh; // TMA maps of the activation operands
+    uint8_t *w_mma_gu, *w_mma_dn;  // decode layout (MMA tiles), null when not built
+    uint8_t *w_tc_gu, *w_tc_dn;    // tensor-core layout, null when not built
     float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
-    // workspace
-    int8_t *qx;
-    const int8_t *zrow;   // zeros, never written after create
+    // workspace: routing
+    int8_t *qx, *qxp;              // q_x rows; the decode kernel's fragment-ordered copy (T <= 64)
+    const int8_t *zrow;
     float *sx;
     int *sumx;
     float *logits;
     int *topk_idx;
     float *topk_w;
     int *counts, *offsets, *perm, *inv, *active, *n_active, *blk_cnt;
-    float *h;
+    // workspace: experts
+    int4 *pieces;
+    int *n_pieces;
+    float *pscale;                 // s_x of each position's token (tensor-core path)
+    float *hscratch;               // per-CTA h rows of the gate/up grouped GEMM [num_sms][128][F]
+    float *h;                      // decode kernel: SwiGLU rows [64*K][F]
     int8_t *qh;
     float *sh;
-    int *sumqh;
-    float *ye;
-    unsigned *tg_cnt, *glob_cnt, *exp_cnt, *comb_cnt;
-    unsigned *arrive;     // [E] finished gate/up items per expert (decode kernel)
-    bool dec_persistent;  // the persistent decode kernel fits this shape
-    int dec_optin;        // shared memory a block may opt in to
-    uint16_t *xn;
+    float *ye;                     // decode kernel: expert outputs [64*K][D]
+    int16_t *acc_hi;               // tensor-core path: down accumulators >> 1 [S][D]
+    uint32_t *acc_lo;              // and their lowest bits [S][D/32]
+    CUtensorMap map_qx, map_qh, map_qxp;   // TMA maps of the activation operands
+    // counters (zero between calls)
+    unsigned *tg_cnt, *glob_cnt, *comb_cnt;
+    unsigned *dx_clear;            // decode kernel: |h| maxima [64*K], unit arrivals, chunk counter
+    uint16_t *xn;                  // stack: normalised input of the current layer
     // flag word in host-mapped memory
     unsigned *flag_host;
     unsigned *flag_dev;
+    // failure handling: limit of every bounded device wait, test hooks, and the
+    // counters a timed-out kernel may leave non-zero (reset before the next call)
+    uint64_t wait_ns;
+    uint32_t debug_flags;
+    bool pending_reset;
+    char *ctr_base;
+    size_t ctr_bytes;
     // optional stage events (profiling)
     cudaEvent_t ev[4];
     bool use_events;
@@ -129,13 +138,14 @@ extern "C" int maple_moe_pack_ternary(const int8_t *values, int64_t rows, int32_
     return launch_status();
 }
 
-// TMA map over an int8 row matrix [rows][cols]: boxes of 128 rows x 128
-// bytes with the 128-byte swizzle (the UMMA K-major operand layout)
+// TMA map over an int8 row matrix [rows][cols]: boxes of box_rows rows x 128
+// bytes, with the 128-byte swizzle (the UMMA K-major operand layout) or none;
+// one-row boxes serve the four-row gathers
 typedef CUresult (*encode_tiled_fn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                     const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-static int make_act_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols)
+static int make_act_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols, int box_rows, bool swizzle)
 {
     static encode_tiled_fn encode = nullptr;
     if (!encode) {
@@ -148,29 +158,32 @@ static int make_act_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols
     }
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)cols};
-    cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)kTcMaxN};
+    cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MAPLE_OK : MAPLE_ERR_CUDA;
 }
 
-static void allow_max_smem(const void *fn, int device)
+// Raise a kernel's dynamic shared-memory limit to what the device offers.
+// Returns false (with the CUDA error state cleared) when that fails.
+static bool allow_max_smem(const void *fn, int device)
 {
     cudaFuncAttributes fa;
     int optin = 0;
     if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess) {
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes) !=
+            cudaSuccess) {
         cudaGetLastError();
-        return;
+        return false;
     }
-    cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+    return true;
 }
 
 typedef void (*route_fn)(RouteArgs);
-typedef void (*gemv_fn)(GemvArgs);
-
 template <int NPER>
 static route_fn pick_route_n(int ni)
 {
@@ -199,28 +212,6 @@ static route_fn pick_qtopk_n(int ni)
 }
 static route_fn pick_qtopk(int D, int E) { return E <= 256 ? pick_qtopk_n<8>(D / 256) : pick_qtopk_n<32>(D / 256); }
 
-static gemv_fn pick_gateup(int D)
-{
-    switch (D / 256) {
-    case 1: return gateup_gemv_kernel<1>;
-    case 2: return gateup_gemv_kernel<2>;
-    case 4: return gateup_gemv_kernel<4>;
-    case 8: return gateup_gemv_kernel<8>;
-    case 16: return gateup_gemv_kernel<16>;
-    default: return nullptr;
-    }
-}
-static gemv_fn pick_down(int F)
-{
-    switch (F / 128) {
-    case 1: return down_gemv_kernel<1>;
-    case 2: return down_gemv_kernel<2>;
-    case 4: return down_gemv_kernel<4>;
-    case 8: return down_gemv_kernel<8>;
-    default: return nullptr;
-    }
-}
-
 static bool pow2_upto(int v, int hi) { return v >= 1 && v <= hi && (v & (v - 1)) == 0; }
 
 static int check_shape(const maple_moe_config *c)
@@ -230,9 +221,13 @@ static int check_shape(const maple_moe_config *c)
     if (c->n_experts < 16 || c->n_experts > kMaxExperts || c->n_experts % 16 != 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     if (c->top_k < 1 || c->top_k > 32 || c->top_k > c->n_experts) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     if (c->max_tokens < 1 || c->max_tokens > 65536) return MAPLE_ERR_UNSUPPORTED_SHAPE;
-    if (c->decode_max_tokens < 0) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    if (c->decode_max_tokens < 0 || c->decode_max_tokens > kRouteSmallT) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     return MAPLE_OK;
 }
+
+// largest unit count of a decode batch: every active expert, plus one unit per
+// further 16 slots of an expert
+static int64_t dx_max_units(int64_t E, int64_t S) { return E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1; }
 
 extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_weights *w, maple_stream_t stream,
                                 maple_moe_t *out)
@@ -241,6 +236,9 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     *out = nullptr;
     int rc = check_shape(config);
     if (rc) return rc;
+    const uint32_t known = MAPLE_CFG_FORCE_GEMV | MAPLE_CFG_FORCE_TC | MAPLE_CFG_DECODE_ONLY;
+    if ((config->flags & ~known) || ((config->flags & MAPLE_CFG_FORCE_TC) && (config->flags & ~MAPLE_CFG_FORCE_TC)))
+        return MAPLE_ERR_INVALID_ARG;
     const void *need[] = {w->w_gate, w->w_up, w->w_down, w->alpha_gate, w->alpha_up, w->alpha_down, w->router_w};
     for (const void *p : need)
         if (!p || !aligned16(p)) return MAPLE_ERR_INVALID_ARG;
@@ -254,34 +252,55 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->K = config->top_k;
     h->F = config->d_ff;
     h->Tm = config->max_tokens;
-    h->dmax = config->decode_max_tokens ? config->decode_max_tokens : 64;
+    h->dmax = config->decode_max_tokens ? config->decode_max_tokens : kRouteSmallT;
     h->cfg_flags = config->flags;
     if (cudaGetDevice(&h->device) != cudaSuccess ||
-        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device) != cudaSuccess) {
+        cudaGetLastError();
         delete h;
         return MAPLE_ERR_CUDA;
     }
     const int64_t D = h->D, E = h->E, K = h->K, F = h->F, Tm = h->Tm;
     const int64_t S = Tm * K;
+    const int64_t T64 = Tm < kRouteSmallT ? Tm : kRouteSmallT, S64 = T64 * K;   // decode batches
+    // which weight layouts the handle needs: the decode kernel's (when it fits the
+    // shape: d_ff <= d_model and its shared memory at one token) unless every T
+    // goes to the tensor cores; the tensor-core one unless the handle is for
+    // decode batches only
+    const bool dec_fits = dx_ring_slots(h->D, h->F, 1, h->K, h->E, (size_t)h->optin) > 0;
+    const bool build_dec = !(h->cfg_flags & MAPLE_CFG_FORCE_TC) && dec_fits;
+    const bool build_tc = !(h->cfg_flags & (MAPLE_CFG_FORCE_GEMV | MAPLE_CFG_DECODE_ONLY)) || !dec_fits;
+    if (!build_dec && (h->cfg_flags & (MAPLE_CFG_FORCE_GEMV | MAPLE_CFG_DECODE_ONLY))) {
+        delete h;
+        return MAPLE_ERR_UNSUPPORTED_SHAPE;   // the decode kernel does not fit this shape
+    }
     const int64_t nblk = (Tm + kPermBlockTokens - 1) / kPermBlockTokens;
     Arena ar;
-    size_t o_gu = ar.take(E * gu_bytes_per_expert(D, F)), o_dn = ar.take(E * dn_bytes_per_expert(D, F));
-    size_t o_tgu = ar.take(E * F * D / 2), o_tdn = ar.take(E * D * F / 4);
-    size_t o_pc = ar.take((E + S / kPieceSlots + 1) * 16), o_npc = ar.take(4);
-    size_t o_xp = ar.take(S * D), o_ps = ar.take(S * 4 + 512);
-    size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
-    size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
-    size_t o_qx = ar.take(Tm * D), o_sx = ar.take(Tm * 4), o_sumx = ar.take(Tm * 4);
-    size_t o_lg = ar.take(Tm * E * 4), o_ti = ar.take(S * 4), o_tw = ar.take(S * 4);
-    size_t o_cnt = ar.take(E * 4), o_off = ar.take((E + 1) * 4), o_perm = ar.take(S * 4), o_inv = ar.take(S * 4);
-    size_t o_act = ar.take(E * 4), o_nact = ar.take(4), o_blk = ar.take(nblk * E * 4);
-    size_t o_h = ar.take(S * F * 4), o_qh = ar.take(S * F), o_sh = ar.take(S * 4), o_sumqh = ar.take(S * 4);
-    size_t o_ye = ar.take(S * D * 4);
-    size_t o_ctr = ar.take(0);
-    size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4), o_ec = ar.take(E * 4);
-    size_t o_cc = ar.take(Tm * (D / 32) * 4), o_rdy = ar.take((E + 1) * 4);
-    size_t o_xn = ar.take(Tm * D * 2);
-    size_t o_zr = ar.take(D > F * 4 ? D : F * 4);   // a row of zeros (padding rows of the decode kernel)
+    const size_t o_mgu = build_dec ? ar.take(E * F * D / 2) : 0, o_mdn = build_dec ? ar.take(E * D * F / 4) : 0;
+    const size_t o_tgu = build_tc ? ar.take(E * F * D / 2) : 0, o_tdn = build_tc ? ar.take(E * D * F / 4) : 0;
+    const size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
+    const size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
+    // workspace (zeroed once below)
+    const size_t o_ws = ar.take(0);
+    const size_t o_qx = ar.take(Tm * D), o_qxp = ar.take(T64 * D), o_zr = ar.take(D);
+    const size_t o_sx = ar.take(Tm * 4), o_sumx = ar.take(Tm * 4);
+    const size_t o_lg = ar.take(Tm * E * 4), o_ti = ar.take(S * 4), o_tw = ar.take(S * 4);
+    const size_t o_cnt = ar.take(E * 4), o_off = ar.take((E + 1) * 4), o_perm = ar.take(S * 4), o_inv = ar.take(S * 4);
+    const size_t o_act = ar.take(E * 4), o_nact = ar.take(4), o_blk = ar.take(nblk * E * 4);
+    const size_t o_pc = build_tc ? ar.take((E + S / kPieceSlots + 1) * 16) : 0, o_npc = ar.take(4);
+    const size_t o_ps = build_tc ? ar.take(S * 4 + 512) : 0;
+    const size_t o_hs = build_tc ? ar.take((size_t)h->num_sms * kTcMaxN * F * 4) : 0;
+    const size_t o_h = build_dec ? ar.take(S64 * F * 4) : 0;
+    const size_t o_qh = build_tc ? ar.take(S * F) : 0, o_sh = build_tc ? ar.take(S * 4) : 0;
+    const size_t o_ye = build_dec ? ar.take(S64 * D * 4) : 0;
+    const size_t o_ahi = build_tc ? ar.take(S * D * 2) : 0, o_alo = build_tc ? ar.take(S * D / 8) : 0;
+    const size_t o_ctr = ar.take(0);   // counters: zero between calls
+    const size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4);
+    const size_t o_cc = ar.take(T64 * (D / 256) * 4);
+    const size_t o_dx = ar.take((S64 + dx_max_units(E, S64) + 1) * 4);
+    const size_t o_ctr_end = ar.take(0);
+    const size_t o_xn = ar.take(Tm * D * 2);
 
     if (cudaMalloc(&h->base, ar.size) != cudaSuccess) {
         cudaGetLastError();
@@ -297,20 +316,18 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     }
     *h->flag_host = 0;
     char *b = h->base;
-    h->w_gu = (uint8_t *)(b + o_gu);
-    h->w_dn = (uint8_t *)(b + o_dn);
-    h->w_tc_gu = (uint8_t *)(b + o_tgu);
-    h->w_tc_dn = (uint8_t *)(b + o_tdn);
-    h->pieces = (int4 *)(b + o_pc);
-    h->n_pieces = (int *)(b + o_npc);
-    h->xperm = (int8_t *)(b + o_xp);
-    h->pscale = (float *)(b + o_ps);
+    h->w_mma_gu = build_dec ? (uint8_t *)(b + o_mgu) : nullptr;
+    h->w_mma_dn = build_dec ? (uint8_t *)(b + o_mdn) : nullptr;
+    h->w_tc_gu = build_tc ? (uint8_t *)(b + o_tgu) : nullptr;
+    h->w_tc_dn = build_tc ? (uint8_t *)(b + o_tdn) : nullptr;
     h->alpha_gate = (float *)(b + o_ag);
     h->alpha_up = (float *)(b + o_au);
     h->alpha_down = (float *)(b + o_ad);
     h->router_w = (float *)(b + o_rw);
     h->router_bias = w->router_bias ? (float *)(b + o_rb) : nullptr;
     h->qx = (int8_t *)(b + o_qx);
+    h->qxp = (int8_t *)(b + o_qxp);
+    h->zrow = (const int8_t *)(b + o_zr);
     h->sx = (float *)(b + o_sx);
     h->sumx = (int *)(b + o_sumx);
     h->logits = (float *)(b + o_lg);
@@ -323,60 +340,59 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->active = (int *)(b + o_act);
     h->n_active = (int *)(b + o_nact);
     h->blk_cnt = (int *)(b + o_blk);
-    h->h = (float *)(b + o_h);
-    h->qh = (int8_t *)(b + o_qh);
-    h->sh = (float *)(b + o_sh);
-    h->sumqh = (int *)(b + o_sumqh);
-    h->ye = (float *)(b + o_ye);
+    h->pieces = build_tc ? (int4 *)(b + o_pc) : nullptr;
+    h->n_pieces = (int *)(b + o_npc);
+    h->pscale = build_tc ? (float *)(b + o_ps) : nullptr;
+    h->hscratch = build_tc ? (float *)(b + o_hs) : nullptr;
+    h->h = build_dec ? (float *)(b + o_h) : nullptr;
+    h->qh = build_tc ? (int8_t *)(b + o_qh) : nullptr;
+    h->sh = build_tc ? (float *)(b + o_sh) : nullptr;
+    h->ye = build_dec ? (float *)(b + o_ye) : nullptr;
+    h->acc_hi = build_tc ? (int16_t *)(b + o_ahi) : nullptr;
+    h->acc_lo = build_tc ? (uint32_t *)(b + o_alo) : nullptr;
     h->tg_cnt = (unsigned *)(b + o_tg);
     h->glob_cnt = (unsigned *)(b + o_gc);
-    h->exp_cnt = (unsigned *)(b + o_ec);
     h->comb_cnt = (unsigned *)(b + o_cc);
-    h->arrive = (unsigned *)(b + o_rdy);
-    {
-        int optin = 0;
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
-        h->dec_optin = optin;
-        h->dec_persistent = decode_smem_bytes(h->D, h->F, 1, h->K, h->E) <= (size_t)optin;
-    }
+    h->dx_clear = (unsigned *)(b + o_dx);
     h->xn = (uint16_t *)(b + o_xn);
-    h->zrow = (const int8_t *)(b + o_zr);
+    h->wait_ns = kDefaultWaitNs;
+    h->ctr_base = b + o_ctr;
+    h->ctr_bytes = o_ctr_end - o_ctr;
 
     cudaStream_t st = (cudaStream_t)stream;
     // the whole workspace starts at zero: counters must, and every index array
     // then holds in-range values even before its first write
-    cudaMemsetAsync(b + o_qx, 0, ar.size - o_qx, st);
+    cudaMemsetAsync(b + o_ws, 0, ar.size - o_ws, st);
     cudaMemcpyAsync(h->alpha_gate, w->alpha_gate, E * F * 4, cudaMemcpyDeviceToDevice, st);
     cudaMemcpyAsync(h->alpha_up, w->alpha_up, E * F * 4, cudaMemcpyDeviceToDevice, st);
     cudaMemcpyAsync(h->alpha_down, w->alpha_down, E * D * 4, cudaMemcpyDeviceToDevice, st);
     cudaMemcpyAsync(h->router_w, w->router_w, E * D * 4, cudaMemcpyDeviceToDevice, st);
     if (w->router_bias) cudaMemcpyAsync(h->router_bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, st);
     const int cap = h->num_sms * 16;
-    repack_gu_kernel<<<grid_for(E * (F / 16) * (D / 64) * 128, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E,
-                                                                                     h->D, h->F, (uint32_t *)h->w_gu);
-    repack_dn_kernel<<<grid_for(E * (D / 32) * (F / 64) * 128, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
-                                                                                    (uint32_t *)h->w_dn);
-    repack_tc_gu_kernel<<<grid_for(E * F * D / 8, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E, h->D, h->F,
-                                                                          (uint32_t *)h->w_tc_gu);
-    repack_tc_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
-                                                                           (uint32_t *)h->w_tc_dn);
-    if (make_act_map(&h->map_xperm, h->xperm, S, D) || make_act_map(&h->map_qh, h->qh, S, F)) {
-        cudaFree(h->base);
-        cudaFreeHost(h->flag_host);
-        delete h;
-        return MAPLE_ERR_CUDA;
+    if (build_dec) {
+        repack_mma_gu_kernel<<<grid_for(E * F * D / 8, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E, h->D, h->F,
+                                                                               (uint32_t *)h->w_mma_gu);
+        repack_mma_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
+                                                                                (uint32_t *)h->w_mma_dn);
     }
+    if (build_tc) {
+        repack_tc_gu_kernel<<<grid_for(E * F * D / 8, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E, h->D, h->F,
+                                                                              (uint32_t *)h->w_tc_gu);
+        repack_tc_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
+                                                                               (uint32_t *)h->w_tc_dn);
+    }
+    bool maps_ok = make_act_map(&h->map_qxp, h->qxp, T64, D, 1, false) == MAPLE_OK;
+    if (build_tc)
+        maps_ok = maps_ok && make_act_map(&h->map_qx, h->qx, Tm, D, 1, true) == MAPLE_OK &&
+                  make_act_map(&h->map_qh, h->qh, S, F, kTcMaxN, true) == MAPLE_OK;
     // allow every kernel the largest dynamic shared memory the device offers, so
     // that handles of different shapes never cap one another's launches
-    allow_max_smem((const void *)tc_gemm_kernel<0>, h->device);
-    allow_max_smem((const void *)tc_gemm_kernel<1>, h->device);
-    allow_max_smem((const void *)pick_route(h->D, h->E), h->device);
-    allow_max_smem((const void *)pick_qtopk(h->D, h->E), h->device);
-    allow_max_smem((const void *)router_gemm_kernel, h->device);
-    allow_max_smem((const void *)pick_gateup(h->D), h->device);
-    allow_max_smem((const void *)pick_down(h->F), h->device);
-    allow_max_smem((const void *)decode_experts_kernel, h->device);
-    if (cudaGetLastError() != cudaSuccess) {
+    const void *kernels[] = {(const void *)tc_gemm_kernel<0>, (const void *)tc_gemm_kernel<1>,
+                             (const void *)pick_route(h->D, h->E), (const void *)pick_qtopk(h->D, h->E),
+                             (const void *)router_gemm_kernel, (const void *)decode_mma_kernel};
+    bool smem_ok = true;
+    for (const void *k : kernels) smem_ok = allow_max_smem(k, h->device) && smem_ok;
+    if (!maps_ok || !smem_ok || cudaGetLastError() != cudaSuccess) {
         cudaFree(h->base);
         cudaFreeHost(h->flag_host);
         delete h;
@@ -392,20 +408,29 @@ static int check_handle(maple_moe_t h)
     return MAPLE_OK;
 }
 
-static int take_flag(maple_moe_t h)
+// Report (and clear) what kernels of earlier calls flagged.  After a timeout the
+// self-resetting counters may hold stale values: zero them on this call's
+// stream first, so that the next call starts from the state create left.
+static int take_flag(maple_moe_t h, cudaStream_t st)
 {
-    unsigned f = __atomic_exchange_n(h->flag_host, 0u, __ATOMIC_ACQ_REL);
+    const unsigned f = __atomic_exchange_n(h->flag_host, 0u, __ATOMIC_ACQ_REL);
+    if ((f & MAPLE_DEVFLAG_TIMEOUT) || h->pending_reset) {
+        h->pending_reset = false;
+        if (cudaMemsetAsync(h->ctr_base, 0, h->ctr_bytes, st) != cudaSuccess) return MAPLE_ERR_CUDA;
+        if (f & MAPLE_DEVFLAG_TIMEOUT) return MAPLE_ERR_TIMEOUT;
+    }
     return f ? MAPLE_ERR_DEVICE_FLAG : MAPLE_OK;
 }
 
 // routing stage: quantise, logits, top-k (+ the permutation)
 static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
                      float *out_w, int32_t *out_counts, bool permute, bool pieces, cudaStream_t st,
-                     unsigned *clear = nullptr, int n_clear = 0)
+                     unsigned *clear = nullptr, int n_clear = 0, bool frag = false)
 {
     RouteArgs a;
     memset(&a, 0, sizeof a);
     a.x = x;
+    a.qxp = frag ? h->qxp : nullptr;   // the decode kernel's fragment-ordered q_x
     a.T = T;
     a.D = h->D;
     a.E = h->E;
@@ -477,6 +502,8 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
         p.tap_perm = a.tap_perm;
         p.pieces = pieces ? h->pieces : nullptr;
         p.n_pieces = h->n_pieces;
+        p.sx = h->sx;
+        p.pscale = pieces ? h->pscale : nullptr;
         p.flag = h->flag_dev;
         const int nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
         perm_count_kernel<<<nblk, 256, 0, st>>>(p);
@@ -486,100 +513,85 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     return launch_status();
 }
 
-// 1 when the persistent decode kernel runs this batch (it fits the shape and T), else 0
-static int decode_ring_slots(maple_moe_t h, int T)
+// Items per claimed chunk of the decode kernel: about a third of a CTA's
+// expected share (claims then even out the load), a power of two dividing
+// the items of a unit.  The expected number of units is the expected number
+// of distinct experts of T tokens under uniform routing.
+static void dx_chunks(maple_moe_t h, int T, int &c1, int &c2)
 {
-    if (!h->dec_persistent || T > kRouteSmallT || (int64_t)T * h->E > kFusedMarkBytes) return 0;
-    return decode_smem_bytes(h->D, h->F, T, h->K, h->E) <= (size_t)h->dec_optin ? 1 : 0;
+    const int G1 = h->F / 8, G2 = h->D / (16 * (h->D / h->F));
+    double miss = 1.0;
+    for (int t = 0; t < T; t++) miss *= 1.0 - (double)h->K / h->E;
+    const double units = h->E * (1.0 - miss);
+    const double want = units * G1 / (3.0 * h->num_sms);
+    c1 = 1;
+    while (c1 * 2 <= G1 && c1 * 2 <= want) c1 *= 2;
+    c2 = 1;
+    while (c2 * 2 <= G2 && c2 * 2 <= (double)c1 * G2 / G1) c2 *= 2;
 }
 
-static int run_experts(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
-                       int nw, cudaStream_t st)
+// the decode kernel: permutation, gate/up + SwiGLU, requantisation, down and
+// combine in one persistent launch (one CTA per SM)
+static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps, int nslot,
+                           cudaStream_t st)
 {
-    GemvArgs g;
-    memset(&g, 0, sizeof g);
-    g.T = T;
-    g.D = h->D;
-    g.E = h->E;
-    g.K = h->K;
-    g.F = h->F;
-    g.active = h->active;
-    g.n_active = h->n_active;
-    g.counts = h->counts;
-    g.offsets = h->offsets;
-    g.perm = h->perm;
-    g.inv = h->inv;
-    g.topk_w = h->topk_w;
-    g.qx = h->qx;
-    g.sx = h->sx;
-    g.sumx = h->sumx;
-    g.w_gu = h->w_gu;
-    g.w_dn = h->w_dn;
-    g.alpha_gate = h->alpha_gate;
-    g.alpha_up = h->alpha_up;
-    g.alpha_down = h->alpha_down;
-    g.h = h->h;
-    g.qh = h->qh;
-    g.sh = h->sh;
-    g.sumqh = h->sumqh;
-    g.ye = h->ye;
-    g.y = y;
-    g.resid = resid;
-    g.exp_cnt = h->exp_cnt;
-    g.comb_cnt = h->comb_cnt;
+    DxArgs d;
+    memset(&d, 0, sizeof d);
+    d.T = T;
+    d.D = h->D;
+    d.E = h->E;
+    d.K = h->K;
+    d.F = h->F;
+    d.topk_idx = h->topk_idx;
+    d.topk_w = h->topk_w;
+    d.sx = h->sx;
+    d.sumx = h->sumx;
+    d.w_gu = h->w_mma_gu;
+    d.w_dn = h->w_mma_dn;
+    d.alpha_gate = h->alpha_gate;
+    d.alpha_up = h->alpha_up;
+    d.alpha_down = h->alpha_down;
+    d.h = h->h;
+    const int S = T * h->K;
+    d.amax = h->dx_clear;
+    d.arrive = h->dx_clear + S;
+    d.claim = (int *)(h->dx_clear + S + dx_max_units(h->E, S));
+    d.comb = h->comb_cnt;
+    d.ye = h->ye;
+    d.y = y;
+    d.resid = resid;
     if (taps) {
-        g.tap_acc_gate = taps->acc_gate;
-        g.tap_acc_up = taps->acc_up;
-        g.tap_acc_down = taps->acc_down;
-        g.tap_qh = taps->q_h;
-        g.tap_sh = taps->s_h;
+        d.tap_acc_gate = taps->acc_gate;
+        d.tap_acc_up = taps->acc_up;
+        d.tap_acc_down = taps->acc_down;
+        d.tap_qh = taps->q_h;
+        d.tap_sh = taps->s_h;
+        d.tap_counts = taps->expert_counts;
+        d.tap_offsets = taps->expert_offsets;
+        d.tap_perm = taps->perm;
     }
-    g.flag_dev = h->flag_dev;
-    if (nw) {
-        // persistent: one CTA per SM builds the permutation from
-        // the router's top-k, then streams gate/up and down
-        DecodeArgs d;
-        memset(&d, 0, sizeof d);
-        d.g = g;
-        d.arrive = h->arrive;
-        d.aslot_bytes = dec_aslot_bytes(h->D, h->F);
-        d.zrow = h->zrow;
-        d.item_ctr = (int *)(h->arrive + h->E);
-        d.topk_idx = h->topk_idx;
-        d.topk_w = h->topk_w;
-        if (taps) {
-            d.tap_counts = taps->expert_counts;
-            d.tap_offsets = taps->expert_offsets;
-            d.tap_perm = taps->perm;
-        }
-        // h->arrive and the item counter were zeroed by the routing kernel.  A plain
-        // launch: the kernel needs no co-residency, since a CTA only ever waits on
-        // items that running CTAs have already claimed (gate/up items, all claimed
-        // before any down item, wait on nothing of other CTAs).
-        // Launched as a programmatic dependent of the routing kernel before it: its
-        // launch and set-up overlap the router's tail, and griddepcontrol.wait in
-        // the kernel orders every read of the routing outputs after that grid.
-        cudaLaunchConfig_t lc;
-        memset(&lc, 0, sizeof lc);
-        lc.gridDim = dim3(h->num_sms);
-        lc.blockDim = dim3(kDecThreads);
-        lc.dynamicSmemBytes = decode_smem_bytes(h->D, h->F, T, h->K, h->E);
-        lc.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        lc.attrs = attr;
-        lc.numAttrs = 1;
-        if (cudaLaunchKernelEx(&lc, decode_experts_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
-        stage_event(h, 2, st);
-        stage_event(h, 3, st);
-        return launch_status();
-    }
-    // one CTA per (active expert, row block); CTAs past the active experts exit at once
-    const int64_t max_active = (int64_t)T * h->K < h->E ? (int64_t)T * h->K : h->E;
-    pick_gateup(h->D)<<<(unsigned)(max_active * (h->F / 32)), kGemvWarps * 32, gemv_smem_bytes(h->D), st>>>(g);
+    d.flag = h->flag_dev;
+    d.wait_ns = h->wait_ns;
+    d.stall = (h->debug_flags & MAPLE_DEBUG_STALL_DOWN) ? 1 : 0;
+    dx_chunks(h, T, d.chunk1, d.chunk2);
+    d.nslot = nslot;
+    // Launched as a programmatic dependent of the routing kernel before it: its
+    // launch and set-up overlap the router's tail, and griddepcontrol.wait in the
+    // kernel orders every read of the routing outputs after that grid.  A plain
+    // launch otherwise: a CTA only waits on work that running CTAs have claimed.
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof lc);
+    lc.gridDim = dim3(h->num_sms);
+    lc.blockDim = dim3(kDxThreads);
+    lc.dynamicSmemBytes = DxSmem(h->D, h->F, T, h->K, h->E, nslot).total;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, decode_mma_kernel, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 2, st);
-    pick_down(h->F)<<<(unsigned)(max_active * (h->D / 128)), kGemvWarps * 32, gemv_smem_bytes(h->F), st>>>(g);
     stage_event(h, 3, st);
     return launch_status();
 }
@@ -600,7 +612,7 @@ extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int3
     int rc = check_handle(h);
     if (rc) return rc;
     if (T < 0 || T > h->Tm) return MAPLE_ERR_INVALID_ARG;
-    if ((rc = take_flag(h))) return rc;
+    if ((rc = take_flag(h, (cudaStream_t)stream))) return rc;
     if (T == 0) return MAPLE_OK;
     if (!x || !aligned16(x)) return MAPLE_ERR_INVALID_ARG;
     for (const void *p : {(const void *)topk_idx, (const void *)topk_w, (const void *)expert_counts})
@@ -609,11 +621,11 @@ extern "C" int maple_moe_route(maple_moe_t h, const uint16_t *x, int32_t T, int3
                      (cudaStream_t)stream);
 }
 
-// tensor-core expert stage: gate/up grouped GEMM, requantise, down grouped GEMM, combine
+// tensor-core expert stage: gate/up grouped GEMM (SwiGLU and the requantisation
+// fused), down grouped GEMM, combine
 static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
                           cudaStream_t st)
 {
-    const int S = T * h->K;
     TcArgs g;
     memset(&g, 0, sizeof g);
     g.D = h->D;
@@ -622,54 +634,67 @@ static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, co
     g.pieces = h->pieces;
     g.n_pieces = h->n_pieces;
     g.perm = h->perm;
-    g.sx = h->sx;
     g.sh = h->sh;
     g.pscale = h->pscale;
     g.flag = h->flag_dev;
+    g.wait_ns = h->wait_ns;
     g.codes = h->w_tc_gu;
     g.alpha0 = h->alpha_gate;
     g.alpha1 = h->alpha_up;
-    g.out = h->h;
+    g.out = h->hscratch;
+    g.qh = h->qh;
     g.tap0 = taps ? taps->acc_gate : nullptr;
     g.tap1 = taps ? taps->acc_up : nullptr;
-    gather_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->qx, h->sx, h->perm, h->K, h->D, S, h->xperm, h->pscale);
-    tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_xperm, g);
-    requant_rows_kernel<<<(S + 7) / 8, 256, 0, st>>>(h->h, S, h->F, h->perm, h->qh, h->sh, taps ? taps->q_h : nullptr,
-                                                   taps ? taps->s_h : nullptr);
+    g.tap_qh = taps ? taps->q_h : nullptr;
+    g.tap_sh = taps ? taps->s_h : nullptr;
+    tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_qx, g);
     stage_event(h, 2, st);
     g.codes = h->w_tc_dn;
     g.alpha0 = h->alpha_down;
     g.alpha1 = nullptr;
-    g.out = h->ye;
+    g.out = nullptr;
+    g.qh = nullptr;
+    g.acc_hi = h->acc_hi;
+    g.acc_lo = h->acc_lo;
     g.tap0 = taps ? taps->acc_down : nullptr;
     g.tap1 = nullptr;
+    g.tap_qh = nullptr;
+    g.tap_sh = nullptr;
     tc_gemm_kernel<1><<<h->num_sms, kTcThreads, TcSmem<1>::kTotal, st>>>(h->map_qh, g);
-    combine_kernel<<<grid_for((int64_t)T * h->D / 4, 256, h->num_sms * 8), 256, 0, st>>>(h->ye, h->inv, h->topk_w, T,
-                                                                                       h->K, h->D, y, resid);
+    combine_kernel<<<grid_for((int64_t)T * h->D / 4, 256, h->num_sms * 8), 256, 0, st>>>(
+        h->acc_hi, h->acc_lo, h->alpha_down, h->sh, h->topk_idx, h->inv, h->topk_w, T, h->K, h->D, y, resid);
     stage_event(h, 3, st);
     return launch_status();
 }
 
-static bool use_tc(maple_moe_t h, int T)
+// ring slots of the decode kernel for a batch of T tokens, 0 when it does not serve it
+static int dec_slots(maple_moe_t h, int T)
 {
-    if (h->cfg_flags & MAPLE_CFG_FORCE_GEMV) return false;
-    if (h->cfg_flags & MAPLE_CFG_FORCE_TC) return true;
-    return T > h->dmax;
+    if (!h->w_mma_gu || T > kRouteSmallT || (int64_t)T * h->E > kFusedMarkBytes) return 0;
+    if (T > h->dmax && !(h->cfg_flags & MAPLE_CFG_FORCE_GEMV)) return 0;
+    return dx_ring_slots(h->D, h->F, T, h->K, h->E, (size_t)h->optin);
 }
 
 static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const float *resid,
                         const maple_moe_taps *taps, cudaStream_t st)
 {
-    const bool tc = use_tc(h, T);
-    const int nw = tc ? 0 : decode_ring_slots(h, T);
+    const int nslot = (h->cfg_flags & MAPLE_CFG_FORCE_TC) ? 0 : dec_slots(h, T);
+    if (!nslot && !h->w_tc_gu) return MAPLE_ERR_UNSUPPORTED_SHAPE;   // decode-only handle, T too large
     stage_event(h, 0, st);
-    // the persistent decode kernel builds its own permutation from the top-k; the
-    // routing kernel zeroes its arrival counters and its work-item counter
-    int rc = nw ? run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, st, h->arrive, h->E + 1)
-                : run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, tc, st);
+    int rc;
+    if (nslot) {
+        // the decode kernel builds its own permutation from the top-k; the routing
+        // kernel zeroes its maxima, unit arrivals and chunk counter, and writes the
+        // fragment-ordered q_x
+        const int S = T * h->K;
+        rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, st, h->dx_clear,
+                       (int)(S + dx_max_units(h->E, S) + 1), true);
+    } else {
+        rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, true, st);
+    }
     if (rc) return rc;
     stage_event(h, 1, st);
-    return tc ? run_experts_tc(h, T, y, resid, taps, st) : run_experts(h, T, y, resid, taps, nw, st);
+    return nslot ? run_experts_dec(h, T, y, resid, taps, nslot, st) : run_experts_tc(h, T, y, resid, taps, st);
 }
 
 extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const maple_moe_taps *taps,
@@ -678,7 +703,7 @@ extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, fl
     int rc = check_handle(h);
     if (rc) return rc;
     if (T < 0 || T > h->Tm) return MAPLE_ERR_INVALID_ARG;
-    if ((rc = take_flag(h))) return rc;
+    if ((rc = take_flag(h, (cudaStream_t)stream))) return rc;
     if (T == 0) return MAPLE_OK;
     if (!x || !y || !aligned16(x) || !aligned16(y)) return MAPLE_ERR_INVALID_ARG;
     if ((rc = check_taps(taps))) return rc;
@@ -698,7 +723,7 @@ extern "C" int maple_moe_stack_forward(const maple_moe_t *layers, int32_t n_laye
         if (T < 0 || T > a->Tm) return MAPLE_ERR_INVALID_ARG;
     }
     for (int l = 0; l < n_layers; l++) {
-        int rc = take_flag(layers[l]);
+        int rc = take_flag(layers[l], (cudaStream_t)stream);
         if (rc) return rc;
     }
     if (T == 0) return MAPLE_OK;
@@ -739,6 +764,17 @@ extern "C" int maple_moe_device_flags(maple_moe_t h, uint32_t *flags, int32_t cl
     if (!flags) return MAPLE_ERR_INVALID_ARG;
     *flags = clear ? __atomic_exchange_n(h->flag_host, 0u, __ATOMIC_ACQ_REL)
                    : __atomic_load_n(h->flag_host, __ATOMIC_ACQUIRE);
+    if (clear && (*flags & MAPLE_DEVFLAG_TIMEOUT)) h->pending_reset = true;
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_set_debug(maple_moe_t h, int32_t wait_limit_us, uint32_t debug_flags)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (wait_limit_us < 0 || wait_limit_us > 60000000 || (debug_flags & ~MAPLE_DEBUG_STALL_DOWN)) return MAPLE_ERR_INVALID_ARG;
+    h->wait_ns = wait_limit_us ? (uint64_t)wait_limit_us * 1000ull : kDefaultWaitNs;
+    h->debug_flags = debug_flags;
     return MAPLE_OK;
 }
 
@@ -781,7 +817,10 @@ void *g_noalloc_addr[kNoallocMaxDevices];   // device address of g_route_scratch
 
 // Once per device, with that device current: look up the device address of
 // the scratch array (in host code its name is only a host-side stand-in) and
-// raise the routing kernels' dynamic shared-memory limit.
+// raise the routing kernels' dynamic shared-memory limit.  Both are cached for
+// the life of the process; a cudaDeviceReset invalidates them (the module is
+// loaded again, at a new address), so a process that resets a device must not
+// call this entry point on that device afterwards.
 int noalloc_scratch(void **out)
 {
     int dev = -1;
@@ -796,10 +835,12 @@ int noalloc_scratch(void **out)
             cudaGetLastError();
             return MAPLE_ERR_CUDA;
         }
+        bool ok = true;
         for (int ni = 1; ni <= 16; ni *= 2) {
-            allow_max_smem((const void *)pick_route(ni * 256, 16), dev);
-            allow_max_smem((const void *)pick_route(ni * 256, 1024), dev);
+            ok = allow_max_smem((const void *)pick_route(ni * 256, 16), dev) && ok;
+            ok = allow_max_smem((const void *)pick_route(ni * 256, 1024), dev) && ok;
         }
+        if (!ok) return MAPLE_ERR_CUDA;
         g_noalloc_addr[dev] = p;
     }
     *out = g_noalloc_addr[dev];

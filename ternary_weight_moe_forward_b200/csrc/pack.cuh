@@ -1,5 +1,5 @@
-// 2-bit ternary packer and the re-layout of packed weights into the GEMV
-// layout (run once, at create).
+// 2-bit ternary packer, the re-layout of packed weights into the decode
+// kernel's MMA-tile layout (run once, at create), and the stack's RMSNorm.
 #pragma once
 
 #include "common.cuh"
@@ -29,39 +29,38 @@ __global__ void pack_ternary_kernel(const int8_t *values, int64_t n_words, uint3
     }
 }
 
-// gate/up interchange [E][F][D/16] (two tensors) -> GEMV layout; one thread per output word
-__global__ void repack_gu_kernel(const uint32_t *gate, const uint32_t *up, int E, int D, int F, uint32_t *out)
+// gate/up interchange -> MMA-tile layout (layout.cuh); one thread per output word
+__global__ void repack_mma_gu_kernel(const uint32_t *gate, const uint32_t *up, int E, int D, int F, uint32_t *out)
 {
-    const int C = D / 64, G = F / 16;
-    const int64_t n = (int64_t)E * G * C * 32 * 4;
+    const int KB = D / 128, NT = F / 8;
+    const int64_t n = (int64_t)E * NT * KB * 128;
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
         int64_t q = o;
-        const int w = q % 4; q /= 4;
+        const int i = q % 4; q /= 4;
         const int lane = q % 32; q /= 32;
-        const int c = q % C; q /= C;
-        const int g = q % G; q /= G;
+        const int kb = q % KB; q /= KB;
+        const int t = q % NT; q /= NT;
         const int e = (int)q;
-        const int r = 16 * g + (lane & 15);
-        const uint32_t *src = (lane < 16 ? gate : up) + ((int64_t)e * F + r) * (D / 16);
-        out[o] = gemv_word(src[4 * c + w]);
+        const int r = mma_word_row(lane, i);   // rows 0..7 gate, 8..15 up, outputs 8t .. 8t+7
+        const uint32_t *src = (r < 8 ? gate : up) + ((int64_t)e * F + 8 * t + (r & 7)) * (D / 16);
+        out[o] = mma_word(src, lane, i, kb);
     }
 }
 
-// down interchange [E][D][F/16] -> GEMV layout
-__global__ void repack_dn_kernel(const uint32_t *down, int E, int D, int F, uint32_t *out)
+// down interchange -> MMA-tile layout
+__global__ void repack_mma_dn_kernel(const uint32_t *down, int E, int D, int F, uint32_t *out)
 {
-    const int C = F / 64, G = D / 32;
-    const int64_t n = (int64_t)E * G * C * 32 * 4;
+    const int KB = F / 128, NT = D / 16;
+    const int64_t n = (int64_t)E * NT * KB * 128;
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
         int64_t q = o;
-        const int w = q % 4; q /= 4;
+        const int i = q % 4; q /= 4;
         const int lane = q % 32; q /= 32;
-        const int c = q % C; q /= C;
-        const int g = q % G; q /= G;
+        const int kb = q % KB; q /= KB;
+        const int t = q % NT; q /= NT;
         const int e = (int)q;
-        const int row = 32 * g + lane;
-        const uint32_t *src = down + ((int64_t)e * D + row) * (F / 16);
-        out[o] = gemv_word(src[4 * c + w]);
+        const uint32_t *src = down + ((int64_t)e * D + 16 * t + mma_word_row(lane, i)) * (F / 16);
+        out[o] = mma_word(src, lane, i, kb);
     }
 }
 

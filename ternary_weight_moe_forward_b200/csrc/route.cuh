@@ -3,6 +3,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "layout.cuh"
 
 namespace maple {
 
@@ -19,6 +20,7 @@ struct RouteArgs {
     const float *Wr, *bias;
     // workspace outputs
     int8_t *qx;
+    int8_t *qxp;   // optional: q_x rows in the fragment order of the decode kernel (frag_word_pos)
     float *sx;
     int *sumx;
     float *logits;
@@ -146,6 +148,12 @@ __device__ void quantize_token_warp(const RouteArgs &a, int t, const uint16_t *x
         size_t off = (size_t)t * a.D + 256 * i + 8 * lane;
         *reinterpret_cast<uint2 *>(a.qx + off) = pv;
         if (a.tap_qx) *reinterpret_cast<uint2 *>(a.tap_qx + off) = pv;
+        if (a.qxp) {
+            // the two words sit at word positions 2(l%16), +1 of 128-column block 2i + l/16
+            uint32_t *blk = reinterpret_cast<uint32_t *>(a.qxp + (size_t)t * a.D + 256 * i + 128 * (lane >> 4));
+            blk[frag_word_pos(2 * (lane & 15))] = packed[0];
+            blk[frag_word_pos(2 * (lane & 15) + 1)] = packed[1];
+        }
     }
     sum = warp_sum_int(sum);
     if (lane == 0) {
@@ -267,7 +275,7 @@ __device__ void build_marks(uint8_t *mark, const int *idx, int t0, int nt, int K
 // place the block's slots: expert e's first slot in this block goes to base_e(e)
 template <class BaseFn>
 __device__ void scatter_marks(const uint8_t *mark, int t0, int nt, int K, int E, BaseFn base_e, int *perm, int *inv,
-                              int *tap_perm)
+                              int *tap_perm, const float *sx = nullptr, float *pscale = nullptr)
 {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int p = base_e(e);
@@ -278,6 +286,7 @@ __device__ void scatter_marks(const uint8_t *mark, int t0, int nt, int K, int E,
                 perm[p] = s;
                 inv[s] = p;
                 if (tap_perm) tap_perm[p] = s;
+                if (pscale) pscale[p] = sx[t0 + t];
                 p++;
             }
         }
@@ -424,6 +433,8 @@ struct PermArgs {
     int *out_counts, *tap_offsets, *tap_perm;
     int4 *pieces;   // optional: expert slot ranges of at most kPieceSlots for the grouped GEMM
     int *n_pieces;
+    const float *sx;   // with pscale: s_x of every token
+    float *pscale;     // optional: s_x of each position's token (the tensor-core path's column scales)
     unsigned *flag;
 };
 
@@ -484,18 +495,35 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(PermArgs a)
         }
     }
     if (a.pieces) {
-        // split every expert's slots into ceil(count / kPieceSlots) near-equal ranges
+        // split every expert's slots into ceil(count / kPieceSlots) near-equal
+        // ranges, listed by size, largest first (a counting sort over the sizes;
+        // the order of equal sizes is arbitrary: every piece is computed on its
+        // own, so it changes no result, only which CTA takes which piece)
+        __shared__ int s_size[kPieceSlots + 1];
+        for (int i = threadIdx.x; i <= kPieceSlots; i += blockDim.x) s_size[i] = 0;
+        __syncthreads();
         const int e = threadIdx.x;
         const int cnt = e < a.E ? s_cnt[e] : 0;
         const int np = (cnt + kPieceSlots - 1) / kPieceSlots;
-        int total;
-        const int base = block_excl_scan(np, s_warp, &total);
-        for (int i = 0; i < np; i++) {
-            const int q = cnt / np, rem = cnt % np;
-            const int start = i * q + min(i, rem);
-            a.pieces[base + i] = make_int4(e, s_off[e] + start, q + (i < rem ? 1 : 0), 0);
+        const int q = np ? cnt / np : 0, rem = np ? cnt % np : 0;
+        if (rem) atomicAdd(&s_size[q + 1], rem);
+        if (np - rem) atomicAdd(&s_size[q], np - rem);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = 0;   // first list position of each size, sizes in descending order
+            for (int z = kPieceSlots; z >= 1; z--) {
+                const int c = s_size[z];
+                s_size[z] = run;
+                run += c;
+            }
+            *a.n_pieces = run;
         }
-        if (threadIdx.x == 0) *a.n_pieces = total;
+        __syncthreads();
+        for (int i = 0; i < np; i++) {
+            const int sz = q + (i < rem ? 1 : 0);
+            const int start = i * q + min(i, rem);
+            a.pieces[atomicAdd(&s_size[sz], 1)] = make_int4(e, s_off[e] + start, sz, 0);
+        }
     }
 }
 
@@ -506,7 +534,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(PermArgs a)
     const int nt = min(kPermBlockTokens, a.T - t0);
     build_marks(s_mark, a.idx, t0, nt, a.K, a.E, nullptr);
     const int *base = a.blk_cnt + (size_t)blockIdx.x * a.E;
-    scatter_marks(s_mark, t0, nt, a.K, a.E, [&](int e) { return base[e]; }, a.perm, a.inv, a.tap_perm);
+    scatter_marks(s_mark, t0, nt, a.K, a.E, [&](int e) { return base[e]; }, a.perm, a.inv, a.tap_perm, a.sx,
+                  a.pscale);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,30 +1,43 @@
 // Prefill expert stage on the 5th-generation tensor cores (tcgen05, int8).
 //
 // Grouped GEMM over "pieces": a piece is up to 128 consecutive slots of one
-// expert in the permutation.  A tile is (piece, 128-row block of the weight
-// matrix).  The MMA computes D[128 weight rows][N slots] (M = 128, N = the
-// piece size rounded up to 16, K = 32 per instruction) with
+// expert in the permutation (the routing stage lists them largest first).  A
+// tile is (piece, 128-row block of the weight matrix).  The MMA computes
+// D[128 weight rows][N slots] (M = 128, N = the piece size rounded up to 16,
+// K = 32 per instruction) with
 //   A = ternary weights, expanded in shared memory from 2-bit codes to int8
 //       {0, +64, -64} (64 * t: the code sits in the two top bits of the byte),
-//   B = int8 activation rows of the piece's slots, loaded by the tensor
-//       memory accelerator (TMA) from a slot-ordered copy of the rows,
+//   B = int8 activation rows of the piece's slots,
 // both K-major with the 128-byte swizzle, the int32 accumulator in tensor
 // memory (two accumulator buffers, so the epilogue of one tile overlaps the
-// MMAs of the next).  The accumulator is 64x the ternary dot product; the epilogue shifts
-// it back (exact).
+// MMAs of the next).  The accumulator is 64x the ternary dot product; the
+// epilogue shifts it back (exact).
 //
-// Warp roles (16 warps): warp 0 issues the bulk copies of the 2-bit codes
-// and the TMA loads of the activation tiles, warp 1 issues the MMAs (and owns
-// the TMEM allocation), warps 4..7 run the epilogue (TMEM lane quarter =
-// warp % 4), warps 8..15 expand the codes into int8 tiles.  Stage hand-off uses mbarriers; every wait is
-// bounded in time and a timeout makes the whole CTA drain and return with a
-// device flag set.
+// Warp roles (20 warps): warp 0 issues the bulk copies of the 2-bit codes and
+// the activation loads, warp 1 issues the MMAs (and owns the TMEM
+// allocation), warps 4..11 run the epilogue (TMEM lane quarter = warp % 4,
+// two warps per quarter splitting the columns), warps 12..19 expand the codes
+// into int8 tiles.  Stage hand-off uses mbarriers; every wait is bounded in
+// time and a timeout makes the whole CTA drain and return with a device flag
+// set.
 //
 // Mode 0 (gate/up): A = gate rows and up rows of one 128-row block (two MMAs
-// per K step, gate and up accumulators 128 columns apart), B = q_x rows of the
-// slots' tokens; the epilogue writes h = SiLU(g) * u (fp32, slot order).
+// per K step, gate and up accumulators 128 columns apart), B = the q_x rows of
+// the slots' tokens, fetched straight from q_x by TMA gather (four rows per
+// copy).  A CTA takes whole pieces (all F/128 row blocks of one piece in a
+// row, pieces dealt out in a snake order over the size-sorted list), so that
+// it holds every h value of its slots: the epilogue writes h = SiLU(g) * u
+// (fp32) to a per-CTA scratch area that stays in L2 and keeps each slot's
+// running absmax in shared memory; after the piece's last row block the
+// epilogue warps requantise the slots (int8 absmax codes q_h, scale s_h),
+// so no fp32 h leaves the chip.
 // Mode 1 (down): A = 128 output channels of the down matrix, B = q_h rows
-// (consecutive slot positions); the epilogue writes yE (fp32, slot order).
+// (consecutive slot positions, a plain 2-D TMA load); tiles are dealt out
+// round robin.  The epilogue stores the exact int32 accumulators, which need
+// 17 bits (|acc| <= 127 * 512): acc >> 1 as int16 and the lowest bit in a bit
+// plane (one 32-bit word per 32 channels, by warp ballot), 2.125 bytes per
+// value instead of 4 for fp32 yE; combine_kernel rebuilds acc and scales it
+// exactly as the oracle does.
 #pragma once
 
 #include <cuda.h>
@@ -33,7 +46,9 @@
 
 namespace maple {
 
-constexpr int kTcThreads = 512;
+constexpr int kTcThreads = 640;
+constexpr int kTcEpiWarp0 = 4, kTcEpiWarps = 8;     // epilogue warps 4..11
+constexpr int kTcProdWarp0 = 12, kTcProdWarps = 8;  // code-expanding warps 12..19
 constexpr int kTcMaxN = 128;
 constexpr int kTcBK = 128;  // K elements (bytes) per stage = one swizzle row
 
@@ -74,22 +89,29 @@ struct TcSmem {
     static constexpr int kA = 0, kB = TcCfg<MODE>::kABytes, kCodes = kB + kBBytes;
     static constexpr int kBars = TcCfg<MODE>::kStages * kStage;   // barriers, TMEM holder, abort word: 256 B
     static constexpr int kMeta = kBars + 256;                       // epilogue column metadata [2][2][128]
-    static constexpr int kTotal = kMeta + 2 * 2 * kTcMaxN * 4;
+    static constexpr int kAmax = kMeta + 2 * 2 * kTcMaxN * 4;       // mode 0: per-slot absmax of h [128]
+    static constexpr int kTotal = kAmax + kTcMaxN * 4;
     static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
 };
 
 struct TcArgs {
     int D, F, K;
-    const int4 *pieces;      // {expert, first position, count, 0}
+    const int4 *pieces;      // {expert, first position, count, 0}, largest first
     const int *n_pieces;
     const uint8_t *codes;    // tensor-core layout
     const int *perm;         // position -> slot
-    const float *sx, *sh;
+    float *sh;               // mode 0: written (s_h per position); mode 1: read
     const float *pscale;     // mode 0: s_x of each position's token
     const float *alpha0, *alpha1;  // mode 0: gate, up; mode 1: down, unused
-    float *out;              // mode 0: h [S][F]; mode 1: yE [S][D]
+    float *out;              // mode 0: per-CTA h scratch [gridDim][128][F]
+    int8_t *qh;              // mode 0: q_h [S][F] (position order)
+    int16_t *acc_hi;         // mode 1: down accumulators >> 1 [S][D] (position order)
+    uint32_t *acc_lo;        // mode 1: their lowest bits, [S][D/32] words (bit c%32 = channel c)
     int *tap0, *tap1;        // mode 0: acc_gate, acc_up; mode 1: acc_down
+    int8_t *tap_qh;          // mode 0 (slot order, may be null)
+    float *tap_sh;
     unsigned *flag;
+    uint64_t wait_ns;        // limit of every bounded wait
 };
 
 // ---------------------------------------------------------------------------
@@ -121,26 +143,20 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, far above any legitimate wait
+__device__ __forceinline__ uint64_t global_ns() { return global_timer_ns(); }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up
-// after kWaitLimitNs, or at once when another role of the CTA has given up;
+// after `limit` ns, or at once when another role of the CTA has given up;
 // returns false then (and raises the CTA abort word and the device flag).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, unsigned *flag)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort, unsigned *flag,
+                                          uint64_t limit)
 {
     if (mbar_test(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_test(bar, parity)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit) {
             *abort = 1u;
             set_flag(flag, MAPLE_DEVFLAG_TIMEOUT);
             return false;
@@ -153,6 +169,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+// four rows (y0..y3) of 128 bytes starting at column x, gathered by the TMA
+// unit from a row-major int8 matrix (tensor map box: 128 bytes x 1 row, 128-byte
+// swizzle) into 512 consecutive bytes of shared memory
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int x, int y0, int y1, int y2, int y3,
+                                            uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+        : "memory");
 }
 // 2-D tiled TMA load (box given by the tensor map) into 128B-swizzled shared memory
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
@@ -211,6 +239,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, int (&v)[32])
         : "r"(taddr)
         : "memory");
 }
+// 32 lanes x 16 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, int *v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // K-major operand, 128-byte swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart
@@ -239,7 +278,48 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w)
     return make_uint4((w << 6) & 0xC0C0C0C0u, (w << 4) & 0xC0C0C0C0u, (w << 2) & 0xC0C0C0C0u, w & 0xC0C0C0C0u);
 }
 
+// Column maxima of a warp's 32 x 32 block (lane = row, v[j] = column j, values
+// >= 0): after the five exchange levels lane l holds the maximum of column l.
+// At the level with distance o a lane keeps the half of its columns selected by
+// its bit o and sends the other half to lane l ^ o.
+__device__ __forceinline__ float warp_column_max(float (&v)[32])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+        const bool upper = lane & o;
+#pragma unroll
+        for (int j = 0; j < n / 2; j++) {
+            const float send = upper ? v[j] : v[j + n / 2];
+            const float keep = upper ? v[j + n / 2] : v[j];
+            v[j] = fmaxf(keep, __shfl_xor_sync(FULL, send, o));
+        }
+    }
+    return v[0];
+}
+
 // ---------------------------------------------------------------------------
+// The CTA's u-th tile: piece (index into the size-sorted list) and row block;
+// false once the CTA has no more.  Mode 0 deals out whole pieces: the j-th
+// piece of CTA b is j*G + b for even j and j*G + G-1-b for odd j (a snake over
+// the sorted list, which evens out the work), its R row blocks one after the
+// other.  Mode 1 deals out tiles round robin over the piece-major tile list.
+template <int MODE>
+__device__ __forceinline__ bool tc_tile(int u, int R, int n_pc, int &pc, int &rb)
+{
+    const int G = gridDim.x, b = blockIdx.x;
+    if (MODE == 0) {
+        const int j = u / R;
+        pc = j * G + ((j & 1) ? G - 1 - b : b);
+        rb = u - j * R;
+        return pc < n_pc;
+    }
+    const int t = b + u * G;
+    pc = t / R;
+    rb = t - pc * R;
+    return pc < n_pc;
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_constant__ CUtensorMap act_map, TcArgs a)
 {
@@ -254,6 +334,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
     int *meta_slot = (int *)(smem + L::kMeta);                      // [2][kTcMaxN]
     float *meta_scale = (float *)(smem + L::kMeta + 2 * kTcMaxN * 4);
+    unsigned *s_amax = (unsigned *)(smem + L::kAmax);               // mode 0: [kTcMaxN] |h| maxima (float bits)
     uint64_t *bars = (uint64_t *)(smem + L::kBars);
     // bars: codes_full[S], full[S], empty[S], acc_full[2], acc_empty[2], drain
     uint32_t *tmem_holder = (uint32_t *)(bars + 3 * S + 5);
@@ -266,17 +347,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; s++) {
             mbar_init(b_codes_full + 8 * s, 1);
-            mbar_init(b_full + 8 * s, 8);      // one arrival per producer warp
-            mbar_init(b_empty + 8 * s, 1);     // MMA commit
+            mbar_init(b_full + 8 * s, kTcProdWarps);   // one arrival per producer warp
+            mbar_init(b_empty + 8 * s, 1);             // MMA commit
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(b_acc_full + 8 * b, 1);
-            mbar_init(b_acc_empty + 8 * b, 4);  // one arrival per epilogue warp
+            mbar_init(b_acc_empty + 8 * b, kTcEpiWarps);  // one arrival per epilogue warp
         }
         mbar_init(b_drain, 1);
         *abort = 0u;
         fence_barrier_init();
     }
+    if (MODE == 0 && threadIdx.x < kTcMaxN) s_amax[threadIdx.x] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(tmem_holder), 512);
     tc_fence_before();
     __syncthreads();
@@ -285,61 +367,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 
     const int R = MODE == 0 ? a.F / 128 : a.D / 128;   // row blocks per piece
     const int KS = MODE == 0 ? a.D / kTcBK : a.F / kTcBK;
-    const int n_tiles = __ldg(a.n_pieces) * R;
+    const int n_pc = __ldg(a.n_pieces);
 
     if (warp == 0) {
-        // ---------------- bulk copies of the 2-bit codes
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            int4 npc = blockIdx.x < n_tiles ? a.pieces[blockIdx.x / R] : make_int4(0, 0, 0, 0);
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-                const int4 pc = npc;   // fetched one tile ahead
-                if (tile + (int)gridDim.x < n_tiles) npc = a.pieces[(tile + gridDim.x) / R];
-                const int rt = tile % R;
-                const uint8_t *src = a.codes + ((size_t)pc.x * R + rt) * KS * Cfg::kCodeBytes;
-                for (int ks = 0; ks < KS; ks++, it++) {
-                    const int s = it % S;
-                    if (!mbar_wait(b_empty + 8 * s, ((it / S) & 1) ^ 1, abort, a.flag)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_expect_tx(b_codes_full + 8 * s, Cfg::kCodeBytes + L::kBBytes);
-                    bulk_g2s(smem_addr(smem + s * L::kStage + L::kCodes), src + (size_t)ks * Cfg::kCodeBytes,
-                             Cfg::kCodeBytes, b_codes_full + 8 * s);
-                    tma_load_2d(smem_addr(smem + s * L::kStage + L::kB), &act_map, ks * kTcBK, pc.y,
-                                b_codes_full + 8 * s);
+        // ---------------- copies: the 2-bit codes (bulk) and the activation rows (TMA)
+        uint32_t it = 0;
+        bool ok = true;
+        int cur = -1;
+        int y[4] = {0, 0, 0, 0};   // mode 0: tokens of rows 4*lane .. 4*lane+3 of the current piece
+        int pc, rb;
+        for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++) {
+            const int4 P = a.pieces[pc];
+            const int npad = (P.z + 15) & ~15;
+            if (MODE == 0 && pc != cur) {
+                cur = pc;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int row = min(4 * lane + i, P.z - 1);   // padding rows repeat the last slot's token
+                    y[i] = __ldg(a.perm + P.y + row) / a.K;
                 }
             }
-            if (!ok) {
-                // drain: wait (bounded) for the copies still in flight, the last S issued
-                for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; j++) {
-                    const uint64_t t0 = global_ns();
-                    while (!mbar_test(b_codes_full + 8 * (j % S), (j / S) & 1) && global_ns() - t0 < kWaitLimitNs) {
-                    }
+            const uint8_t *src = a.codes + ((size_t)P.x * R + rb) * KS * Cfg::kCodeBytes;
+            for (int ks = 0; ks < KS; ks++, it++) {
+                const int s = it % S;
+                if (lane == 0) ok = mbar_wait(b_empty + 8 * s, ((it / S) & 1) ^ 1, abort, a.flag, a.wait_ns);
+                ok = __shfl_sync(FULL, ok, 0);
+                if (!ok) break;
+                const uint32_t cf = b_codes_full + 8 * s;
+                const uint32_t bdst = smem_addr(smem + s * L::kStage + L::kB);
+                if (lane == 0) {
+                    mbar_expect_tx(cf, Cfg::kCodeBytes + (MODE == 0 ? npad * kTcBK : L::kBBytes));
+                    bulk_g2s(smem_addr(smem + s * L::kStage + L::kCodes), src + (size_t)ks * Cfg::kCodeBytes,
+                             Cfg::kCodeBytes, cf);
+                    if (MODE == 1) tma_load_2d(bdst, &act_map, ks * kTcBK, P.y, cf);
+                }
+                __syncwarp();
+                if (MODE == 0 && 4 * lane < npad)
+                    tma_gather4(bdst + 4 * lane * kTcBK, &act_map, ks * kTcBK, y[0], y[1], y[2], y[3], cf);
+            }
+        }
+        if (!ok && lane == 0) {
+            // drain: wait (bounded) for the copies still in flight, the last S issued
+            for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; j++) {
+                const uint64_t t0 = global_ns();
+                while (!mbar_test(b_codes_full + 8 * (j % S), (j / S) & 1) && global_ns() - t0 < a.wait_ns) {
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issue
         if (lane == 0) {
-            uint32_t it = 0, tc = 0;
+            uint32_t it = 0, tcount = 0;
             bool ok = true;
-            int4 npc = blockIdx.x < n_tiles ? a.pieces[blockIdx.x / R] : make_int4(0, 0, 0, 0);
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, tc++) {
-                const int4 pc = npc;   // fetched one tile ahead
-                if (tile + (int)gridDim.x < n_tiles) npc = a.pieces[(tile + gridDim.x) / R];
-                const int npad = (pc.z + 15) & ~15;
+            int pc, rb;
+            for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++, tcount++) {
+                const int4 P = a.pieces[pc];
+                const int npad = (P.z + 15) & ~15;
                 const uint32_t idesc = idesc_i8(npad);
-                const uint32_t ab = tc & 1, dt = tmem + 256 * ab;
-                if (!mbar_wait(b_acc_empty + 8 * ab, ((tc >> 1) & 1) ^ 1, abort, a.flag)) {
+                const uint32_t ab = tcount & 1, dt = tmem + 256 * ab;
+                if (!mbar_wait(b_acc_empty + 8 * ab, ((tcount >> 1) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < KS; ks++, it++) {
                     const int s = it % S;
-                    if (!mbar_wait(b_full + 8 * s, (it / S) & 1, abort, a.flag)) {
+                    if (!mbar_wait(b_full + 8 * s, (it / S) & 1, abort, a.flag, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -362,110 +455,159 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             // make sure every issued MMA has finished before TMEM is released
             mma_commit(b_drain);
             const uint64_t t0 = global_ns();
-            while (!mbar_test(b_drain, 0) && global_ns() - t0 < kWaitLimitNs) {
+            while (!mbar_test(b_drain, 0) && global_ns() - t0 < a.wait_ns) {
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= kTcEpiWarp0 && warp < kTcEpiWarp0 + kTcEpiWarps) {
         // ---------------- epilogue: TMEM -> registers -> global
-        // The next tile's per-column metadata (slot ids and token / slot
-        // scales, both contiguous per piece) is copied with cp.async and its
-        // row scales loaded into registers while this tile is processed, so
-        // no global latency sits between the MMAs and the stores.
-        const int q = warp & 3;
+        // Warp ew takes lane quarter q = warp % 4 (rows 32q .. 32q+31 of the
+        // block) and every other chunk of 32 columns (half hf = ew / 4).  The
+        // next tile's per-column metadata (slot ids and token / slot scales,
+        // contiguous per piece) is copied with cp.async and its row scales loaded
+        // into registers while this tile is processed.
+        const int ew = warp - kTcEpiWarp0;
+        const int q = warp & 3, hf = ew >> 2;
         const int r = q * 32 + lane;
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
         const int ldo = MODE == 0 ? a.F : a.D;
         const float *scale_src = MODE == 0 ? a.pscale : a.sh;
-        auto fetch = [&](int tile, int buf, const int4 &pc, float &al0, float &al1) {
-            const int row = (tile % R) * 128 + r;
-            al0 = a.alpha0[(size_t)pc.x * ldo + row];
-            al1 = MODE == 0 ? a.alpha1[(size_t)pc.x * ldo + row] : 0.0f;
-            if (r < pc.z) {   // one slot id and one scale per column (4-byte copies: any alignment of p0)
-                cp_async4_tc(meta_slot + buf * kTcMaxN + r, a.perm + pc.y + r);
-                cp_async4_tc(meta_scale + buf * kTcMaxN + r, scale_src + pc.y + r);
+        float *hs = MODE == 0 ? a.out + (size_t)blockIdx.x * kTcMaxN * a.F : nullptr;   // [128 slots][F]
+        auto fetch = [&](int buf, const int4 &P, int rbk, float &al0, float &al1) {
+            const int row = rbk * 128 + r;
+            al0 = a.alpha0[(size_t)P.x * ldo + row];
+            al1 = MODE == 0 ? a.alpha1[(size_t)P.x * ldo + row] : 0.0f;
+            if (hf == 0 && r < P.z) {   // one slot id and one scale per column (4-byte copies: any alignment)
+                cp_async4_tc(meta_slot + buf * kTcMaxN + r, a.perm + P.y + r);
+                cp_async4_tc(meta_scale + buf * kTcMaxN + r, scale_src + P.y + r);
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
         };
-        uint32_t tc = 0;
-        bool dead = false;   // after a failed wait: keep the loop (and its named barrier) in step, do nothing
-        int4 npc = make_int4(0, 0, 0, 0), nnpc = make_int4(0, 0, 0, 0);
+        uint32_t tcount = 0;
+        bool dead = false;   // after a failed wait: keep the loop (and its named barriers) in step, do nothing
+        int npc = 0, nrb = 0;
         float nal0 = 0.0f, nal1 = 0.0f;
-        if (blockIdx.x < n_tiles) {
-            npc = a.pieces[blockIdx.x / R];
-            fetch(blockIdx.x, 0, npc, nal0, nal1);
-        }
-        if (blockIdx.x + (int)gridDim.x < n_tiles) nnpc = a.pieces[(blockIdx.x + gridDim.x) / R];
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, tc++) {
-            const int4 pc = npc;
+        bool have = tc_tile<MODE>(0, R, n_pc, npc, nrb);
+        int4 nP = have ? a.pieces[npc] : make_int4(0, 0, 0, 0);
+        if (have) fetch(0, nP, nrb, nal0, nal1);
+        while (have) {
+            const int rb = nrb;
+            const int4 P = nP;
             const float al0 = nal0, al1 = nal1;
-            const int rt = tile % R;
-            const int row = rt * 128 + r;
-            const uint32_t ab = tc & 1, tb = tbase + 256 * ab;
-            const int p0 = pc.y, n = pc.z;
+            const uint32_t ab = tcount & 1, tb = tbase + 256 * ab;
+            const int row = rb * 128 + r;
+            const int p0 = P.y, n = P.z;
             const int *ms = meta_slot + ab * kTcMaxN;
             const float *mf = meta_scale + ab * kTcMaxN;
             asm volatile("cp.async.wait_group 0;" ::: "memory");
-            asm volatile("bar.sync 2, 128;" ::: "memory");   // this tile's metadata is in place
-            if (tile + (int)gridDim.x < n_tiles) {
-                npc = nnpc;
-                fetch(tile + gridDim.x, ab ^ 1, npc, nal0, nal1);
-                if (tile + 2 * (int)gridDim.x < n_tiles) nnpc = a.pieces[(tile + 2 * gridDim.x) / R];
+            asm volatile("bar.sync 2, 256;" ::: "memory");   // this tile's metadata is in place
+            have = tc_tile<MODE>((int)tcount + 1, R, n_pc, npc, nrb);
+            if (have) {
+                nP = a.pieces[npc];
+                fetch(ab ^ 1, nP, nrb, nal0, nal1);
             }
-            if (!dead && !mbar_wait(b_acc_full + 8 * ab, (tc >> 1) & 1, abort, a.flag)) dead = true;
-            if (dead) continue;
-            tc_fence_after();
-            if (MODE == 0) {
-                for (int c0 = 0; c0 < n; c0 += 32) {
-                    int g[32], u[32];
-                    tmem_ld32(tb + c0, g);
-                    tmem_ld32(tb + 128 + c0, u);
-                    tmem_wait_ld();
+            if (!dead && !mbar_wait(b_acc_full + 8 * ab, (tcount >> 1) & 1, abort, a.flag, a.wait_ns)) dead = true;
+            if (!dead) {
+                tc_fence_after();
+                if (MODE == 0) {
+                    for (int c0 = 32 * hf; c0 < n; c0 += 64) {
+                        float v[32];
+                        int g[16], u[16];   // sixteen columns at a time (register budget)
 #pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int col = c0 + j;
-                        if (col < n) {
-                            const int p = p0 + col;
-                            const int slot = ms[col];
-                            const float sxt = mf[col];
-                            const int gi = g[j] >> 6, ui = u[j] >> 6;
-                            const float gv = __fmul_rn((float)gi, __fmul_rn(al0, sxt));
-                            const float uv = __fmul_rn((float)ui, __fmul_rn(al1, sxt));
-                            a.out[(size_t)p * a.F + row] = swiglu(gv, uv);
-                            if (a.tap0) a.tap0[(size_t)slot * a.F + row] = gi;
-                            if (a.tap1) a.tap1[(size_t)slot * a.F + row] = ui;
+                        for (int j = 0; j < 32; j++) {
+                            const int col = c0 + j;
+                            if ((j & 15) == 0) {
+                                tmem_ld16(tb + c0 + j, g);
+                                tmem_ld16(tb + 128 + c0 + j, u);
+                                tmem_wait_ld();
+                            }
+                            v[j] = 0.0f;
+                            if (col < n) {
+                                const float sxt = mf[col];
+                                const int gi = g[j & 15] >> 6, ui = u[j & 15] >> 6;
+                                const float gv = __fmul_rn((float)gi, __fmul_rn(al0, sxt));
+                                const float uv = __fmul_rn((float)ui, __fmul_rn(al1, sxt));
+                                const float hv = swiglu(gv, uv);
+                                hs[(size_t)col * a.F + row] = hv;
+                                v[j] = fabsf(hv);
+                                if (a.tap0) a.tap0[(size_t)ms[col] * a.F + row] = gi;
+                                if (a.tap1) a.tap1[(size_t)ms[col] * a.F + row] = ui;
+                            }
+                        }
+                        // |h| maximum of each column over this warp's 32 rows, then over the CTA
+                        const float m = warp_column_max(v);
+                        if (c0 + lane < n) atomicMax(s_amax + c0 + lane, __float_as_uint(m));
+                    }
+                } else {
+                    for (int c0 = 32 * hf; c0 < n; c0 += 64) {
+                        int dd[32];
+                        tmem_ld32(tb + c0, dd);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; j++) {
+                            const int col = c0 + j;   // the same column in every lane
+                            if (col < n) {
+                                const int p = p0 + col;
+                                const int di = dd[j] >> 6;
+                                a.acc_hi[(size_t)p * a.D + row] = (int16_t)(di >> 1);
+                                const uint32_t lo = __ballot_sync(FULL, di & 1);
+                                if (lane == 0) a.acc_lo[(size_t)p * (a.D / 32) + (row >> 5)] = lo;
+                                if (a.tap0) a.tap0[(size_t)ms[col] * a.D + row] = di;
+                            }
+                        }
+                    }
+                    (void)al0;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_acc_empty + 8 * ab);
+            }
+            if (MODE == 0 && rb == R - 1) {
+                // the piece's last row block: requantise its slots (h from the scratch
+                // area, read past L1; the absmax from shared memory)
+                __threadfence_block();
+                asm volatile("bar.sync 3, 256;" ::: "memory");
+                if (!dead) {
+                    for (int i = ew; i < n; i += kTcEpiWarps) {
+                        const int p = p0 + i, slot = ms[i];
+                        const float amax = __uint_as_float(s_amax[i]);
+                        const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+                        const float4 *hr = reinterpret_cast<const float4 *>(hs + (size_t)i * a.F);
+                        for (int c = lane; c < a.F / 4; c += 32) {
+                            const float4 hv = __ldcg(hr + c);
+                            int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+                            if (amax > 0.0f) {
+                                q0 = quant_code(hv.x, inv);
+                                q1 = quant_code(hv.y, inv);
+                                q2 = quant_code(hv.z, inv);
+                                q3 = quant_code(hv.w, inv);
+                            }
+                            const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                                                ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+                            reinterpret_cast<uint32_t *>(a.qh + (size_t)p * a.F)[c] = pk;
+                            if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * a.F)[c] = pk;
+                        }
+                        if (lane == 0) {
+                            const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+                            a.sh[p] = sv;
+                            if (a.tap_sh) a.tap_sh[slot] = sv;
                         }
                     }
                 }
-            } else {
-                for (int c0 = 0; c0 < n; c0 += 32) {
-                    int dd[32];
-                    tmem_ld32(tb + c0, dd);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; j++) {
-                        const int col = c0 + j;
-                        if (col < n) {
-                            const int p = p0 + col;
-                            const int di = dd[j] >> 6;
-                            a.out[(size_t)p * a.D + row] = __fmul_rn((float)di, __fmul_rn(al0, mf[col]));
-                            if (a.tap0) a.tap0[(size_t)ms[col] * a.D + row] = di;
-                        }
-                    }
-                }
+                asm volatile("bar.sync 3, 256;" ::: "memory");   // every read of the maxima and the scratch is done
+                if (ew < 4) s_amax[ew * 32 + lane] = 0u;       // (ordered before the next piece's maxima by bar 2)
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_acc_empty + 8 * ab);
+            tcount++;
         }
-    } else if (warp >= 8) {
+    } else if (warp >= kTcProdWarp0) {
         // ---------------- producers: expand the 2-bit codes into int8 A tiles
-        const int pid = threadIdx.x - 256;
+        const int pid = threadIdx.x - kTcProdWarp0 * 32;
         uint32_t it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+        int pc, rb;
+        for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++) {
             for (int ks = 0; ks < KS; ks++, it++) {
                 const int s = it % S;
-                if (!mbar_wait(b_codes_full + 8 * s, (it / S) & 1, abort, a.flag)) {
+                if (!mbar_wait(b_codes_full + 8 * s, (it / S) & 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -473,8 +615,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 const uint4 *codes = (const uint4 *)(st + L::kCodes);
                 constexpr int kQuads = Cfg::kCodeBytes / 16;   // four words = one row's half stage
 #pragma unroll
-                for (int i = 0; i < kQuads / 256; i++) {
-                    const int qi = pid + 256 * i;
+                for (int i = 0; i < kQuads / (kTcProdWarps * 32); i++) {
+                    const int qi = pid + kTcProdWarps * 32 * i;
                     const int mrow = qi >> 1, w0 = (qi & 1) * 4;  // row within gate|up (or down), first word
                     const uint4 c4 = codes[qi];
                     *(uint4 *)(st + L::kA + sw128(mrow, w0 + 0)) = expand_word(c4.x);
@@ -497,78 +639,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
 }
 
-// ---------------------------------------------------------------------------
-// slot-ordered copy of the int8 activation rows: xperm[p] = q_x[perm[p] / K]
-// (one warp per position)
-// ---------------------------------------------------------------------------
-__global__ void gather_rows_kernel(const int8_t *qx, const float *sx, const int *perm, int K, int D, int S,
-                                   int8_t *xperm, float *pscale)
-{
-    const int lane = threadIdx.x & 31;
-    const int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (p >= S) return;
-    const int t = perm[p] / K;
-    if (lane == 0) pscale[p] = sx[t];
-    const uint4 *src = reinterpret_cast<const uint4 *>(qx + (size_t)t * D);
-    uint4 *dst = reinterpret_cast<uint4 *>(xperm + (size_t)p * D);
-    for (int i = lane; i < D / 16; i += 32) dst[i] = __ldg(src + i);
-}
-
-// ---------------------------------------------------------------------------
-// requantise h rows (one warp per slot position) for the tensor-core path
-// ---------------------------------------------------------------------------
-__global__ void requant_rows_kernel(const float *h, int S, int F, const int *perm, int8_t *qh, float *sh,
-                                    int8_t *tap_qh, float *tap_sh)
-{
-    const int lane = threadIdx.x & 31;
-    const int p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (p >= S) return;
-    const float4 *hr = reinterpret_cast<const float4 *>(h + (size_t)p * F);
-    float amax = 0.0f;
-    for (int i = lane; i < F / 4; i += 32) {
-        float4 v = hr[i];
-        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v.x)), fmaxf(fabsf(v.y), fabsf(v.z))), fabsf(v.w));
-    }
-    amax = warp_max(amax);
-    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-    const int slot = perm[p];
-    for (int i = lane; i < F / 4; i += 32) {
-        float4 v = hr[i];
-        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-        if (amax > 0.0f) {
-            q0 = quant_code(v.x, inv);
-            q1 = quant_code(v.y, inv);
-            q2 = quant_code(v.z, inv);
-            q3 = quant_code(v.w, inv);
-        }
-        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
-                            ((uint32_t)(q3 & 0xff) << 24);
-        reinterpret_cast<uint32_t *>(qh + (size_t)p * F)[i] = pk;
-        if (tap_qh) reinterpret_cast<uint32_t *>(tap_qh + (size_t)slot * F)[i] = pk;
-    }
-    if (lane == 0) {
-        const float s = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-        sh[p] = s;
-        if (tap_sh) tap_sh[slot] = s;
-    }
-}
-
-// y[t][c] = (resid[t][c] +) sum_k fmaf(w[t][k], yE[inv[t*K+k]][c]) in rank order
-__global__ void combine_kernel(const float *ye, const int *inv, const float *topk_w, int T, int K, int D, float *y,
+// y[t][c] = (resid[t][c] +) sum_k fmaf(w[t][k], yE_k[c]) in rank order, with
+// yE_k[c] = f32(acc) * (alpha_down[e_k][c] * s_h) rebuilt from the stored
+// accumulator (acc = 2 * acc_hi + its bit in acc_lo); one thread per 4 channels
+__global__ void combine_kernel(const int16_t *acc_hi, const uint32_t *acc_lo, const float *alpha_down, const float *sh,
+                               const int *topk_idx, const int *inv, const float *topk_w, int T, int K, int D, float *y,
                                const float *resid)
 {
     const int64_t n4 = (int64_t)T * D / 4;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
         const int t = (int)(i / (D / 4));
-        const int c4 = (int)(i % (D / 4));
+        const int c = 4 * (int)(i % (D / 4));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < K; k++) {
-            const float w = topk_w[t * K + k];
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(ye + (size_t)inv[t * K + k] * D) + c4);
-            acc.x = __fmaf_rn(w, v.x, acc.x);
-            acc.y = __fmaf_rn(w, v.y, acc.y);
-            acc.z = __fmaf_rn(w, v.z, acc.z);
-            acc.w = __fmaf_rn(w, v.w, acc.w);
+            const int sl = t * K + k, p = __ldg(inv + sl), e = __ldg(topk_idx + sl);
+            const float w = __ldg(topk_w + sl), s = __ldg(sh + p);
+            const uint2 hv = __ldcs(reinterpret_cast<const uint2 *>(acc_hi + (size_t)p * D + c));
+            const uint32_t lo = __ldg(acc_lo + (size_t)p * (D / 32) + (c >> 5)) >> (c & 31);
+            const float4 al = __ldg(reinterpret_cast<const float4 *>(alpha_down + (size_t)e * D + c));
+            const int a0 = 2 * (int)(int16_t)(hv.x & 0xffffu) + (int)(lo & 1u);
+            const int a1 = 2 * (int)(int16_t)(hv.x >> 16) + (int)((lo >> 1) & 1u);
+            const int a2 = 2 * (int)(int16_t)(hv.y & 0xffffu) + (int)((lo >> 2) & 1u);
+            const int a3 = 2 * (int)(int16_t)(hv.y >> 16) + (int)((lo >> 3) & 1u);
+            acc.x = __fmaf_rn(w, __fmul_rn((float)a0, __fmul_rn(al.x, s)), acc.x);
+            acc.y = __fmaf_rn(w, __fmul_rn((float)a1, __fmul_rn(al.y, s)), acc.y);
+            acc.z = __fmaf_rn(w, __fmul_rn((float)a2, __fmul_rn(al.z, s)), acc.z);
+            acc.w = __fmaf_rn(w, __fmul_rn((float)a3, __fmul_rn(al.w, s)), acc.w);
         }
         if (resid) {
             const float4 r = reinterpret_cast<const float4 *>(resid)[i];

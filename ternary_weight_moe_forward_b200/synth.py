@@ -136,3 +136,38 @@ def residual(n_tokens: int, d_model: int, seed: int) -> np.ndarray:
     """fp32 residual stream input for the layer stack: N(0, 1) values that are bf16-exact."""
     rng = _rng(seed, 0, _T_RESID, n_tokens)
     return bf16_bits_to_f32(f32_to_bf16_bits(rng.standard_normal((n_tokens, d_model)).astype(np.float32)))
+
+
+def layer_weights_device(shape: LayerShape, seed: int, layer: int = 0, zipf: float | None = None, device="cuda"):
+    """The same distributions as layer_weights, drawn on a CUDA device with
+    torch's counter-based generator (one seeded stream per tensor), for
+    workloads too large to draw on the host in time (the 24-layer stack).
+    These are different numbers from layer_weights' numpy streams.  Returns
+    torch tensors on `device`: gate/up/down int8, the rest fp32."""
+    import torch
+
+    E, D, F = shape.n_experts, shape.d_model, shape.d_ff
+    lut = torch.tensor(_TERNARY_LUT, dtype=torch.int8, device=device)
+
+    def gen(tensor):
+        g = torch.Generator(device=device)
+        g.manual_seed(int(np.random.SeedSequence([seed, layer, tensor]).generate_state(1, np.uint64)[0] >> 1))
+        return g
+
+    def ternary(tensor, shp):
+        return lut[torch.randint(0, 10, shp, generator=gen(tensor), device=device, dtype=torch.int64)]
+
+    def alpha(tensor, shp):
+        return 0.02 * torch.exp(0.25 * torch.randn(shp, generator=gen(tensor), device=device, dtype=torch.float32))
+
+    w = {
+        "gate": ternary(_T_GATE, (E, F, D)),
+        "up": ternary(_T_UP, (E, F, D)),
+        "down": ternary(_T_DOWN, (E, D, F)),
+        "alpha_gate": alpha(_T_AGATE, (E, F)),
+        "alpha_up": alpha(_T_AUP, (E, F)),
+        "alpha_down": alpha(_T_ADOWN, (E, D)),
+        "router_w": torch.randn((E, D), generator=gen(_T_ROUTER), device=device, dtype=torch.float32) / float(np.sqrt(D)),
+        "router_bias": None if zipf is None else torch.from_numpy(zipf_bias(E, zipf, seed, layer)).to(device),
+    }
+    return w

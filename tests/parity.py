@@ -60,3 +60,50 @@ def compare_permutation(shape, g: dict, idx_ref: np.ndarray):
     assert np.array_equal(g["expert_counts"], counts), "expert_counts"
     assert np.array_equal(g["expert_offsets"], offsets), "expert_offsets"
     assert np.array_equal(g["perm"], perm), "perm"
+
+
+# ---------------------------------------------------------------------------- the oracle over many tokens
+# Tokens are independent in the layer, so the single-threaded oracle can run on
+# shards of tokens in parallel processes; each worker builds the layer once from
+# the seeded generator (nothing of the GPU path crosses into the workers).
+_WORKER_LAYER = None
+
+
+def _oracle_worker_init(shape, seed: int, zipf):
+    global _WORKER_LAYER
+    _WORKER_LAYER = oracle.Layer(shape, synth.layer_weights(shape, seed=seed, zipf=zipf))
+
+
+def _oracle_worker_run(job):
+    t0, x_rows = job
+    return t0, _WORKER_LAYER.forward_tokens(x_rows, np.arange(x_rows.shape[0], dtype=np.int32))
+
+
+def oracle_shards(shape, seed: int, zipf, x_bits: np.ndarray, shard: int = 32, workers: int | None = None):
+    """Yield (tokens, oracle taps for those tokens) over every token of x_bits,
+    computed by a pool of spawned processes (started fresh, so it is safe after
+    CUDA is initialised in this process)."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    T = x_bits.shape[0]
+    workers = workers or max(1, min(os.cpu_count() or 1, 64))
+    jobs = [(t0, np.ascontiguousarray(x_bits[t0:t0 + shard])) for t0 in range(0, T, shard)]
+    ctx = mp.get_context("spawn")
+    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=ctx, initializer=_oracle_worker_init,
+                                initargs=(shape, seed, zipf)) as pool:
+        for t0, ref in pool.map(_oracle_worker_run, jobs, chunksize=1):
+            yield np.arange(t0, t0 + ref["y"].shape[0], dtype=np.int32), ref
+
+
+def compare_all_tokens(shape, g: dict, seed: int, zipf, x_bits: np.ndarray) -> dict:
+    """Every token of a GPU forward (taps in g) against the oracle; asserts.
+    Returns the worst y error and whether y agreed bit for bit everywhere."""
+    worst, exact, n = 0.0, True, 0
+    for tokens, ref in oracle_shards(shape, seed, zipf, x_bits):
+        res = compare_tokens(shape, g, ref, tokens)
+        worst = max(worst, res["y_rel"])
+        exact = exact and res["y_bit_exact"]
+        n += tokens.size
+    assert n == x_bits.shape[0]
+    return {"y_rel": worst, "y_bit_exact": exact}

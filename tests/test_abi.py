@@ -71,6 +71,11 @@ def test_argument_errors_before_any_cuda_call(lib):
     assert lib.maple_moe_create(C.byref(cfg), C.byref(w), None, C.byref(h)) == tw.MAPLE_ERR_UNSUPPORTED_SHAPE
     cfg = tw.maple_moe_config(256, 16, 2, 128, 8, 0, 0)
     assert lib.maple_moe_create(C.byref(cfg), C.byref(w), None, C.byref(h)) == tw.MAPLE_ERR_INVALID_ARG  # NULL weights
+    cfg = tw.maple_moe_config(256, 16, 2, 128, 8, 65, 0)   # decode kernel serves at most 64 tokens
+    assert lib.maple_moe_create(C.byref(cfg), C.byref(w), None, C.byref(h)) == tw.MAPLE_ERR_UNSUPPORTED_SHAPE
+    for flags in (0x80, tw.MAPLE_CFG_FORCE_TC | tw.MAPLE_CFG_DECODE_ONLY):   # unknown, conflicting
+        cfg = tw.maple_moe_config(256, 16, 2, 128, 8, 0, flags)
+        assert lib.maple_moe_create(C.byref(cfg), C.byref(w), None, C.byref(h)) == tw.MAPLE_ERR_INVALID_ARG
     assert lib.maple_moe_forward(None, None, 1, None, None, None) == tw.MAPLE_ERR_INVALID_ARG
     assert lib.maple_moe_route(None, None, 1, None, None, None, None) == tw.MAPLE_ERR_INVALID_ARG
     assert lib.maple_moe_pack_ternary(None, 4, 15, None, None, None) == tw.MAPLE_ERR_INVALID_ARG

@@ -13,7 +13,8 @@ import oracle
 from ternary_weight_moe_forward_b200 import synth
 from ternary_weight_moe_forward_b200.layer import Layer, bf16_from_bits
 
-from parity import Y_TOL, compare_permutation, compare_tokens, gpu_forward_with_taps, max_rel
+from parity import (Y_TOL, compare_all_tokens, compare_permutation, compare_tokens, gpu_forward_with_taps,
+                    max_rel)
 
 pytestmark = pytest.mark.gpu
 
@@ -161,22 +162,17 @@ def test_nan_input_sets_the_device_flag(tiny):
     assert L_gpu.device_flags() == 0
 
 
-def test_prefill_config_sampled_parity(big):
-    """T=4096: routing of every token and the permutation against the oracle,
-    full per-token comparison on a sample spread over the batch."""
+def test_prefill_config_full_parity(big):
+    """T=4096 (the tensor-core path): every tap of every token against the
+    oracle, which runs on token shards in parallel processes."""
     L_orc, L_gpu = big
     T = 4096
     x = synth.activations(T, BIG.d_model, seed=0)
     g = gpu_forward_with_taps(L_gpu, x)
     logits, idx, w = L_orc.route(x)
-    assert np.array_equal(g["topk_idx"], idx)
-    assert np.array_equal(g["topk_w"].view(np.uint32), w.view(np.uint32))
-    assert np.array_equal(g["logits"].view(np.uint32), logits.view(np.uint32))
     compare_permutation(BIG, g, idx)
-    tokens = np.unique(np.concatenate([[0, 1, T - 1], np.random.default_rng(0).choice(T, 21, replace=False)]))
-    tokens = tokens.astype(np.int32)
-    ref = L_orc.forward_tokens(x, tokens)
-    compare_tokens(BIG, g, ref, tokens)
+    res = compare_all_tokens(BIG, g, 0, None, x)
+    assert res["y_rel"] <= Y_TOL
 
 
 # ---------------------------------------------------------------------------- both expert paths
@@ -193,12 +189,29 @@ def test_tensor_core_path_forced_tiny(tiny, T):
     Lg.close()
 
 
-@pytest.mark.parametrize("T", [65, 300])
-def test_gemv_path_forced_large_T(tiny, T):
+@pytest.mark.parametrize("T", [9, 33, 64])
+def test_decode_kernel_forced_beyond_its_default_limit(tiny, T):
+    """MAPLE_CFG_FORCE_GEMV runs the decode kernel for every T <= 64, here
+    above a handle's decode_max_tokens of 8 (units of 16 slots, 2 n-tiles)."""
     w, L_orc, _ = tiny
-    Lg = Layer(TINY, w, max_tokens=512, flags=tw.MAPLE_CFG_FORCE_GEMV)
+    Lg = Layer(TINY, w, max_tokens=512, decode_max_tokens=8, flags=tw.MAPLE_CFG_FORCE_GEMV)
     x = synth.activations(T, TINY.d_model, seed=200 + T)
     _full_check(TINY, L_orc, Lg, x)
+    with pytest.raises(tw.MapleError) as e:   # beyond 64 tokens there is no decode kernel
+        Lg.forward(bf16_from_bits(synth.activations(65, TINY.d_model, seed=1), "cuda"))
+    assert e.value.code == tw.MAPLE_ERR_UNSUPPORTED_SHAPE
+    Lg.close()
+
+
+def test_decode_only_handle(big_weights, big):
+    """A handle with only the decode layout serves T <= 64 and rejects more."""
+    L_orc, _ = big
+    Lg = Layer(BIG, big_weights, max_tokens=128, flags=tw.MAPLE_CFG_DECODE_ONLY)
+    x = synth.activations(16, BIG.d_model, seed=400)
+    _full_check(BIG, L_orc, Lg, x)
+    with pytest.raises(tw.MapleError) as e:
+        Lg.forward(bf16_from_bits(synth.activations(65, BIG.d_model, seed=1), "cuda"))
+    assert e.value.code == tw.MAPLE_ERR_UNSUPPORTED_SHAPE
     Lg.close()
 
 
@@ -212,10 +225,10 @@ def test_tensor_core_path_forced_decode_shape(big_weights, big):
 
 
 def test_paths_agree_bitwise(big_weights, big):
-    """GEMV and tensor-core paths give identical bits on the same input."""
-    Lt = Layer(BIG, big_weights, max_tokens=128, flags=tw.MAPLE_CFG_FORCE_TC)
-    Lv = Layer(BIG, big_weights, max_tokens=128, flags=tw.MAPLE_CFG_FORCE_GEMV)
-    x = bf16_from_bits(synth.activations(128, BIG.d_model, seed=7), "cuda")
+    """The decode kernel and the tensor-core path give identical bits on the same input."""
+    Lt = Layer(BIG, big_weights, max_tokens=64, flags=tw.MAPLE_CFG_FORCE_TC)
+    Lv = Layer(BIG, big_weights, max_tokens=64, flags=tw.MAPLE_CFG_FORCE_GEMV)
+    x = bf16_from_bits(synth.activations(64, BIG.d_model, seed=7), "cuda")
     yt, yv = Lt.forward(x), Lv.forward(x)
     torch.cuda.synchronize()
     assert torch.equal(yt.view(torch.int32), yv.view(torch.int32))

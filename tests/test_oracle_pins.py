@@ -99,19 +99,30 @@ def test_quantize_is_nearest_code_and_scale_invariant():
 
 # ------------------------------------------------------------------ router
 def _golden_router_cases():
+    """(D, [(j, w_j)], expected logit, exact sum) per line; a leading D=... token
+    gives the row length (256 otherwise)."""
     cases = []
     for line in open(os.path.join(GOLDEN, "router_order.txt")):
         if line.startswith("#") or not line.strip():
             continue
         terms, expect, exact = line.split("|")
-        cases.append(([tuple(int(a) for a in t.split("=")) for t in terms.split()], float(expect), float(exact)))
+        D, pairs = 256, []
+        for t in terms.split():
+            k, v = t.split("=")
+            if k == "D":
+                D = int(v)
+            else:
+                pairs.append((int(k), int(v)))
+        cases.append((D, pairs, float(expect), float(exact)))
     return cases
 
 
 def test_router_order_hand_worked_cases():
-    for terms, expect, exact in _golden_router_cases():
-        x = np.zeros(256, np.float32)
-        w = np.zeros(256, np.float32)
+    cases = _golden_router_cases()
+    assert {c[0] for c in cases} >= {256, 512, 2048}
+    for D, terms, expect, exact in cases:
+        x = np.zeros(D, np.float32)
+        w = np.zeros(D, np.float32)
         for j, wj in terms:
             x[j] = 1.0
             w[j] = wj

@@ -14,7 +14,6 @@ import ternary_weight_moe_forward_b200 as tw
 from ternary_weight_moe_forward_b200 import synth
 from ternary_weight_moe_forward_b200.layer import Layer, bf16_from_bits
 
-from parity import Y_TOL, max_rel
 
 pytestmark = pytest.mark.gpu
 
@@ -32,10 +31,16 @@ def _route_weights(shape, seed, zipf=None):
     return w
 
 
+# d_model 4096 needs the raised shared-memory limit of the routing kernel; 1024
+# experts take its wide top-k variant, and T * E = 16384 fills the array's limit
+_SHAPES = {"tiny": synth.CONFIGS["tiny"]["shape"], "decode": synth.CONFIGS["decode"]["shape"],
+           "d4096": synth.LayerShape(4096, 256, 8, 128), "e1024": synth.LayerShape(256, 1024, 8, 128)}
+
+
 @pytest.mark.parametrize("name,T,zipf", [("tiny", 8, None), ("decode", 1, None), ("decode", 64, None),
-                                         ("decode", 37, 1.1)])
+                                         ("decode", 37, 1.1), ("d4096", 8, None), ("e1024", 16, None)])
 def test_route_noalloc_matches_route(name, T, zipf):
-    shape = synth.CONFIGS[name]["shape"]
+    shape = _SHAPES[name]
     w = _route_weights(shape, seed=3, zipf=zipf)
     ref_layer = Layer(shape, w, max_tokens=64)
     x = bf16_from_bits(synth.activations(T, shape.d_model, seed=11), "cuda")
@@ -53,7 +58,8 @@ def test_route_noalloc_matches_route(name, T, zipf):
         torch.cuda.synchronize()
         assert torch.equal(idx, idx_ref)
         assert torch.equal(cnt, cnt_ref)
-        assert max_rel(wt.cpu().numpy(), w_ref.cpu().numpy()) <= Y_TOL
+        # the same routing kernel computes both: the weights agree bit for bit
+        assert torch.equal(wt.view(torch.int32), w_ref.view(torch.int32))
     ref_layer.close()
 
 

@@ -132,4 +132,34 @@ __device__ __forceinline__ void set_flag(unsigned *flag, unsigned bits)
     if (flag) atomicOr(flag, bits);
 }
 
+// One token's pre-norm input, one warp: out = bf16(r / rms) with
+// rms = sqrt(sum(r^2) / D + 1e-6), norm weights 1; the sum of squares in the
+// router's fixed order (lane l takes j = 256i + 8l + m with fmaf, then the
+// pairwise tree).  `out` may be global or shared memory.
+__device__ __forceinline__ void rmsnorm_token_warp(const float *r, int D, uint16_t *out)
+{
+    const int lane = threadIdx.x & 31;
+    float acc = 0.0f;
+    for (int i = 0; i < D / 256; i++) {
+        const float4 v0 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane);
+        const float4 v1 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane + 4);
+        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int m = 0; m < 8; m++) acc = __fmaf_rn(v[m], v[m], acc);
+    }
+    const float ms = __fdiv_rn(warp_tree_sum(acc), (float)D);
+    const float rms = __fsqrt_rn(__fadd_rn(ms, 1e-6f));
+    for (int i = 0; i < D / 256; i++) {
+        const float4 v0 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane);
+        const float4 v1 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane + 4);
+        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t pk[4];
+#pragma unroll
+        for (int m = 0; m < 4; m++)
+            pk[m] = (uint32_t)f32_to_bf16_bits(__fdiv_rn(v[2 * m], rms)) |
+                    ((uint32_t)f32_to_bf16_bits(__fdiv_rn(v[2 * m + 1], rms)) << 16);
+        *reinterpret_cast<uint4 *>(out + 256 * i + 8 * lane) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
 }  // namespace maple

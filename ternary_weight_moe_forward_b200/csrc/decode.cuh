@@ -13,7 +13,7 @@
 // a chunk never spans two units), so a CTA only ever waits on work that
 // running CTAs have claimed: no grid-wide residency is assumed.
 //
-// Warp roles (18 warps, one CTA per SM):
+// Warp roles (10 warps, one CTA per SM):
 //   warp 0      claims chunks, publishes them in a shared queue and streams
 //               every item's codes into a ring of shared-memory slots with one
 //               bulk copy each, as far ahead as the ring allows (stage-2 codes
@@ -24,7 +24,7 @@
 //               every stage-1 item of the unit has finished (arrival counter),
 //               by requantising the unit's SwiGLU rows h (int8 absmax per slot,
 //               the absmax taken from stage 1's per-slot maxima);
-//   warps 2-17  compute: item j of the CTA's stream goes to warp j % 16.  Per
+//   warps 2-9   compute: item j of the CTA's stream goes to warp j % 8.  Per
 //               128-column block one 16-byte shared load gives the lane its four
 //               code words; w & (0x03030303 << 2q) is the A fragment of the MMA
 //               over columns 32q.. of the block, scaled by 4^q, so four plane
@@ -47,11 +47,15 @@
 
 namespace maple {
 
-constexpr int kDxComputeWarps = 16;
-constexpr int kDxThreads = (2 + kDxComputeWarps) * 32;   // 576
+// Eight compute warps: each holds a ring slot only while it computes, so that most
+// of the ring's slots are always copies in flight (the ring, not the MMAs, sets
+// how many bytes per SM are on their way from HBM).
+constexpr int kDxComputeWarps = 8;
+constexpr int kDxThreads = (2 + kDxComputeWarps) * 32;   // 320
 constexpr int kDxUnitTokens = 16;                        // tokens of a unit: two MMA n-tiles
 constexpr int kDxQueue = 16;                             // chunk entries in flight
 constexpr int kDxNB = 2;                                 // B-operand buffers
+constexpr int kDxMaxF = 1024;                            // largest d_ff (the shape limit)
 
 struct DxArgs {
     int T, D, E, K, F;
@@ -236,6 +240,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         *s_last_tma = -1;
         fence_barrier_init();
     }
+    // A routing kernel launched after this one as a programmatic dependent (the next
+    // layer of a stack) may start loading its router weights now; it waits for
+    // this grid's completion before it reads anything this kernel writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // The kernel may be launched while the routing kernel still runs (programmatic
     // dependent launch): nothing it writes is read before this point.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -456,12 +464,19 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     continue;
                 }
                 const int pos = p0 + n, slot = t_perm[pos];
+                const float4 *hr = reinterpret_cast<const float4 *>(a.h + (size_t)pos * F);
+                float4 hrow[kDxMaxF / 128];   // this lane's words, all loads in flight together
+#pragma unroll
+                for (int i = 0; i < kDxMaxF / 128; i++)
+                    if (i < F / 128) hrow[i] = __ldcg(hr + lane + 32 * i);
                 const float amax = __uint_as_float(__ldcg(a.amax + pos));
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                const float4 *hr = reinterpret_cast<const float4 *>(a.h + (size_t)pos * F);
                 int sum = 0;
-                for (int w = lane; w < F / 4; w += 32) {   // word w: columns 4w .. 4w+3
-                    const float4 hv = __ldcg(hr + w);
+#pragma unroll
+                for (int i = 0; i < kDxMaxF / 128; i++) {
+                    if (i >= F / 128) break;
+                    const int w = lane + 32 * i;   // word w: columns 4w .. 4w+3
+                    const float4 hv = hrow[i];
                     int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
                     if (amax > 0.0f) {
                         q0 = quant_code(hv.x, inv);
@@ -510,9 +525,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         const int unit = ch.unit, e = sd->e, cnt = sd->cnt;
         const int ntiles = (cnt + 7) / 8;
         const uint32_t bb = smem_addr(bbuf + (size_t)b * L.b_bytes) + lane * 32;
-        // the first of this warp's items in the chunk: stream index = cw (mod 16)
+        // the first of this warp's items in the chunk: stream index = cw (mod the warps)
         int k = (cw - ch.stream) % kDxComputeWarps;
         if (k < 0) k += kDxComputeWarps;
+        int done_items = 0;   // stage-1 items of the chunk this warp finished
         for (; k < ch.n; k += kDxComputeWarps) {
             const int j = ch.stream + k, s = j % a.nslot;
             if (!mbar_wait(b_rfull + 8 * s, (j / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
@@ -530,6 +546,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     dx_tile<2>(aa, bb, KB1, KB1 * 1024, acc);
                 else
                     dx_tile<1>(aa, bb, KB1, KB1 * 1024, acc);
+                // the codes are in registers' results: hand the slot back to the producer now
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_rempty + 8 * s);
 #pragma unroll
                 for (int nt = 0; nt < 2; nt++) {
                     if (nt >= ntiles) break;
@@ -565,10 +584,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         }
                     }
                 }
-                // publish: h and the maxima before the unit's arrival count
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicAdd(a.arrive + unit, 1u);
+                done_items++;
             } else {
                 // ---- down item `it`: tiles S2*it .. S2*it + S2-1, channels 16*S2*it ..
                 for (int d = 0; d < S2; d++) {
@@ -577,6 +593,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         dx_tile<2>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
                     else
                         dx_tile<1>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                    if (d == S2 - 1) {   // the item's last tile is read: hand the slot back
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(b_rempty + 8 * s);
+                    }
                     const int ch0 = 16 * dt + g;
                     const float ad0 = __ldg(a.alpha_down + (size_t)e * D + ch0);
                     const float ad1 = __ldg(a.alpha_down + (size_t)e * D + ch0 + 8);
@@ -642,10 +662,14 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     if (lane == jn) a.comb[(size_t)tt * NCB + blk] = 0u;
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_rempty + 8 * s);
         }
         if (!ok) break;
+        if (done_items) {
+            // publish this warp's h and maxima of the chunk, then count its items on the unit
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicAdd(a.arrive + unit, (unsigned)done_items);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(b_bempty + 8 * b);
     }

@@ -425,11 +425,13 @@ static int take_flag(maple_moe_t h, cudaStream_t st)
 // routing stage: quantise, logits, top-k (+ the permutation)
 static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_taps *taps, int32_t *out_idx,
                      float *out_w, int32_t *out_counts, bool permute, bool pieces, cudaStream_t st,
-                     unsigned *clear = nullptr, int n_clear = 0, bool frag = false)
+                     unsigned *clear = nullptr, int n_clear = 0, bool frag = false, const float *norm_resid = nullptr,
+                     bool pdl = false)
 {
     RouteArgs a;
     memset(&a, 0, sizeof a);
     a.x = x;
+    a.resid = norm_resid;   // (T <= 64 only) x = bf16(RMSNorm(resid)), computed by the routing kernel
     a.qxp = frag ? h->qxp : nullptr;   // the decode kernel's fragment-ordered q_x
     a.T = T;
     a.D = h->D;
@@ -475,8 +477,20 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
         a.n_clear = n_clear;
     }
     if (small) {
-        dim3 grid(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
-        pick_route(h->D, h->E)<<<grid, 256, route_smem_bytes(h->D), st>>>(a);
+        // as a programmatic dependent (the layer stack) the kernel loads its router
+        // rows while the previous layer finishes, then waits for it
+        cudaLaunchConfig_t lc;
+        memset(&lc, 0, sizeof lc);
+        lc.gridDim = dim3(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
+        lc.blockDim = dim3(256);
+        lc.dynamicSmemBytes = route_smem_bytes(h->D);
+        lc.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = pdl ? 1 : 0;
+        if (cudaLaunchKernelEx(&lc, pick_route(h->D, h->E), a) != cudaSuccess) return MAPLE_ERR_CUDA;
     } else {
         dim3 grid((T + kRgTok - 1) / kRgTok, h->E / kRgExp);
         router_gemm_kernel<<<grid, 256, 2 * kRgStage, st>>>(x, T, h->D, h->E, h->router_w, h->router_bias,
@@ -675,11 +689,16 @@ static int dec_slots(maple_moe_t h, int T)
     return dx_ring_slots(h->D, h->F, T, h->K, h->E, (size_t)h->optin);
 }
 
+// norm_resid (decode batches only): the layer input is bf16(RMSNorm(norm_resid)),
+// computed by the routing kernel, and x is unused; pdl: launch the routing
+// kernel as a programmatic dependent of the kernel before it (the layer stack)
 static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const float *resid,
-                        const maple_moe_taps *taps, cudaStream_t st)
+                        const maple_moe_taps *taps, cudaStream_t st, const float *norm_resid = nullptr,
+                        bool pdl = false)
 {
     const int nslot = (h->cfg_flags & MAPLE_CFG_FORCE_TC) ? 0 : dec_slots(h, T);
     if (!nslot && !h->w_tc_gu) return MAPLE_ERR_UNSUPPORTED_SHAPE;   // decode-only handle, T too large
+    if (norm_resid && !nslot) return MAPLE_ERR_INVALID_ARG;          // (callers check dec_slots first)
     stage_event(h, 0, st);
     int rc;
     if (nslot) {
@@ -688,7 +707,7 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
         // fragment-ordered q_x
         const int S = T * h->K;
         rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, st, h->dx_clear,
-                       (int)(S + dx_max_units(h->E, S) + 1), true);
+                       (int)(S + dx_max_units(h->E, S) + 1), true, norm_resid, pdl);
     } else {
         rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, true, st);
     }
@@ -730,11 +749,21 @@ extern "C" int maple_moe_stack_forward(const maple_moe_t *layers, int32_t n_laye
     if (!resid || !aligned16(resid)) return MAPLE_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
     uint16_t *xn = layers[0]->xn;
+    bool chained = false;   // the previous layer ended with the decode kernel
     for (int l = 0; l < n_layers; l++) {
-        rmsnorm_bf16_kernel<<<(T + 7) / 8, 256, 0, st>>>(resid, T, layers[l]->D, xn);
-        int rc = launch_status();
-        if (rc) return rc;
-        rc = forward_impl(layers[l], xn, T, resid, resid, nullptr, st);
+        maple_moe_t L = layers[l];
+        int rc;
+        if (!(L->cfg_flags & MAPLE_CFG_FORCE_TC) && dec_slots(L, T)) {
+            // decode batch: the routing kernel normalises the residual itself, and
+            // after a decode kernel it is launched as that kernel's dependent
+            rc = forward_impl(L, nullptr, T, resid, resid, nullptr, st, resid, chained);
+            chained = true;
+        } else {
+            rmsnorm_bf16_kernel<<<(T + 7) / 8, 256, 0, st>>>(resid, T, L->D, xn);
+            if ((rc = launch_status())) return rc;
+            rc = forward_impl(L, xn, T, resid, resid, nullptr, st);
+            chained = false;
+        }
         if (rc) return rc;
     }
     return MAPLE_OK;

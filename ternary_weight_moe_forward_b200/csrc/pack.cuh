@@ -68,31 +68,9 @@ __global__ void repack_mma_dn_kernel(const uint32_t *down, int E, int D, int F, 
 // in the router's order: lane l takes j = 256*i + 8*l + m (fmaf), xor tree.
 __global__ void rmsnorm_bf16_kernel(const float *resid, int T, int D, uint16_t *out)
 {
-    const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (t >= T) return;
-    const float *r = resid + (size_t)t * D;
-    float acc = 0.0f;
-    for (int i = 0; i < D / 256; i++) {
-        const float4 v0 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane);
-        const float4 v1 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane + 4);
-        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int m = 0; m < 8; m++) acc = __fmaf_rn(v[m], v[m], acc);
-    }
-    const float ms = __fdiv_rn(warp_tree_sum(acc), (float)D);
-    const float rms = __fsqrt_rn(__fadd_rn(ms, 1e-6f));
-    for (int i = 0; i < D / 256; i++) {
-        const float4 v0 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane);
-        const float4 v1 = *reinterpret_cast<const float4 *>(r + 256 * i + 8 * lane + 4);
-        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t pk[4];
-#pragma unroll
-        for (int m = 0; m < 4; m++)
-            pk[m] = (uint32_t)f32_to_bf16_bits(__fdiv_rn(v[2 * m], rms)) |
-                    ((uint32_t)f32_to_bf16_bits(__fdiv_rn(v[2 * m + 1], rms)) << 16);
-        *reinterpret_cast<uint4 *>(out + (size_t)t * D + 256 * i + 8 * lane) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
+    rmsnorm_token_warp(resid + (size_t)t * D, D, out + (size_t)t * D);
 }
 
 }  // namespace maple

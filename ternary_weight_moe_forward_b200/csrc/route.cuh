@@ -16,6 +16,7 @@ constexpr int kRouteSmallT = 64;       // up to this many tokens the latency-ori
 
 struct RouteArgs {
     const uint16_t *x;
+    const float *resid;   // optional (route_kernel): x = bf16(RMSNorm(resid)) computed here, x unused
     int T, D, E, K;
     const float *Wr, *bias;
     // workspace outputs
@@ -324,10 +325,9 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
     // let a kernel launched after this one as a programmatic dependent start its
     // set-up now (it waits for this grid's completion before reading any output)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    if (a.clear && eb == 0 && tg == 0)
-        for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
 
-    // this lane's part of the router row, all in flight at once
+    // this lane's part of the router row, all in flight at once (the router
+    // weights are not written by any kernel, so this may run before the wait)
     const float *wr = a.Wr + (size_t)e * a.D;
     float4 w0[NI], w1[NI];
 #pragma unroll
@@ -335,9 +335,17 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
         w0[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane));
         w1[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane + 4));
     }
-    // stage the token rows (nt * D/8 16-byte units, at most NI per thread) with
-    // asynchronous copies, all in flight at once
-    {
+    // launched as a programmatic dependent (the layer stack), wait here for the
+    // grid before, which wrote the input; otherwise this returns at once
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (a.clear && eb == 0 && tg == 0)
+        for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
+    if (a.resid) {
+        // the layer stack: each warp normalises one of the CTA's tokens
+        if (warp < nt) rmsnorm_token_warp(a.resid + (size_t)(t0 + warp) * a.D, a.D, xs + (size_t)warp * a.D);
+    } else {
+        // stage the token rows (nt * D/8 16-byte units, at most NI per thread) with
+        // asynchronous copies, all in flight at once
         const int n16 = nt * (a.D / 8);
         const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D);
 #pragma unroll

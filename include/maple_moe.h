@@ -233,8 +233,8 @@ int maple_moe_route_noalloc(const uint16_t *x, int32_t T, int32_t d_model, int32
 int maple_moe_device_flags(maple_moe_t layer, uint32_t *flags, int32_t clear);
 
 /* maple_moe_set_debug flags (testing the failure handling only) */
-#define MAPLE_DEBUG_STALL_DOWN 0x1u   /* the decode expert kernel's down stage waits for an arrival
-                                         count that is never reached, so that its bounded wait expires */
+#define MAPLE_DEBUG_STALL_DOWN 0x1u   /* the decode path's down kernel waits for a device word that
+                                         nothing sets, so that its bounded wait expires */
 
 /*
  * Failure-handling knobs of a handle, for tests.  wait_limit_us: the limit of

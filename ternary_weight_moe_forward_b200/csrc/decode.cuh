@@ -1,40 +1,48 @@
-// Persistent expert-stage kernel for decode batches (T <= 64) on warp-level
-// int8 MMA (mma.sync m16n8k32, A = 2-bit weight codes as unsigned byte planes,
-// B = int8 activations, int32 accumulators).
+// Expert stage for decode batches (T <= 64) on warp-level int8 MMA
+// (mma.sync m16n8k32: A = 2-bit weight codes as unsigned byte planes,
+// B = int8 activations, int32 accumulators), as two persistent streaming
+// kernels, one CTA per SM:
 //
-// Work.  The kernel's prologue builds, in every CTA, the token -> expert
-// permutation from the router's top-k (as a token bitmask per expert) and
-// cuts every active expert's slots into units of at most 16 (two 8-token MMA
-// n-tiles).  Stage 1 (gate/up) has F/8 items per unit, one 16-row weight tile
-// each (8 gate rows and the up rows of the same 8 outputs, all of K); stage 2
-// (down) has D/(16*S2) items per unit, each S2 consecutive 16-channel tiles,
-// so that an item of either stage is 4*D bytes of codes.  Items are claimed in
-// chunks (one atomic per chunk, all stage-1 chunks before any stage-2 chunk,
-// a chunk never spans two units), so a CTA only ever waits on work that
-// running CTAs have claimed: no grid-wide residency is assumed.
+//   decode_stage_kernel<1>  gate/up: h = SiLU(g) * u per (slot, output), fp32,
+//                           and the per-slot |h| maxima (atomicMax);
+//   decode_stage_kernel<2>  down: requantise h (int8 absmax per slot), the down
+//                           contraction, yE, and the rank-order combine.
 //
-// Warp roles (10 warps, one CTA per SM):
-//   warp 0      claims chunks, publishes them in a shared queue and streams
-//               every item's codes into a ring of shared-memory slots with one
-//               bulk copy each, as far ahead as the ring allows (stage-2 codes
-//               are fetched while stage 1 still runs elsewhere);
-//   warp 1      builds each chunk's B operand (the unit's activations in MMA
-//               fragment order) in one of two buffers: stage 1 by four-row TMA
-//               gathers from the fragment-ordered copy of q_x; stage 2, once
-//               every stage-1 item of the unit has finished (arrival counter),
-//               by requantising the unit's SwiGLU rows h (int8 absmax per slot,
-//               the absmax taken from stage 1's per-slot maxima);
-//   warps 2-9   compute: item j of the CTA's stream goes to warp j % 8.  Per
-//               128-column block one 16-byte shared load gives the lane its four
-//               code words; w & (0x03030303 << 2q) is the A fragment of the MMA
-//               over columns 32q.. of the block, scaled by 4^q, so four plane
-//               accumulators hold exact multiples of 4^q and combine exactly.
-//               Stage 1 epilogue: SwiGLU in the lane (its gate and up values of
-//               one output sit in c0/c2 and c1/c3), h to L2, per-slot |h| maxima
-//               by atomics, then the unit's arrival counter.  Stage 2 epilogue:
-//               yE to L2, then one arrival per (token, channel block); the last
-//               of a token's arrivals on a block combines that block in rank
-//               order (fmaf from 0, plus the residual).
+// The second is launched as a programmatic dependent of the first: its CTAs
+// start as the first kernel's CTAs retire, stream their down codes into shared
+// memory, and only then wait for the first grid (griddepcontrol.wait) before
+// reading h.  The grid boundary is the only synchronisation between the two
+// contractions; inside a kernel no CTA waits on another CTA's work, so no
+// grid-wide residency is assumed.
+//
+// Work.  The routing kernel has built the token -> expert permutation and
+// cut every active expert's slots into units of at most 16 (two 8-token MMA
+// n-tiles); every CTA loads those tables into shared memory.  Stage 1
+// has F/8 items per unit (one 16-row tile: 8 gate rows and the up rows of the
+// same 8 outputs over all of K); stage 2 has D/(16*S2) items per unit (S2 =
+// D/F consecutive 16-channel tiles), so that every item is 4*D bytes of codes.
+// CTA b takes the contiguous item range [N*b/G, N*(b+1)/G).
+//
+// Warp roles (10 warps):
+//   warp 0     streams the range's codes into a ring of shared-memory slots,
+//              one bulk copy per item, as far ahead as the ring allows;
+//   warp 1     builds each unit's B operand (the unit's activations in MMA
+//              fragment order) in one of two buffers: stage 1 by four-row TMA
+//              gathers from the fragment-ordered copy of q_x; stage 2 (after
+//              griddepcontrol.wait) by requantising the unit's rows of h with
+//              the per-slot maxima, with each slot's scale and code sum;
+//   warps 2-9  compute: item j of the range goes to warp j % 8.  Per 128-column
+//              block one 16-byte shared load gives the lane its four code words;
+//              w & (0x03030303 << 2q) is the A fragment of the MMA over columns
+//              32q.. of the block, scaled by 4^q, so four plane accumulators hold
+//              exact multiples of 4^q and combine exactly; subtracting the row's
+//              code sum gives the ternary dot product.  A warp hands its ring slot
+//              back as soon as its MMAs have read it.  Stage-1 epilogue: SwiGLU in
+//              the lane (gate and up of one output sit in c0/c2 and c1/c3), h to
+//              global memory, the slot maxima by shuffles and one atomicMax.
+//              Stage-2 epilogue: yE to global memory, then one arrival per
+//              (token, channel block); the last of a token's arrivals on a block
+//              combines it in rank order (fmaf from 0, plus the residual).
 // Every wait is bounded (the handle's limit) and raises the device flag on
 // expiry; the CTA then drains its copies in flight and returns.
 #pragma once
@@ -43,17 +51,17 @@
 
 #include "common.cuh"
 #include "layout.cuh"
+#include "route.cuh"
 #include "tc_gemm.cuh"
 
 namespace maple {
 
-// Eight compute warps: each holds a ring slot only while it computes, so that most
-// of the ring's slots are always copies in flight (the ring, not the MMAs, sets
-// how many bytes per SM are on their way from HBM).
+// Eight compute warps: each holds a ring slot only while its MMAs read it, so
+// that most of the ring's slots are always copies in flight (the ring, not the
+// MMAs, sets how many bytes per SM are on their way from HBM).
 constexpr int kDxComputeWarps = 8;
 constexpr int kDxThreads = (2 + kDxComputeWarps) * 32;   // 320
-constexpr int kDxUnitTokens = 16;                        // tokens of a unit: two MMA n-tiles
-constexpr int kDxQueue = 16;                             // chunk entries in flight
+constexpr int kDxUnitTokens = kUnitTokens;               // tokens of a unit: two MMA n-tiles
 constexpr int kDxNB = 2;                                 // B-operand buffers
 constexpr int kDxMaxF = 1024;                            // largest d_ff (the shape limit)
 
@@ -65,63 +73,60 @@ struct DxArgs {
     const int *sumx;       // [T] sum of q_x's codes
     const uint8_t *w_gu, *w_dn;   // MMA-tile layouts
     const float *alpha_gate, *alpha_up, *alpha_down;
+    const int *perm;       // [T*K] position -> slot (the routing kernel's permutation)
+    const int *inv;        // [T*K] slot -> position
+    const int2 *units;     // the units: {expert, first position | count << 16}
+    const int *n_units;
     float *h;              // [T*K][F] SwiGLU outputs, position order
-    unsigned *amax;        // [T*K] |h| maxima (float bits), zero at launch
-    unsigned *arrive;      // [units] finished stage-1 items per unit, zero at launch
-    int *claim;            // chunks claimed so far, zero at launch
+    unsigned *amax;        // [T*K] |h| maxima (float bits), zero before stage 1
     unsigned *comb;        // [T][D/cb] arrivals per (token, channel block), zero between launches
+    const unsigned *never; // a word that stays 0 (the stall test hook waits for it to become 1)
     float *ye;             // [T*K][D] expert outputs, position order
     float *y;              // [T][D]
     const float *resid;    // [T][D] or null: y = resid + combine
     int *tap_acc_gate, *tap_acc_up, *tap_acc_down;
     int8_t *tap_qh;
     float *tap_sh;
-    int *tap_counts, *tap_offsets, *tap_perm;
     unsigned *flag;
     uint64_t wait_ns;
-    int stall;             // test hook: stage 2 waits for one stage-1 arrival more than will ever come
-    int chunk1, chunk2;    // items per chunk in the two stages (powers of two dividing F/8 and D/(16*S2))
-    int nslot;             // weight ring slots of 4*D bytes
+    int stall;             // test hook: stage 2 waits for `never` to become 1
+    int nslot;             // weight ring slots (4*D bytes of codes + the item's scales)
 };
 
-struct DxChunk {
-    int stage;    // 1, 2; 0 = no more work
-    int unit, first, n;
-    int stream;   // index of the chunk's first item in the CTA's item stream
-};
-
-struct DxSide {                 // per-slot data of a chunk's unit, next to its B operand
+struct DxSide {                 // per-slot data of a unit, next to its B operand
     float s[kDxUnitTokens];     // stage 1: s_x of the token; stage 2: s_h of the slot
     int sum[kDxUnitTokens];     // sum of the row's int8 codes (q_x or q_h)
     int pos[kDxUnitTokens];     // position of the slot in the permutation
     int e, cnt;
 };
 
-// shared-memory layout of the decode kernel
+// shared-memory layout of the decode kernels
 struct DxSmem {
-    int ring, bbuf, side, queue, bars, tables, total;
-    int slot_bytes, b_bytes;
+    int ring, bbuf, side, bars, tables, total;
+    int code_bytes, alpha_bytes, slot_bytes, b_bytes;
     __host__ __device__ DxSmem(int D, int F, int T, int K, int E, int nslot)
     {
-        slot_bytes = 4 * D;
+        // a ring slot: an item's codes, then its scales (stage 1: alpha_gate and
+        // alpha_up of 8 outputs; stage 2: alpha_down of its 16*D/F channels)
+        code_bytes = 4 * D;
+        alpha_bytes = 64 * (D / F) > 64 ? 64 * (D / F) : 64;
+        slot_bytes = code_bytes + alpha_bytes;
         b_bytes = 2 * (D / 128) * 1024;
         ring = 0;
         bbuf = ring + nslot * slot_bytes;
         side = bbuf + kDxNB * b_bytes;
-        queue = side + kDxNB * (int)sizeof(DxSide);
-        bars = (queue + kDxQueue * (int)sizeof(DxChunk) + 7) & ~7;
-        const int n_bars = 2 * nslot + 2 * kDxNB + 2 * kDxQueue;
-        tables = bars + 8 * n_bars + 16;   // + abort word, issued count, last gathered chunk, spare
+        bars = (side + kDxNB * (int)sizeof(DxSide) + 7) & ~7;
+        const int n_bars = 2 * nslot + 2 * kDxNB;
+        tables = bars + 8 * n_bars + 16;   // + abort word, issued count, last gathered unit, spare
         const int S = T * K, units = E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;
-        // t_idx, t_w, t_perm, t_inv [S]; t_cnt, t_act [E]; t_off [E+2] (E+1 used, keeps 8-byte
-        // alignment); t_sx, t_sumx [T]; misc [16]; units [units] (int2); tmask [E] (u64)
-        int tb = 4 * S * 4 + 2 * E * 4 + (E + 2) * 4 + 2 * T * 4 + 16 * 4 + units * 8;
+        // t_w, t_perm, t_inv [S]; t_sx, t_sumx [T]; misc [2]; units [units] (int2, 8-byte aligned)
+        int tb = 3 * S * 4 + 2 * T * 4 + 2 * 4;
         tb = (tb + 7) & ~7;
-        total = tables + tb + E * 8;
+        total = tables + tb + units * 8;
     }
 };
 
-// ring slots for a shape within a shared-memory budget (0: the kernel does not fit)
+// ring slots for a shape within a shared-memory budget (0: the kernels do not fit)
 __host__ inline int dx_ring_slots(int D, int F, int T, int K, int E, size_t budget)
 {
     if (F > D) return 0;
@@ -181,8 +186,9 @@ __device__ __forceinline__ int dx_total(const int (&acc)[2][4][4], int nt, int i
     return acc[nt][0][i] + (acc[nt][1][i] >> 2) + (acc[nt][2][i] >> 4) + (acc[nt][3][i] >> 6);
 }
 
+template <int STAGE>
 __global__ void __launch_bounds__(kDxThreads, 1)
-    decode_mma_kernel(const __grid_constant__ CUtensorMap qxp_map, DxArgs a)
+    decode_stage_kernel(const __grid_constant__ CUtensorMap qxp_map, DxArgs a)
 {
     extern __shared__ __align__(1024) uint8_t dsm[];
     const DxSmem L(a.D, a.F, a.T, a.K, a.E, a.nslot);
@@ -190,6 +196,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const int KB1 = D / 128, KB2 = F / 128;
     const int S2 = D / F;                      // down tiles per stage-2 item
     const int G1 = F / 8, G2 = D / (16 * S2);  // items per unit
+    const int GS = STAGE == 1 ? G1 : G2;
     const int CB = 16 * S2 > 256 ? 16 * S2 : 256;   // channels per combine block
     const int NCB = D / CB;
     const int comb_target = K * (CB / (16 * S2));
@@ -197,29 +204,20 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     uint8_t *ring = dsm + L.ring;
     uint8_t *bbuf = dsm + L.bbuf;
     DxSide *side = (DxSide *)(dsm + L.side);
-    DxChunk *queue = (DxChunk *)(dsm + L.queue);
     uint64_t *bars = (uint64_t *)(dsm + L.bars);
     const uint32_t b_rfull = smem_addr(bars), b_rempty = b_rfull + 8 * a.nslot;
     const uint32_t b_bfull = b_rempty + 8 * a.nslot, b_bempty = b_bfull + 8 * kDxNB;
-    const uint32_t b_qfull = b_bempty + 8 * kDxNB, b_qempty = b_qfull + 8 * kDxQueue;
-    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * a.nslot + 2 * kDxNB + 2 * kDxQueue);
+    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * a.nslot + 2 * kDxNB);
     volatile int *s_issued = (volatile int *)(abort + 1);   // items whose codes the producer copied
-    volatile int *s_last_tma = s_issued + 1;                // the last chunk whose B operand was gathered
-    // routing tables
-    int *t_idx = (int *)(dsm + L.tables);
-    float *t_w = (float *)(t_idx + S);
+    volatile int *s_last_tma = s_issued + 1;                // the last unit whose B operand was gathered
+    // routing tables (loaded from the routing kernel's outputs)
+    float *t_w = (float *)(dsm + L.tables);
     int *t_perm = (int *)(t_w + S);
     int *t_inv = t_perm + S;
-    int *t_cnt = t_inv + S;
-    int *t_act = t_cnt + E;
-    int *t_off = t_act + E;
-    float *t_sx = (float *)(t_off + E + 2);
+    float *t_sx = (float *)(t_inv + S);
     int *t_sumx = (int *)(t_sx + T);
-    int *t_misc = t_sumx + T;   // [0] n_active, [1] n_units
-    int2 *t_unit = (int2 *)(t_misc + 16);   // {expert, first position | count << 16}
-    const int max_units = E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;
-    unsigned long long *tmask =
-        (unsigned long long *)(((uintptr_t)(t_unit + max_units) + 7) & ~(uintptr_t)7);
+    int *t_misc = t_sumx + T;   // [1] n_units
+    int2 *t_unit = (int2 *)(((uintptr_t)(t_misc + 2) + 7) & ~(uintptr_t)7);   // {expert, first | count << 16}
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -231,181 +229,104 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             mbar_init(b_bfull + 8 * b, 1);
             mbar_init(b_bempty + 8 * b, kDxComputeWarps);
         }
-        for (int c = 0; c < kDxQueue; c++) {
-            mbar_init(b_qfull + 8 * c, 1);
-            mbar_init(b_qempty + 8 * c, 1 + kDxComputeWarps);
-        }
         *abort = 0u;
         *s_issued = 0;
         *s_last_tma = -1;
         fence_barrier_init();
     }
-    // A routing kernel launched after this one as a programmatic dependent (the next
-    // layer of a stack) may start loading its router weights now; it waits for
-    // this grid's completion before it reads anything this kernel writes.
+    if (STAGE == 1) {
+        // Launched as a programmatic dependent of the routing kernel: nothing it
+        // wrote is read before this wait.  Only after it may the down kernel
+        // launch, so that when a down CTA runs the routing outputs are complete.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
+    // the next kernel (the down kernel, or the next layer's routing kernel) may
+    // launch; it waits for this grid before it reads anything this grid writes
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    // The kernel may be launched while the routing kernel still runs (programmatic
-    // dependent launch): nothing it writes is read before this point.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---------------- prologue: the permutation of the T*K slots (T <= 64) from the
-    // router's choices (a token bitmask per expert: counts by popcount, a slot's rank
-    // within its expert by the number of earlier tokens), and the units
-    const bool writer = blockIdx.x == 0;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) tmask[e] = 0ull;
+    // ---------------- prologue: the routing tables, one round of loads
+    // (stage 2 reads only the routing outputs here; h and the maxima of the
+    // gate/up kernel are read after its own wait, by the B-operand warp)
+    const int n_units_g = __ldcg(a.n_units);
     for (int q = threadIdx.x; q < S; q += blockDim.x) {
-        t_idx[q] = __ldcg(a.topk_idx + q);
         t_w[q] = __ldcg(a.topk_w + q);
+        t_perm[q] = __ldcg(a.perm + q);
+        t_inv[q] = __ldcg(a.inv + q);
     }
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
         t_sx[t] = __ldcg(a.sx + t);
         t_sumx[t] = __ldcg(a.sumx + t);
     }
-    __syncthreads();
-    for (int q = threadIdx.x; q < S; q += blockDim.x) {
-        const int e = t_idx[q];
-        if (e >= 0 && e < E)
-            atomicOr(tmask + e, 1ull << (q / K));
-        else if (writer)
-            set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        const int per = (E + 31) / 32, e0 = lane * per;
-        int csum = 0, asum = 0, usum = 0;
-        for (int i = 0; i < per; i++) {
-            const int e = e0 + i;
-            if (e < E) {
-                const int c = __popcll(tmask[e]);
-                csum += c;
-                asum += c > 0;
-                usum += (c + kDxUnitTokens - 1) / kDxUnitTokens;
-            }
-        }
-        int cs = csum, as = asum, us = usum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(FULL, cs, o), w = __shfl_up_sync(FULL, as, o), x = __shfl_up_sync(FULL, us, o);
-            if (lane >= o) {
-                cs += v;
-                as += w;
-                us += x;
-            }
-        }
-        int coff = cs - csum, aoff = as - asum, uoff = us - usum;
-        for (int i = 0; i < per; i++) {
-            const int e = e0 + i;
-            if (e < E) {
-                const int c = __popcll(tmask[e]);
-                t_cnt[e] = c;
-                t_off[e] = coff;
-                if (writer && a.tap_counts) a.tap_counts[e] = c;
-                if (writer && a.tap_offsets) a.tap_offsets[e] = coff;
-                for (int u0 = 0; u0 < c; u0 += kDxUnitTokens)
-                    t_unit[uoff++] = make_int2(e, (coff + u0) | (min(kDxUnitTokens, c - u0) << 16));
-                coff += c;
-                if (c) t_act[aoff++] = e;
-            }
-        }
-        if (lane == 31) {
-            t_off[E] = cs;
-            t_misc[0] = as;
-            t_misc[1] = us;
-            if (writer && a.tap_offsets) a.tap_offsets[E] = cs;
-        }
-    }
-    __syncthreads();
-    for (int q = threadIdx.x; q < S; q += blockDim.x) {
-        const int e = t_idx[q];
-        if (e < 0 || e >= E) continue;
-        const int t = q / K;
-        const int p = t_off[e] + __popcll(tmask[e] & ((1ull << t) - 1ull));
-        t_perm[p] = q;
-        t_inv[q] = p;
-        if (writer && a.tap_perm) a.tap_perm[p] = q;
-    }
+    for (int u = threadIdx.x; u < n_units_g; u += blockDim.x) t_unit[u] = __ldcg(a.units + u);
+    if (threadIdx.x == 0) t_misc[1] = n_units_g;
     __syncthreads();
     const int n_units = t_misc[1];
-    const int cpu1 = G1 / a.chunk1, cpu2 = G2 / a.chunk2;   // chunks per unit
-    const int nc1 = n_units * cpu1, nc_tot = nc1 + n_units * cpu2;
+    // this CTA's item range and the units it touches (unit ordinals 0 .. n_uo-1)
+    const int N = n_units * GS;
+    const int j0 = (int)((int64_t)N * blockIdx.x / gridDim.x), j1 = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
+    const int u_first = j0 / GS, n_uo = j1 > j0 ? (j1 - 1) / GS - u_first + 1 : 0;
 
     if (warp == 0) {
-        // ---------------- claims, queue, weight stream
-        int stream = 0;
+        // ---------------- weight stream
         bool ok = true;
-        // one claim is always in flight ahead of the chunk being issued, so the
-        // atomic's round trip overlaps the copies
-        int next = lane == 0 ? atomicAdd(a.claim, 1) : 0;
-        for (int c = 0; ok; c++) {
-            int x = __shfl_sync(FULL, next, 0);
-            if (lane == 0 && x < nc_tot) next = atomicAdd(a.claim, 1);
-            DxChunk ch;
-            ch.stream = stream;
-            if (x >= nc_tot) {
-                ch.stage = 0;
-                ch.unit = ch.first = ch.n = 0;
-            } else if (x < nc1) {
-                ch.stage = 1;
-                ch.unit = x / cpu1;
-                ch.first = (x - ch.unit * cpu1) * a.chunk1;
-                ch.n = a.chunk1;
-            } else {
-                ch.stage = 2;
-                ch.unit = (x - nc1) / cpu2;
-                ch.first = (x - nc1 - ch.unit * cpu2) * a.chunk2;
-                ch.n = a.chunk2;
-            }
-            const int qs = c % kDxQueue;
+        int issued = 0;
+        for (int j = j0; j < j1 && ok; j++) {
+            const int s = (j - j0) % a.nslot;
             if (lane == 0) {
-                if (c >= kDxQueue && !mbar_wait(b_qempty + 8 * qs, ((c / kDxQueue) & 1) ^ 1, abort, a.flag, a.wait_ns))
+                if (!mbar_wait(b_rempty + 8 * s, (((j - j0) / a.nslot) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
-                if (ok) {
-                    queue[qs] = ch;
-                    mbar_arrive(b_qfull + 8 * qs);
+                } else {
+                    const int u = j / GS, it = j - u * GS, e = t_unit[u].x;
+                    const uint32_t dst = smem_addr(ring + (size_t)s * L.slot_bytes), full = b_rfull + 8 * s;
+                    if (STAGE == 1) {
+                        mbar_expect_tx(full, (uint32_t)(L.code_bytes + 64));
+                        bulk_g2s(dst, a.w_gu + ((size_t)e * G1 + it) * L.code_bytes, (uint32_t)L.code_bytes, full);
+                        bulk_g2s(dst + L.code_bytes, a.alpha_gate + (size_t)e * F + 8 * it, 32, full);
+                        bulk_g2s(dst + L.code_bytes + 32, a.alpha_up + (size_t)e * F + 8 * it, 32, full);
+                    } else {
+                        mbar_expect_tx(full, (uint32_t)(L.code_bytes + 64 * S2));
+                        bulk_g2s(dst, a.w_dn + ((size_t)e * G2 + it) * L.code_bytes, (uint32_t)L.code_bytes, full);
+                        bulk_g2s(dst + L.code_bytes, a.alpha_down + (size_t)e * D + 16 * S2 * it, 64 * S2, full);
+                    }
+                    issued = j - j0 + 1;
                 }
             }
             ok = __shfl_sync(FULL, ok, 0);
-            if (!ok || ch.stage == 0) break;
-            const int2 un = t_unit[ch.unit];
-            const int e = un.x;
-            for (int k = 0; k < ch.n; k++, stream++) {
-                const int s = stream % a.nslot;
-                if (lane == 0) {
-                    if (!mbar_wait(b_rempty + 8 * s, ((stream / a.nslot) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
+        }
+        if (lane == 0) *s_issued = issued;
+    } else if (warp == 1) {
+        // ---------------- B operands, one per unit of the range
+        bool ok = true;
+        if (STAGE == 2) {
+            // h and the maxima come from the gate/up kernel: wait for its grid
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            if (a.stall && lane == 0) {
+                // test hook: wait for a word nothing sets, so that the bounded wait expires
+                const uint64_t t0 = global_ns();
+                while (true) {
+                    unsigned v;
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.never) : "memory");
+                    if (v == 1u) break;
+                    __nanosleep(256);
+                    if (*abort || global_ns() - t0 > a.wait_ns) {
+                        *abort = 1u;
+                        set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
                         ok = false;
-                    } else {
-                        const int it = ch.first + k;
-                        const uint8_t *src = ch.stage == 1
-                                                 ? a.w_gu + ((size_t)e * G1 + it) * L.slot_bytes
-                                                 : a.w_dn + ((size_t)e * G2 + it) * L.slot_bytes;
-                        mbar_expect_tx(b_rfull + 8 * s, (uint32_t)L.slot_bytes);
-                        bulk_g2s(smem_addr(ring + (size_t)s * L.slot_bytes), src, (uint32_t)L.slot_bytes,
-                                 b_rfull + 8 * s);
+                        break;
                     }
                 }
-                ok = __shfl_sync(FULL, ok, 0);
-                if (!ok) break;
             }
+            ok = __shfl_sync(FULL, ok, 0);
         }
-        if (lane == 0) *s_issued = stream;
-    } else if (warp == 1) {
-        // ---------------- B operands
-        bool ok = true;
-        for (int c = 0; ok; c++) {
-            const int qs = c % kDxQueue;
-            if (!mbar_wait(b_qfull + 8 * qs, (c / kDxQueue) & 1, abort, a.flag, a.wait_ns)) break;
-            const DxChunk ch = queue[qs];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(b_qempty + 8 * qs);
-            if (ch.stage == 0) break;
-            const int b = c % kDxNB;
-            if (c >= kDxNB && !mbar_wait(b_bempty + 8 * b, ((c / kDxNB) & 1) ^ 1, abort, a.flag, a.wait_ns)) break;
-            const int2 un = t_unit[ch.unit];
+        for (int uo = 0; uo < n_uo && ok; uo++) {
+            const int b = uo % kDxNB;
+            if (uo >= kDxNB && !mbar_wait(b_bempty + 8 * b, ((uo / kDxNB) & 1) ^ 1, abort, a.flag, a.wait_ns)) break;
+            const int2 un = t_unit[u_first + uo];
             const int e = un.x, p0 = un.y & 0xffff, cnt = un.y >> 16;
             DxSide *sd = side + b;
             uint8_t *bb = bbuf + (size_t)b * L.b_bytes;
             const int ntiles = (cnt + 7) / 8;
-            if (ch.stage == 1) {
+            if (STAGE == 1) {
                 if (lane < kDxUnitTokens) {
                     const int n = min(lane, cnt - 1);
                     const int slot = t_perm[p0 + n], t = slot / K;
@@ -417,9 +338,6 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     sd->e = e;
                     sd->cnt = cnt;
                 }
-                // the buffer may hold an earlier stage-2 operand written by plain stores:
-                // order those before the gathers' asynchronous writes
-                fence_async_smem();
                 __threadfence_block();
                 __syncwarp();
                 if (lane == 0) mbar_expect_tx(b_bfull + 8 * b, (uint32_t)(ntiles * KB1 * 1024));
@@ -433,28 +351,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     tma_gather4(smem_addr(bb + nt * KB1 * 1024 + kb * 1024 + hh * 512), &qxp_map, kb * 128, tk[0],
                                 tk[1], tk[2], tk[3], b_bfull + 8 * b);
                 }
-                if (lane == 0) *s_last_tma = c;
+                if (lane == 0) *s_last_tma = uo;
                 continue;
             }
-            // stage 2: wait until every stage-1 item of the unit has finished
-            if (lane == 0) {
-                const uint64_t t0 = global_ns();
-                unsigned v = 0;
-                while (true) {
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.arrive + ch.unit) : "memory");
-                    if (v >= (unsigned)(G1 + a.stall)) break;
-                    __nanosleep(64);
-                    if (*abort || global_ns() - t0 > a.wait_ns) {
-                        *abort = 1u;
-                        set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
-                        ok = false;
-                        break;
-                    }
-                }
-            }
-            ok = __shfl_sync(FULL, ok, 0);
-            if (!ok) break;
-            const bool taps = ch.first == 0;   // the unit's first chunk writes the q_h / s_h taps
+            // stage 2: requantise the unit's rows of h (int8 absmax per slot) into
+            // fragment order, with each slot's scale and code sum (every CTA that
+            // holds items of the unit does this; their q_h / s_h taps agree bitwise)
             for (int n = 0; n < ntiles * 8; n++) {
                 const int nt = n >> 3, g = n & 7;
                 uint8_t *dst = bb + nt * KB2 * 1024 + g * 128;
@@ -488,7 +390,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
                                         ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
                     reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024)[frag_word_pos(w & 31)] = pk;
-                    if (taps && a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * F)[w] = pk;
+                    if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * F)[w] = pk;
                 }
                 sum = warp_sum_int(sum);
                 if (lane == 0) {
@@ -496,7 +398,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     sd->s[n] = sv;
                     sd->sum[n] = sum;
                     sd->pos[n] = pos;
-                    if (taps && a.tap_sh) a.tap_sh[slot] = sv;
+                    if (a.tap_sh) a.tap_sh[slot] = sv;
                 }
             }
             if (lane == 0) {
@@ -508,171 +410,160 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             if (lane == 0) mbar_arrive(b_bfull + 8 * b);
         }
     } else {
-    // ---------------- compute warp cw
-    const int cw = warp - 2;
-    const int g = lane >> 2, tig = lane & 3;
-    bool ok = true;
-    for (int c = 0; ok; c++) {
-        const int qs = c % kDxQueue;
-        if (!mbar_wait(b_qfull + 8 * qs, (c / kDxQueue) & 1, abort, a.flag, a.wait_ns)) break;
-        const DxChunk ch = queue[qs];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_qempty + 8 * qs);
-        if (ch.stage == 0) break;
-        const int b = c % kDxNB;
-        if (!mbar_wait(b_bfull + 8 * b, (c / kDxNB) & 1, abort, a.flag, a.wait_ns)) break;
-        const DxSide *sd = side + b;
-        const int unit = ch.unit, e = sd->e, cnt = sd->cnt;
-        const int ntiles = (cnt + 7) / 8;
-        const uint32_t bb = smem_addr(bbuf + (size_t)b * L.b_bytes) + lane * 32;
-        // the first of this warp's items in the chunk: stream index = cw (mod the warps)
-        int k = (cw - ch.stream) % kDxComputeWarps;
-        if (k < 0) k += kDxComputeWarps;
-        int done_items = 0;   // stage-1 items of the chunk this warp finished
-        for (; k < ch.n; k += kDxComputeWarps) {
-            const int j = ch.stream + k, s = j % a.nslot;
-            if (!mbar_wait(b_rfull + 8 * s, (j / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
-                ok = false;
-                break;
-            }
-            const uint32_t aa = smem_addr(ring + (size_t)s * L.slot_bytes) + lane * 16;
-            const int it = ch.first + k;
-            int acc[2][4][4];
-            if (ch.stage == 1) {
-                // ---- gate/up tile `it`: outputs 8it .. 8it+7 (this lane: output 8it + g)
-                const int o = 8 * it + g;
-                const float ag = __ldg(a.alpha_gate + (size_t)e * F + o), au = __ldg(a.alpha_up + (size_t)e * F + o);
-                if (ntiles == 2)
-                    dx_tile<2>(aa, bb, KB1, KB1 * 1024, acc);
-                else
-                    dx_tile<1>(aa, bb, KB1, KB1 * 1024, acc);
-                // the codes are in registers' results: hand the slot back to the producer now
-                __syncwarp();
-                if (lane == 0) mbar_arrive(b_rempty + 8 * s);
-#pragma unroll
-                for (int nt = 0; nt < 2; nt++) {
-                    if (nt >= ntiles) break;
-                    float hm[2];
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; h2++) {
-                        const int n = 8 * nt + 2 * tig + h2;
-                        hm[h2] = 0.0f;
-                        if (n < cnt) {
-                            const int pos = sd->pos[n], slot = t_perm[pos];
-                            const int gd = dx_total(acc, nt, h2) - sd->sum[n];
-                            const int ud = dx_total(acc, nt, 2 + h2) - sd->sum[n];
-                            const float gv = __fmul_rn((float)gd, __fmul_rn(ag, sd->s[n]));
-                            const float uv = __fmul_rn((float)ud, __fmul_rn(au, sd->s[n]));
-                            const float hv = swiglu(gv, uv);
-                            a.h[(size_t)pos * F + o] = hv;
-                            hm[h2] = fabsf(hv);
-                            if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot * F + o] = gd;
-                            if (a.tap_acc_up) a.tap_acc_up[(size_t)slot * F + o] = ud;
-                        }
-                    }
-                    // maxima over the tile's 8 outputs (lanes of equal tig), then over the unit
-#pragma unroll
-                    for (int o2 = 4; o2 <= 16; o2 <<= 1) {
-                        hm[0] = fmaxf(hm[0], __shfl_xor_sync(FULL, hm[0], o2));
-                        hm[1] = fmaxf(hm[1], __shfl_xor_sync(FULL, hm[1], o2));
-                    }
-                    if (g == 0) {
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; h2++) {
-                            const int n = 8 * nt + 2 * tig + h2;
-                            if (n < cnt) atomicMax(a.amax + sd->pos[n], __float_as_uint(hm[h2]));
-                        }
-                    }
+        // ---------------- compute warp cw: items j0 + cw, j0 + cw + 8, ...
+        const int cw = warp - 2;
+        const int g = lane >> 2, tig = lane & 3;
+        bool ok = true;
+        for (int uo = 0; uo < n_uo && ok; uo++) {
+            const int b = uo % kDxNB;
+            if (!mbar_wait(b_bfull + 8 * b, (uo / kDxNB) & 1, abort, a.flag, a.wait_ns)) break;
+            const DxSide *sd = side + b;
+            const int u = u_first + uo, e = sd->e, cnt = sd->cnt;
+            const int ntiles = (cnt + 7) / 8;
+            const uint32_t bb = smem_addr(bbuf + (size_t)b * L.b_bytes) + lane * 32;
+            // this unit's items within the range, and this warp's first among them
+            const int ja = max(j0, u * GS), jb = min(j1, (u + 1) * GS);
+            int j = ja + ((cw - (ja - j0)) % kDxComputeWarps + kDxComputeWarps) % kDxComputeWarps;
+            for (; j < jb; j += kDxComputeWarps) {
+                const int s = (j - j0) % a.nslot;
+                if (!mbar_wait(b_rfull + 8 * s, ((j - j0) / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
+                    ok = false;
+                    break;
                 }
-                done_items++;
-            } else {
-                // ---- down item `it`: tiles S2*it .. S2*it + S2-1, channels 16*S2*it ..
-                for (int d = 0; d < S2; d++) {
-                    const int dt = S2 * it + d;
+                const uint8_t *slot_p = ring + (size_t)s * L.slot_bytes;
+                const float *alpha_s = reinterpret_cast<const float *>(slot_p + L.code_bytes);   // the item's scales
+                const uint32_t aa = smem_addr(slot_p) + lane * 16;
+                const int it = j - u * GS;
+                int acc[2][4][4];
+                if (STAGE == 1) {
+                    // ---- gate/up tile `it`: outputs 8it .. 8it+7 (this lane: output 8it + g)
+                    const int o = 8 * it + g;
+                    const float ag = alpha_s[g], au = alpha_s[8 + g];
                     if (ntiles == 2)
-                        dx_tile<2>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                        dx_tile<2>(aa, bb, KB1, KB1 * 1024, acc);
                     else
-                        dx_tile<1>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
-                    if (d == S2 - 1) {   // the item's last tile is read: hand the slot back
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(b_rempty + 8 * s);
-                    }
-                    const int ch0 = 16 * dt + g;
-                    const float ad0 = __ldg(a.alpha_down + (size_t)e * D + ch0);
-                    const float ad1 = __ldg(a.alpha_down + (size_t)e * D + ch0 + 8);
+                        dx_tile<1>(aa, bb, KB1, KB1 * 1024, acc);
+                    // the codes have been read: hand the slot back to the weight stream
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(b_rempty + 8 * s);
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++) {
                         if (nt >= ntiles) break;
+                        float hm[2];
 #pragma unroll
                         for (int h2 = 0; h2 < 2; h2++) {
                             const int n = 8 * nt + 2 * tig + h2;
+                            hm[h2] = 0.0f;
                             if (n < cnt) {
-                                const int pos = sd->pos[n];
-                                const int d0 = dx_total(acc, nt, h2) - sd->sum[n];
-                                const int d1 = dx_total(acc, nt, 2 + h2) - sd->sum[n];
-                                a.ye[(size_t)pos * D + ch0] = __fmul_rn((float)d0, __fmul_rn(ad0, sd->s[n]));
-                                a.ye[(size_t)pos * D + ch0 + 8] = __fmul_rn((float)d1, __fmul_rn(ad1, sd->s[n]));
-                                if (a.tap_acc_down) {
-                                    const int slot = t_perm[pos];
-                                    a.tap_acc_down[(size_t)slot * D + ch0] = d0;
-                                    a.tap_acc_down[(size_t)slot * D + ch0 + 8] = d1;
+                                const int pos = sd->pos[n], slot = t_perm[pos];
+                                const int gd = dx_total(acc, nt, h2) - sd->sum[n];
+                                const int ud = dx_total(acc, nt, 2 + h2) - sd->sum[n];
+                                const float gv = __fmul_rn((float)gd, __fmul_rn(ag, sd->s[n]));
+                                const float uv = __fmul_rn((float)ud, __fmul_rn(au, sd->s[n]));
+                                const float hv = swiglu(gv, uv);
+                                a.h[(size_t)pos * F + o] = hv;
+                                hm[h2] = fabsf(hv);
+                                if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot * F + o] = gd;
+                                if (a.tap_acc_up) a.tap_acc_up[(size_t)slot * F + o] = ud;
+                            }
+                        }
+                        // maxima over the tile's 8 outputs (lanes of equal tig), then over the unit
+#pragma unroll
+                        for (int o2 = 4; o2 <= 16; o2 <<= 1) {
+                            hm[0] = fmaxf(hm[0], __shfl_xor_sync(FULL, hm[0], o2));
+                            hm[1] = fmaxf(hm[1], __shfl_xor_sync(FULL, hm[1], o2));
+                        }
+                        if (g == 0) {
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; h2++) {
+                                const int n = 8 * nt + 2 * tig + h2;
+                                if (n < cnt) atomicMax(a.amax + sd->pos[n], __float_as_uint(hm[h2]));
+                            }
+                        }
+                    }
+                } else {
+                    // ---- down item `it`: tiles S2*it .. S2*it + S2-1, channels 16*S2*it ..
+                    for (int d = 0; d < S2; d++) {
+                        const int dt = S2 * it + d;
+                        if (ntiles == 2)
+                            dx_tile<2>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                        else
+                            dx_tile<1>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                        const int ch0 = 16 * dt + g;
+                        const float ad0 = alpha_s[16 * d + g], ad1 = alpha_s[16 * d + 8 + g];
+                        if (d == S2 - 1) {   // the item's codes and scales are read: hand the slot back
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(b_rempty + 8 * s);
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < 2; nt++) {
+                            if (nt >= ntiles) break;
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; h2++) {
+                                const int n = 8 * nt + 2 * tig + h2;
+                                if (n < cnt) {
+                                    const int pos = sd->pos[n];
+                                    const int d0 = dx_total(acc, nt, h2) - sd->sum[n];
+                                    const int d1 = dx_total(acc, nt, 2 + h2) - sd->sum[n];
+                                    a.ye[(size_t)pos * D + ch0] = __fmul_rn((float)d0, __fmul_rn(ad0, sd->s[n]));
+                                    a.ye[(size_t)pos * D + ch0 + 8] = __fmul_rn((float)d1, __fmul_rn(ad1, sd->s[n]));
+                                    if (a.tap_acc_down) {
+                                        const int slot = t_perm[pos];
+                                        a.tap_acc_down[(size_t)slot * D + ch0] = d0;
+                                        a.tap_acc_down[(size_t)slot * D + ch0 + 8] = d1;
+                                    }
                                 }
                             }
                         }
                     }
-                }
-                // arrivals on (token, channel block); the last of a token's arrivals combines the block
-                __threadfence();
-                __syncwarp();
-                const int blk = (16 * S2 * it) / CB;
-                unsigned prev = 0;
-                int t = 0;
-                if (lane < cnt) {
-                    t = t_perm[sd->pos[lane]] / K;
-                    prev = atomicAdd(a.comb + (size_t)t * NCB + blk, 1u);
-                }
-                unsigned done = __ballot_sync(FULL, lane < cnt && prev == (unsigned)(comb_target - 1));
-                if (done) __threadfence();
-                while (done) {
-                    const int jn = __ffs(done) - 1;
-                    done &= done - 1;
-                    const int tt = __shfl_sync(FULL, t, jn);
-                    for (int c4 = lane; c4 < CB / 4; c4 += 32) {
-                        const int cc = blk * CB + 4 * c4;
-                        float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int kk = 0; kk < K; kk++) {
-                            const int sl = tt * K + kk;
-                            const float wk = t_w[sl];
-                            const float4 ev = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)t_inv[sl] * D + cc));
-                            yv.x = __fmaf_rn(wk, ev.x, yv.x);
-                            yv.y = __fmaf_rn(wk, ev.y, yv.y);
-                            yv.z = __fmaf_rn(wk, ev.z, yv.z);
-                            yv.w = __fmaf_rn(wk, ev.w, yv.w);
-                        }
-                        const size_t oo = (size_t)tt * D + cc;
-                        if (a.resid) {
-                            const float4 rv = *reinterpret_cast<const float4 *>(a.resid + oo);
-                            yv.x = __fadd_rn(rv.x, yv.x);
-                            yv.y = __fadd_rn(rv.y, yv.y);
-                            yv.z = __fadd_rn(rv.z, yv.z);
-                            yv.w = __fadd_rn(rv.w, yv.w);
-                        }
-                        *reinterpret_cast<float4 *>(a.y + oo) = yv;
+                    // arrivals on (token, channel block); the last of a token's arrivals
+                    // combines the block (GPU-scope release before, acquire after)
+                    fence_gpu();
+                    __syncwarp();
+                    const int blk = (16 * S2 * it) / CB;
+                    unsigned prev = 0;
+                    int t = 0;
+                    if (lane < cnt) {
+                        t = t_perm[sd->pos[lane]] / K;
+                        prev = atomicAdd(a.comb + (size_t)t * NCB + blk, 1u);
                     }
-                    if (lane == jn) a.comb[(size_t)tt * NCB + blk] = 0u;
+                    unsigned done = __ballot_sync(FULL, lane < cnt && prev == (unsigned)(comb_target - 1));
+                    if (done) fence_gpu();
+                    while (done) {
+                        const int jn = __ffs(done) - 1;
+                        done &= done - 1;
+                        const int tt = __shfl_sync(FULL, t, jn);
+                        for (int c4 = lane; c4 < CB / 4; c4 += 32) {
+                            const int cc = blk * CB + 4 * c4;
+                            float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int kk = 0; kk < K; kk++) {
+                                const int sl = tt * K + kk;
+                                const float wk = t_w[sl];
+                                const float4 ev =
+                                    __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)t_inv[sl] * D + cc));
+                                yv.x = __fmaf_rn(wk, ev.x, yv.x);
+                                yv.y = __fmaf_rn(wk, ev.y, yv.y);
+                                yv.z = __fmaf_rn(wk, ev.z, yv.z);
+                                yv.w = __fmaf_rn(wk, ev.w, yv.w);
+                            }
+                            const size_t oo = (size_t)tt * D + cc;
+                            if (a.resid) {
+                                const float4 rv = *reinterpret_cast<const float4 *>(a.resid + oo);
+                                yv.x = __fadd_rn(rv.x, yv.x);
+                                yv.y = __fadd_rn(rv.y, yv.y);
+                                yv.z = __fadd_rn(rv.z, yv.z);
+                                yv.w = __fadd_rn(rv.w, yv.w);
+                            }
+                            *reinterpret_cast<float4 *>(a.y + oo) = yv;
+                        }
+                        if (lane == jn) a.comb[(size_t)tt * NCB + blk] = 0u;
+                    }
                 }
             }
-        }
-        if (!ok) break;
-        if (done_items) {
-            // publish this warp's h and maxima of the chunk, then count its items on the unit
-            __threadfence();
+            if (!ok) break;
             __syncwarp();
-            if (lane == 0) atomicAdd(a.arrive + unit, (unsigned)done_items);
+            if (lane == 0) mbar_arrive(b_bempty + 8 * b);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_bempty + 8 * b);
-    }
     }
 
     // ---------------- common exit: no copy may still be landing when the CTA exits.

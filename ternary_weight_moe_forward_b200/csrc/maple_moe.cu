@@ -67,7 +67,10 @@ struct maple_moe_s {
     CUtensorMap map_qx, map_qh, map_qxp;   // TMA maps of the activation operands
     // counters (zero between calls)
     unsigned *tg_cnt, *glob_cnt, *comb_cnt;
-    unsigned *dx_clear;            // decode kernel: |h| maxima [64*K], unit arrivals, chunk counter
+    unsigned *dx_clear;            // decode kernels: |h| maxima [64*K] (zeroed by the routing kernel)
+    int2 *units;                   // decode kernels: units of <= 16 slots of one expert (routing kernel)
+    int *n_units;
+    const unsigned *dx_never;      // a word that stays 0 (the stall test hook)
     uint16_t *xn;                  // stack: normalised input of the current layer
     // flag word in host-mapped memory
     unsigned *flag_host;
@@ -225,10 +228,6 @@ static int check_shape(const maple_moe_config *c)
     return MAPLE_OK;
 }
 
-// largest unit count of a decode batch: every active expert, plus one unit per
-// further 16 slots of an expert
-static int64_t dx_max_units(int64_t E, int64_t S) { return E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1; }
-
 extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_weights *w, maple_stream_t stream,
                                 maple_moe_t *out)
 {
@@ -298,7 +297,8 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     const size_t o_ctr = ar.take(0);   // counters: zero between calls
     const size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4);
     const size_t o_cc = ar.take(T64 * (D / 256) * 4);
-    const size_t o_dx = ar.take((S64 + dx_max_units(E, S64) + 1) * 4);
+    const size_t o_dx = ar.take((S64 + 1) * 4);
+    const size_t o_un = ar.take((E + (S64 + kUnitTokens - 1) / kUnitTokens + 1) * 8), o_nun = ar.take(4);
     const size_t o_ctr_end = ar.take(0);
     const size_t o_xn = ar.take(Tm * D * 2);
 
@@ -354,6 +354,9 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->glob_cnt = (unsigned *)(b + o_gc);
     h->comb_cnt = (unsigned *)(b + o_cc);
     h->dx_clear = (unsigned *)(b + o_dx);
+    h->dx_never = h->dx_clear + S64;   // zeroed at create, written by nothing
+    h->units = (int2 *)(b + o_un);
+    h->n_units = (int *)(b + o_nun);
     h->xn = (uint16_t *)(b + o_xn);
     h->wait_ns = kDefaultWaitNs;
     h->ctr_base = b + o_ctr;
@@ -387,9 +390,10 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
                   make_act_map(&h->map_qh, h->qh, S, F, kTcMaxN, true) == MAPLE_OK;
     // allow every kernel the largest dynamic shared memory the device offers, so
     // that handles of different shapes never cap one another's launches
-    const void *kernels[] = {(const void *)tc_gemm_kernel<0>, (const void *)tc_gemm_kernel<1>,
-                             (const void *)pick_route(h->D, h->E), (const void *)pick_qtopk(h->D, h->E),
-                             (const void *)router_gemm_kernel, (const void *)decode_mma_kernel};
+    const void *kernels[] = {(const void *)tc_gemm_kernel<0>,         (const void *)tc_gemm_kernel<1>,
+                             (const void *)pick_route(h->D, h->E),    (const void *)pick_qtopk(h->D, h->E),
+                             (const void *)router_gemm_kernel,        (const void *)decode_stage_kernel<1>,
+                             (const void *)decode_stage_kernel<2>};
     bool smem_ok = true;
     for (const void *k : kernels) smem_ok = allow_max_smem(k, h->device) && smem_ok;
     if (!maps_ok || !smem_ok || cudaGetLastError() != cudaSuccess) {
@@ -432,7 +436,9 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     memset(&a, 0, sizeof a);
     a.x = x;
     a.resid = norm_resid;   // (T <= 64 only) x = bf16(RMSNorm(resid)), computed by the routing kernel
-    a.qxp = frag ? h->qxp : nullptr;   // the decode kernel's fragment-ordered q_x
+    a.qxp = frag ? h->qxp : nullptr;   // the decode kernels' fragment-ordered q_x
+    a.units = frag ? h->units : nullptr;   // and their units (built with the fused permutation)
+    a.n_units = h->n_units;
     a.T = T;
     a.D = h->D;
     a.E = h->E;
@@ -527,25 +533,8 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     return launch_status();
 }
 
-// Items per claimed chunk of the decode kernel: about a third of a CTA's
-// expected share (claims then even out the load), a power of two dividing
-// the items of a unit.  The expected number of units is the expected number
-// of distinct experts of T tokens under uniform routing.
-static void dx_chunks(maple_moe_t h, int T, int &c1, int &c2)
-{
-    const int G1 = h->F / 8, G2 = h->D / (16 * (h->D / h->F));
-    double miss = 1.0;
-    for (int t = 0; t < T; t++) miss *= 1.0 - (double)h->K / h->E;
-    const double units = h->E * (1.0 - miss);
-    const double want = units * G1 / (3.0 * h->num_sms);
-    c1 = 1;
-    while (c1 * 2 <= G1 && c1 * 2 <= want) c1 *= 2;
-    c2 = 1;
-    while (c2 * 2 <= G2 && c2 * 2 <= (double)c1 * G2 / G1) c2 *= 2;
-}
-
-// the decode kernel: permutation, gate/up + SwiGLU, requantisation, down and
-// combine in one persistent launch (one CTA per SM)
+// the two decode kernels: gate/up (+ SwiGLU, per-slot maxima), then down (+
+// requantisation and combine), each a persistent launch of one CTA per SM
 static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps, int nslot,
                            cudaStream_t st)
 {
@@ -560,16 +549,18 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     d.topk_w = h->topk_w;
     d.sx = h->sx;
     d.sumx = h->sumx;
+    d.perm = h->perm;
+    d.inv = h->inv;
+    d.units = h->units;
+    d.n_units = h->n_units;
     d.w_gu = h->w_mma_gu;
     d.w_dn = h->w_mma_dn;
     d.alpha_gate = h->alpha_gate;
     d.alpha_up = h->alpha_up;
     d.alpha_down = h->alpha_down;
     d.h = h->h;
-    const int S = T * h->K;
     d.amax = h->dx_clear;
-    d.arrive = h->dx_clear + S;
-    d.claim = (int *)(h->dx_clear + S + dx_max_units(h->E, S));
+    d.never = h->dx_never;
     d.comb = h->comb_cnt;
     d.ye = h->ye;
     d.y = y;
@@ -580,19 +571,15 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
         d.tap_acc_down = taps->acc_down;
         d.tap_qh = taps->q_h;
         d.tap_sh = taps->s_h;
-        d.tap_counts = taps->expert_counts;
-        d.tap_offsets = taps->expert_offsets;
-        d.tap_perm = taps->perm;
     }
     d.flag = h->flag_dev;
     d.wait_ns = h->wait_ns;
     d.stall = (h->debug_flags & MAPLE_DEBUG_STALL_DOWN) ? 1 : 0;
-    dx_chunks(h, T, d.chunk1, d.chunk2);
     d.nslot = nslot;
-    // Launched as a programmatic dependent of the routing kernel before it: its
-    // launch and set-up overlap the router's tail, and griddepcontrol.wait in the
-    // kernel orders every read of the routing outputs after that grid.  A plain
-    // launch otherwise: a CTA only waits on work that running CTAs have claimed.
+    // Each is a programmatic dependent of the kernel before it (the routing
+    // kernel, then the gate/up kernel): its launch and set-up overlap that
+    // kernel's tail, and griddepcontrol.wait orders every read of that kernel's
+    // outputs after its grid.  No CTA waits on another CTA of its own grid.
     cudaLaunchConfig_t lc;
     memset(&lc, 0, sizeof lc);
     lc.gridDim = dim3(h->num_sms);
@@ -604,8 +591,9 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&lc, decode_mma_kernel, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<1>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 2, st);
+    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<2>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 3, st);
     return launch_status();
 }
@@ -702,12 +690,11 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
     stage_event(h, 0, st);
     int rc;
     if (nslot) {
-        // the decode kernel builds its own permutation from the top-k; the routing
-        // kernel zeroes its maxima, unit arrivals and chunk counter, and writes the
+        // the routing kernel also builds the permutation and the decode kernels'
+        // units (its last CTA), zeroes the per-slot maxima and writes the
         // fragment-ordered q_x
-        const int S = T * h->K;
-        rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, false, false, st, h->dx_clear,
-                       (int)(S + dx_max_units(h->E, S) + 1), true, norm_resid, pdl);
+        rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, false, st, h->dx_clear, T * h->K, true,
+                       norm_resid, pdl);
     } else {
         rc = run_route(h, x, T, taps, nullptr, nullptr, nullptr, true, true, st);
     }

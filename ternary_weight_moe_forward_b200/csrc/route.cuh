@@ -40,8 +40,12 @@ struct RouteArgs {
     int n_clear;
     int *counts, *offsets, *perm, *inv, *active, *n_active;
     int *out_counts, *tap_offsets, *tap_perm;
+    int2 *units;   // optional (with fuse_permute): the decode kernels' units, {expert, first | count << 16}
+    int *n_units;
     unsigned *flag;
 };
+
+constexpr int kUnitTokens = 16;   // slots of a decode unit (two 8-token MMA n-tiles)
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred)
 {
@@ -174,11 +178,85 @@ __device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be)
     return v > bv || (v == bv && e < be);
 }
 
+// (value, index) pairs in rank order: larger value first, equal values by
+// lower index; cas() leaves the pair ranking first in (va, ia)
+__device__ __forceinline__ void rank_cas(float &va, int &ia, float &vb, int &ib)
+{
+    const bool swap = ranks_before(vb, ib, va, ia);
+    const float tv = swap ? vb : va, uv = swap ? va : vb;
+    const int ti = swap ? ib : ia, ui = swap ? ia : ib;
+    va = tv;
+    ia = ti;
+    vb = uv;
+    ib = ui;
+}
+
+// Sort 8 pairs in rank order (bitonic network, fully unrolled)
+__device__ __forceinline__ void rank_sort8(float (&v)[8], int (&id)[8])
+{
+#pragma unroll
+    for (int k = 2; k <= 8; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j >= 1; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int l = i ^ j;
+                if (l > i) {
+                    if ((i & k) == 0)
+                        rank_cas(v[i], id[i], v[l], id[l]);
+                    else
+                        rank_cas(v[l], id[l], v[i], id[i]);
+                }
+            }
+}
+
+// Top 8 of a warp's row held as up to 8 values per lane (NPER <= 8): each lane
+// sorts its pairs, then five exchange levels (lane l with l^1, l^2, .. l^16)
+// merge two sorted lists of 8 into the first 8 of their union (a bitonic
+// merge), so every lane ends with the row's 8 first pairs in rank order.
+template <int NPER>
+__device__ __forceinline__ void warp_top8(const float (&lv)[NPER], int E, float (&v)[8], int (&id)[8])
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const int e = lane + 32 * j;
+        const bool ok = j < NPER && e < E;
+        v[j] = ok ? lv[j < NPER ? j : 0] : -INFINITY;
+        id[j] = ok ? e : 0x7fffffff;
+    }
+    rank_sort8(v, id);
+#pragma unroll
+    for (int o = 1; o <= 16; o <<= 1) {
+        float pv[8];
+        int pi[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            pv[i] = __shfl_xor_sync(FULL, v[i], o);
+            pi[i] = __shfl_xor_sync(FULL, id[i], o);
+        }
+        // first 8 of the two lists: a bitonic sequence, then its merge
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+            if (ranks_before(pv[7 - i], pi[7 - i], v[i], id[i])) {
+                v[i] = pv[7 - i];
+                id[i] = pi[7 - i];
+            }
+#pragma unroll
+        for (int j = 4; j >= 1; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const int l = i ^ j;
+                if (l > i) rank_cas(v[i], id[i], v[l], id[l]);
+            }
+    }
+}
+
 // Top-k of one row of E logits (one warp); lane k < K ends with the k-th
 // choice (my_e) and its softmax weight (my_w).  A NaN logit ranks last and
 // raises the flag.
 template <int NPER>
-__device__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
+__device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
 {
     const int lane = threadIdx.x & 31;
     float lv[NPER];
@@ -197,9 +275,26 @@ __device__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, in
         lv[j] = v;
     }
     if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
-    uint32_t taken = 0;
     float my_v = 0.0f;
     my_e = 0;
+    if (NPER <= 8 && K <= 8) {
+        float v8[8];
+        int i8[8];
+        warp_top8<NPER>(lv, E, v8, i8);
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+            if (lane == k) {
+                my_v = v8[k];
+                my_e = i8[k];
+            }
+        const float l0 = __shfl_sync(FULL, my_v, 0);
+        const float ek = exp_ref(__fsub_rn(my_v, l0));
+        float S = 0.0f;
+        for (int k = 0; k < K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
+        my_w = __fdiv_rn(ek, S);
+        return;
+    }
+    uint32_t taken = 0;
     for (int k = 0; k < K; k++) {
         float bv = -INFINITY;
         int be = 0x7fffffff;
@@ -360,24 +455,41 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
 
     if (eb == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
 
-    for (int tt = 0; tt < nt; tt++) {
-        float acc = 0.0f;
+    // two tokens at a time: two independent fmaf chains, each in the pinned order
+    const float bias_e = a.bias ? a.bias[e] : 0.0f;
+    for (int tt = 0; tt < nt; tt += 2) {
+        const int tb = min(tt + 1, nt - 1);   // an odd last token is computed twice, stored once
+        float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
         for (int i = 0; i < NI; i++) {
-            const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)tt * a.D + 256 * i + 8 * lane);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            const uint4 xa = *reinterpret_cast<const uint4 *>(xs + (size_t)tt * a.D + 256 * i + 8 * lane);
+            const uint4 xb = *reinterpret_cast<const uint4 *>(xs + (size_t)tb * a.D + 256 * i + 8 * lane);
+            const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
             const float wv[8] = {w0[i].x, w0[i].y, w0[i].z, w0[i].w, w1[i].x, w1[i].y, w1[i].z, w1[i].w};
 #pragma unroll
             for (int m = 0; m < 8; m++) {
-                uint32_t bits = (m & 1) ? (xw[m >> 1] >> 16) : (xw[m >> 1] & 0xffffu);
-                acc = __fmaf_rn(bf16_bits_to_f32(bits), wv[m], acc);
+                const uint32_t ba = (m & 1) ? (wa[m >> 1] >> 16) : (wa[m >> 1] & 0xffffu);
+                const uint32_t bb = (m & 1) ? (wb[m >> 1] >> 16) : (wb[m >> 1] & 0xffffu);
+                acc0 = __fmaf_rn(bf16_bits_to_f32(ba), wv[m], acc0);
+                acc1 = __fmaf_rn(bf16_bits_to_f32(bb), wv[m], acc1);
             }
         }
-        float v = warp_tree_sum(acc);
-        if (a.bias) v = __fadd_rn(v, a.bias[e]);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {   // the pairwise tree of warp_tree_sum, two rows at once
+            acc0 = __fadd_rn(acc0, __shfl_xor_sync(FULL, acc0, o));
+            acc1 = __fadd_rn(acc1, __shfl_xor_sync(FULL, acc1, o));
+        }
+        if (a.bias) {
+            acc0 = __fadd_rn(acc0, bias_e);
+            acc1 = __fadd_rn(acc1, bias_e);
+        }
         if (lane == 0) {
-            a.logits[(size_t)(t0 + tt) * a.E + e] = v;
-            if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = v;
+            a.logits[(size_t)(t0 + tt) * a.E + e] = acc0;
+            if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = acc0;
+            if (tb != tt) {
+                a.logits[(size_t)(t0 + tb) * a.E + e] = acc1;
+                if (a.tap_logits) a.tap_logits[(size_t)(t0 + tb) * a.E + e] = acc1;
+            }
         }
     }
 
@@ -427,6 +539,19 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
         }
     }
     scatter_marks(s_mark, 0, a.T, a.K, a.E, [&](int ee) { return s_off[ee]; }, a.perm, a.inv, a.tap_perm);
+    if (a.units) {
+        // units: every expert's slots cut into runs of at most kUnitTokens, in expert order
+        const int per = (a.E + blockDim.x - 1) / blockDim.x;
+        const int lo = min(a.E, (int)threadIdx.x * per), hi = min(a.E, lo + per);
+        int nu = 0;
+        for (int ee = lo; ee < hi; ee++) nu += (s_cnt[ee] + kUnitTokens - 1) / kUnitTokens;
+        int total;
+        int u = block_excl_scan(nu, s_warp, &total);
+        for (int ee = lo; ee < hi; ee++)
+            for (int u0 = 0; u0 < s_cnt[ee]; u0 += kUnitTokens)
+                a.units[u++] = make_int2(ee, (s_off[ee] + u0) | (min(kUnitTokens, s_cnt[ee] - u0) << 16));
+        if (threadIdx.x == 0) *a.n_units = total;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -574,7 +699,7 @@ __device__ __forceinline__ void tree_level(float (&v)[64], int off, bool upper)
 // dynamic shared memory: two stages of (32 token rows x 256 bf16, 16 router rows x 256 fp32)
 constexpr int kRgStage = kRgTok * 256 * 2 + kRgExp * 256 * 4;
 
-__global__ void __launch_bounds__(256, 2) router_gemm_kernel(const uint16_t *x, int T, int D, int E, const float *Wr,
+__global__ void __launch_bounds__(256, 1) router_gemm_kernel(const uint16_t *x, int T, int D, int E, const float *Wr,
                                                              const float *bias, float *logits, float *tap_logits)
 {
     extern __shared__ __align__(16) uint8_t rg_smem[];

@@ -13,13 +13,16 @@
 // MMAs of the next).  The accumulator is 64x the ternary dot product; the
 // epilogue shifts it back (exact).
 //
-// Warp roles (20 warps): warp 0 issues the bulk copies of the 2-bit codes and
-// the activation loads, warp 1 issues the MMAs (and owns the TMEM
+// Warp roles (20 warps): warp 0 issues the bulk copies of the 2-bit codes,
+// warp 2 the activation loads, warp 1 the MMAs (and owns the TMEM
 // allocation), warps 4..11 run the epilogue (TMEM lane quarter = warp % 4,
 // two warps per quarter splitting the columns), warps 12..19 expand the codes
-// into int8 tiles.  Stage hand-off uses mbarriers; every wait is bounded in
-// time and a timeout makes the whole CTA drain and return with a device flag
-// set.
+// into int8 tiles.  Three rings of K stages with their own lifetimes: the
+// codes (small, deep: freed as soon as they are expanded), the activation
+// tiles (freed by the MMAs) and the expanded weight tiles (two or three
+// stages: expansion is quick and local), so that the loads run many stages
+// ahead of the MMAs.  Hand-off uses mbarriers; every wait is bounded in time
+// and a timeout makes the whole CTA drain and return with a device flag set.
 //
 // Mode 0 (gate/up): A = gate rows and up rows of one 128-row block (two MMAs
 // per K step, gate and up accumulators 128 columns apart), B = the q_x rows of
@@ -71,27 +74,31 @@ template <int MODE>
 struct TcCfg;
 template <>
 struct TcCfg<0> {
-    static constexpr int kStages = 4;
+    static constexpr int kCS = 8, kBS = 4, kAS = 2;   // stages of the code, activation and weight rings
     static constexpr int kABytes = 2 * 128 * kTcBK;   // gate + up blocks
     static constexpr int kCodeBytes = 2 * 128 * 32;   // 8 words of 4 bytes per row
 };
 template <>
 struct TcCfg<1> {
-    static constexpr int kStages = 6;
+    static constexpr int kCS = 8, kBS = 6, kAS = 3;
     static constexpr int kABytes = 128 * kTcBK;
     static constexpr int kCodeBytes = 128 * 32;
 };
 
 template <int MODE>
 struct TcSmem {
+    using C = TcCfg<MODE>;
     static constexpr int kBBytes = kTcMaxN * kTcBK;
-    static constexpr int kStage = TcCfg<MODE>::kABytes + kBBytes + TcCfg<MODE>::kCodeBytes;
-    static constexpr int kA = 0, kB = TcCfg<MODE>::kABytes, kCodes = kB + kBBytes;
-    static constexpr int kBars = TcCfg<MODE>::kStages * kStage;   // barriers, TMEM holder, abort word: 256 B
-    static constexpr int kMeta = kBars + 256;                       // epilogue column metadata [2][2][128]
-    static constexpr int kAmax = kMeta + 2 * 2 * kTcMaxN * 4;       // mode 0: per-slot absmax of h [128]
+    static constexpr int kA = 0;                                   // [kAS] expanded weight tiles
+    static constexpr int kB = kA + C::kAS * C::kABytes;            // [kBS] activation tiles
+    static constexpr int kCodes = kB + C::kBS * kBBytes;           // [kCS] 2-bit codes
+    static constexpr int kBars = kCodes + C::kCS * C::kCodeBytes;  // barriers, TMEM holder, abort word: 512 B
+    static constexpr int kMeta = kBars + 512;                      // epilogue column metadata [2][2][128]
+    static constexpr int kAmax = kMeta + 2 * 2 * kTcMaxN * 4;      // mode 0: per-slot absmax of h [128]
     static constexpr int kTotal = kAmax + kTcMaxN * 4;
-    static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+    static constexpr int kNumBars = 2 * (C::kCS + C::kBS + C::kAS) + 5;
+    static_assert(C::kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(8 * kNumBars + 8 <= 512, "barrier area");
 };
 
 struct TcArgs {
@@ -325,7 +332,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
 {
     using Cfg = TcCfg<MODE>;
     using L = TcSmem<MODE>;
-    constexpr int S = Cfg::kStages;
+    constexpr int CS = Cfg::kCS, BS = Cfg::kBS, AS = Cfg::kAS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw;
     if (smem_addr(smem) & 1023u) {   // the 128-byte-swizzled tiles need 1024-byte alignment
@@ -336,19 +343,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     float *meta_scale = (float *)(smem + L::kMeta + 2 * kTcMaxN * 4);
     unsigned *s_amax = (unsigned *)(smem + L::kAmax);               // mode 0: [kTcMaxN] |h| maxima (float bits)
     uint64_t *bars = (uint64_t *)(smem + L::kBars);
-    // bars: codes_full[S], full[S], empty[S], acc_full[2], acc_empty[2], drain
-    uint32_t *tmem_holder = (uint32_t *)(bars + 3 * S + 5);
+    // bars: codes_full[CS], codes_empty[CS], act_full[BS], act_empty[BS], w_full[AS], w_empty[AS],
+    // acc_full[2], acc_empty[2], drain
+    uint32_t *tmem_holder = (uint32_t *)(bars + L::kNumBars);
     volatile uint32_t *abort = tmem_holder + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t b_codes_full = smem_addr(bars), b_full = b_codes_full + 8 * S, b_empty = b_full + 8 * S;
-    const uint32_t b_acc_full = b_empty + 8 * S, b_acc_empty = b_acc_full + 16, b_drain = b_acc_empty + 16;
+    const uint32_t b_codes_full = smem_addr(bars), b_codes_empty = b_codes_full + 8 * CS;
+    const uint32_t b_act_full = b_codes_empty + 8 * CS, b_act_empty = b_act_full + 8 * BS;
+    const uint32_t b_w_full = b_act_empty + 8 * BS, b_w_empty = b_w_full + 8 * AS;
+    const uint32_t b_acc_full = b_w_empty + 8 * AS, b_acc_empty = b_acc_full + 16, b_drain = b_acc_empty + 16;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; s++) {
-            mbar_init(b_codes_full + 8 * s, 1);
-            mbar_init(b_full + 8 * s, kTcProdWarps);   // one arrival per producer warp
-            mbar_init(b_empty + 8 * s, 1);             // MMA commit
+        for (int s = 0; s < CS; s++) {
+            mbar_init(b_codes_full + 8 * s, 1);                 // bulk copy
+            mbar_init(b_codes_empty + 8 * s, kTcProdWarps);     // one arrival per producer warp
+        }
+        for (int s = 0; s < BS; s++) {
+            mbar_init(b_act_full + 8 * s, 1);                   // TMA
+            mbar_init(b_act_empty + 8 * s, 1);                  // MMA commit
+        }
+        for (int s = 0; s < AS; s++) {
+            mbar_init(b_w_full + 8 * s, kTcProdWarps);          // one arrival per producer warp
+            mbar_init(b_w_empty + 8 * s, 1);                    // MMA commit
         }
         for (int b = 0; b < 2; b++) {
             mbar_init(b_acc_full + 8 * b, 1);
@@ -370,7 +387,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     const int n_pc = __ldg(a.n_pieces);
 
     if (warp == 0) {
-        // ---------------- copies: the 2-bit codes (bulk) and the activation rows (TMA)
+        // ---------------- bulk copies of the 2-bit codes, up to CS stages ahead
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            int pc, rb;
+            for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++) {
+                const int4 P = a.pieces[pc];
+                const uint8_t *src = a.codes + ((size_t)P.x * R + rb) * KS * Cfg::kCodeBytes;
+                for (int ks = 0; ks < KS; ks++, it++) {
+                    const int s = it % CS;
+                    if (!mbar_wait(b_codes_empty + 8 * s, ((it / CS) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(b_codes_full + 8 * s, Cfg::kCodeBytes);
+                    bulk_g2s(smem_addr(smem + L::kCodes + s * Cfg::kCodeBytes), src + (size_t)ks * Cfg::kCodeBytes,
+                             Cfg::kCodeBytes, b_codes_full + 8 * s);
+                }
+            }
+            if (!ok) {
+                // drain: wait (bounded) for the copies still in flight, the last CS issued
+                for (uint32_t j = (it > (uint32_t)CS ? it - CS : 0); j < it; j++) {
+                    const uint64_t t0 = global_ns();
+                    while (!mbar_test(b_codes_full + 8 * (j % CS), (j / CS) & 1) && global_ns() - t0 < a.wait_ns) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // ---------------- activation tiles, up to BS stages ahead: mode 0 gathers the
+        // rows of the piece's tokens from q_x (four per copy, one copy per lane),
+        // mode 1 loads 128 consecutive q_h rows
         uint32_t it = 0;
         bool ok = true;
         int cur = -1;
@@ -387,30 +435,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     y[i] = __ldg(a.perm + P.y + row) / a.K;
                 }
             }
-            const uint8_t *src = a.codes + ((size_t)P.x * R + rb) * KS * Cfg::kCodeBytes;
             for (int ks = 0; ks < KS; ks++, it++) {
-                const int s = it % S;
-                if (lane == 0) ok = mbar_wait(b_empty + 8 * s, ((it / S) & 1) ^ 1, abort, a.flag, a.wait_ns);
+                const int s = it % BS;
+                if (lane == 0) ok = mbar_wait(b_act_empty + 8 * s, ((it / BS) & 1) ^ 1, abort, a.flag, a.wait_ns);
                 ok = __shfl_sync(FULL, ok, 0);
                 if (!ok) break;
-                const uint32_t cf = b_codes_full + 8 * s;
-                const uint32_t bdst = smem_addr(smem + s * L::kStage + L::kB);
+                const uint32_t full = b_act_full + 8 * s;
+                const uint32_t bdst = smem_addr(smem + L::kB + s * L::kBBytes);
                 if (lane == 0) {
-                    mbar_expect_tx(cf, Cfg::kCodeBytes + (MODE == 0 ? npad * kTcBK : L::kBBytes));
-                    bulk_g2s(smem_addr(smem + s * L::kStage + L::kCodes), src + (size_t)ks * Cfg::kCodeBytes,
-                             Cfg::kCodeBytes, cf);
-                    if (MODE == 1) tma_load_2d(bdst, &act_map, ks * kTcBK, P.y, cf);
+                    mbar_expect_tx(full, MODE == 0 ? npad * kTcBK : L::kBBytes);
+                    if (MODE == 1) tma_load_2d(bdst, &act_map, ks * kTcBK, P.y, full);
                 }
                 __syncwarp();
                 if (MODE == 0 && 4 * lane < npad)
-                    tma_gather4(bdst + 4 * lane * kTcBK, &act_map, ks * kTcBK, y[0], y[1], y[2], y[3], cf);
+                    tma_gather4(bdst + 4 * lane * kTcBK, &act_map, ks * kTcBK, y[0], y[1], y[2], y[3], full);
             }
         }
         if (!ok && lane == 0) {
-            // drain: wait (bounded) for the copies still in flight, the last S issued
-            for (uint32_t j = (it > (uint32_t)S ? it - S : 0); j < it; j++) {
+            for (uint32_t j = (it > (uint32_t)BS ? it - BS : 0); j < it; j++) {
                 const uint64_t t0 = global_ns();
-                while (!mbar_test(b_codes_full + 8 * (j % S), (j / S) & 1) && global_ns() - t0 < a.wait_ns) {
+                while (!mbar_test(b_act_full + 8 * (j % BS), (j / BS) & 1) && global_ns() - t0 < a.wait_ns) {
                 }
             }
         }
@@ -431,14 +475,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 tc_fence_after();
                 for (int ks = 0; ks < KS; ks++, it++) {
-                    const int s = it % S;
-                    if (!mbar_wait(b_full + 8 * s, (it / S) & 1, abort, a.flag, a.wait_ns)) {
+                    const int sw = it % AS, sb_ = it % BS;
+                    if (!mbar_wait(b_w_full + 8 * sw, (it / AS) & 1, abort, a.flag, a.wait_ns) ||
+                        !mbar_wait(b_act_full + 8 * sb_, (it / BS) & 1, abort, a.flag, a.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(smem + s * L::kStage + L::kA);
-                    const uint32_t sb = smem_addr(smem + s * L::kStage + L::kB);
+                    const uint32_t sa = smem_addr(smem + L::kA + sw * Cfg::kABytes);
+                    const uint32_t sb = smem_addr(smem + L::kB + sb_ * L::kBBytes);
                     const uint64_t da0 = desc_sw128(sa), db = desc_sw128(sb);
                     const uint64_t da1 = desc_sw128(sa + 128 * kTcBK);
 #pragma unroll
@@ -447,7 +492,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         mma_i8(dt, da0 + 2 * k, db + 2 * k, idesc, acc);
                         if (MODE == 0) mma_i8(dt + 128, da1 + 2 * k, db + 2 * k, idesc, acc);
                     }
-                    mma_commit(b_empty + 8 * s);
+                    mma_commit(b_w_empty + 8 * sw);     // both tiles are free once these MMAs are done
+                    mma_commit(b_act_empty + 8 * sb_);
                 }
                 if (!ok) break;
                 mma_commit(b_acc_full + 8 * ab);
@@ -606,13 +652,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         int pc, rb;
         for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++) {
             for (int ks = 0; ks < KS; ks++, it++) {
-                const int s = it % S;
-                if (!mbar_wait(b_codes_full + 8 * s, (it / S) & 1, abort, a.flag, a.wait_ns)) {
+                const int sc = it % CS, sw = it % AS;
+                if (!mbar_wait(b_codes_full + 8 * sc, (it / CS) & 1, abort, a.flag, a.wait_ns) ||
+                    !mbar_wait(b_w_empty + 8 * sw, ((it / AS) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
-                uint8_t *st = smem + s * L::kStage;
-                const uint4 *codes = (const uint4 *)(st + L::kCodes);
+                uint8_t *st = smem + sw * Cfg::kABytes;   // this stage's weight tile is at st + L::kA (kA = 0)
+                const uint4 *codes = (const uint4 *)(smem + L::kCodes + sc * Cfg::kCodeBytes);
                 constexpr int kQuads = Cfg::kCodeBytes / 16;   // four words = one row's half stage
 #pragma unroll
                 for (int i = 0; i < kQuads / (kTcProdWarps * 32); i++) {
@@ -626,7 +673,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 }
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(b_full + 8 * s);
+                if (lane == 0) {
+                    mbar_arrive(b_w_full + 8 * sw);
+                    mbar_arrive(b_codes_empty + 8 * sc);
+                }
             }
         }
     }

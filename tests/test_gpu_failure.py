@@ -1,8 +1,7 @@
 """Failure handling on the GPU, without a fault: a bounded wait made to run out.
 
 maple_moe_set_debug shortens every bounded wait of a handle to 1 ms and makes
-the decode expert kernel's down stage wait for one arrival more than its
-gate/up stage will ever give.  The forward pass must come back in bounded
+the decode path's down kernel wait for a device word that nothing sets.  The forward pass must come back in bounded
 time with MAPLE_FLAG_TIMEOUT raised, the next call must report
 MAPLE_ERR_TIMEOUT (after resetting the handle's counters), and the call after
 that, with the hook off, must match the oracle bit for bit.  Nothing faults,

@@ -2,16 +2,21 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Workload: one decode-shape layer (d_model 2048, 256 experts, top-8, d_ff 512,
-ternary 2-bit weights, seed 0) run on the four decode batches T = 1, 8, 32
-and 64 (105 tokens).  A step is one forward pass of the whole layer (routing,
-permutation, gate/up, down, combine) for each of the four batches.  Before
-every forward pass L2 is flushed (a 256 MB write, outside the timed events),
-so the weights come from HBM.  Each forward is a replay of a CUDA graph of the
-library call (its two kernels), timed with CUDA events on its stream; the step
-time is their sum.  value = tokens per second over all ranks.  The per-stage
-split (routing / experts) comes from a second set of graphs that also record
-the library's stage events, replayed after the timed region.
+Workload: the decode-shape layer (d_model 2048, 256 experts, top-8, d_ff 512,
+ternary 2-bit weights) run on the four decode batches T = 1, 8, 32 and 64 (105
+tokens), each through 32 independently seeded layers (6.4 GB of packed
+weights), one forward pass of the whole layer (routing, permutation, gate/up,
+down, combine) per layer: a step is 4 x 32 layer forwards.  The inputs are
+larger than L2: consecutive forwards read different layers' weights, as a
+model's layers follow one another (at T = 1 the 32 layers touch about 270 MB,
+twice the 126 MB L2).  Per batch size one CUDA graph holds the 32 forwards
+(four kernels each); its replay is timed with CUDA events on the stream, and
+the step time is the sum over the four batch sizes.  value = layer-tokens per
+second (tokens x layers) over all ranks.  The per-stage split (routing /
+gate-up / down + combine) comes from single-forward graphs that also record
+the library's stage events, replayed once per layer after the timed region.
+per_T also reports each batch with L2 flushed before every forward (a 256 MB
+write, outside the events), which also evicts the kernels' instructions.
 
 The JSON line adds: roofline (dominant kernel vs measured HBM bandwidth),
 cpu_baseline (the CPU oracle timed on a sample, pinned to one host core),
@@ -182,11 +187,18 @@ def decode_bytes(n_active: int, T: int) -> int:
 
 
 def experts_bytes(n_active: int, T: int) -> int:
-    """Algorithmic bytes of the expert-stage kernel (decode_experts_kernel):
+    """Algorithmic bytes of the expert stage (gate/up, down and combine kernels):
     packed codes and scales of the experts touched (gate, up, down), the int8
     activations in and the fp32 layer output."""
     D, F = 2048, 512
     return n_active * (3 * F * D // 4 + (2 * F + D) * 4) + T * D + T * D * 4
+
+
+def gate_up_bytes(n_active: int, T: int) -> int:
+    """Algorithmic bytes of the gate/up kernel: gate and up codes and scales of
+    the experts touched, the int8 activations in, h out (fp32, T*K rows)."""
+    D, F, K = 2048, 512, 8
+    return n_active * (2 * F * D // 4 + 2 * F * 4) + T * D + T * K * F * 4
 
 
 
@@ -377,6 +389,9 @@ def bench_tiny(args, dev, stream, flush):
             "tokens_per_s": 8 / (statistics.mean(t) * 1e-3), "bound": "latency"}
 
 
+N_ROT = 32   # layers in rotation: their weights (6.4 GB) are the inputs larger than L2
+
+
 def run_gpu(args, rank: int, world: int):
     import torch
     import torch.distributed as dist
@@ -388,29 +403,39 @@ def run_gpu(args, rank: int, world: int):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     shape = synth.CONFIGS["decode"]["shape"]
-    weights = synth.layer_weights(shape, seed=0)
-    layer = Layer(shape, weights, max_tokens=max(DECODE_T), device=dev)
-    del weights
+    layers = []
+    for l in range(N_ROT):
+        w = synth.layer_weights_device(shape, seed=0, layer=l, device=dev)
+        layers.append(Layer(shape, w, max_tokens=max(DECODE_T), device=dev, flags=tw.MAPLE_CFG_DECODE_ONLY))
+        del w
     stream = torch.cuda.current_stream(dev)
     xs = {T: bf16_from_bits(synth.activations(T, shape.d_model, seed=0, stream=rank), dev) for T in DECODE_T}
     ys = {T: torch.empty((T, shape.d_model), dtype=torch.float32, device=dev) for T in DECODE_T}
-    n_active = {}
+    n_active = {T: [] for T in DECODE_T}   # experts touched, per layer
     for T in DECODE_T:
-        _, _, counts = layer.route(xs[T])
-        n_active[T] = int((counts > 0).sum().item())
+        for L in layers:
+            _, _, counts = L.route(xs[T])
+            n_active[T].append(int((counts > 0).sum().item()))
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    no_flush = torch.empty(0, dtype=torch.float32, device=dev)
 
-    # One CUDA graph per batch size: the forward (routing kernel and expert
-    # kernel) replays without host launch gaps.  A second graph per batch size
-    # also records the library's per-stage events (an event between the routing
-    # and the expert kernel keeps them from overlapping their launch), replayed
-    # after the timed region for the stage split.
-    timers = {T: GraphTimer(lambda T=T: layer.forward(xs[T], y=ys[T]), stream, flush,
-                            lambda ev: tw.maple_moe_set_stage_events(layer.handle, ev)) for T in DECODE_T}
+    # The timed unit: per batch size one CUDA graph holding the forwards of all
+    # N_ROT layers in order (each forward is four kernels, each a programmatic
+    # dependent of the one before); one replay = N_ROT forwards, back to back,
+    # timed with CUDA events on the stream.  Consecutive forwards read different
+    # layers' weights.
+    seq = {T: GraphTimer(lambda T=T: [L.forward(xs[T], y=ys[T]) for L in layers], stream, no_flush)
+           for T in DECODE_T}
+    # one forward per graph, with the library's stage events (an event between two
+    # kernels keeps them from overlapping their launch): the stage split, replayed
+    # once per layer after the timed region
+    single = {(T, l): GraphTimer(lambda T=T, L=L: L.forward(xs[T], y=ys[T]), stream, no_flush,
+                                 lambda ev, L=L: tw.maple_moe_set_stage_events(L.handle, ev))
+              for T in DECODE_T for l, L in enumerate(layers)}
 
     def one_step(timed: list | None):
         for T in DECODE_T:
-            ms = timers[T].replay_ms()
+            ms = seq[T].replay_ms()
             if timed is not None:
                 timed.append((T, ms))
 
@@ -431,14 +456,25 @@ def run_gpu(args, rank: int, world: int):
     torch.cuda.synchronize(dev)
     clocks = clk.stop()
 
-    # stage split: the same number of forwards again, from the graphs with events
-    split = {T: [timers[T].stages_ms() for _ in range(args.steps)] for T in DECODE_T}
-    stage_src = "events inside a second set of graphs (untimed replays)"
+    # stage split: every layer once more, from the graphs with events
+    split = {T: [(l, single[(T, l)].stages_ms()) for l in range(N_ROT)] for T in DECODE_T}
+    stage_src = "events inside single-forward graphs (untimed replays, every layer once)"
+    # the same batches with L2 flushed before each forward (layer 0): code and data cold
+    flushed = {T: [] for T in DECODE_T}
+    for T in DECODE_T:
+        gt = single[(T, 0)]
+        gt.flush = flush
+        for _ in range(args.warmup):
+            gt.replay_ms()
+        flushed[T] = [gt.replay_ms() for _ in range(args.steps)]
+        gt.flush = no_flush
 
     total_ms = sum(t[1] for t in timed)
-    fwd_T = {T: [t[1] for t in timed if t[0] == T] for T in DECODE_T}
-    experts_ms = sum(x[2] - x[0] for T in DECODE_T for x in split[T])
-    experts_alg = sum(experts_bytes(n_active[T], T) for T in DECODE_T) * args.steps
+    fwd_T = {T: [t[1] / N_ROT for t in timed if t[0] == T] for T in DECODE_T}
+    experts_ms = sum(x[2] - x[0] for T in DECODE_T for _, x in split[T])
+    experts_alg = sum(experts_bytes(n_active[T][l], T) for T in DECODE_T for l, _ in split[T])
+    gu_ms = sum(x[1] - x[0] for T in DECODE_T for _, x in split[T])
+    gu_alg = sum(gate_up_bytes(n_active[T][l], T) for T in DECODE_T for l, _ in split[T])
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host, all timed
     hx = {T: xs[T].cpu().pin_memory() for T in DECODE_T}
@@ -448,24 +484,28 @@ def run_gpu(args, rank: int, world: int):
     e2e_ms = 0.0
     for it in range(args.warmup + args.steps):
         for T in DECODE_T:
-            flush.fill_(1.0)
             e0.record(stream)
             dx[T].copy_(hx[T], non_blocking=True)
-            layer.forward(dx[T], y=ys[T])
+            for L in layers:
+                L.forward(dx[T], y=ys[T])
             hy[T].copy_(ys[T], non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             if it >= args.warmup:
                 e2e_ms += e0.elapsed_time(e1)
-    del timers
-    layer.close()
+    del seq, single
+    for L in layers:
+        L.close()
+    del layers
+    torch.cuda.empty_cache()
 
     # ---- max over ranks
     total_ms, e2e_ms, experts_ms = reduce_max_over_ranks([total_ms, e2e_ms, experts_ms], device=dev)
-    tokens_rank = sum(DECODE_T) * args.steps
+    tokens_rank = sum(DECODE_T) * N_ROT * args.steps   # each step: the four batches through every layer
     hbm, peak_kind = peaks()
     achieved = experts_alg / (experts_ms * 1e-3) / 1e9
-    layer_bytes = sum(decode_bytes(n_active[T], T) for T in DECODE_T) * args.steps
+    layer_bytes = sum(decode_bytes(n_active[T][l], T) for T in DECODE_T for l in range(N_ROT)) * args.steps
+    gu_achieved = gu_alg / (gu_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": whole_job_rate(tokens_rank, world, total_ms),
@@ -480,26 +520,35 @@ def run_gpu(args, rank: int, world: int):
         "dtype": "int8",
         "data": "synthetic (seeded ternary weights P=.3/.4/.3, lognormal alpha, N(0,1) bf16 x)",
         "config": config_of(world),
-        "experts_touched": {str(T): n_active[T] for T in DECODE_T},
-        "l2": "flushed before every timed forward (256 MB write, outside the events)",
+        "experts_touched_mean": {str(T): statistics.mean(n_active[T]) for T in DECODE_T},
+        "l2": f"inputs larger than L2: {N_ROT} independently seeded layers (6.4 GB of packed weights) "
+              "in rotation, one per forward; no flush inside the timed region",
         "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(fwd_T[T]) * 1e-3),
                            "us_per_forward": 1e3 * statistics.mean(fwd_T[T]),
-                           "us_route": 1e3 * statistics.mean(x[0] for x in split[T]),
-                           "us_experts": 1e3 * statistics.mean(x[2] - x[0] for x in split[T]),
-                           "layer_hbm_frac": decode_bytes(n_active[T], T) /
+                           "us_per_forward_l2_flushed": 1e3 * statistics.mean(flushed[T]),
+                           "us_route": 1e3 * statistics.mean(x[0] for _, x in split[T]),
+                           "us_gate_up": 1e3 * statistics.mean(x[1] - x[0] for _, x in split[T]),
+                           "us_down_combine": 1e3 * statistics.mean(x[2] - x[1] for _, x in split[T]),
+                           "layer_hbm_frac": statistics.mean(decode_bytes(n, T) for n in n_active[T]) /
                            (statistics.mean(fwd_T[T]) * 1e-3) / 1e9 / hbm,
-                           "experts_hbm_frac": experts_bytes(n_active[T], T) /
-                           (statistics.mean(x[2] - x[0] for x in split[T]) * 1e-3) / 1e9 / hbm}
+                           "experts_hbm_frac": statistics.mean(experts_bytes(n_active[T][l], T) / (
+                               (x[2] - x[0]) * 1e-3) / 1e9 / hbm for l, x in split[T]),
+                           "gate_up_hbm_frac": statistics.mean(gate_up_bytes(n_active[T][l], T) / (
+                               (x[1] - x[0]) * 1e-3) / 1e9 / hbm for l, x in split[T])}
                   for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
-        "roofline": {"kernel": "decode expert stage", "bound": "hbm", "achieved": achieved, "peak": hbm,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": measured_traffic(), "traffic_launch": "T=64 (ncu, profiles/)",
-                     "algorithmic_bytes_T64": experts_bytes(n_active[64], 64)},
+        "roofline": {"kernel": "decode_stage_kernel<1> (gate/up: the dominant kernel)", "bound": "hbm",
+                     "achieved": gu_achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": gu_achieved / hbm, "traffic": measured_traffic(),
+                     "traffic_launch": "T=64 (ncu, profiles/)",
+                     "algorithmic_bytes_T64": gate_up_bytes(round(statistics.mean(n_active[64])), 64)},
+        "roofline_expert_stage": {"kernels": "decode_stage_kernel<1>, decode_stage_kernel<2>, dx_combine_kernel",
+                                  "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                                  "frac": achieved / hbm},
         "e2e": {"value": whole_job_rate(tokens_rank, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(T * shape.d_model * 2 for T in DECODE_T),
                 "d2h_bytes_per_step": sum(T * shape.d_model * 4 for T in DECODE_T)},
-        "gpu_launches": 2 * len(DECODE_T) * args.steps,
+        "gpu_launches": 4 * len(DECODE_T) * N_ROT * args.steps,   # routing, gate/up, down, combine per forward
         "cuda_graphs": True,
         "stage_split_from": stage_src,
         "clocks": clocks,
@@ -517,7 +566,7 @@ def run_gpu(args, rank: int, world: int):
 
 
 def config_of(world: int) -> dict:
-    return {"workload": WORKLOAD, "tokens_per_step": sum(DECODE_T), "layers": 1,
+    return {"workload": WORKLOAD, "layers": N_ROT, "layer_tokens_per_step": sum(DECODE_T) * N_ROT,
             "parallelism": f"replicas x{world}"}
 
 

@@ -1,48 +1,52 @@
 // Expert stage for decode batches (T <= 64) on warp-level int8 MMA
 // (mma.sync m16n8k32: A = 2-bit weight codes as unsigned byte planes,
 // B = int8 activations, int32 accumulators), as two persistent streaming
-// kernels, one CTA per SM:
+// kernels, one CTA per SM, and a combine kernel:
 //
 //   decode_stage_kernel<1>  gate/up: h = SiLU(g) * u per (slot, output), fp32,
 //                           and the per-slot |h| maxima (atomicMax);
 //   decode_stage_kernel<2>  down: requantise h (int8 absmax per slot), the down
-//                           contraction, yE, and the rank-order combine.
+//                           contraction, yE;
+//   dx_combine_kernel       y = resid + the rank-order combine of yE.
 //
-// The second is launched as a programmatic dependent of the first: its CTAs
-// start as the first kernel's CTAs retire, stream their down codes into shared
-// memory, and only then wait for the first grid (griddepcontrol.wait) before
-// reading h.  The grid boundary is the only synchronisation between the two
-// contractions; inside a kernel no CTA waits on another CTA's work, so no
-// grid-wide residency is assumed.
+// Each is launched as a programmatic dependent of the kernel before it: its
+// CTAs start as the previous kernel's CTAs retire (the down kernel streams its
+// codes into shared memory at once) and wait for the previous grid
+// (griddepcontrol.wait) before reading its outputs.  The grid boundaries are
+// the only synchronisation between the phases; no CTA waits on another CTA of
+// its own grid, so no grid-wide residency is assumed.
 //
 // Work.  The routing kernel has built the token -> expert permutation and
 // cut every active expert's slots into units of at most 16 (two 8-token MMA
-// n-tiles); every CTA loads those tables into shared memory.  Stage 1
-// has F/8 items per unit (one 16-row tile: 8 gate rows and the up rows of the
-// same 8 outputs over all of K); stage 2 has D/(16*S2) items per unit (S2 =
-// D/F consecutive 16-channel tiles), so that every item is 4*D bytes of codes.
-// CTA b takes the contiguous item range [N*b/G, N*(b+1)/G).
+// n-tiles); every CTA loads those tables into shared memory.  Stage 1 has F/8
+// items per unit (one 16-row tile: 8 gate rows and the up rows of the same 8
+// outputs over all of K), stage 2 has F/16 items per unit (D/F consecutive
+// 16-channel tiles); an item is 4*D bytes of codes followed by its row scales
+// (layout.cuh).  CTA b takes the contiguous item range [N*b/G, N*(b+1)/G).
 //
-// Warp roles (10 warps):
-//   warp 0     streams the range's codes into a ring of shared-memory slots,
-//              one bulk copy per item, as far ahead as the ring allows;
-//   warp 1     builds each unit's B operand (the unit's activations in MMA
+// Warp roles (11 warps):
+//   warps 0-1  stream the range's items into a ring of shared-memory slots in
+//              groups of kDxCopyItems consecutive items (one mbarrier pair per
+//              group; warp p fills the groups g = p mod 2), one bulk copy per run
+//              of items of one unit (consecutive in memory), as far ahead as the
+//              ring allows.  Two issuing warps and large copies: one thread
+//              issuing one copy per item does not keep HBM busy;
+//   warp 2     builds each unit's B operand (the unit's activations in MMA
 //              fragment order) in one of two buffers: stage 1 by four-row TMA
 //              gathers from the fragment-ordered copy of q_x; stage 2 (after
-//              griddepcontrol.wait) by requantising the unit's rows of h with
-//              the per-slot maxima, with each slot's scale and code sum;
-//   warps 2-9  compute: item j of the range goes to warp j % 8.  Per 128-column
+//              griddepcontrol.wait) from the unit's rows of h, brought in by one
+//              bulk copy, requantised with the per-slot maxima, with each
+//              slot's scale and code sum;
+//   warps 3-10 compute: item j of the range goes to warp j % 8.  Per 128-column
 //              block one 16-byte shared load gives the lane its four code words;
 //              w & (0x03030303 << 2q) is the A fragment of the MMA over columns
 //              32q.. of the block, scaled by 4^q, so four plane accumulators hold
 //              exact multiples of 4^q and combine exactly; subtracting the row's
-//              code sum gives the ternary dot product.  A warp hands its ring slot
-//              back as soon as its MMAs have read it.  Stage-1 epilogue: SwiGLU in
-//              the lane (gate and up of one output sit in c0/c2 and c1/c3), h to
-//              global memory, the slot maxima by shuffles and one atomicMax.
-//              Stage-2 epilogue: yE to global memory, then one arrival per
-//              (token, channel block); the last of a token's arrivals on a block
-//              combines it in rank order (fmaf from 0, plus the residual).
+//              code sum gives the ternary dot product.  A warp hands its item back
+//              as soon as its MMAs have read it.  Stage-1 epilogue: SwiGLU in the
+//              lane (gate and up of one output sit in c0/c2 and c1/c3), h to global
+//              memory, the slot maxima by shuffles and one atomicMax.  Stage-2
+//              epilogue: yE to global memory.
 // Every wait is bounded (the handle's limit) and raises the device flag on
 // expiry; the CTA then drains its copies in flight and returns.
 #pragma once
@@ -57,40 +61,38 @@
 namespace maple {
 
 // Eight compute warps: each holds a ring slot only while its MMAs read it, so
-// that most of the ring's slots are always copies in flight (the ring, not the
-// MMAs, sets how many bytes per SM are on their way from HBM).
+// that most of the ring's slots are always copies in flight.
 constexpr int kDxComputeWarps = 8;
-constexpr int kDxThreads = (2 + kDxComputeWarps) * 32;   // 320
+constexpr int kDxProducers = 2;                          // weight-stream warps
+constexpr int kDxBuilder = kDxProducers;                 // the B-operand warp
+constexpr int kDxCompute0 = kDxProducers + 1;            // first compute warp
+constexpr int kDxThreads = (kDxCompute0 + kDxComputeWarps) * 32;   // 352
 constexpr int kDxUnitTokens = kUnitTokens;               // tokens of a unit: two MMA n-tiles
 constexpr int kDxNB = 2;                                 // B-operand buffers
 constexpr int kDxMaxF = 1024;                            // largest d_ff (the shape limit)
+// Items per ring group (one copy per run of an expert's items): few large copies
+// stream faster than many small ones.  Divides kDxComputeWarps.
+constexpr int kDxCopyItems = 4;
 
 struct DxArgs {
     int T, D, E, K, F;
-    const int *topk_idx;   // [T][K] the router's choices (distinct per token)
-    const float *topk_w;   // [T][K] their softmax weights
     const float *sx;       // [T] scale of q_x
     const int *sumx;       // [T] sum of q_x's codes
-    const uint8_t *w_gu, *w_dn;   // MMA-tile layouts
-    const float *alpha_gate, *alpha_up, *alpha_down;
+    const uint8_t *w_gu, *w_dn;   // MMA-tile layouts (codes and row scales per item)
     const int *perm;       // [T*K] position -> slot (the routing kernel's permutation)
-    const int *inv;        // [T*K] slot -> position
     const int2 *units;     // the units: {expert, first position | count << 16}
     const int *n_units;
     float *h;              // [T*K][F] SwiGLU outputs, position order
     unsigned *amax;        // [T*K] |h| maxima (float bits), zero before stage 1
-    unsigned *comb;        // [T][D/cb] arrivals per (token, channel block), zero between launches
     const unsigned *never; // a word that stays 0 (the stall test hook waits for it to become 1)
     float *ye;             // [T*K][D] expert outputs, position order
-    float *y;              // [T][D]
-    const float *resid;    // [T][D] or null: y = resid + combine
     int *tap_acc_gate, *tap_acc_up, *tap_acc_down;
     int8_t *tap_qh;
     float *tap_sh;
     unsigned *flag;
     uint64_t wait_ns;
     int stall;             // test hook: stage 2 waits for `never` to become 1
-    int nslot;             // weight ring slots (4*D bytes of codes + the item's scales)
+    int nslot;             // ring slots (a multiple of kDxComputeWarps)
 };
 
 struct DxSide {                 // per-slot data of a unit, next to its B operand
@@ -100,38 +102,48 @@ struct DxSide {                 // per-slot data of a unit, next to its B operan
     int e, cnt;
 };
 
-// shared-memory layout of the decode kernels
+// shared-memory layout of a decode kernel
 struct DxSmem {
-    int ring, bbuf, side, bars, tables, total;
-    int code_bytes, alpha_bytes, slot_bytes, b_bytes;
-    __host__ __device__ DxSmem(int D, int F, int T, int K, int E, int nslot)
+    int ring, bbuf, hst, side, bars, tables, total;
+    int code_bytes, item_bytes, b_bytes, hst_bytes, ngroups;
+    __host__ __device__ DxSmem(int stage, int D, int F, int T, int K, int E, int nslot)
     {
-        // a ring slot: an item's codes, then its scales (stage 1: alpha_gate and
-        // alpha_up of 8 outputs; stage 2: alpha_down of its 16*D/F channels)
         code_bytes = 4 * D;
-        alpha_bytes = 64 * (D / F) > 64 ? 64 * (D / F) : 64;
-        slot_bytes = code_bytes + alpha_bytes;
-        b_bytes = 2 * (D / 128) * 1024;
+        item_bytes = stage == 1 ? (int)mma_gu_item_bytes(D) : (int)mma_dn_item_bytes(D, F);
+        b_bytes = 2 * ((stage == 1 ? D : F) / 128) * 1024;            // two 8-token n-tiles
+        hst_bytes = stage == 1 ? 0 : 2 * kDxUnitTokens * F * 4;      // two units' rows of h
+        ngroups = nslot / kDxCopyItems;
         ring = 0;
-        bbuf = ring + nslot * slot_bytes;
-        side = bbuf + kDxNB * b_bytes;
+        bbuf = (ring + nslot * item_bytes + 1023) & ~1023;
+        hst = bbuf + kDxNB * b_bytes;
+        side = hst + hst_bytes;
         bars = (side + kDxNB * (int)sizeof(DxSide) + 7) & ~7;
-        const int n_bars = 2 * nslot + 2 * kDxNB;
-        tables = bars + 8 * n_bars + 16;   // + abort word, issued count, last gathered unit, spare
+        const int n_bars = 2 * ngroups + 2 * kDxNB + 2;   // ring groups full/empty, B full/empty, h staged [2]
+        // + abort word, last gathered unit, copies into each h buffer; per ring group the copies issued into it
+        tables = bars + 8 * n_bars + 16 + 4 * ngroups;
         const int S = T * K, units = E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;
-        // t_w, t_perm, t_inv [S]; t_sx, t_sumx [T]; misc [2]; units [units] (int2, 8-byte aligned)
-        int tb = 3 * S * 4 + 2 * T * 4 + 2 * 4;
+        // t_perm [S]; t_sx, t_sumx [T]; misc [2]; units [units] (int2, 8-byte aligned)
+        int tb = S * 4 + 2 * T * 4 + 2 * 4;
         tb = (tb + 7) & ~7;
         total = tables + tb + units * 8;
     }
 };
 
-// ring slots for a shape within a shared-memory budget (0: the kernels do not fit)
-__host__ inline int dx_ring_slots(int D, int F, int T, int K, int E, size_t budget)
+// Ring slots of a decode kernel within a shared-memory budget (0: it does not
+// fit).  Item j of a CTA's range goes to compute warp j % 8 and to slot
+// j % nslot; with nslot a multiple of 8, items j and j + nslot (the next use of
+// the slot) belong to the same warp (and with nslot a multiple of
+// kDxCopyItems * kDxProducers, every ring group to one producer warp).  Otherwise the warp of item j + nslot could
+// test the slot group's full barrier while item j's copy is still landing, see
+// the barrier in the phase before and take it as complete (a parity wait
+// accepts the current phase and the one before it).
+__host__ inline int dx_ring_slots(int stage, int D, int F, int T, int K, int E, size_t budget)
 {
-    if (F > D) return 0;
-    for (int n = 32; n >= 4; n--)
-        if ((size_t)DxSmem(D, F, T, K, E, n).total <= budget) return n;
+    if (F > D || D % F) return 0;
+    constexpr int step = kDxComputeWarps > kDxCopyItems * kDxProducers ? kDxComputeWarps : kDxCopyItems * kDxProducers;
+    static_assert(step % kDxComputeWarps == 0 && step % (kDxCopyItems * kDxProducers) == 0, "ring step");
+    for (int n = 32; n >= step; n -= step)
+        if ((size_t)DxSmem(stage, D, F, T, K, E, n).total <= budget) return n;
     return 0;
 }
 
@@ -153,8 +165,10 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
 
 // One 16-row tile over nkb 128-column blocks against NT n-tiles of 8 tokens:
 // acc[nt][q][i] is plane q of C-fragment register i (a multiple of 4^q).
+// b_lo / b_hi: this lane's two 16-byte B chunks in the first block (the B
+// operand is 128-byte swizzled, see dx_b_chunk).
 template <int NT>
-__device__ __forceinline__ void dx_tile(uint32_t a_addr, uint32_t b_addr, int nkb, int b_nt_stride,
+__device__ __forceinline__ void dx_tile(uint32_t a_addr, uint32_t b_lo, uint32_t b_hi, int nkb, int b_nt_stride,
                                         int (&acc)[2][4][4])
 {
 #pragma unroll
@@ -168,8 +182,8 @@ __device__ __forceinline__ void dx_tile(uint32_t a_addr, uint32_t b_addr, int nk
         const uint4 w = lds128(a_addr + kb * 512);
 #pragma unroll
         for (int nt = 0; nt < NT; nt++) {
-            const uint4 b0 = lds128(b_addr + nt * b_nt_stride + kb * 1024);
-            const uint4 b1 = lds128(b_addr + nt * b_nt_stride + kb * 1024 + 16);
+            const uint4 b0 = lds128(b_lo + nt * b_nt_stride + kb * 1024);
+            const uint4 b1 = lds128(b_hi + nt * b_nt_stride + kb * 1024);
             const uint32_t bq[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int q = 0; q < 4; q++) {
@@ -179,6 +193,13 @@ __device__ __forceinline__ void dx_tile(uint32_t a_addr, uint32_t b_addr, int nk
         }
     }
 }
+
+// B operand layout: per n-tile and 128-column block 1 KB, token g's 128 bytes
+// (fragment order, frag_word_pos) in row g, its 16-byte chunk c stored at
+// chunk c ^ g (the TMA's 128-byte swizzle).  Lane 4g + c2 reads chunks 2c2 and
+// 2c2 + 1 of token g, which lands the eight lanes of every quarter warp on
+// distinct banks.  Byte offset of chunk c of token g within a block:
+__device__ __forceinline__ uint32_t dx_b_chunk(int g, int c) { return (uint32_t)(g * 128 + ((c ^ g) << 4)); }
 
 // the exact row total of register i: acc_0 + acc_1/4 + acc_2/16 + acc_3/64
 __device__ __forceinline__ int dx_total(const int (&acc)[2][4][4], int nt, int i)
@@ -191,47 +212,48 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     decode_stage_kernel(const __grid_constant__ CUtensorMap qxp_map, DxArgs a)
 {
     extern __shared__ __align__(1024) uint8_t dsm[];
-    const DxSmem L(a.D, a.F, a.T, a.K, a.E, a.nslot);
-    const int D = a.D, F = a.F, T = a.T, K = a.K, E = a.E, S = T * K;
+    const DxSmem L(STAGE, a.D, a.F, a.T, a.K, a.E, a.nslot);
+    const int D = a.D, F = a.F, T = a.T, K = a.K, S = T * K;
     const int KB1 = D / 128, KB2 = F / 128;
-    const int S2 = D / F;                      // down tiles per stage-2 item
-    const int G1 = F / 8, G2 = D / (16 * S2);  // items per unit
-    const int GS = STAGE == 1 ? G1 : G2;
-    const int CB = 16 * S2 > 256 ? 16 * S2 : 256;   // channels per combine block
-    const int NCB = D / CB;
-    const int comb_target = K * (CB / (16 * S2));
+    const int S2 = D / F;                                     // down tiles per stage-2 item
+    const int GS = STAGE == 1 ? mma_gu_items(F) : mma_dn_items(F);   // items per unit (= per expert)
+    const uint8_t *wsrc = STAGE == 1 ? a.w_gu : a.w_dn;
 
     uint8_t *ring = dsm + L.ring;
     uint8_t *bbuf = dsm + L.bbuf;
+    uint8_t *hst = dsm + L.hst;
     DxSide *side = (DxSide *)(dsm + L.side);
     uint64_t *bars = (uint64_t *)(dsm + L.bars);
-    const uint32_t b_rfull = smem_addr(bars), b_rempty = b_rfull + 8 * a.nslot;
-    const uint32_t b_bfull = b_rempty + 8 * a.nslot, b_bempty = b_bfull + 8 * kDxNB;
-    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * a.nslot + 2 * kDxNB);
-    volatile int *s_issued = (volatile int *)(abort + 1);   // items whose codes the producer copied
-    volatile int *s_last_tma = s_issued + 1;                // the last unit whose B operand was gathered
+    const uint32_t b_rfull = smem_addr(bars), b_rempty = b_rfull + 8 * L.ngroups;
+    const uint32_t b_bfull = b_rempty + 8 * L.ngroups, b_bempty = b_bfull + 8 * kDxNB;
+    const uint32_t b_hst = b_bempty + 8 * kDxNB;   // [2]: the two h staging buffers
+    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * L.ngroups + 2 * kDxNB + 2);
+    volatile int *s_last_tma = (volatile int *)(abort + 1);   // stage 1: the last unit whose B operand was gathered
+    volatile int *s_hgen = s_last_tma + 1;                    // stage 2: [2] copies issued into each h buffer
+    volatile int *s_gen = s_last_tma + 3;                     // [ngroups] copies issued into each ring group
     // routing tables (loaded from the routing kernel's outputs)
-    float *t_w = (float *)(dsm + L.tables);
-    int *t_perm = (int *)(t_w + S);
-    int *t_inv = t_perm + S;
-    float *t_sx = (float *)(t_inv + S);
+    int *t_perm = (int *)(dsm + L.tables);
+    float *t_sx = (float *)(t_perm + S);
     int *t_sumx = (int *)(t_sx + T);
     int *t_misc = t_sumx + T;   // [1] n_units
     int2 *t_unit = (int2 *)(((uintptr_t)(t_misc + 2) + 7) & ~(uintptr_t)7);   // {expert, first | count << 16}
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.nslot; s++) {
-            mbar_init(b_rfull + 8 * s, 1);
-            mbar_init(b_rempty + 8 * s, 1);
+        for (int g = 0; g < L.ngroups; g++) {
+            mbar_init(b_rfull + 8 * g, 1);
+            mbar_init(b_rempty + 8 * g, kDxCopyItems);
         }
         for (int b = 0; b < kDxNB; b++) {
             mbar_init(b_bfull + 8 * b, 1);
             mbar_init(b_bempty + 8 * b, kDxComputeWarps);
         }
+        mbar_init(b_hst, 1);
+        mbar_init(b_hst + 8, 1);
         *abort = 0u;
-        *s_issued = 0;
         *s_last_tma = -1;
+        s_hgen[0] = s_hgen[1] = 0;
+        for (int g = 0; g < L.ngroups; g++) s_gen[g] = 0;
         fence_barrier_init();
     }
     if (STAGE == 1) {
@@ -240,23 +262,20 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         // launch, so that when a down CTA runs the routing outputs are complete.
         asm volatile("griddepcontrol.wait;" ::: "memory");
     }
-    // the next kernel (the down kernel, or the next layer's routing kernel) may
-    // launch; it waits for this grid before it reads anything this grid writes
+    // the next kernel may launch; it waits for this grid before it reads
+    // anything this grid writes
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---------------- prologue: the routing tables, one round of loads
     // (stage 2 reads only the routing outputs here; h and the maxima of the
     // gate/up kernel are read after its own wait, by the B-operand warp)
     const int n_units_g = __ldcg(a.n_units);
-    for (int q = threadIdx.x; q < S; q += blockDim.x) {
-        t_w[q] = __ldcg(a.topk_w + q);
-        t_perm[q] = __ldcg(a.perm + q);
-        t_inv[q] = __ldcg(a.inv + q);
-    }
-    for (int t = threadIdx.x; t < T; t += blockDim.x) {
-        t_sx[t] = __ldcg(a.sx + t);
-        t_sumx[t] = __ldcg(a.sumx + t);
-    }
+    for (int q = threadIdx.x; q < S; q += blockDim.x) t_perm[q] = __ldcg(a.perm + q);
+    if (STAGE == 1)
+        for (int t = threadIdx.x; t < T; t += blockDim.x) {
+            t_sx[t] = __ldcg(a.sx + t);
+            t_sumx[t] = __ldcg(a.sumx + t);
+        }
     for (int u = threadIdx.x; u < n_units_g; u += blockDim.x) t_unit[u] = __ldcg(a.units + u);
     if (threadIdx.x == 0) t_misc[1] = n_units_g;
     __syncthreads();
@@ -266,35 +285,35 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const int j0 = (int)((int64_t)N * blockIdx.x / gridDim.x), j1 = (int)((int64_t)N * (blockIdx.x + 1) / gridDim.x);
     const int u_first = j0 / GS, n_uo = j1 > j0 ? (j1 - 1) / GS - u_first + 1 : 0;
 
-    if (warp == 0) {
-        // ---------------- weight stream
+    if (warp < kDxProducers) {
+        // ---------------- weight stream: group gi of the range (items j0 + M*gi ..) goes to
+        // ring group gi mod ngroups; this warp takes the groups gi = warp mod kDxProducers
         bool ok = true;
-        int issued = 0;
-        for (int j = j0; j < j1 && ok; j++) {
-            const int s = (j - j0) % a.nslot;
+        const int n_grp = (j1 - j0 + kDxCopyItems - 1) / kDxCopyItems;
+        for (int gi = warp; gi < n_grp && ok; gi += kDxProducers) {
+            const int sg = gi % L.ngroups;
             if (lane == 0) {
-                if (!mbar_wait(b_rempty + 8 * s, (((j - j0) / a.nslot) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
+                if (!mbar_wait(b_rempty + 8 * sg, ((gi / L.ngroups) & 1) ^ 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                 } else {
-                    const int u = j / GS, it = j - u * GS, e = t_unit[u].x;
-                    const uint32_t dst = smem_addr(ring + (size_t)s * L.slot_bytes), full = b_rfull + 8 * s;
-                    if (STAGE == 1) {
-                        mbar_expect_tx(full, (uint32_t)(L.code_bytes + 64));
-                        bulk_g2s(dst, a.w_gu + ((size_t)e * G1 + it) * L.code_bytes, (uint32_t)L.code_bytes, full);
-                        bulk_g2s(dst + L.code_bytes, a.alpha_gate + (size_t)e * F + 8 * it, 32, full);
-                        bulk_g2s(dst + L.code_bytes + 32, a.alpha_up + (size_t)e * F + 8 * it, 32, full);
-                    } else {
-                        mbar_expect_tx(full, (uint32_t)(L.code_bytes + 64 * S2));
-                        bulk_g2s(dst, a.w_dn + ((size_t)e * G2 + it) * L.code_bytes, (uint32_t)L.code_bytes, full);
-                        bulk_g2s(dst + L.code_bytes, a.alpha_down + (size_t)e * D + 16 * S2 * it, 64 * S2, full);
+                    const int ja = j0 + kDxCopyItems * gi, jb = min(j1, ja + kDxCopyItems);
+                    const uint32_t full = b_rfull + 8 * sg;
+                    mbar_expect_tx(full, (uint32_t)((jb - ja) * L.item_bytes));
+                    uint32_t dst = smem_addr(ring + (size_t)sg * kDxCopyItems * L.item_bytes);
+                    for (int j = ja; j < jb;) {
+                        // a run of items of one unit: consecutive in memory
+                        const int u = j / GS, it = j - u * GS, e = t_unit[u].x;
+                        const int n = min(jb - j, GS - it);
+                        bulk_g2s(dst, wsrc + ((size_t)e * GS + it) * L.item_bytes, (uint32_t)(n * L.item_bytes), full);
+                        dst += n * L.item_bytes;
+                        j += n;
                     }
-                    issued = j - j0 + 1;
+                    s_gen[sg] = gi / L.ngroups + 1;
                 }
             }
             ok = __shfl_sync(FULL, ok, 0);
         }
-        if (lane == 0) *s_issued = issued;
-    } else if (warp == 1) {
+    } else if (warp == kDxBuilder) {
         // ---------------- B operands, one per unit of the range
         bool ok = true;
         if (STAGE == 2) {
@@ -354,31 +373,46 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                 if (lane == 0) *s_last_tma = uo;
                 continue;
             }
-            // stage 2: requantise the unit's rows of h (int8 absmax per slot) into
+            // stage 2: the unit's rows of h (consecutive positions) came in one copy
+            // (issued one unit ahead, into the other of two staging buffers), the
+            // per-slot maxima by the lanes; requantise (int8 absmax per slot) into
             // fragment order, with each slot's scale and code sum (every CTA that
             // holds items of the unit does this; their q_h / s_h taps agree bitwise)
+            auto stage_h = [&](int un_o) {   // copy unit un_o's rows of h into buffer un_o & 1
+                const int2 uu = t_unit[u_first + un_o];
+                const int q0 = uu.y & 0xffff, qc = uu.y >> 16, hb = un_o & 1;
+                fence_async_smem();   // earlier reads of the buffer come first
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_expect_tx(b_hst + 8 * hb, (uint32_t)(qc * F * 4));
+                    bulk_g2s(smem_addr(hst + (size_t)hb * (L.hst_bytes / 2)), a.h + (size_t)q0 * F, (uint32_t)(qc * F * 4),
+                             b_hst + 8 * hb);
+                    s_hgen[hb] = s_hgen[hb] + 1;
+                }
+            };
+            if (uo == 0) stage_h(0);
+            const float am_lane = lane < cnt ? __uint_as_float(__ldcg(a.amax + p0 + lane)) : 0.0f;
+            if (!__all_sync(FULL, mbar_wait(b_hst + 8 * (uo & 1), (uo >> 1) & 1, abort, a.flag, a.wait_ns))) break;
+            if (uo + 1 < n_uo) stage_h(uo + 1);
+            const uint8_t *hsrc = hst + (size_t)(uo & 1) * (L.hst_bytes / 2);
             for (int n = 0; n < ntiles * 8; n++) {
                 const int nt = n >> 3, g = n & 7;
-                uint8_t *dst = bb + nt * KB2 * 1024 + g * 128;
+                uint8_t *dst = bb + nt * KB2 * 1024;   // token g's row: 128 bytes at g * 128 of each block
                 if (n >= cnt) {   // padding token of the last n-tile: zeros
                     for (int w = lane; w < KB2 * 32; w += 32)
-                        reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024)[w & 31] = 0u;
+                        reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024 + g * 128)[w & 31] = 0u;
                     continue;
                 }
                 const int pos = p0 + n, slot = t_perm[pos];
-                const float4 *hr = reinterpret_cast<const float4 *>(a.h + (size_t)pos * F);
-                float4 hrow[kDxMaxF / 128];   // this lane's words, all loads in flight together
-#pragma unroll
-                for (int i = 0; i < kDxMaxF / 128; i++)
-                    if (i < F / 128) hrow[i] = __ldcg(hr + lane + 32 * i);
-                const float amax = __uint_as_float(__ldcg(a.amax + pos));
+                const float4 *hr = reinterpret_cast<const float4 *>(hsrc + (size_t)n * F * 4);
+                const float amax = __shfl_sync(FULL, am_lane, n);
                 const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
                 int sum = 0;
 #pragma unroll
                 for (int i = 0; i < kDxMaxF / 128; i++) {
                     if (i >= F / 128) break;
                     const int w = lane + 32 * i;   // word w: columns 4w .. 4w+3
-                    const float4 hv = hrow[i];
+                    const float4 hv = hr[w];
                     int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
                     if (amax > 0.0f) {
                         q0 = quant_code(hv.x, inv);
@@ -389,7 +423,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     sum += q0 + q1 + q2 + q3;
                     const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
                                         ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
-                    reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024)[frag_word_pos(w & 31)] = pk;
+                    const int fp = frag_word_pos(w & 31);   // word of token g's row, swizzled by chunk
+                    reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024 + dx_b_chunk(g, fp >> 2))[fp & 3] = pk;
                     if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * F)[w] = pk;
                 }
                 sum = warp_sum_int(sum);
@@ -411,26 +446,27 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         }
     } else {
         // ---------------- compute warp cw: items j0 + cw, j0 + cw + 8, ...
-        const int cw = warp - 2;
+        const int cw = warp - kDxCompute0;
         const int g = lane >> 2, tig = lane & 3;
         bool ok = true;
         for (int uo = 0; uo < n_uo && ok; uo++) {
             const int b = uo % kDxNB;
             if (!mbar_wait(b_bfull + 8 * b, (uo / kDxNB) & 1, abort, a.flag, a.wait_ns)) break;
             const DxSide *sd = side + b;
-            const int u = u_first + uo, e = sd->e, cnt = sd->cnt;
+            const int u = u_first + uo, cnt = sd->cnt;
             const int ntiles = (cnt + 7) / 8;
-            const uint32_t bb = smem_addr(bbuf + (size_t)b * L.b_bytes) + lane * 32;
+            const uint32_t bbase = smem_addr(bbuf + (size_t)b * L.b_bytes);
+            const uint32_t bb_lo = bbase + dx_b_chunk(g, 2 * tig), bb_hi = bbase + dx_b_chunk(g, 2 * tig + 1);
             // this unit's items within the range, and this warp's first among them
             const int ja = max(j0, u * GS), jb = min(j1, (u + 1) * GS);
             int j = ja + ((cw - (ja - j0)) % kDxComputeWarps + kDxComputeWarps) % kDxComputeWarps;
             for (; j < jb; j += kDxComputeWarps) {
-                const int s = (j - j0) % a.nslot;
-                if (!mbar_wait(b_rfull + 8 * s, ((j - j0) / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
+                const int rel = j - j0, slot = rel % a.nslot, sg = slot / kDxCopyItems;
+                if (!mbar_wait(b_rfull + 8 * sg, (rel / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
-                const uint8_t *slot_p = ring + (size_t)s * L.slot_bytes;
+                const uint8_t *slot_p = ring + (size_t)slot * L.item_bytes;
                 const float *alpha_s = reinterpret_cast<const float *>(slot_p + L.code_bytes);   // the item's scales
                 const uint32_t aa = smem_addr(slot_p) + lane * 16;
                 const int it = j - u * GS;
@@ -440,12 +476,12 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     const int o = 8 * it + g;
                     const float ag = alpha_s[g], au = alpha_s[8 + g];
                     if (ntiles == 2)
-                        dx_tile<2>(aa, bb, KB1, KB1 * 1024, acc);
+                        dx_tile<2>(aa, bb_lo, bb_hi, KB1, KB1 * 1024, acc);
                     else
-                        dx_tile<1>(aa, bb, KB1, KB1 * 1024, acc);
-                    // the codes have been read: hand the slot back to the weight stream
+                        dx_tile<1>(aa, bb_lo, bb_hi, KB1, KB1 * 1024, acc);
+                    // the codes and scales have been read: hand the item back to the weight stream
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(b_rempty + 8 * s);
+                    if (lane == 0) mbar_arrive(b_rempty + 8 * sg);
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++) {
                         if (nt >= ntiles) break;
@@ -455,7 +491,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                             const int n = 8 * nt + 2 * tig + h2;
                             hm[h2] = 0.0f;
                             if (n < cnt) {
-                                const int pos = sd->pos[n], slot = t_perm[pos];
+                                const int pos = sd->pos[n], slot_t = t_perm[pos];
                                 const int gd = dx_total(acc, nt, h2) - sd->sum[n];
                                 const int ud = dx_total(acc, nt, 2 + h2) - sd->sum[n];
                                 const float gv = __fmul_rn((float)gd, __fmul_rn(ag, sd->s[n]));
@@ -463,8 +499,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                                 const float hv = swiglu(gv, uv);
                                 a.h[(size_t)pos * F + o] = hv;
                                 hm[h2] = fabsf(hv);
-                                if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot * F + o] = gd;
-                                if (a.tap_acc_up) a.tap_acc_up[(size_t)slot * F + o] = ud;
+                                if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot_t * F + o] = gd;
+                                if (a.tap_acc_up) a.tap_acc_up[(size_t)slot_t * F + o] = ud;
                             }
                         }
                         // maxima over the tile's 8 outputs (lanes of equal tig), then over the unit
@@ -486,14 +522,14 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     for (int d = 0; d < S2; d++) {
                         const int dt = S2 * it + d;
                         if (ntiles == 2)
-                            dx_tile<2>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                            dx_tile<2>(aa + d * KB2 * 512, bb_lo, bb_hi, KB2, KB2 * 1024, acc);
                         else
-                            dx_tile<1>(aa + d * KB2 * 512, bb, KB2, KB2 * 1024, acc);
+                            dx_tile<1>(aa + d * KB2 * 512, bb_lo, bb_hi, KB2, KB2 * 1024, acc);
                         const int ch0 = 16 * dt + g;
                         const float ad0 = alpha_s[16 * d + g], ad1 = alpha_s[16 * d + 8 + g];
-                        if (d == S2 - 1) {   // the item's codes and scales are read: hand the slot back
+                        if (d == S2 - 1) {   // the item's codes and scales are read: hand it back
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(b_rempty + 8 * s);
+                            if (lane == 0) mbar_arrive(b_rempty + 8 * sg);
                         }
 #pragma unroll
                         for (int nt = 0; nt < 2; nt++) {
@@ -508,55 +544,13 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                                     a.ye[(size_t)pos * D + ch0] = __fmul_rn((float)d0, __fmul_rn(ad0, sd->s[n]));
                                     a.ye[(size_t)pos * D + ch0 + 8] = __fmul_rn((float)d1, __fmul_rn(ad1, sd->s[n]));
                                     if (a.tap_acc_down) {
-                                        const int slot = t_perm[pos];
-                                        a.tap_acc_down[(size_t)slot * D + ch0] = d0;
-                                        a.tap_acc_down[(size_t)slot * D + ch0 + 8] = d1;
+                                        const int slot_t = t_perm[pos];
+                                        a.tap_acc_down[(size_t)slot_t * D + ch0] = d0;
+                                        a.tap_acc_down[(size_t)slot_t * D + ch0 + 8] = d1;
                                     }
                                 }
                             }
                         }
-                    }
-                    // arrivals on (token, channel block); the last of a token's arrivals
-                    // combines the block (GPU-scope release before, acquire after)
-                    fence_gpu();
-                    __syncwarp();
-                    const int blk = (16 * S2 * it) / CB;
-                    unsigned prev = 0;
-                    int t = 0;
-                    if (lane < cnt) {
-                        t = t_perm[sd->pos[lane]] / K;
-                        prev = atomicAdd(a.comb + (size_t)t * NCB + blk, 1u);
-                    }
-                    unsigned done = __ballot_sync(FULL, lane < cnt && prev == (unsigned)(comb_target - 1));
-                    if (done) fence_gpu();
-                    while (done) {
-                        const int jn = __ffs(done) - 1;
-                        done &= done - 1;
-                        const int tt = __shfl_sync(FULL, t, jn);
-                        for (int c4 = lane; c4 < CB / 4; c4 += 32) {
-                            const int cc = blk * CB + 4 * c4;
-                            float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
-                            for (int kk = 0; kk < K; kk++) {
-                                const int sl = tt * K + kk;
-                                const float wk = t_w[sl];
-                                const float4 ev =
-                                    __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)t_inv[sl] * D + cc));
-                                yv.x = __fmaf_rn(wk, ev.x, yv.x);
-                                yv.y = __fmaf_rn(wk, ev.y, yv.y);
-                                yv.z = __fmaf_rn(wk, ev.z, yv.z);
-                                yv.w = __fmaf_rn(wk, ev.w, yv.w);
-                            }
-                            const size_t oo = (size_t)tt * D + cc;
-                            if (a.resid) {
-                                const float4 rv = *reinterpret_cast<const float4 *>(a.resid + oo);
-                                yv.x = __fadd_rn(rv.x, yv.x);
-                                yv.y = __fadd_rn(rv.y, yv.y);
-                                yv.z = __fadd_rn(rv.z, yv.z);
-                                yv.w = __fadd_rn(rv.w, yv.w);
-                            }
-                            *reinterpret_cast<float4 *>(a.y + oo) = yv;
-                        }
-                        if (lane == jn) a.comb[(size_t)tt * NCB + blk] = 0u;
                     }
                 }
             }
@@ -568,20 +562,63 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 
     // ---------------- common exit: no copy may still be landing when the CTA exits.
     // After a normal run every copy has been waited for; after a failed wait the
-    // last nslot weight copies and the last gather are waited for (bounded).
+    // last copy into every ring group and the last B-operand (or h) copy are
+    // waited for (bounded).
     __syncthreads();
     if (threadIdx.x == 0 && *abort) {
-        const int issued = *s_issued, lt = *s_last_tma;
-        for (int j = issued > a.nslot ? issued - a.nslot : 0; j < issued; j++) {
+        const int lt = *s_last_tma;
+        for (int g = 0; g < L.ngroups; g++) {
+            const int gen = s_gen[g];   // copies issued into group g; the last one has phase gen - 1
+            if (!gen) continue;
             const uint64_t t0 = global_ns();
-            while (!mbar_test(b_rfull + 8 * (j % a.nslot), (j / a.nslot) & 1) && global_ns() - t0 < a.wait_ns) {
+            while (!mbar_test(b_rfull + 8 * g, (gen - 1) & 1) && global_ns() - t0 < a.wait_ns) {
             }
         }
-        if (lt >= 0) {
+        if (STAGE == 1 && lt >= 0) {
             const uint64_t t0 = global_ns();
             while (!mbar_test(b_bfull + 8 * (lt % kDxNB), (lt / kDxNB) & 1) && global_ns() - t0 < a.wait_ns) {
             }
         }
+        for (int hb = 0; STAGE == 2 && hb < 2; hb++) {
+            const int gen = s_hgen[hb];   // copies issued into h buffer hb; the last one has phase gen - 1
+            if (!gen) continue;
+            const uint64_t t0 = global_ns();
+            while (!mbar_test(b_hst + 8 * hb, (gen - 1) & 1) && global_ns() - t0 < a.wait_ns) {
+            }
+        }
+    }
+}
+
+// y[t] = resid[t] + sum over ranks k of topk_w[t][k] * yE[inv[t*K + k]]: fmaf
+// from 0 in rank order, then the residual added; one thread per 4 channels.
+// A programmatic dependent of the down kernel (and itself the primary of the
+// next layer's routing kernel).
+__global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const int *inv, const float *topk_w, int T,
+                                                         int K, int D, float *y, const float *resid)
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int d4 = D / 4;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T * d4; i += gridDim.x * blockDim.x) {
+        const int t = i / d4, c = 4 * (i - t * d4);
+        float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < K; k++) {
+            const float wk = __ldcg(topk_w + t * K + k);
+            const float4 ev = __ldcg(reinterpret_cast<const float4 *>(ye + (size_t)__ldcg(inv + t * K + k) * D + c));
+            yv.x = __fmaf_rn(wk, ev.x, yv.x);
+            yv.y = __fmaf_rn(wk, ev.y, yv.y);
+            yv.z = __fmaf_rn(wk, ev.z, yv.z);
+            yv.w = __fmaf_rn(wk, ev.w, yv.w);
+        }
+        const size_t o = (size_t)t * D + c;
+        if (resid) {
+            const float4 rv = *reinterpret_cast<const float4 *>(resid + o);
+            yv.x = __fadd_rn(rv.x, yv.x);
+            yv.y = __fadd_rn(rv.y, yv.y);
+            yv.z = __fadd_rn(rv.z, yv.z);
+            yv.w = __fadd_rn(rv.w, yv.w);
+        }
+        *reinterpret_cast<float4 *>(y + o) = yv;
     }
 }
 

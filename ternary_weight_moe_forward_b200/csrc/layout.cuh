@@ -7,12 +7,18 @@
 // GEMM layout (tcgen05 int8 grouped GEMM, T > decode_max_tokens): see
 // tc_gemm.cuh.
 //
-// MMA-tile layout (the persistent decode kernel, warp-level int8 MMA
-// m16n8k32 with the weights as the 16 x 32 A operand).  A tile is 16 rows
-// over the whole K, stored as K/128 blocks of 512 bytes (32 lanes x 4 words):
-//   gate/up  [E][F/8 tiles][D/128][32][4]  rows 0..7 = gate rows 8t..8t+7,
-//                                          rows 8..15 = the up rows of the same outputs
-//   down     [E][D/16 tiles][F/128][32][4] row r = channel 16t + r
+// MMA-tile layout (the decode kernels, warp-level int8 MMA m16n8k32 with
+// the weights as the 16 x 32 A operand).  A tile is 16 rows over the whole K,
+// stored as K/128 blocks of 512 bytes (32 lanes x 4 words).  Tiles are grouped
+// into items, the unit of the kernels' weight stream, each followed by the
+// row scales it needs, so that one copy brings both:
+//   gate/up  [E][F/8 items]  item t = one tile (rows 0..7 = gate rows 8t..8t+7,
+//            rows 8..15 = the up rows of the same outputs) over D/128 blocks,
+//            then alpha_gate[8t..8t+7], alpha_up[8t..8t+7]   (4D + 64 bytes)
+//   down     [E][F/16 items] item t = S2 = D/F consecutive tiles (tile 16c +
+//            r = channel of row r) over F/128 blocks each, then alpha_down of
+//            its 16*S2 channels                               (4D + 64*S2 bytes)
+// Consecutive items of one expert are contiguous, so a run of them is one copy.
 // Lane l (g = l/4, c = l%4), word i, byte j, plane q (bits 8j + 2q) holds the
 // offset code t + 1 of row g + 8*(i%2), column 128*kb + 32q + 16*(i/2) + 4c + j.
 // So w_i & (0x03030303 << 2q) is A-fragment register i of the MMA over
@@ -31,8 +37,11 @@
 
 namespace maple {
 
-__host__ __device__ constexpr int64_t gu_bytes_per_expert(int D, int F) { return (int64_t)F * D / 2; }
-__host__ __device__ constexpr int64_t dn_bytes_per_expert(int D, int F) { return (int64_t)D * F / 4; }
+// bytes of one item of the MMA-tile layout (codes and scales) and items per expert
+__host__ __device__ constexpr int64_t mma_gu_item_bytes(int D) { return 4 * (int64_t)D + 64; }
+__host__ __device__ constexpr int64_t mma_dn_item_bytes(int D, int F) { return 4 * (int64_t)D + 64 * (int64_t)(D / F); }
+__host__ __device__ constexpr int mma_gu_items(int F) { return F / 8; }
+__host__ __device__ constexpr int mma_dn_items(int F) { return F / 16; }
 
 // map an interchange code to the offset code t + 1 (invalid 3 -> value 0 -> 1)
 __host__ __device__ inline uint32_t offset_code(uint32_t code)

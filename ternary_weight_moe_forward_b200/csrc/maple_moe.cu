@@ -66,7 +66,7 @@ struct maple_moe_s {
     uint32_t *acc_lo;              // and their lowest bits [S][D/32]
     CUtensorMap map_qx, map_qh, map_qxp;   // TMA maps of the activation operands
     // counters (zero between calls)
-    unsigned *tg_cnt, *glob_cnt, *comb_cnt;
+    unsigned *tg_cnt, *glob_cnt;
     unsigned *dx_clear;            // decode kernels: |h| maxima [64*K] (zeroed by the routing kernel)
     int2 *units;                   // decode kernels: units of <= 16 slots of one expert (routing kernel)
     int *n_units;
@@ -267,7 +267,8 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     // shape: d_ff <= d_model and its shared memory at one token) unless every T
     // goes to the tensor cores; the tensor-core one unless the handle is for
     // decode batches only
-    const bool dec_fits = dx_ring_slots(h->D, h->F, 1, h->K, h->E, (size_t)h->optin) > 0;
+    const bool dec_fits = dx_ring_slots(1, h->D, h->F, 1, h->K, h->E, (size_t)h->optin) > 0 &&
+                          dx_ring_slots(2, h->D, h->F, 1, h->K, h->E, (size_t)h->optin) > 0;
     const bool build_dec = !(h->cfg_flags & MAPLE_CFG_FORCE_TC) && dec_fits;
     const bool build_tc = !(h->cfg_flags & (MAPLE_CFG_FORCE_GEMV | MAPLE_CFG_DECODE_ONLY)) || !dec_fits;
     if (!build_dec && (h->cfg_flags & (MAPLE_CFG_FORCE_GEMV | MAPLE_CFG_DECODE_ONLY))) {
@@ -276,7 +277,8 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     }
     const int64_t nblk = (Tm + kPermBlockTokens - 1) / kPermBlockTokens;
     Arena ar;
-    const size_t o_mgu = build_dec ? ar.take(E * F * D / 2) : 0, o_mdn = build_dec ? ar.take(E * D * F / 4) : 0;
+    const size_t o_mgu = build_dec ? ar.take(E * mma_gu_items((int)F) * mma_gu_item_bytes((int)D)) : 0;
+    const size_t o_mdn = build_dec ? ar.take(E * mma_dn_items((int)F) * mma_dn_item_bytes((int)D, (int)F)) : 0;
     const size_t o_tgu = build_tc ? ar.take(E * F * D / 2) : 0, o_tdn = build_tc ? ar.take(E * D * F / 4) : 0;
     const size_t o_ag = ar.take(E * F * 4), o_au = ar.take(E * F * 4), o_ad = ar.take(E * D * 4);
     const size_t o_rw = ar.take(E * D * 4), o_rb = ar.take(E * 4);
@@ -296,7 +298,6 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     const size_t o_ahi = build_tc ? ar.take(S * D * 2) : 0, o_alo = build_tc ? ar.take(S * D / 8) : 0;
     const size_t o_ctr = ar.take(0);   // counters: zero between calls
     const size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4);
-    const size_t o_cc = ar.take(T64 * (D / 256) * 4);
     const size_t o_dx = ar.take((S64 + 1) * 4);
     const size_t o_un = ar.take((E + (S64 + kUnitTokens - 1) / kUnitTokens + 1) * 8), o_nun = ar.take(4);
     const size_t o_ctr_end = ar.take(0);
@@ -352,7 +353,6 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->acc_lo = build_tc ? (uint32_t *)(b + o_alo) : nullptr;
     h->tg_cnt = (unsigned *)(b + o_tg);
     h->glob_cnt = (unsigned *)(b + o_gc);
-    h->comb_cnt = (unsigned *)(b + o_cc);
     h->dx_clear = (unsigned *)(b + o_dx);
     h->dx_never = h->dx_clear + S64;   // zeroed at create, written by nothing
     h->units = (int2 *)(b + o_un);
@@ -377,6 +377,8 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
                                                                                (uint32_t *)h->w_mma_gu);
         repack_mma_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
                                                                                 (uint32_t *)h->w_mma_dn);
+        mma_item_scales_kernel<<<grid_for(E * (2 * F + D), 256, cap), 256, 0, st>>>(
+            h->alpha_gate, h->alpha_up, h->alpha_down, h->E, h->D, h->F, (float *)h->w_mma_gu, (float *)h->w_mma_dn);
     }
     if (build_tc) {
         repack_tc_gu_kernel<<<grid_for(E * F * D / 8, 256, cap), 256, 0, st>>>(w->w_gate, w->w_up, h->E, h->D, h->F,
@@ -384,7 +386,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
         repack_tc_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
                                                                                (uint32_t *)h->w_tc_dn);
     }
-    bool maps_ok = make_act_map(&h->map_qxp, h->qxp, T64, D, 1, false) == MAPLE_OK;
+    bool maps_ok = make_act_map(&h->map_qxp, h->qxp, T64, D, 1, true) == MAPLE_OK;   // 128-byte swizzle: see dx_b_chunk
     if (build_tc)
         maps_ok = maps_ok && make_act_map(&h->map_qx, h->qx, Tm, D, 1, true) == MAPLE_OK &&
                   make_act_map(&h->map_qh, h->qh, S, F, kTcMaxN, true) == MAPLE_OK;
@@ -533,11 +535,14 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     return launch_status();
 }
 
-// the two decode kernels: gate/up (+ SwiGLU, per-slot maxima), then down (+
-// requantisation and combine), each a persistent launch of one CTA per SM
-static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps, int nslot,
+// the decode kernels: gate/up (+ SwiGLU, per-slot maxima), down (+
+// requantisation), combine; the first two persistent, one CTA per SM
+static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
                            cudaStream_t st)
 {
+    const int n1 = dx_ring_slots(1, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
+    const int n2 = dx_ring_slots(2, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
+    if (!n1 || !n2) return MAPLE_ERR_UNSUPPORTED_SHAPE;
     DxArgs d;
     memset(&d, 0, sizeof d);
     d.T = T;
@@ -545,26 +550,17 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     d.E = h->E;
     d.K = h->K;
     d.F = h->F;
-    d.topk_idx = h->topk_idx;
-    d.topk_w = h->topk_w;
     d.sx = h->sx;
     d.sumx = h->sumx;
     d.perm = h->perm;
-    d.inv = h->inv;
     d.units = h->units;
     d.n_units = h->n_units;
     d.w_gu = h->w_mma_gu;
     d.w_dn = h->w_mma_dn;
-    d.alpha_gate = h->alpha_gate;
-    d.alpha_up = h->alpha_up;
-    d.alpha_down = h->alpha_down;
     d.h = h->h;
     d.amax = h->dx_clear;
     d.never = h->dx_never;
-    d.comb = h->comb_cnt;
     d.ye = h->ye;
-    d.y = y;
-    d.resid = resid;
     if (taps) {
         d.tap_acc_gate = taps->acc_gate;
         d.tap_acc_up = taps->acc_up;
@@ -575,25 +571,34 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     d.flag = h->flag_dev;
     d.wait_ns = h->wait_ns;
     d.stall = (h->debug_flags & MAPLE_DEBUG_STALL_DOWN) ? 1 : 0;
-    d.nslot = nslot;
     // Each is a programmatic dependent of the kernel before it (the routing
-    // kernel, then the gate/up kernel): its launch and set-up overlap that
-    // kernel's tail, and griddepcontrol.wait orders every read of that kernel's
-    // outputs after its grid.  No CTA waits on another CTA of its own grid.
+    // kernel, the gate/up kernel, the down kernel): its launch and set-up
+    // overlap that kernel's tail, and griddepcontrol.wait orders every read of
+    // that kernel's outputs after its grid.  No CTA waits on another CTA of its
+    // own grid.
     cudaLaunchConfig_t lc;
     memset(&lc, 0, sizeof lc);
     lc.gridDim = dim3(h->num_sms);
     lc.blockDim = dim3(kDxThreads);
-    lc.dynamicSmemBytes = DxSmem(h->D, h->F, T, h->K, h->E, nslot).total;
     lc.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
+    d.nslot = n1;
+    lc.dynamicSmemBytes = DxSmem(1, h->D, h->F, T, h->K, h->E, n1).total;
     if (cudaLaunchKernelEx(&lc, decode_stage_kernel<1>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 2, st);
+    d.nslot = n2;
+    lc.dynamicSmemBytes = DxSmem(2, h->D, h->F, T, h->K, h->E, n2).total;
     if (cudaLaunchKernelEx(&lc, decode_stage_kernel<2>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+    lc.gridDim = dim3((unsigned)((T * (h->D / 4) + 255) / 256));
+    lc.blockDim = dim3(256);
+    lc.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&lc, dx_combine_kernel, (const float *)h->ye, (const int *)h->inv, (const float *)h->topk_w,
+                           T, h->K, h->D, y, resid) != cudaSuccess)
+        return MAPLE_ERR_CUDA;
     stage_event(h, 3, st);
     return launch_status();
 }
@@ -674,7 +679,9 @@ static int dec_slots(maple_moe_t h, int T)
 {
     if (!h->w_mma_gu || T > kRouteSmallT || (int64_t)T * h->E > kFusedMarkBytes) return 0;
     if (T > h->dmax && !(h->cfg_flags & MAPLE_CFG_FORCE_GEMV)) return 0;
-    return dx_ring_slots(h->D, h->F, T, h->K, h->E, (size_t)h->optin);
+    const int n1 = dx_ring_slots(1, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
+    const int n2 = dx_ring_slots(2, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
+    return n1 < n2 ? n1 : n2;
 }
 
 // norm_resid (decode batches only): the layer input is bf16(RMSNorm(norm_resid)),
@@ -700,7 +707,7 @@ static int forward_impl(maple_moe_t h, const uint16_t *x, int32_t T, float *y, c
     }
     if (rc) return rc;
     stage_event(h, 1, st);
-    return nslot ? run_experts_dec(h, T, y, resid, taps, nslot, st) : run_experts_tc(h, T, y, resid, taps, st);
+    return nslot ? run_experts_dec(h, T, y, resid, taps, st) : run_experts_tc(h, T, y, resid, taps, st);
 }
 
 extern "C" int maple_moe_forward(maple_moe_t h, const uint16_t *x, int32_t T, float *y, const maple_moe_taps *taps,

@@ -29,10 +29,11 @@ __global__ void pack_ternary_kernel(const int8_t *values, int64_t n_words, uint3
     }
 }
 
-// gate/up interchange -> MMA-tile layout (layout.cuh); one thread per output word
+// gate/up interchange -> MMA-tile layout (layout.cuh); one thread per code word
 __global__ void repack_mma_gu_kernel(const uint32_t *gate, const uint32_t *up, int E, int D, int F, uint32_t *out)
 {
-    const int KB = D / 128, NT = F / 8;
+    const int KB = D / 128, NT = mma_gu_items(F);
+    const int64_t item_words = mma_gu_item_bytes(D) / 4;
     const int64_t n = (int64_t)E * NT * KB * 128;
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
         int64_t q = o;
@@ -43,14 +44,15 @@ __global__ void repack_mma_gu_kernel(const uint32_t *gate, const uint32_t *up, i
         const int e = (int)q;
         const int r = mma_word_row(lane, i);   // rows 0..7 gate, 8..15 up, outputs 8t .. 8t+7
         const uint32_t *src = (r < 8 ? gate : up) + ((int64_t)e * F + 8 * t + (r & 7)) * (D / 16);
-        out[o] = mma_word(src, lane, i, kb);
+        out[((int64_t)e * NT + t) * item_words + (kb * 32 + lane) * 4 + i] = mma_word(src, lane, i, kb);
     }
 }
 
-// down interchange -> MMA-tile layout
+// down interchange -> MMA-tile layout; one thread per code word
 __global__ void repack_mma_dn_kernel(const uint32_t *down, int E, int D, int F, uint32_t *out)
 {
-    const int KB = F / 128, NT = D / 16;
+    const int KB = F / 128, NT = D / 16, S2 = D / F, NI = mma_dn_items(F);
+    const int64_t item_words = mma_dn_item_bytes(D, F) / 4;
     const int64_t n = (int64_t)E * NT * KB * 128;
     for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
         int64_t q = o;
@@ -60,7 +62,31 @@ __global__ void repack_mma_dn_kernel(const uint32_t *down, int E, int D, int F, 
         const int t = q % NT; q /= NT;
         const int e = (int)q;
         const uint32_t *src = down + ((int64_t)e * D + 16 * t + mma_word_row(lane, i)) * (F / 16);
-        out[o] = mma_word(src, lane, i, kb);
+        out[((int64_t)e * NI + t / S2) * item_words + (int64_t)(t % S2) * F + (kb * 32 + lane) * 4 + i] =
+            mma_word(src, lane, i, kb);
+    }
+}
+
+// the row scales behind the codes of every MMA-tile item: gate/up item t of
+// expert e ends in alpha_gate[e][8t..8t+7], alpha_up[e][8t..8t+7]; down item t
+// in alpha_down[e][16*S2*t ..] (16*S2 values); one thread per value
+__global__ void mma_item_scales_kernel(const float *alpha_gate, const float *alpha_up, const float *alpha_down, int E,
+                                       int D, int F, float *gu, float *dn)
+{
+    const int S2 = D / F;
+    const int64_t gu_words = mma_gu_item_bytes(D) / 4, dn_words = mma_dn_item_bytes(D, F) / 4;
+    const int64_t n_gu = (int64_t)E * F * 2, n = n_gu + (int64_t)E * D;
+    for (int64_t o = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; o < n; o += (int64_t)gridDim.x * blockDim.x) {
+        if (o < n_gu) {   // (e, output f, gate|up)
+            const int64_t e = o / (2 * F);
+            const int f = (int)(o / 2 % F), m = (int)(o & 1);
+            const float v = (m ? alpha_up : alpha_gate)[e * F + f];
+            gu[(e * mma_gu_items(F) + f / 8) * gu_words + D + 8 * m + (f & 7)] = v;
+        } else {          // (e, channel c)
+            const int64_t q = o - n_gu, e = q / D;
+            const int c = (int)(q % D);
+            dn[(e * mma_dn_items(F) + c / (16 * S2)) * dn_words + D + c % (16 * S2)] = alpha_down[q];
+        }
     }
 }
 

@@ -173,84 +173,23 @@ __device__ void quantize_token_warp(const RouteArgs &a, int t, const uint16_t *x
 // top-k (ties to the lower index) and softmax over the kept logits, one warp
 // per token; NPER = logits held per lane (E <= 32*NPER)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool ranks_before(float v, int e, float bv, int be)
+// A logit and its expert index as one 64-bit key whose unsigned order is the
+// rank order (larger logit first, equal logits by lower index): the float's
+// bits made order-preserving in the high word (-0 taken as +0, which compares
+// equal), the complement of the index in the low word.  No key is 0.
+__device__ __forceinline__ unsigned long long rank_key(float v, int e)
 {
-    return v > bv || (v == bv && e < be);
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;
+    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)o << 32) | (uint32_t)(0xffffffffu - (uint32_t)e);
 }
-
-// (value, index) pairs in rank order: larger value first, equal values by
-// lower index; cas() leaves the pair ranking first in (va, ia)
-__device__ __forceinline__ void rank_cas(float &va, int &ia, float &vb, int &ib)
+__device__ __forceinline__ float rank_key_value(unsigned long long k)
 {
-    const bool swap = ranks_before(vb, ib, va, ia);
-    const float tv = swap ? vb : va, uv = swap ? va : vb;
-    const int ti = swap ? ib : ia, ui = swap ? ia : ib;
-    va = tv;
-    ia = ti;
-    vb = uv;
-    ib = ui;
+    const uint32_t o = (uint32_t)(k >> 32);
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
-
-// Sort 8 pairs in rank order (bitonic network, fully unrolled)
-__device__ __forceinline__ void rank_sort8(float (&v)[8], int (&id)[8])
-{
-#pragma unroll
-    for (int k = 2; k <= 8; k <<= 1)
-#pragma unroll
-        for (int j = k >> 1; j >= 1; j >>= 1)
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const int l = i ^ j;
-                if (l > i) {
-                    if ((i & k) == 0)
-                        rank_cas(v[i], id[i], v[l], id[l]);
-                    else
-                        rank_cas(v[l], id[l], v[i], id[i]);
-                }
-            }
-}
-
-// Top 8 of a warp's row held as up to 8 values per lane (NPER <= 8): each lane
-// sorts its pairs, then five exchange levels (lane l with l^1, l^2, .. l^16)
-// merge two sorted lists of 8 into the first 8 of their union (a bitonic
-// merge), so every lane ends with the row's 8 first pairs in rank order.
-template <int NPER>
-__device__ __forceinline__ void warp_top8(const float (&lv)[NPER], int E, float (&v)[8], int (&id)[8])
-{
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const int e = lane + 32 * j;
-        const bool ok = j < NPER && e < E;
-        v[j] = ok ? lv[j < NPER ? j : 0] : -INFINITY;
-        id[j] = ok ? e : 0x7fffffff;
-    }
-    rank_sort8(v, id);
-#pragma unroll
-    for (int o = 1; o <= 16; o <<= 1) {
-        float pv[8];
-        int pi[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            pv[i] = __shfl_xor_sync(FULL, v[i], o);
-            pi[i] = __shfl_xor_sync(FULL, id[i], o);
-        }
-        // first 8 of the two lists: a bitonic sequence, then its merge
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-            if (ranks_before(pv[7 - i], pi[7 - i], v[i], id[i])) {
-                v[i] = pv[7 - i];
-                id[i] = pi[7 - i];
-            }
-#pragma unroll
-        for (int j = 4; j >= 1; j >>= 1)
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const int l = i ^ j;
-                if (l > i) rank_cas(v[i], id[i], v[l], id[l]);
-            }
-    }
-}
+__device__ __forceinline__ int rank_key_index(unsigned long long k) { return (int)(0xffffffffu - (uint32_t)k); }
 
 // Top-k of one row of E logits (one warp); lane k < K ends with the k-th
 // choice (my_e) and its softmax weight (my_w).  A NaN logit ranks last and
@@ -275,49 +214,29 @@ __device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsig
         lv[j] = v;
     }
     if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
+    // K rounds of a warp-wide maximum of the keys not yet taken (a compact loop:
+    // this runs once per token group on an SM whose instruction cache is cold)
+    unsigned long long key[NPER];
+#pragma unroll
+    for (int j = 0; j < NPER; j++) key[j] = lane + 32 * j < E ? rank_key(lv[j], lane + 32 * j) : 0ull;
     float my_v = 0.0f;
     my_e = 0;
-    if (NPER <= 8 && K <= 8) {
-        float v8[8];
-        int i8[8];
-        warp_top8<NPER>(lv, E, v8, i8);
-#pragma unroll
-        for (int k = 0; k < 8; k++)
-            if (lane == k) {
-                my_v = v8[k];
-                my_e = i8[k];
-            }
-        const float l0 = __shfl_sync(FULL, my_v, 0);
-        const float ek = exp_ref(__fsub_rn(my_v, l0));
-        float S = 0.0f;
-        for (int k = 0; k < K; k++) S = __fadd_rn(S, __shfl_sync(FULL, ek, k));
-        my_w = __fdiv_rn(ek, S);
-        return;
-    }
-    uint32_t taken = 0;
+#pragma unroll 1
     for (int k = 0; k < K; k++) {
-        float bv = -INFINITY;
-        int be = 0x7fffffff;
+        unsigned long long best = 0ull;
 #pragma unroll
-        for (int j = 0; j < NPER; j++) {
-            int e = lane + 32 * j;
-            if (e < E && !((taken >> j) & 1u) && ranks_before(lv[j], e, bv, be)) {
-                bv = lv[j];
-                be = e;
-            }
-        }
+        for (int j = 0; j < NPER; j++) best = key[j] > best ? key[j] : best;
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
-            float ov = __shfl_xor_sync(FULL, bv, o);
-            int oe = __shfl_xor_sync(FULL, be, o);
-            if (ranks_before(ov, oe, bv, be)) {
-                bv = ov;
-                be = oe;
-            }
+            const unsigned long long other = __shfl_xor_sync(FULL, best, o);
+            best = other > best ? other : best;
         }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        const int be = rank_key_index(best);
+#pragma unroll
+        for (int j = 0; j < NPER; j++)
+            if (lane + 32 * j == be) key[j] = 0ull;
         if (lane == k) {
-            my_v = bv;
+            my_v = rank_key_value(best);
             my_e = be;
         }
     }
@@ -519,15 +438,25 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
     fence_gpu();
     if (threadIdx.x == 0) *a.glob_cnt = 0;
 
-    uint8_t *s_mark = rsm;   // reuses the token rows: T*E <= kFusedMarkBytes
+    // T <= 64: per expert the mask of the tokens that chose it (a token's choices
+    // are distinct); a slot's position is its expert's offset plus the number of
+    // earlier tokens in the mask, so every step is a constant number of shared
+    // memory operations per thread (no loop over tokens)
+    unsigned long long *s_mask = reinterpret_cast<unsigned long long *>(rsm);   // [E], reuses the token rows
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_off[kMaxExperts + 1];
-    build_marks(s_mark, a.topk_idx, 0, a.T, a.K, a.E, a.flag);
-    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) {
-        int c = 0;
-        for (int t = 0; t < a.T; t++) c += s_mark[t * a.E + ee] != 0;
-        s_cnt[ee] = c;
+    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_mask[ee] = 0ull;
+    __syncthreads();
+    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
+        const int ee = __ldcg(a.topk_idx + sl);
+        if (ee < 0 || ee >= a.E) {
+            set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
+            continue;
+        }
+        atomicOr(s_mask + ee, 1ull << (sl / a.K));
     }
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_cnt[ee] = __popcll(s_mask[ee]);
     __syncthreads();
     scan_experts(s_cnt, s_off, a.E, a.active, a.n_active, s_warp);
     for (int ee = threadIdx.x; ee <= a.E; ee += blockDim.x) {
@@ -538,7 +467,15 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
             if (a.out_counts) a.out_counts[ee] = s_cnt[ee];
         }
     }
-    scatter_marks(s_mark, 0, a.T, a.K, a.E, [&](int ee) { return s_off[ee]; }, a.perm, a.inv, a.tap_perm);
+    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
+        const int ee = __ldcg(a.topk_idx + sl);
+        if (ee < 0 || ee >= a.E) continue;
+        const int t = sl / a.K;
+        const int p = s_off[ee] + __popcll(s_mask[ee] & ((1ull << t) - 1ull));
+        a.perm[p] = sl;
+        a.inv[sl] = p;
+        if (a.tap_perm) a.tap_perm[p] = sl;
+    }
     if (a.units) {
         // units: every expert's slots cut into runs of at most kUnitTokens, in expert order
         const int per = (a.E + blockDim.x - 1) / blockDim.x;

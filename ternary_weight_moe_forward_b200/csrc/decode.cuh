@@ -32,8 +32,8 @@
 //              ring allows.  Two issuing warps and large copies: one thread
 //              issuing one copy per item does not keep HBM busy;
 //   warp 2     builds each unit's B operand (the unit's activations in MMA
-//              fragment order) in one of two buffers: stage 1 by four-row TMA
-//              gathers from the fragment-ordered copy of q_x; stage 2 (after
+//              fragment order, 128-byte swizzled) in one of two buffers: stage 1
+//              from the fragment-ordered copy of q_x by 16-byte loads; stage 2 (after
 //              griddepcontrol.wait) from the unit's rows of h, brought in by one
 //              bulk copy, requantised with the per-slot maxima, with each
 //              slot's scale and code sum;
@@ -79,6 +79,7 @@ struct DxArgs {
     const float *sx;       // [T] scale of q_x
     const int *sumx;       // [T] sum of q_x's codes
     const uint8_t *w_gu, *w_dn;   // MMA-tile layouts (codes and row scales per item)
+    const int8_t *qxp;     // [T][D] q_x rows in fragment order (frag_word_pos)
     const int *perm;       // [T*K] position -> slot (the routing kernel's permutation)
     const int2 *units;     // the units: {expert, first position | count << 16}
     const int *n_units;
@@ -119,7 +120,7 @@ struct DxSmem {
         side = hst + hst_bytes;
         bars = (side + kDxNB * (int)sizeof(DxSide) + 7) & ~7;
         const int n_bars = 2 * ngroups + 2 * kDxNB + 2;   // ring groups full/empty, B full/empty, h staged [2]
-        // + abort word, last gathered unit, copies into each h buffer; per ring group the copies issued into it
+        // + abort word, spare, copies into each h buffer; per ring group the copies issued into it
         tables = bars + 8 * n_bars + 16 + 4 * ngroups;
         const int S = T * K, units = E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;
         // t_perm [S]; t_sx, t_sumx [T]; misc [2]; units [units] (int2, 8-byte aligned)
@@ -209,7 +210,7 @@ __device__ __forceinline__ int dx_total(const int (&acc)[2][4][4], int nt, int i
 
 template <int STAGE>
 __global__ void __launch_bounds__(kDxThreads, 1)
-    decode_stage_kernel(const __grid_constant__ CUtensorMap qxp_map, DxArgs a)
+    decode_stage_kernel(DxArgs a)
 {
     extern __shared__ __align__(1024) uint8_t dsm[];
     const DxSmem L(STAGE, a.D, a.F, a.T, a.K, a.E, a.nslot);
@@ -228,9 +229,8 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const uint32_t b_bfull = b_rempty + 8 * L.ngroups, b_bempty = b_bfull + 8 * kDxNB;
     const uint32_t b_hst = b_bempty + 8 * kDxNB;   // [2]: the two h staging buffers
     volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * L.ngroups + 2 * kDxNB + 2);
-    volatile int *s_last_tma = (volatile int *)(abort + 1);   // stage 1: the last unit whose B operand was gathered
-    volatile int *s_hgen = s_last_tma + 1;                    // stage 2: [2] copies issued into each h buffer
-    volatile int *s_gen = s_last_tma + 3;                     // [ngroups] copies issued into each ring group
+    volatile int *s_hgen = (volatile int *)(abort + 2);   // stage 2: [2] copies issued into each h buffer
+    volatile int *s_gen = (volatile int *)(abort + 4);    // [ngroups] copies issued into each ring group
     // routing tables (loaded from the routing kernel's outputs)
     int *t_perm = (int *)(dsm + L.tables);
     float *t_sx = (float *)(t_perm + S);
@@ -251,7 +251,6 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         mbar_init(b_hst, 1);
         mbar_init(b_hst + 8, 1);
         *abort = 0u;
-        *s_last_tma = -1;
         s_hgen[0] = s_hgen[1] = 0;
         for (int g = 0; g < L.ngroups; g++) s_gen[g] = 0;
         fence_barrier_init();
@@ -270,13 +269,14 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     // (stage 2 reads only the routing outputs here; h and the maxima of the
     // gate/up kernel are read after its own wait, by the B-operand warp)
     const int n_units_g = __ldcg(a.n_units);
+    const int unit_cap = a.E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;   // the units array's length
     for (int q = threadIdx.x; q < S; q += blockDim.x) t_perm[q] = __ldcg(a.perm + q);
     if (STAGE == 1)
         for (int t = threadIdx.x; t < T; t += blockDim.x) {
             t_sx[t] = __ldcg(a.sx + t);
             t_sumx[t] = __ldcg(a.sumx + t);
         }
-    for (int u = threadIdx.x; u < n_units_g; u += blockDim.x) t_unit[u] = __ldcg(a.units + u);
+    for (int u = threadIdx.x; u < unit_cap; u += blockDim.x) t_unit[u] = __ldcg(a.units + u);   // not waiting for n_units
     if (threadIdx.x == 0) t_misc[1] = n_units_g;
     __syncthreads();
     const int n_units = t_misc[1];
@@ -357,20 +357,24 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     sd->e = e;
                     sd->cnt = cnt;
                 }
+                // the unit's q_x rows (fragment order) by 16-byte asynchronous copies,
+                // all in flight at once, into the B operand's swizzled positions
+                // (dx_b_chunk); the padding tokens of the last n-tile are left as they
+                // are (their outputs are never read)
+                const int cpr = D / 16;   // 16-byte chunks per row
+                for (int idx = lane; idx < cnt * cpr; idx += 32) {
+                    const int n = idx / cpr, cc = idx - n * cpr;
+                    const int t = t_perm[p0 + n] / K;
+                    const uint32_t dst = smem_addr(bb + (n >> 3) * KB1 * 1024 + (cc >> 3) * 1024 + dx_b_chunk(n & 7, cc & 7));
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                                 "l"(reinterpret_cast<const uint4 *>(a.qxp + (size_t)t * D) + cc)
+                                 : "memory");
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
                 __threadfence_block();
                 __syncwarp();
-                if (lane == 0) mbar_expect_tx(b_bfull + 8 * b, (uint32_t)(ntiles * KB1 * 1024));
-                __syncwarp();
-                // gathers: (n-tile, block, half) -> tokens 8nt + 4h .. +3 of the unit
-                for (int gi = lane; gi < ntiles * KB1 * 2; gi += 32) {
-                    const int nt = gi / (2 * KB1), kb = (gi >> 1) % KB1, hh = gi & 1;
-                    int tk[4];
-#pragma unroll
-                    for (int r = 0; r < 4; r++) tk[r] = t_perm[p0 + min(8 * nt + 4 * hh + r, cnt - 1)] / K;
-                    tma_gather4(smem_addr(bb + nt * KB1 * 1024 + kb * 1024 + hh * 512), &qxp_map, kb * 128, tk[0],
-                                tk[1], tk[2], tk[3], b_bfull + 8 * b);
-                }
-                if (lane == 0) *s_last_tma = uo;
+                if (lane == 0) mbar_arrive(b_bfull + 8 * b);
                 continue;
             }
             // stage 2: the unit's rows of h (consecutive positions) came in one copy
@@ -395,14 +399,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             if (!__all_sync(FULL, mbar_wait(b_hst + 8 * (uo & 1), (uo >> 1) & 1, abort, a.flag, a.wait_ns))) break;
             if (uo + 1 < n_uo) stage_h(uo + 1);
             const uint8_t *hsrc = hst + (size_t)(uo & 1) * (L.hst_bytes / 2);
-            for (int n = 0; n < ntiles * 8; n++) {
+            for (int n = 0; n < cnt; n++) {   // (padding tokens: left as they are, never read)
                 const int nt = n >> 3, g = n & 7;
                 uint8_t *dst = bb + nt * KB2 * 1024;   // token g's row: 128 bytes at g * 128 of each block
-                if (n >= cnt) {   // padding token of the last n-tile: zeros
-                    for (int w = lane; w < KB2 * 32; w += 32)
-                        reinterpret_cast<uint32_t *>(dst + (w >> 5) * 1024 + g * 128)[w & 31] = 0u;
-                    continue;
-                }
                 const int pos = p0 + n, slot = t_perm[pos];
                 const float4 *hr = reinterpret_cast<const float4 *>(hsrc + (size_t)n * F * 4);
                 const float amax = __shfl_sync(FULL, am_lane, n);
@@ -562,21 +561,15 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 
     // ---------------- common exit: no copy may still be landing when the CTA exits.
     // After a normal run every copy has been waited for; after a failed wait the
-    // last copy into every ring group and the last B-operand (or h) copy are
-    // waited for (bounded).
+    // last copy into every ring group and into each h staging buffer is waited
+    // for (bounded).
     __syncthreads();
     if (threadIdx.x == 0 && *abort) {
-        const int lt = *s_last_tma;
         for (int g = 0; g < L.ngroups; g++) {
             const int gen = s_gen[g];   // copies issued into group g; the last one has phase gen - 1
             if (!gen) continue;
             const uint64_t t0 = global_ns();
             while (!mbar_test(b_rfull + 8 * g, (gen - 1) & 1) && global_ns() - t0 < a.wait_ns) {
-            }
-        }
-        if (STAGE == 1 && lt >= 0) {
-            const uint64_t t0 = global_ns();
-            while (!mbar_test(b_bfull + 8 * (lt % kDxNB), (lt / kDxNB) & 1) && global_ns() - t0 < a.wait_ns) {
             }
         }
         for (int hb = 0; STAGE == 2 && hb < 2; hb++) {

@@ -39,6 +39,7 @@ struct maple_moe_s {
     int num_sms;
     int device;
     int optin;                     // shared memory a block may opt in to
+    int route_clusters;            // decode batches route with route_cluster_kernel: clusters that fit at once (0: not used)
     char *base;                    // one device allocation: weights + workspace
     // weights
     uint8_t *w_mma_gu, *w_mma_dn;  // decode layout (MMA tiles), null when not built
@@ -64,7 +65,7 @@ struct maple_moe_s {
     float *ye;                     // decode kernel: expert outputs [64*K][D]
     int16_t *acc_hi;               // tensor-core path: down accumulators >> 1 [S][D]
     uint32_t *acc_lo;              // and their lowest bits [S][D/32]
-    CUtensorMap map_qx, map_qh, map_qxp;   // TMA maps of the activation operands
+    CUtensorMap map_qx, map_qh;   // TMA maps of the tensor-core path's activation operands
     // counters (zero between calls)
     unsigned *tg_cnt, *glob_cnt;
     unsigned *dx_clear;            // decode kernels: |h| maxima [64*K] (zeroed by the routing kernel)
@@ -201,6 +202,18 @@ static route_fn pick_route_n(int ni)
 }
 static route_fn pick_route(int D, int E) { return E <= 256 ? pick_route_n<8>(D / 256) : pick_route_n<32>(D / 256); }
 
+// the cluster routing kernel for d_model = 256 * ni (E <= 256): d_model <= 2048
+static route_fn pick_route_cluster(int D)
+{
+    switch (D / 256) {
+    case 1: return route_cluster_kernel<1, 8>;
+    case 2: return route_cluster_kernel<2, 8>;
+    case 4: return route_cluster_kernel<4, 8>;
+    case 8: return route_cluster_kernel<8, 8>;
+    default: return nullptr;
+    }
+}
+
 template <int NPER>
 static route_fn pick_qtopk_n(int ni)
 {
@@ -216,6 +229,61 @@ static route_fn pick_qtopk_n(int ni)
 static route_fn pick_qtopk(int D, int E) { return E <= 256 ? pick_qtopk_n<8>(D / 256) : pick_qtopk_n<32>(D / 256); }
 
 static bool pow2_upto(int v, int hi) { return v >= 1 && v <= hi && (v & (v - 1)) == 0; }
+
+// launch configuration of the cluster routing kernel: one cluster of E/16 CTAs
+// per group of 8 tokens
+static void route_cluster_config(maple_moe_t h, int T, int gt, cudaStream_t st, cudaLaunchConfig_t *lc,
+                                 cudaLaunchAttribute (&attr)[2], bool pdl)
+{
+    memset(lc, 0, sizeof *lc);
+    lc->gridDim = dim3(h->E / kRcExperts, (T + gt - 1) / gt);
+    lc->blockDim = dim3(kRcExperts * 32);
+    lc->dynamicSmemBytes = route_cluster_smem_bytes(h->D, h->E, gt);
+    lc->stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = h->E / kRcExperts;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc->attrs = attr;
+    lc->numAttrs = pdl ? 2 : 1;
+}
+
+// How many clusters of the cluster routing kernel run at once on this device
+// and shape (E <= 256, a multiple of 16; K <= 8; d_model <= 2048), 0 when it cannot run.
+// Sets the kernel's attributes; clears any CUDA error it causes.
+static int cluster_route_ok(maple_moe_t h)
+{
+    if (h->E > kRcMaxExperts || h->E % kRcExperts || h->K > 8) return 0;   // (choices buffer: 8 per token)
+    route_fn k = pick_route_cluster(h->D);
+    if (!k) return 0;
+    const int csize = h->E / kRcExperts;
+    if (cudaFuncSetAttribute((const void *)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)route_cluster_smem_bytes(h->D, h->E, kRcMaxGroup)) != cudaSuccess ||
+        (csize > 8 &&
+         cudaFuncSetAttribute((const void *)k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t lc;
+    cudaLaunchAttribute attr[2];
+    route_cluster_config(h, kRcMaxGroup, kRcMaxGroup, nullptr, &lc, attr, false);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void *)k, &lc) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+// tokens per cluster for a batch of T: 8 when its 8-token groups all fit at
+// once, else 0 (route_kernel serves the batch: 16-token groups measured slower)
+static int route_cluster_group(maple_moe_t h, int T)
+{
+    const int nc = h->route_clusters;
+    return nc >= 1 && (T + kRouteTokens - 1) / kRouteTokens <= nc ? kRouteTokens : 0;
+}
 
 static int check_shape(const maple_moe_config *c)
 {
@@ -386,9 +454,9 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
         repack_tc_dn_kernel<<<grid_for(E * D * F / 16, 256, cap), 256, 0, st>>>(w->w_down, h->E, h->D, h->F,
                                                                                (uint32_t *)h->w_tc_dn);
     }
-    bool maps_ok = make_act_map(&h->map_qxp, h->qxp, T64, D, 1, true) == MAPLE_OK;   // 128-byte swizzle: see dx_b_chunk
+    bool maps_ok = true;
     if (build_tc)
-        maps_ok = maps_ok && make_act_map(&h->map_qx, h->qx, Tm, D, 1, true) == MAPLE_OK &&
+        maps_ok = make_act_map(&h->map_qx, h->qx, Tm, D, 1, true) == MAPLE_OK &&
                   make_act_map(&h->map_qh, h->qh, S, F, kTcMaxN, true) == MAPLE_OK;
     // allow every kernel the largest dynamic shared memory the device offers, so
     // that handles of different shapes never cap one another's launches
@@ -398,6 +466,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
                              (const void *)decode_stage_kernel<2>};
     bool smem_ok = true;
     for (const void *k : kernels) smem_ok = allow_max_smem(k, h->device) && smem_ok;
+    h->route_clusters = cluster_route_ok(h);
     if (!maps_ok || !smem_ok || cudaGetLastError() != cudaSuccess) {
         cudaFree(h->base);
         cudaFreeHost(h->flag_host);
@@ -484,9 +553,16 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
         a.clear = clear;
         a.n_clear = n_clear;
     }
-    if (small) {
+    const int gt = small ? route_cluster_group(h, T) : 0;
+    if (gt) {
         // as a programmatic dependent (the layer stack) the kernel loads its router
         // rows while the previous layer finishes, then waits for it
+        a.group_tokens = gt;
+        cudaLaunchConfig_t lc;
+        cudaLaunchAttribute attr[2];
+        route_cluster_config(h, T, gt, st, &lc, attr, pdl);
+        if (cudaLaunchKernelEx(&lc, pick_route_cluster(h->D), a) != cudaSuccess) return MAPLE_ERR_CUDA;
+    } else if (small) {
         cudaLaunchConfig_t lc;
         memset(&lc, 0, sizeof lc);
         lc.gridDim = dim3(h->E / kRouteExperts, (T + kRouteTokens - 1) / kRouteTokens);
@@ -552,6 +628,7 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     d.F = h->F;
     d.sx = h->sx;
     d.sumx = h->sumx;
+    d.qxp = h->qxp;
     d.perm = h->perm;
     d.units = h->units;
     d.n_units = h->n_units;
@@ -588,11 +665,11 @@ static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, c
     lc.numAttrs = 1;
     d.nslot = n1;
     lc.dynamicSmemBytes = DxSmem(1, h->D, h->F, T, h->K, h->E, n1).total;
-    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<1>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<1>, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 2, st);
     d.nslot = n2;
     lc.dynamicSmemBytes = DxSmem(2, h->D, h->F, T, h->K, h->E, n2).total;
-    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<2>, h->map_qxp, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&lc, decode_stage_kernel<2>, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     lc.gridDim = dim3((unsigned)((T * (h->D / 4) + 255) / 256));
     lc.blockDim = dim3(256);
     lc.dynamicSmemBytes = 0;

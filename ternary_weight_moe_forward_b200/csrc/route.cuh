@@ -2,6 +2,8 @@
 // kept logits, and the token -> expert permutation.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "layout.cuh"
 
@@ -43,6 +45,7 @@ struct RouteArgs {
     int2 *units;   // optional (with fuse_permute): the decode kernels' units, {expert, first | count << 16}
     int *n_units;
     unsigned *flag;
+    int group_tokens;   // route_cluster_kernel: tokens per cluster (8 or 16)
 };
 
 constexpr int kUnitTokens = 16;   // slots of a decode unit (two 8-token MMA n-tiles)
@@ -194,7 +197,7 @@ __device__ __forceinline__ int rank_key_index(unsigned long long k) { return (in
 // Top-k of one row of E logits (one warp); lane k < K ends with the k-th
 // choice (my_e) and its softmax weight (my_w).  A NaN logit ranks last and
 // raises the flag.
-template <int NPER>
+template <int NPER, bool SMEM = false>
 __device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
 {
     const int lane = threadIdx.x & 31;
@@ -205,7 +208,7 @@ __device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsig
         int e = lane + 32 * j;
         float v = -INFINITY;
         if (e < E) {
-            v = __ldcg(row + e);
+            v = SMEM ? row[e] : __ldcg(row + e);
             if (isnan(v)) {
                 nan_seen = true;
                 v = -INFINITY;
@@ -248,13 +251,15 @@ __device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsig
     my_w = __fdiv_rn(ek, S);
 }
 
-template <int NPER>
-__device__ void topk_token_warp(const RouteArgs &a, int t)
+// top-k of token t from its logits (global, or a row in shared memory), written
+// to the routing outputs; returns the lane's choice (lanes < K)
+template <int NPER, bool SMEM = false>
+__device__ int topk_token_warp(const RouteArgs &a, int t, const float *row = nullptr)
 {
     const int lane = threadIdx.x & 31;
     int my_e;
     float my_w;
-    topk_row_warp<NPER>(a.logits + (size_t)t * a.E, a.E, a.K, a.flag, my_e, my_w);
+    topk_row_warp<NPER, SMEM>(SMEM ? row : a.logits + (size_t)t * a.E, a.E, a.K, a.flag, my_e, my_w);
     if (lane < a.K) {
         const size_t o = (size_t)t * a.K + lane;
         a.topk_idx[o] = my_e;
@@ -262,6 +267,7 @@ __device__ void topk_token_warp(const RouteArgs &a, int t)
         if (a.out_idx) a.out_idx[o] = my_e;
         if (a.out_w) a.out_w[o] = my_w;
     }
+    return my_e;
 }
 
 // ---------------------------------------------------------------------------
@@ -324,6 +330,124 @@ __host__ __device__ inline size_t route_smem_bytes(int D)
     return xb > (size_t)kFusedMarkBytes ? xb : (size_t)kFusedMarkBytes;
 }
 
+// Stage the bf16 rows of tokens t0 .. t0+nt-1 in shared memory: from x by
+// asynchronous copies (all in flight at once), or, for the layer stack, as
+// bf16(RMSNorm(resid)) with one warp per token.  Ends with __syncthreads.
+template <int NI>
+__device__ __forceinline__ void route_stage_tokens(const RouteArgs &a, uint16_t *xs, int t0, int nt)
+{
+    const int warp = threadIdx.x >> 5;
+    if (a.resid) {
+        if (warp < nt) rmsnorm_token_warp(a.resid + (size_t)(t0 + warp) * a.D, a.D, xs + (size_t)warp * a.D);
+    } else {
+        const int n16 = nt * (a.D / 8);
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D);
+        for (int idx = threadIdx.x; idx < n16; idx += blockDim.x)
+            cp_async16(reinterpret_cast<uint4 *>(xs) + idx, src + idx, true);
+        cp_async_commit();
+        cp_async_wait<0>();
+    }
+    __syncthreads();
+}
+
+// Logits of one expert (this warp's router row, in registers as w0/w1) for the
+// nt staged tokens, two tokens at a time (two independent fmaf chains, each in
+// the pinned order); store(t, logit) is called by lane 0 for t = 0 .. nt-1.
+template <int NI, class Store>
+__device__ __forceinline__ void route_logits_warp(const RouteArgs &a, const float4 (&w0)[NI], const float4 (&w1)[NI],
+                                                  const uint16_t *xs, int nt, float bias_e, Store store)
+{
+    const int lane = threadIdx.x & 31;
+    for (int tt = 0; tt < nt; tt += 2) {
+        const int tb = min(tt + 1, nt - 1);   // an odd last token is computed twice, stored once
+        float acc0 = 0.0f, acc1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NI; i++) {
+            const uint4 xa = *reinterpret_cast<const uint4 *>(xs + (size_t)tt * a.D + 256 * i + 8 * lane);
+            const uint4 xb = *reinterpret_cast<const uint4 *>(xs + (size_t)tb * a.D + 256 * i + 8 * lane);
+            const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+            const float wv[8] = {w0[i].x, w0[i].y, w0[i].z, w0[i].w, w1[i].x, w1[i].y, w1[i].z, w1[i].w};
+#pragma unroll
+            for (int m = 0; m < 8; m++) {
+                const uint32_t ba = (m & 1) ? (wa[m >> 1] >> 16) : (wa[m >> 1] & 0xffffu);
+                const uint32_t bb = (m & 1) ? (wb[m >> 1] >> 16) : (wb[m >> 1] & 0xffffu);
+                acc0 = __fmaf_rn(bf16_bits_to_f32(ba), wv[m], acc0);
+                acc1 = __fmaf_rn(bf16_bits_to_f32(bb), wv[m], acc1);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {   // the pairwise tree of warp_tree_sum, two rows at once
+            acc0 = __fadd_rn(acc0, __shfl_xor_sync(FULL, acc0, o));
+            acc1 = __fadd_rn(acc1, __shfl_xor_sync(FULL, acc1, o));
+        }
+        if (a.bias) {
+            acc0 = __fadd_rn(acc0, bias_e);
+            acc1 = __fadd_rn(acc1, bias_e);
+        }
+        if (lane == 0) {
+            store(tt, acc0);
+            if (tb != tt) store(tb, acc1);
+        }
+    }
+}
+
+// The permutation of all T*K slots (T <= 64) in one CTA, from every token's
+// choices (expert_of(slot)).  Per expert the mask of the tokens that chose it
+// (a token's choices are distinct); a slot's position is its expert's offset
+// plus the number of earlier tokens in the mask, so every step is a constant
+// number of shared-memory operations per thread (no loop over tokens).  Also
+// writes the decode kernels' units.  s_mask: E words of shared memory.
+template <class ExpertOf>
+__device__ void route_fused_permutation(const RouteArgs &a, unsigned long long *s_mask, int *s_warp, ExpertOf expert_of)
+{
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_off[kMaxExperts + 1];
+    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_mask[ee] = 0ull;
+    __syncthreads();
+    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
+        const int ee = expert_of(sl);
+        if (ee < 0 || ee >= a.E) {
+            set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
+            continue;
+        }
+        atomicOr(s_mask + ee, 1ull << (sl / a.K));
+    }
+    __syncthreads();
+    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_cnt[ee] = __popcll(s_mask[ee]);
+    __syncthreads();
+    scan_experts(s_cnt, s_off, a.E, a.active, a.n_active, s_warp);
+    for (int ee = threadIdx.x; ee <= a.E; ee += blockDim.x) {
+        a.offsets[ee] = s_off[ee];
+        if (a.tap_offsets) a.tap_offsets[ee] = s_off[ee];
+        if (ee < a.E) {
+            a.counts[ee] = s_cnt[ee];
+            if (a.out_counts) a.out_counts[ee] = s_cnt[ee];
+        }
+    }
+    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
+        const int ee = expert_of(sl);
+        if (ee < 0 || ee >= a.E) continue;
+        const int t = sl / a.K;
+        const int p = s_off[ee] + __popcll(s_mask[ee] & ((1ull << t) - 1ull));
+        a.perm[p] = sl;
+        a.inv[sl] = p;
+        if (a.tap_perm) a.tap_perm[p] = sl;
+    }
+    if (a.units) {
+        // units: every expert's slots cut into runs of at most kUnitTokens, in expert order
+        const int per = (a.E + blockDim.x - 1) / blockDim.x;
+        const int lo = min(a.E, (int)threadIdx.x * per), hi = min(a.E, lo + per);
+        int nu = 0;
+        for (int ee = lo; ee < hi; ee++) nu += (s_cnt[ee] + kUnitTokens - 1) / kUnitTokens;
+        int total;
+        int u = block_excl_scan(nu, s_warp, &total);
+        for (int ee = lo; ee < hi; ee++)
+            for (int u0 = 0; u0 < s_cnt[ee]; u0 += kUnitTokens)
+                a.units[u++] = make_int2(ee, (s_off[ee] + u0) | (min(kUnitTokens, s_cnt[ee] - u0) << 16));
+        if (threadIdx.x == 0) *a.n_units = total;
+    }
+}
+
 template <int NI, int NPER>
 __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
 {
@@ -354,63 +478,14 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (a.clear && eb == 0 && tg == 0)
         for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
-    if (a.resid) {
-        // the layer stack: each warp normalises one of the CTA's tokens
-        if (warp < nt) rmsnorm_token_warp(a.resid + (size_t)(t0 + warp) * a.D, a.D, xs + (size_t)warp * a.D);
-    } else {
-        // stage the token rows (nt * D/8 16-byte units, at most NI per thread) with
-        // asynchronous copies, all in flight at once
-        const int n16 = nt * (a.D / 8);
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)t0 * a.D);
-#pragma unroll
-        for (int i = 0; i < NI; i++) {
-            const int idx = threadIdx.x + 256 * i;
-            if (idx < n16) cp_async16(reinterpret_cast<uint4 *>(xs) + idx, src + idx, true);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-    }
-    __syncthreads();
+    route_stage_tokens<NI>(a, xs, t0, nt);
 
     if (eb == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
 
-    // two tokens at a time: two independent fmaf chains, each in the pinned order
-    const float bias_e = a.bias ? a.bias[e] : 0.0f;
-    for (int tt = 0; tt < nt; tt += 2) {
-        const int tb = min(tt + 1, nt - 1);   // an odd last token is computed twice, stored once
-        float acc0 = 0.0f, acc1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < NI; i++) {
-            const uint4 xa = *reinterpret_cast<const uint4 *>(xs + (size_t)tt * a.D + 256 * i + 8 * lane);
-            const uint4 xb = *reinterpret_cast<const uint4 *>(xs + (size_t)tb * a.D + 256 * i + 8 * lane);
-            const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
-            const float wv[8] = {w0[i].x, w0[i].y, w0[i].z, w0[i].w, w1[i].x, w1[i].y, w1[i].z, w1[i].w};
-#pragma unroll
-            for (int m = 0; m < 8; m++) {
-                const uint32_t ba = (m & 1) ? (wa[m >> 1] >> 16) : (wa[m >> 1] & 0xffffu);
-                const uint32_t bb = (m & 1) ? (wb[m >> 1] >> 16) : (wb[m >> 1] & 0xffffu);
-                acc0 = __fmaf_rn(bf16_bits_to_f32(ba), wv[m], acc0);
-                acc1 = __fmaf_rn(bf16_bits_to_f32(bb), wv[m], acc1);
-            }
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {   // the pairwise tree of warp_tree_sum, two rows at once
-            acc0 = __fadd_rn(acc0, __shfl_xor_sync(FULL, acc0, o));
-            acc1 = __fadd_rn(acc1, __shfl_xor_sync(FULL, acc1, o));
-        }
-        if (a.bias) {
-            acc0 = __fadd_rn(acc0, bias_e);
-            acc1 = __fadd_rn(acc1, bias_e);
-        }
-        if (lane == 0) {
-            a.logits[(size_t)(t0 + tt) * a.E + e] = acc0;
-            if (a.tap_logits) a.tap_logits[(size_t)(t0 + tt) * a.E + e] = acc0;
-            if (tb != tt) {
-                a.logits[(size_t)(t0 + tb) * a.E + e] = acc1;
-                if (a.tap_logits) a.tap_logits[(size_t)(t0 + tb) * a.E + e] = acc1;
-            }
-        }
-    }
+    route_logits_warp<NI>(a, w0, w1, xs, nt, a.bias ? a.bias[e] : 0.0f, [&](int t, float v) {
+        a.logits[(size_t)(t0 + t) * a.E + e] = v;
+        if (a.tap_logits) a.tap_logits[(size_t)(t0 + t) * a.E + e] = v;
+    });
 
     // ---- last CTA of this token group: top-k + softmax
     fence_gpu();
@@ -438,57 +513,100 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
     fence_gpu();
     if (threadIdx.x == 0) *a.glob_cnt = 0;
 
-    // T <= 64: per expert the mask of the tokens that chose it (a token's choices
-    // are distinct); a slot's position is its expert's offset plus the number of
-    // earlier tokens in the mask, so every step is a constant number of shared
-    // memory operations per thread (no loop over tokens)
-    unsigned long long *s_mask = reinterpret_cast<unsigned long long *>(rsm);   // [E], reuses the token rows
-    __shared__ int s_cnt[kMaxExperts];
-    __shared__ int s_off[kMaxExperts + 1];
-    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_mask[ee] = 0ull;
+    route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp,
+                            [&](int sl) { return __ldcg(a.topk_idx + sl); });
+}
+
+// ---------------------------------------------------------------------------
+// The routing kernel on thread-block clusters (T <= 64, E <= 256 and a
+// multiple of 16): one cluster of E/16 CTAs per group of 8 or 16 tokens (16
+// when 8-token groups would need more clusters than fit at once), 16 warps per
+// CTA, warp w of cluster rank r scoring expert 16r + w with the same
+// arithmetic in the same order as route_kernel.  Every warp writes its logits
+// straight into rank 0's shared memory (distributed shared memory); after the
+// cluster barrier rank 0 runs top-k for the group's tokens from there, so no
+// logit goes through global memory and no CTA waits on a counter.  With one
+// token group (T <= 8) rank 0 builds the permutation at once from its own
+// choices; with several, the last group to finish does (as in route_kernel).
+// Dynamic shared memory: route_cluster_smem_bytes(D, E, group_tokens).
+// ---------------------------------------------------------------------------
+constexpr int kRcExperts = 16;   // experts per CTA (one per warp)
+constexpr int kRcMaxExperts = 256;
+constexpr int kRcMaxGroup = 16;  // tokens per cluster at most (one top-k warp each)
+__host__ __device__ inline size_t route_cluster_rows_bytes(int D, int E, int gt)
+{
+    const size_t xb = (size_t)gt * D * 2, mb = (size_t)E * 8;   // token rows, later the experts' masks
+    return xb > mb ? xb : mb;
+}
+__host__ __device__ inline size_t route_cluster_smem_bytes(int D, int E, int gt)
+{
+    // + the group's logits [gt][E] and its choices [gt][8]
+    return route_cluster_rows_bytes(D, E, gt) + (size_t)gt * E * 4 + (size_t)gt * 8 * 4;
+}
+
+template <int NI, int NPER>
+__global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
+{
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(16) uint8_t rsm[];
+    uint16_t *xs = (uint16_t *)rsm;                                       // [nt][D] bf16
+    const int gt = a.group_tokens;
+    float *lg = (float *)(rsm + route_cluster_rows_bytes(a.D, a.E, gt));  // [gt][E] (rank 0)
+    int *ch = (int *)(lg + gt * a.E);                                     // [gt][K] (rank 0, one group)
+    __shared__ unsigned s_last;
+    __shared__ int s_warp[33];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tg = blockIdx.y, t0 = tg * gt;
+    const int nt = min(gt, a.T - t0);
+    const int e = rank * kRcExperts + warp;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    const float *wr = a.Wr + (size_t)e * a.D;
+    float4 w0[NI], w1[NI];
+#pragma unroll
+    for (int i = 0; i < NI; i++) {
+        w0[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane));
+        w1[i] = __ldg(reinterpret_cast<const float4 *>(wr + 256 * i + 8 * lane + 4));
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (a.clear && rank == 0 && tg == 0)
+        for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
+    route_stage_tokens<NI>(a, xs, t0, nt);
+    if (rank == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
+
+    float *lg0 = cluster.map_shared_rank(lg, 0);   // rank 0's logit rows
+    route_logits_warp<NI>(a, w0, w1, xs, nt, a.bias ? a.bias[e] : 0.0f, [&](int t, float v) {
+        lg0[t * a.E + e] = v;
+        if (a.tap_logits) a.tap_logits[(size_t)(t0 + t) * a.E + e] = v;
+    });
+    cluster.sync();   // every logit of the group is in rank 0's shared memory
+    if (rank != 0) return;
+
+    int my_e = 0;
+    if (warp < nt) my_e = topk_token_warp<NPER, true>(a, t0 + warp, lg + warp * a.E);
+    if (!a.fuse_permute) return;
+    if (gridDim.y == 1) {
+        // one token group: the choices are this CTA's own
+        if (warp < nt && lane < a.K) ch[warp * a.K + lane] = my_e;
+        __syncthreads();
+        route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp, [&](int sl) { return ch[sl]; });
+        return;
+    }
+    // several token groups: the last to finish builds the permutation
+    fence_gpu();
     __syncthreads();
-    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
-        const int ee = __ldcg(a.topk_idx + sl);
-        if (ee < 0 || ee >= a.E) {
-            set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
-            continue;
-        }
-        atomicOr(s_mask + ee, 1ull << (sl / a.K));
+    if (threadIdx.x == 0) {
+        unsigned prev = atomicAdd(a.glob_cnt, 1u);
+        s_last = (prev == gridDim.y - 1);
     }
     __syncthreads();
-    for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_cnt[ee] = __popcll(s_mask[ee]);
-    __syncthreads();
-    scan_experts(s_cnt, s_off, a.E, a.active, a.n_active, s_warp);
-    for (int ee = threadIdx.x; ee <= a.E; ee += blockDim.x) {
-        a.offsets[ee] = s_off[ee];
-        if (a.tap_offsets) a.tap_offsets[ee] = s_off[ee];
-        if (ee < a.E) {
-            a.counts[ee] = s_cnt[ee];
-            if (a.out_counts) a.out_counts[ee] = s_cnt[ee];
-        }
-    }
-    for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
-        const int ee = __ldcg(a.topk_idx + sl);
-        if (ee < 0 || ee >= a.E) continue;
-        const int t = sl / a.K;
-        const int p = s_off[ee] + __popcll(s_mask[ee] & ((1ull << t) - 1ull));
-        a.perm[p] = sl;
-        a.inv[sl] = p;
-        if (a.tap_perm) a.tap_perm[p] = sl;
-    }
-    if (a.units) {
-        // units: every expert's slots cut into runs of at most kUnitTokens, in expert order
-        const int per = (a.E + blockDim.x - 1) / blockDim.x;
-        const int lo = min(a.E, (int)threadIdx.x * per), hi = min(a.E, lo + per);
-        int nu = 0;
-        for (int ee = lo; ee < hi; ee++) nu += (s_cnt[ee] + kUnitTokens - 1) / kUnitTokens;
-        int total;
-        int u = block_excl_scan(nu, s_warp, &total);
-        for (int ee = lo; ee < hi; ee++)
-            for (int u0 = 0; u0 < s_cnt[ee]; u0 += kUnitTokens)
-                a.units[u++] = make_int2(ee, (s_off[ee] + u0) | (min(kUnitTokens, s_cnt[ee] - u0) << 16));
-        if (threadIdx.x == 0) *a.n_units = total;
-    }
+    if (!s_last) return;
+    fence_gpu();
+    if (threadIdx.x == 0) *a.glob_cnt = 0;
+    route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp,
+                            [&](int sl) { return __ldcg(a.topk_idx + sl); });
 }
 
 // ---------------------------------------------------------------------------

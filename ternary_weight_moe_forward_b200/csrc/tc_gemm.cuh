@@ -74,7 +74,7 @@ template <int MODE>
 struct TcCfg;
 template <>
 struct TcCfg<0> {
-    static constexpr int kCS = 8, kBS = 4, kAS = 2;   // stages of the code, activation and weight rings
+    static constexpr int kCS = 6, kBS = 4, kAS = 3;   // stages of the code, activation and weight rings
     static constexpr int kABytes = 2 * 128 * kTcBK;   // gate + up blocks
     static constexpr int kCodeBytes = 2 * 128 * 32;   // 8 words of 4 bytes per row
 };
@@ -95,7 +95,8 @@ struct TcSmem {
     static constexpr int kBars = kCodes + C::kCS * C::kCodeBytes;  // barriers, TMEM holder, abort word: 512 B
     static constexpr int kMeta = kBars + 512;                      // epilogue column metadata [2][2][128]
     static constexpr int kAmax = kMeta + 2 * 2 * kTcMaxN * 4;      // mode 0: per-slot absmax of h [128]
-    static constexpr int kTotal = kAmax + kTcMaxN * 4;
+    static constexpr int kTr = kAmax + kTcMaxN * 4;                 // mode 1: per epilogue warp a 32 x 32 int16 tile
+    static constexpr int kTotal = kTr + (MODE == 1 ? kTcEpiWarps * 2048 : 0);
     static constexpr int kNumBars = 2 * (C::kCS + C::kBS + C::kAS) + 5;
     static_assert(C::kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(8 * kNumBars + 8 <= 512, "barrier area");
@@ -584,22 +585,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         if (c0 + lane < n) atomicMax(s_amax + c0 + lane, __float_as_uint(m));
                     }
                 } else {
+                    // The warp's 32 channels x 32 slot columns, transposed through its
+                    // shared-memory tile (row = slot, 64 bytes of int16, 16-byte chunks
+                    // swizzled by (slot / 2) % 4 so that both sides are free of bank
+                    // conflicts), then written back per slot as four 16-byte stores of
+                    // acc >> 1 and one word of low bits (the column's ballot).
+                    uint8_t *tile = smem + L::kTr + ew * 2048;
+                    const int row0 = rb * 128 + q * 32;   // this warp's first channel
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
                         int dd[32];
                         tmem_ld32(tb + c0, dd);
                         tmem_wait_ld();
+                        uint32_t my_lo = 0;   // lane j: the low bits of column j
 #pragma unroll
                         for (int j = 0; j < 32; j++) {
-                            const int col = c0 + j;   // the same column in every lane
-                            if (col < n) {
-                                const int p = p0 + col;
-                                const int di = dd[j] >> 6;
-                                a.acc_hi[(size_t)p * a.D + row] = (int16_t)(di >> 1);
-                                const uint32_t lo = __ballot_sync(FULL, di & 1);
-                                if (lane == 0) a.acc_lo[(size_t)p * (a.D / 32) + (row >> 5)] = lo;
-                                if (a.tap0) a.tap0[(size_t)ms[col] * a.D + row] = di;
-                            }
+                            const int di = dd[j] >> 6;
+                            const int ck = (lane >> 3) ^ ((j >> 1) & 3);
+                            *reinterpret_cast<int16_t *>(tile + j * 64 + ck * 16 + (lane & 7) * 2) = (int16_t)(di >> 1);
+                            const uint32_t lo = __ballot_sync(FULL, di & 1);
+                            if (lane == j) my_lo = lo;
+                            if (a.tap0 && c0 + j < n) a.tap0[(size_t)ms[c0 + j] * a.D + row] = di;
                         }
+                        __syncwarp();
+                        if (c0 + lane < n) {
+                            const size_t p = (size_t)p0 + c0 + lane;
+                            uint4 *dst = reinterpret_cast<uint4 *>(a.acc_hi + p * a.D + row0);
+#pragma unroll
+                            for (int k = 0; k < 4; k++)
+                                dst[k] = *reinterpret_cast<const uint4 *>(tile + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4));
+                            a.acc_lo[p * (a.D / 32) + (row0 >> 5)] = my_lo;
+                        }
+                        __syncwarp();   // the tile is read before the next chunk overwrites it
                     }
                     (void)al0;
                 }
@@ -613,29 +629,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 __threadfence_block();
                 asm volatile("bar.sync 3, 256;" ::: "memory");
                 if (!dead) {
-                    for (int i = ew; i < n; i += kTcEpiWarps) {
-                        const int p = p0 + i, slot = ms[i];
-                        const float amax = __uint_as_float(s_amax[i]);
-                        const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-                        const float4 *hr = reinterpret_cast<const float4 *>(hs + (size_t)i * a.F);
-                        for (int c = lane; c < a.F / 4; c += 32) {
-                            const float4 hv = __ldcg(hr + c);
-                            int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-                            if (amax > 0.0f) {
-                                q0 = quant_code(hv.x, inv);
-                                q1 = quant_code(hv.y, inv);
-                                q2 = quant_code(hv.z, inv);
-                                q3 = quant_code(hv.w, inv);
+                    // two slots per round and 512 columns at a time, all eight of a
+                    // lane's loads in flight together
+                    for (int i = ew; i < n; i += 2 * kTcEpiWarps) {
+                        const int ib = i + kTcEpiWarps;   // the round's second slot (if any)
+                        const float am0 = __uint_as_float(s_amax[i]);
+                        const float am1 = ib < n ? __uint_as_float(s_amax[ib]) : 0.0f;
+                        const float inv0 = am0 > 0.0f ? __fdiv_rn(127.0f, am0) : 0.0f;
+                        const float inv1 = am1 > 0.0f ? __fdiv_rn(127.0f, am1) : 0.0f;
+                        for (int c0 = 0; c0 < a.F / 4; c0 += 128) {
+                            float4 hv[2][4];
+#pragma unroll
+                            for (int k = 0; k < 4; k++) {
+                                const int c = c0 + lane + 32 * k;   // d_ff need not be a multiple of 512
+                                hv[0][k] = hv[1][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                if (c < a.F / 4) {
+                                    hv[0][k] = __ldcg(reinterpret_cast<const float4 *>(hs + (size_t)i * a.F) + c);
+                                    if (ib < n) hv[1][k] = __ldcg(reinterpret_cast<const float4 *>(hs + (size_t)ib * a.F) + c);
+                                }
                             }
-                            const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
-                                                ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
-                            reinterpret_cast<uint32_t *>(a.qh + (size_t)p * a.F)[c] = pk;
-                            if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * a.F)[c] = pk;
+#pragma unroll
+                            for (int r = 0; r < 2; r++) {
+                                const int ii = r ? ib : i;
+                                if (ii >= n) break;
+                                const float am = r ? am1 : am0, inv = r ? inv1 : inv0;
+                                const int p = p0 + ii, slot = ms[ii];
+#pragma unroll
+                                for (int k = 0; k < 4; k++) {
+                                    const int c = c0 + lane + 32 * k;
+                                    if (c >= a.F / 4) break;
+                                    int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+                                    if (am > 0.0f) {
+                                        q0 = quant_code(hv[r][k].x, inv);
+                                        q1 = quant_code(hv[r][k].y, inv);
+                                        q2 = quant_code(hv[r][k].z, inv);
+                                        q3 = quant_code(hv[r][k].w, inv);
+                                    }
+                                    const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                                                        ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+                                    reinterpret_cast<uint32_t *>(a.qh + (size_t)p * a.F)[c] = pk;
+                                    if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)slot * a.F)[c] = pk;
+                                }
+                            }
                         }
                         if (lane == 0) {
-                            const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-                            a.sh[p] = sv;
-                            if (a.tap_sh) a.tap_sh[slot] = sv;
+#pragma unroll
+                            for (int r = 0; r < 2; r++) {
+                                const int ii = r ? ib : i;
+                                if (ii >= n) break;
+                                const float am = r ? am1 : am0;
+                                const float sv = am > 0.0f ? __fdiv_rn(am, 127.0f) : 0.0f;
+                                a.sh[p0 + ii] = sv;
+                                if (a.tap_sh) a.tap_sh[ms[ii]] = sv;
+                            }
                         }
                     }
                 }

@@ -60,18 +60,20 @@
 
 namespace maple {
 
-// Eight compute warps: each holds a ring slot only while its MMAs read it, so
-// that most of the ring's slots are always copies in flight.
-constexpr int kDxComputeWarps = 8;
+// Twelve compute warps, claiming the CTA's items one at a time: each holds a
+// ring slot only while its MMAs read it, so most of the ring's slots are
+// always copies in flight, and three warps per scheduler hide the latency of
+// the MMA chains and the SwiGLU epilogue.
+constexpr int kDxComputeWarps = 12;
 constexpr int kDxProducers = 2;                          // weight-stream warps
 constexpr int kDxBuilder = kDxProducers;                 // the B-operand warp
 constexpr int kDxCompute0 = kDxProducers + 1;            // first compute warp
-constexpr int kDxThreads = (kDxCompute0 + kDxComputeWarps) * 32;   // 352
+constexpr int kDxThreads = (kDxCompute0 + kDxComputeWarps) * 32;   // 480
 constexpr int kDxUnitTokens = kUnitTokens;               // tokens of a unit: two MMA n-tiles
 constexpr int kDxNB = 2;                                 // B-operand buffers
 constexpr int kDxMaxF = 1024;                            // largest d_ff (the shape limit)
 // Items per ring group (one copy per run of an expert's items): few large copies
-// stream faster than many small ones.  Divides kDxComputeWarps.
+// stream faster than many small ones.
 constexpr int kDxCopyItems = 4;
 
 struct DxArgs {
@@ -93,7 +95,7 @@ struct DxArgs {
     unsigned *flag;
     uint64_t wait_ns;
     int stall;             // test hook: stage 2 waits for `never` to become 1
-    int nslot;             // ring slots (a multiple of kDxComputeWarps)
+    int nslot;             // ring slots (a multiple of kDxCopyItems * kDxProducers)
 };
 
 struct DxSide {                 // per-slot data of a unit, next to its B operand
@@ -120,8 +122,9 @@ struct DxSmem {
         side = hst + hst_bytes;
         bars = (side + kDxNB * (int)sizeof(DxSide) + 7) & ~7;
         const int n_bars = 2 * ngroups + 2 * kDxNB + 2;   // ring groups full/empty, B full/empty, h staged [2]
-        // + abort word, spare, copies into each h buffer; per ring group the copies issued into it
-        tables = bars + 8 * n_bars + 16 + 4 * ngroups;
+        // + abort word, item claim counter, copies into each h buffer; per ring group the
+        // copies issued into it; per ring slot the items consumed from it
+        tables = bars + 8 * n_bars + 16 + 4 * ngroups + 4 * nslot;
         const int S = T * K, units = E + (S + kDxUnitTokens - 1) / kDxUnitTokens + 1;
         // t_perm [S]; t_sx, t_sumx [T]; misc [2]; units [units] (int2, 8-byte aligned)
         int tb = S * 4 + 2 * T * 4 + 2 * 4;
@@ -131,19 +134,21 @@ struct DxSmem {
 };
 
 // Ring slots of a decode kernel within a shared-memory budget (0: it does not
-// fit).  Item j of a CTA's range goes to compute warp j % 8 and to slot
-// j % nslot; with nslot a multiple of 8, items j and j + nslot (the next use of
-// the slot) belong to the same warp (and with nslot a multiple of
-// kDxCopyItems * kDxProducers, every ring group to one producer warp).  Otherwise the warp of item j + nslot could
+// fit): a multiple of kDxCopyItems * kDxProducers, so that every ring group
+// belongs to one producer warp.  Item j of a CTA's range goes to slot
+// j % nslot, round j / nslot; the warp that claims it first waits until item
+// j - nslot has been consumed (a per-slot count), so that when it tests the
+// group's full barrier the barrier is in round j / nslot or later.  (A parity
+// wait accepts the current phase and the one before it: without that count a
+// warp could take the previous round's phase as complete.)  Otherwise the warp of item j + nslot could
 // test the slot group's full barrier while item j's copy is still landing, see
 // the barrier in the phase before and take it as complete (a parity wait
 // accepts the current phase and the one before it).
 __host__ inline int dx_ring_slots(int stage, int D, int F, int T, int K, int E, size_t budget)
 {
     if (F > D || D % F) return 0;
-    constexpr int step = kDxComputeWarps > kDxCopyItems * kDxProducers ? kDxComputeWarps : kDxCopyItems * kDxProducers;
-    static_assert(step % kDxComputeWarps == 0 && step % (kDxCopyItems * kDxProducers) == 0, "ring step");
-    for (int n = 32; n >= step; n -= step)
+    constexpr int step = kDxCopyItems * kDxProducers;
+    for (int n = 32; n >= 2 * step; n -= step)
         if ((size_t)DxSmem(stage, D, F, T, K, E, n).total <= budget) return n;
     return 0;
 }
@@ -229,8 +234,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     const uint32_t b_bfull = b_rempty + 8 * L.ngroups, b_bempty = b_bfull + 8 * kDxNB;
     const uint32_t b_hst = b_bempty + 8 * kDxNB;   // [2]: the two h staging buffers
     volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * L.ngroups + 2 * kDxNB + 2);
+    int *s_claim = (int *)(abort + 1);                    // the CTA's next unclaimed item (relative)
     volatile int *s_hgen = (volatile int *)(abort + 2);   // stage 2: [2] copies issued into each h buffer
     volatile int *s_gen = (volatile int *)(abort + 4);    // [ngroups] copies issued into each ring group
+    volatile int *s_done = s_gen + L.ngroups;             // [nslot] items consumed from each ring slot
     // routing tables (loaded from the routing kernel's outputs)
     int *t_perm = (int *)(dsm + L.tables);
     float *t_sx = (float *)(t_perm + S);
@@ -251,8 +258,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
         mbar_init(b_hst, 1);
         mbar_init(b_hst + 8, 1);
         *abort = 0u;
+        *s_claim = 0;
         s_hgen[0] = s_hgen[1] = 0;
         for (int g = 0; g < L.ngroups; g++) s_gen[g] = 0;
+        for (int q = 0; q < a.nslot; q++) s_done[q] = 0;
         fence_barrier_init();
     }
     if (STAGE == 1) {
@@ -444,10 +453,16 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             if (lane == 0) mbar_arrive(b_bfull + 8 * b);
         }
     } else {
-        // ---------------- compute warp cw: items j0 + cw, j0 + cw + 8, ...
-        const int cw = warp - kDxCompute0;
+        // ---------------- compute warps: claim the range's items one at a time (in
+        // order), visiting every unit's B operand in turn
         const int g = lane >> 2, tig = lane & 3;
         bool ok = true;
+        auto claim = [&]() {
+            int c = 0;
+            if (lane == 0) c = atomicAdd(s_claim, 1);
+            return j0 + __shfl_sync(FULL, c, 0);
+        };
+        int j = claim();
         for (int uo = 0; uo < n_uo && ok; uo++) {
             const int b = uo % kDxNB;
             if (!mbar_wait(b_bfull + 8 * b, (uo / kDxNB) & 1, abort, a.flag, a.wait_ns)) break;
@@ -456,12 +471,22 @@ __global__ void __launch_bounds__(kDxThreads, 1)
             const int ntiles = (cnt + 7) / 8;
             const uint32_t bbase = smem_addr(bbuf + (size_t)b * L.b_bytes);
             const uint32_t bb_lo = bbase + dx_b_chunk(g, 2 * tig), bb_hi = bbase + dx_b_chunk(g, 2 * tig + 1);
-            // this unit's items within the range, and this warp's first among them
-            const int ja = max(j0, u * GS), jb = min(j1, (u + 1) * GS);
-            int j = ja + ((cw - (ja - j0)) % kDxComputeWarps + kDxComputeWarps) % kDxComputeWarps;
-            for (; j < jb; j += kDxComputeWarps) {
-                const int rel = j - j0, slot = rel % a.nslot, sg = slot / kDxCopyItems;
-                if (!mbar_wait(b_rfull + 8 * sg, (rel / a.nslot) & 1, abort, a.flag, a.wait_ns)) {
+            const int jb = min(j1, (u + 1) * GS);   // this unit's items end here
+            for (; j < jb; j = claim()) {
+                const int rel = j - j0, slot = rel % a.nslot, sg = slot / kDxCopyItems, round = rel / a.nslot;
+                // item j - nslot consumed first: the group's barrier is then in this round or later
+                if (lane == 0) {
+                    const uint64_t t0 = global_ns();
+                    while (s_done[slot] < round) {
+                        if (*abort || global_ns() - t0 > a.wait_ns) {
+                            *abort = 1u;
+                            set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
+                            break;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (!mbar_wait(b_rfull + 8 * sg, round & 1, abort, a.flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -480,7 +505,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         dx_tile<1>(aa, bb_lo, bb_hi, KB1, KB1 * 1024, acc);
                     // the codes and scales have been read: hand the item back to the weight stream
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(b_rempty + 8 * sg);
+                    if (lane == 0) {
+                        mbar_arrive(b_rempty + 8 * sg);
+                        s_done[slot] = round + 1;
+                    }
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++) {
                         if (nt >= ntiles) break;
@@ -528,7 +556,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                         const float ad0 = alpha_s[16 * d + g], ad1 = alpha_s[16 * d + 8 + g];
                         if (d == S2 - 1) {   // the item's codes and scales are read: hand it back
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(b_rempty + 8 * sg);
+                            if (lane == 0) {
+                                mbar_arrive(b_rempty + 8 * sg);
+                                s_done[slot] = round + 1;
+                            }
                         }
 #pragma unroll
                         for (int nt = 0; nt < 2; nt++) {

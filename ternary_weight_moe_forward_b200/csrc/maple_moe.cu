@@ -47,6 +47,7 @@ struct maple_moe_s {
     float *alpha_gate, *alpha_up, *alpha_down, *router_w, *router_bias;
     // workspace: routing
     int8_t *qx, *qxp;              // q_x rows; the decode kernel's fragment-ordered copy (T <= 64)
+    int8_t *xpos;                  // tensor-core path: the q_x row of every position (position order)
     const int8_t *zrow;
     float *sx;
     int *sumx;
@@ -65,7 +66,7 @@ struct maple_moe_s {
     float *ye;                     // decode kernel: expert outputs [64*K][D]
     int16_t *acc_hi;               // tensor-core path: down accumulators >> 1 [S][D]
     uint32_t *acc_lo;              // and their lowest bits [S][D/32]
-    CUtensorMap map_qx, map_qh;   // TMA maps of the tensor-core path's activation operands
+    CUtensorMap map_xpos, map_qh;   // TMA maps of the tensor-core path's activation operands
     // counters (zero between calls)
     unsigned *tg_cnt, *glob_cnt;
     unsigned *dx_clear;            // decode kernels: |h| maxima [64*K] (zeroed by the routing kernel)
@@ -362,6 +363,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     const size_t o_hs = build_tc ? ar.take((size_t)h->num_sms * kTcMaxN * F * 4) : 0;
     const size_t o_h = build_dec ? ar.take(S64 * F * 4) : 0;
     const size_t o_qh = build_tc ? ar.take(S * F) : 0, o_sh = build_tc ? ar.take(S * 4) : 0;
+    const size_t o_xpos = build_tc ? ar.take(S * D) : 0;
     const size_t o_ye = build_dec ? ar.take(S64 * D * 4) : 0;
     const size_t o_ahi = build_tc ? ar.take(S * D * 2) : 0, o_alo = build_tc ? ar.take(S * D / 8) : 0;
     const size_t o_ctr = ar.take(0);   // counters: zero between calls
@@ -415,6 +417,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->hscratch = build_tc ? (float *)(b + o_hs) : nullptr;
     h->h = build_dec ? (float *)(b + o_h) : nullptr;
     h->qh = build_tc ? (int8_t *)(b + o_qh) : nullptr;
+    h->xpos = build_tc ? (int8_t *)(b + o_xpos) : nullptr;
     h->sh = build_tc ? (float *)(b + o_sh) : nullptr;
     h->ye = build_dec ? (float *)(b + o_ye) : nullptr;
     h->acc_hi = build_tc ? (int16_t *)(b + o_ahi) : nullptr;
@@ -456,7 +459,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     }
     bool maps_ok = true;
     if (build_tc)
-        maps_ok = make_act_map(&h->map_qx, h->qx, Tm, D, 1, true) == MAPLE_OK &&
+        maps_ok = make_act_map(&h->map_xpos, h->xpos, S, D, kTcMaxN, true) == MAPLE_OK &&
                   make_act_map(&h->map_qh, h->qh, S, F, kTcMaxN, true) == MAPLE_OK;
     // allow every kernel the largest dynamic shared memory the device offers, so
     // that handles of different shapes never cap one another's launches
@@ -731,7 +734,11 @@ static int run_experts_tc(maple_moe_t h, int T, float *y, const float *resid, co
     g.tap1 = taps ? taps->acc_up : nullptr;
     g.tap_qh = taps ? taps->q_h : nullptr;
     g.tap_sh = taps ? taps->s_h : nullptr;
-    tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_qx, g);
+    // the q_x row of every position, so that the gate/up GEMM loads its activation
+    // tiles with one 2-D copy per stage
+    gather_rows_kernel<<<grid_for((int64_t)T * h->K, 8, h->num_sms * 16), 256, 0, st>>>(h->qx, h->perm, T * h->K,
+                                                                                       h->K, h->D, h->xpos);
+    tc_gemm_kernel<0><<<h->num_sms, kTcThreads, TcSmem<0>::kTotal, st>>>(h->map_xpos, g);
     stage_event(h, 2, st);
     g.codes = h->w_tc_dn;
     g.alpha0 = h->alpha_down;

@@ -49,6 +49,9 @@ struct RouteArgs {
 };
 
 constexpr int kUnitTokens = 16;   // slots of a decode unit (two 8-token MMA n-tiles)
+constexpr int kRcExperts = 16;    // route_cluster_kernel: experts per CTA (one per warp)
+constexpr int kRcMaxExperts = 256;
+constexpr int kRcMaxGroup = 16;   // route_cluster_kernel: tokens per cluster at most (one top-k warp each)
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pred)
 {
@@ -517,6 +520,81 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
                             [&](int sl) { return __ldcg(a.topk_idx + sl); });
 }
 
+// The same permutation for T <= 8 (K <= 8, E <= 256) by one warp, from the
+// choices in shared memory (ch[slot]): per expert an 8-bit token mask,
+// counts, offsets and the active list by warp scans, so no block-wide barrier
+// is taken.  Every active expert is one unit (at most 8 slots).
+__device__ void route_perm_warp(const RouteArgs &a, const int *ch)
+{
+    __shared__ uint32_t s_m8[kRcMaxExperts / 4];   // 8-bit token masks, four experts a word
+    __shared__ int s_off[kRcMaxExperts];
+    const int lane = threadIdx.x & 31;
+    const int S = a.T * a.K, per = (a.E + 31) / 32, e0 = lane * per;
+    for (int w = lane; w < a.E / 4; w += 32) s_m8[w] = 0u;
+    __syncwarp();
+    for (int sl = lane; sl < S; sl += 32) {
+        const int e = ch[sl];
+        if (e < 0 || e >= a.E) {
+            set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
+            continue;
+        }
+        atomicOr(s_m8 + e / 4, 1u << (8 * (e & 3) + sl / a.K));
+    }
+    __syncwarp();
+    int cnt[8], sum = 0, nz = 0;   // this lane's experts e0 .. e0+per-1 (per <= 8)
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int e = e0 + i;
+        cnt[i] = (i < per && e < a.E) ? __popc((s_m8[e / 4] >> (8 * (e & 3))) & 0xffu) : 0;
+        sum += cnt[i];
+        nz += cnt[i] > 0;
+    }
+    int off = sum, act = nz;   // inclusive warp scans, made exclusive below
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(FULL, off, o), w = __shfl_up_sync(FULL, act, o);
+        if (lane >= o) {
+            off += v;
+            act += w;
+        }
+    }
+    const int total = __shfl_sync(FULL, off, 31), n_act = __shfl_sync(FULL, act, 31);
+    off -= sum;
+    act -= nz;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int e = e0 + i;
+        if (i >= per || e >= a.E) break;
+        s_off[e] = off;
+        a.offsets[e] = off;
+        a.counts[e] = cnt[i];
+        if (a.tap_offsets) a.tap_offsets[e] = off;
+        if (a.out_counts) a.out_counts[e] = cnt[i];
+        if (cnt[i]) {
+            a.active[act] = e;
+            if (a.units) a.units[act] = make_int2(e, off | (cnt[i] << 16));
+            act++;
+        }
+        off += cnt[i];
+    }
+    if (lane == 0) {
+        a.offsets[a.E] = total;
+        if (a.tap_offsets) a.tap_offsets[a.E] = total;
+        *a.n_active = n_act;
+        if (a.units) *a.n_units = n_act;
+    }
+    __syncwarp();
+    for (int sl = lane; sl < S; sl += 32) {
+        const int e = ch[sl];
+        if (e < 0 || e >= a.E) continue;
+        const int t = sl / a.K;
+        const int p = s_off[e] + __popc((s_m8[e / 4] >> (8 * (e & 3))) & ((1u << t) - 1u));
+        a.perm[p] = sl;
+        a.inv[sl] = p;
+        if (a.tap_perm) a.tap_perm[p] = sl;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // The routing kernel on thread-block clusters (T <= 64, E <= 256 and a
 // multiple of 16): one cluster of E/16 CTAs per group of 8 or 16 tokens (16
@@ -530,9 +608,6 @@ __global__ void __launch_bounds__(256, 2) route_kernel(RouteArgs a)
 // choices; with several, the last group to finish does (as in route_kernel).
 // Dynamic shared memory: route_cluster_smem_bytes(D, E, group_tokens).
 // ---------------------------------------------------------------------------
-constexpr int kRcExperts = 16;   // experts per CTA (one per warp)
-constexpr int kRcMaxExperts = 256;
-constexpr int kRcMaxGroup = 16;  // tokens per cluster at most (one top-k warp each)
 __host__ __device__ inline size_t route_cluster_rows_bytes(int D, int E, int gt)
 {
     const size_t xb = (size_t)gt * D * 2, mb = (size_t)E * 8;   // token rows, later the experts' masks
@@ -574,7 +649,6 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
     if (a.clear && rank == 0 && tg == 0)
         for (int i = threadIdx.x; i < a.n_clear; i += blockDim.x) a.clear[i] = 0u;
     route_stage_tokens<NI>(a, xs, t0, nt);
-    if (rank == 0 && warp < nt) quantize_token_warp<NI>(a, t0 + warp, xs + (size_t)warp * a.D);
 
     float *lg0 = cluster.map_shared_rank(lg, 0);   // rank 0's logit rows
     route_logits_warp<NI>(a, w0, w1, xs, nt, a.bias ? a.bias[e] : 0.0f, [&](int t, float v) {
@@ -584,14 +658,22 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
     cluster.sync();   // every logit of the group is in rank 0's shared memory
     if (rank != 0) return;
 
+    // top-k by warps 0 .. nt-1 while warps 16-nt .. 15 quantise the tokens
+    // (q_x feeds the expert kernels, not the router)
     int my_e = 0;
     if (warp < nt) my_e = topk_token_warp<NPER, true>(a, t0 + warp, lg + warp * a.E);
+    if (warp >= kRcExperts - nt) quantize_token_warp<NI>(a, t0 + warp - (kRcExperts - nt), xs + (size_t)(warp - (kRcExperts - nt)) * a.D);
     if (!a.fuse_permute) return;
     if (gridDim.y == 1) {
-        // one token group: the choices are this CTA's own
+        // one token group: the choices are this CTA's own; one warp builds the
+        // permutation (T <= 8: no block-wide barrier)
         if (warp < nt && lane < a.K) ch[warp * a.K + lane] = my_e;
         __syncthreads();
-        route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp, [&](int sl) { return ch[sl]; });
+        if (a.T <= 8) {
+            if (warp == 0) route_perm_warp(a, ch);
+        } else {
+            route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp, [&](int sl) { return ch[sl]; });
+        }
         return;
     }
     // several token groups: the last to finish builds the permutation

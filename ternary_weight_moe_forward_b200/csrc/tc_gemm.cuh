@@ -14,7 +14,7 @@
 // epilogue shifts it back (exact).
 //
 // Warp roles (20 warps): warp 0 issues the bulk copies of the 2-bit codes,
-// warp 2 the activation loads, warp 1 the MMAs (and owns the TMEM
+// warp 2 the activation loads (lane 0), warp 1 the MMAs (and owns the TMEM
 // allocation), warps 4..11 run the epilogue (TMEM lane quarter = warp % 4,
 // two warps per quarter splitting the columns), warps 12..19 expand the codes
 // into int8 tiles.  Three rings of K stages with their own lifetimes: the
@@ -26,8 +26,10 @@
 //
 // Mode 0 (gate/up): A = gate rows and up rows of one 128-row block (two MMAs
 // per K step, gate and up accumulators 128 columns apart), B = the q_x rows of
-// the slots' tokens, fetched straight from q_x by TMA gather (four rows per
-// copy).  A CTA takes whole pieces (all F/128 row blocks of one piece in a
+// the piece's positions (gather_rows_kernel has laid out the q_x row of every
+// position in position order), one 2-D TMA copy per stage.  (Fetching them
+// straight from q_x by four-row TMA gathers, 32 per stage, kept the loading
+// warp issuing for most of the kernel.)  A CTA takes whole pieces (all F/128 row blocks of one piece in a
 // row, pieces dealt out in a snake order over the size-sorted list), so that
 // it holds every h value of its slots: the epilogue writes h = SiLU(g) * u
 // (fp32) to a per-CTA scratch area that stays in L2 and keeps each slot's
@@ -177,18 +179,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
-}
-// four rows (y0..y3) of 128 bytes starting at column x, gathered by the TMA
-// unit from a row-major int8 matrix (tensor map box: 128 bytes x 1 row, 128-byte
-// swizzle) into 512 consecutive bytes of shared memory
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, int x, int y0, int y1, int y2, int y3,
-                                            uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
 }
 // 2-D tiled TMA load (box given by the tensor map) into 128B-swizzled shared memory
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
@@ -417,39 +407,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
         }
     } else if (warp == 2) {
-        // ---------------- activation tiles, up to BS stages ahead: mode 0 gathers the
-        // rows of the piece's tokens from q_x (four per copy, one copy per lane),
-        // mode 1 loads 128 consecutive q_h rows
+        // ---------------- activation tiles, up to BS stages ahead: 128 consecutive
+        // position rows (mode 0: the q_x row of every position, mode 1: q_h), one
+        // 2-D copy per stage
         uint32_t it = 0;
         bool ok = true;
-        int cur = -1;
-        int y[4] = {0, 0, 0, 0};   // mode 0: tokens of rows 4*lane .. 4*lane+3 of the current piece
         int pc, rb;
         for (int u = 0; ok && tc_tile<MODE>(u, R, n_pc, pc, rb); u++) {
             const int4 P = a.pieces[pc];
-            const int npad = (P.z + 15) & ~15;
-            if (MODE == 0 && pc != cur) {
-                cur = pc;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const int row = min(4 * lane + i, P.z - 1);   // padding rows repeat the last slot's token
-                    y[i] = __ldg(a.perm + P.y + row) / a.K;
-                }
-            }
             for (int ks = 0; ks < KS; ks++, it++) {
                 const int s = it % BS;
                 if (lane == 0) ok = mbar_wait(b_act_empty + 8 * s, ((it / BS) & 1) ^ 1, abort, a.flag, a.wait_ns);
                 ok = __shfl_sync(FULL, ok, 0);
                 if (!ok) break;
                 const uint32_t full = b_act_full + 8 * s;
-                const uint32_t bdst = smem_addr(smem + L::kB + s * L::kBBytes);
                 if (lane == 0) {
-                    mbar_expect_tx(full, MODE == 0 ? npad * kTcBK : L::kBBytes);
-                    if (MODE == 1) tma_load_2d(bdst, &act_map, ks * kTcBK, P.y, full);
+                    mbar_expect_tx(full, L::kBBytes);
+                    tma_load_2d(smem_addr(smem + L::kB + s * L::kBBytes), &act_map, ks * kTcBK, P.y, full);
                 }
                 __syncwarp();
-                if (MODE == 0 && 4 * lane < npad)
-                    tma_gather4(bdst + 4 * lane * kTcBK, &act_map, ks * kTcBK, y[0], y[1], y[2], y[3], full);
             }
         }
         if (!ok && lane == 0) {
@@ -732,6 +708,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// The q_x row of every position (xpos[p] = q_x[perm[p] / K]), so that the gate/up
+// GEMM loads 128 positions' rows with one 2-D copy; one warp per row.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const int8_t *qx, const int *perm, int S, int K, int D,
+                                                          int8_t *xpos)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5, nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t p = w0; p < S; p += nw) {
+        const int t = __ldg(perm + p) / K;
+        const uint4 *src = reinterpret_cast<const uint4 *>(qx + (size_t)t * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(xpos + (size_t)p * D);
+        for (int c = lane; c < D / 16; c += 32) dst[c] = __ldg(src + c);
     }
 }
 

@@ -147,24 +147,30 @@ def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
 
 
 # ---------------------------------------------------------------------------- measured traffic
-PROFILE_T64 = os.path.join(ROOT, "profiles", "decode_experts_kernel__decode_T64.md")
+PROFILE_T64 = os.path.join(ROOT, "profiles", "decode_stage_kernel__decode_T64.md")
+# the sources of the dominant kernel (decode_stage_kernel): its own file and
+# the helpers and layout it is built from
+TRAFFIC_SOURCES = ("common.cuh", "decode.cuh", "layout.cuh")
 
 
 def csrc_digest() -> str:
-    """sha256 over the CUDA sources (file names and contents, sorted)."""
-    import glob
+    """sha256 over the dominant kernel's CUDA sources (file names and contents,
+    in TRAFFIC_SOURCES order; a missing file counts as empty)."""
     import hashlib
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "ternary_weight_moe_forward_b200", "csrc", "*"))):
-        h.update(os.path.basename(p).encode())
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for name in TRAFFIC_SOURCES:
+        h.update(name.encode())
+        try:
+            with open(os.path.join(ROOT, "ternary_weight_moe_forward_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        except OSError:
+            pass
     return h.hexdigest()
 
 
 def measured_traffic():
-    """DRAM bytes (read + write) of one T=64 launch of decode_experts_kernel from
-    the committed ncu summary, or None when the sources changed since."""
+    """DRAM bytes (read + write) of one T=64 launch of decode_stage_kernel<1>
+    from the committed ncu summary, or None when its sources changed since."""
     try:
         with open(PROFILE_T64) as f:
             txt = f.read()

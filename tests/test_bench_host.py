@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _fake_tree(tmp_path, text):
     csrc = tmp_path / "ternary_weight_moe_forward_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "a.cuh").write_text(text)
+    (csrc / "decode.cuh").write_text(text)
     return tmp_path
 
 
@@ -23,7 +23,7 @@ def test_digest_follows_the_sources(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "ROOT", str(root))
     d0 = bench.csrc_digest()
     assert d0 == bench.csrc_digest()
-    (root / "ternary_weight_moe_forward_b200" / "csrc" / "a.cuh").write_text("int y;\n")
+    (root / "ternary_weight_moe_forward_b200" / "csrc" / "decode.cuh").write_text("int y;\n")
     assert bench.csrc_digest() != d0
 
 

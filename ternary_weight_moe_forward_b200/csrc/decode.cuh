@@ -207,6 +207,35 @@ __device__ __forceinline__ void dx_tile(uint32_t a_addr, uint32_t b_lo, uint32_t
 // distinct banks.  Byte offset of chunk c of token g within a block:
 __device__ __forceinline__ uint32_t dx_b_chunk(int g, int c) { return (uint32_t)(g * 128 + ((c ^ g) << 4)); }
 
+// Four 16-row tiles (a_addr + d * tile_stride) against one n-tile at once: the
+// four tiles' accumulator chains interleave, instead of four short chains one
+// after another.  acc[d][q][i] as in dx_tile.
+__device__ __forceinline__ void dx_tile4(uint32_t a_addr, int tile_stride, uint32_t b_lo, uint32_t b_hi, int nkb,
+                                         int (&acc)[4][4][4])
+{
+#pragma unroll
+    for (int d = 0; d < 4; d++)
+#pragma unroll
+        for (int q = 0; q < 4; q++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) acc[d][q][i] = 0;
+#pragma unroll 1
+    for (int kb = 0; kb < nkb; kb++) {
+        const uint4 b0 = lds128(b_lo + kb * 1024);
+        const uint4 b1 = lds128(b_hi + kb * 1024);
+        const uint32_t bq[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int d = 0; d < 4; d++) {
+            const uint4 w = lds128(a_addr + d * tile_stride + kb * 512);
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint32_t m = 0x03030303u << (2 * q);
+                mma_u8s8(acc[d][q], w.x & m, w.y & m, w.z & m, w.w & m, bq[2 * q], bq[2 * q + 1]);
+            }
+        }
+    }
+}
+
 // the exact row total of register i: acc_0 + acc_1/4 + acc_2/16 + acc_3/64
 __device__ __forceinline__ int dx_total(const int (&acc)[2][4][4], int nt, int i)
 {
@@ -546,6 +575,47 @@ __global__ void __launch_bounds__(kDxThreads, 1)
                     }
                 } else {
                     // ---- down item `it`: tiles S2*it .. S2*it + S2-1, channels 16*S2*it ..
+                    if (S2 == 4 && ntiles == 1) {
+                        // the common decode shape (d_ff = d_model / 4, at most 8 tokens):
+                        // the four tiles' chains together
+                        int acc4[4][4][4];
+                        dx_tile4(aa, KB2 * 512, bb_lo, bb_hi, KB2, acc4);
+                        float ad[4][2];   // this lane's channel scales, read before the slot is handed back
+#pragma unroll
+                        for (int d = 0; d < 4; d++) {
+                            ad[d][0] = alpha_s[16 * d + g];
+                            ad[d][1] = alpha_s[16 * d + 8 + g];
+                        }
+                        __syncwarp();
+                        if (lane == 0) {   // the item's codes and scales are read: hand it back
+                            mbar_arrive(b_rempty + 8 * sg);
+                            s_done[slot] = round + 1;
+                        }
+#pragma unroll
+                        for (int d = 0; d < 4; d++) {
+                            const int ch0 = 16 * (4 * it + d) + g;
+                            const float ad0 = ad[d][0], ad1 = ad[d][1];
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; h2++) {
+                                const int n = 2 * tig + h2;
+                                if (n < cnt) {
+                                    const int pos = sd->pos[n];
+                                    const int d0 = acc4[d][0][h2] + (acc4[d][1][h2] >> 2) + (acc4[d][2][h2] >> 4) +
+                                                   (acc4[d][3][h2] >> 6) - sd->sum[n];
+                                    const int d1 = acc4[d][0][2 + h2] + (acc4[d][1][2 + h2] >> 2) +
+                                                   (acc4[d][2][2 + h2] >> 4) + (acc4[d][3][2 + h2] >> 6) - sd->sum[n];
+                                    a.ye[(size_t)pos * D + ch0] = __fmul_rn((float)d0, __fmul_rn(ad0, sd->s[n]));
+                                    a.ye[(size_t)pos * D + ch0 + 8] = __fmul_rn((float)d1, __fmul_rn(ad1, sd->s[n]));
+                                    if (a.tap_acc_down) {
+                                        const int slot_t = t_perm[pos];
+                                        a.tap_acc_down[(size_t)slot_t * D + ch0] = d0;
+                                        a.tap_acc_down[(size_t)slot_t * D + ch0 + 8] = d1;
+                                    }
+                                }
+                            }
+                        }
+                        continue;
+                    }
                     for (int d = 0; d < S2; d++) {
                         const int dt = S2 * it + d;
                         if (ntiles == 2)

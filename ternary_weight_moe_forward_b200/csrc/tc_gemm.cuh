@@ -32,10 +32,10 @@
 // warp issuing for most of the kernel.)  A CTA takes whole pieces (all F/128 row blocks of one piece in a
 // row, pieces dealt out in a snake order over the size-sorted list), so that
 // it holds every h value of its slots: the epilogue writes h = SiLU(g) * u
-// (fp32) to a per-CTA scratch area that stays in L2 and keeps each slot's
-// running absmax in shared memory; after the piece's last row block the
-// epilogue warps requantise the slots (int8 absmax codes q_h, scale s_h),
-// so no fp32 h leaves the chip.
+// (fp32) to a per-CTA scratch area that stays in L2; after the piece's last
+// row block the epilogue warps requantise the slots, a slot's row at a time
+// in registers (its |h| maximum by a warp reduction, then the int8 absmax
+// codes q_h and the scale s_h), so no fp32 h leaves the chip.
 // Mode 1 (down): A = 128 output channels of the down matrix, B = q_h rows
 // (consecutive slot positions, a plain 2-D TMA load); tiles are dealt out
 // round robin.  The epilogue stores the exact int32 accumulators, which need
@@ -96,8 +96,7 @@ struct TcSmem {
     static constexpr int kCodes = kB + C::kBS * kBBytes;           // [kCS] 2-bit codes
     static constexpr int kBars = kCodes + C::kCS * C::kCodeBytes;  // barriers, TMEM holder, abort word: 512 B
     static constexpr int kMeta = kBars + 512;                      // epilogue column metadata [2][2][128]
-    static constexpr int kAmax = kMeta + 2 * 2 * kTcMaxN * 4;      // mode 0: per-slot absmax of h [128]
-    static constexpr int kTr = kAmax + kTcMaxN * 4;                 // mode 1: per epilogue warp a 32 x 32 int16 tile
+    static constexpr int kTr = kMeta + 2 * 2 * kTcMaxN * 4;        // mode 1: per epilogue warp a 32 x 32 int16 tile
     static constexpr int kTotal = kTr + (MODE == 1 ? kTcEpiWarps * 2048 : 0);
     static constexpr int kNumBars = 2 * (C::kCS + C::kBS + C::kAS) + 5;
     static_assert(C::kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
@@ -276,26 +275,6 @@ __device__ __forceinline__ uint4 expand_word(uint32_t w)
     return make_uint4((w << 6) & 0xC0C0C0C0u, (w << 4) & 0xC0C0C0C0u, (w << 2) & 0xC0C0C0C0u, w & 0xC0C0C0C0u);
 }
 
-// Column maxima of a warp's 32 x 32 block (lane = row, v[j] = column j, values
-// >= 0): after the five exchange levels lane l holds the maximum of column l.
-// At the level with distance o a lane keeps the half of its columns selected by
-// its bit o and sends the other half to lane l ^ o.
-__device__ __forceinline__ float warp_column_max(float (&v)[32])
-{
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
-        const bool upper = lane & o;
-#pragma unroll
-        for (int j = 0; j < n / 2; j++) {
-            const float send = upper ? v[j] : v[j + n / 2];
-            const float keep = upper ? v[j + n / 2] : v[j];
-            v[j] = fmaxf(keep, __shfl_xor_sync(FULL, send, o));
-        }
-    }
-    return v[0];
-}
-
 // ---------------------------------------------------------------------------
 // The CTA's u-th tile: piece (index into the size-sorted list) and row block;
 // false once the CTA has no more.  Mode 0 deals out whole pieces: the j-th
@@ -332,7 +311,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     }
     int *meta_slot = (int *)(smem + L::kMeta);                      // [2][kTcMaxN]
     float *meta_scale = (float *)(smem + L::kMeta + 2 * kTcMaxN * 4);
-    unsigned *s_amax = (unsigned *)(smem + L::kAmax);               // mode 0: [kTcMaxN] |h| maxima (float bits)
     uint64_t *bars = (uint64_t *)(smem + L::kBars);
     // bars: codes_full[CS], codes_empty[CS], act_full[BS], act_empty[BS], w_full[AS], w_empty[AS],
     // acc_full[2], acc_empty[2], drain
@@ -366,7 +344,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         *abort = 0u;
         fence_barrier_init();
     }
-    if (MODE == 0 && threadIdx.x < kTcMaxN) s_amax[threadIdx.x] = 0u;
     if (warp == 1) tmem_alloc(smem_addr(tmem_holder), 512);
     tc_fence_before();
     __syncthreads();
@@ -532,8 +509,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             if (!dead) {
                 tc_fence_after();
                 if (MODE == 0) {
+                    // h = SiLU(g) * u to the scratch; the slots' |h| maxima are taken
+                    // when the piece is requantised (each slot's row is then in registers)
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
-                        float v[32];
                         int g[16], u[16];   // sixteen columns at a time (register budget)
 #pragma unroll
                         for (int j = 0; j < 32; j++) {
@@ -543,22 +521,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                 tmem_ld16(tb + 128 + c0 + j, u);
                                 tmem_wait_ld();
                             }
-                            v[j] = 0.0f;
                             if (col < n) {
                                 const float sxt = mf[col];
                                 const int gi = g[j & 15] >> 6, ui = u[j & 15] >> 6;
                                 const float gv = __fmul_rn((float)gi, __fmul_rn(al0, sxt));
                                 const float uv = __fmul_rn((float)ui, __fmul_rn(al1, sxt));
-                                const float hv = swiglu(gv, uv);
-                                hs[(size_t)col * a.F + row] = hv;
-                                v[j] = fabsf(hv);
+                                hs[(size_t)col * a.F + row] = swiglu(gv, uv);
                                 if (a.tap0) a.tap0[(size_t)ms[col] * a.F + row] = gi;
                                 if (a.tap1) a.tap1[(size_t)ms[col] * a.F + row] = ui;
                             }
                         }
-                        // |h| maximum of each column over this warp's 32 rows, then over the CTA
-                        const float m = warp_column_max(v);
-                        if (c0 + lane < n) atomicMax(s_amax + c0 + lane, __float_as_uint(m));
                     }
                 } else {
                     // The warp's 32 channels x 32 slot columns, transposed through its
@@ -601,20 +573,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
             }
             if (MODE == 0 && rb == R - 1) {
                 // the piece's last row block: requantise its slots (h from the scratch
-                // area, read past L1; the absmax from shared memory)
+                // area, read past L1)
                 __threadfence_block();
                 asm volatile("bar.sync 3, 256;" ::: "memory");
                 if (!dead) {
                     // two slots per round and 512 columns at a time, all eight of a
-                    // lane's loads in flight together
+                    // lane's loads in flight together: first each slot's |h| maximum
+                    // (over the lane's values, then the warp), then the codes (for
+                    // d_ff <= 512 from the same registers, else from a second pass)
                     for (int i = ew; i < n; i += 2 * kTcEpiWarps) {
                         const int ib = i + kTcEpiWarps;   // the round's second slot (if any)
-                        const float am0 = __uint_as_float(s_amax[i]);
-                        const float am1 = ib < n ? __uint_as_float(s_amax[ib]) : 0.0f;
-                        const float inv0 = am0 > 0.0f ? __fdiv_rn(127.0f, am0) : 0.0f;
-                        const float inv1 = am1 > 0.0f ? __fdiv_rn(127.0f, am1) : 0.0f;
-                        for (int c0 = 0; c0 < a.F / 4; c0 += 128) {
-                            float4 hv[2][4];
+                        float4 hv[2][4];
+                        float am[2] = {0.0f, 0.0f};
+                        auto load = [&](int c0) {
 #pragma unroll
                             for (int k = 0; k < 4; k++) {
                                 const int c = c0 + lane + 32 * k;   // d_ff need not be a multiple of 512
@@ -624,18 +595,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                     if (ib < n) hv[1][k] = __ldcg(reinterpret_cast<const float4 *>(hs + (size_t)ib * a.F) + c);
                                 }
                             }
+                        };
+                        for (int c0 = 0; c0 < a.F / 4; c0 += 128) {
+                            load(c0);
+#pragma unroll
+                            for (int r = 0; r < 2; r++)
+#pragma unroll
+                                for (int k = 0; k < 4; k++)
+                                    am[r] = fmaxf(fmaxf(am[r], fmaxf(fabsf(hv[r][k].x), fabsf(hv[r][k].y))),
+                                                  fmaxf(fabsf(hv[r][k].z), fabsf(hv[r][k].w)));
+                        }
+#pragma unroll
+                        for (int o = 16; o >= 1; o >>= 1) {
+                            am[0] = fmaxf(am[0], __shfl_xor_sync(FULL, am[0], o));
+                            am[1] = fmaxf(am[1], __shfl_xor_sync(FULL, am[1], o));
+                        }
+                        const float inv0 = am[0] > 0.0f ? __fdiv_rn(127.0f, am[0]) : 0.0f;
+                        const float inv1 = am[1] > 0.0f ? __fdiv_rn(127.0f, am[1]) : 0.0f;
+                        for (int c0 = 0; c0 < a.F / 4; c0 += 128) {
+                            if (a.F / 4 > 128) load(c0);   // the registers hold only the last 512 columns
 #pragma unroll
                             for (int r = 0; r < 2; r++) {
                                 const int ii = r ? ib : i;
                                 if (ii >= n) break;
-                                const float am = r ? am1 : am0, inv = r ? inv1 : inv0;
+                                const float amx = am[r], inv = r ? inv1 : inv0;
                                 const int p = p0 + ii, slot = ms[ii];
 #pragma unroll
                                 for (int k = 0; k < 4; k++) {
                                     const int c = c0 + lane + 32 * k;
                                     if (c >= a.F / 4) break;
                                     int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-                                    if (am > 0.0f) {
+                                    if (amx > 0.0f) {
                                         q0 = quant_code(hv[r][k].x, inv);
                                         q1 = quant_code(hv[r][k].y, inv);
                                         q2 = quant_code(hv[r][k].z, inv);
@@ -653,16 +643,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             for (int r = 0; r < 2; r++) {
                                 const int ii = r ? ib : i;
                                 if (ii >= n) break;
-                                const float am = r ? am1 : am0;
-                                const float sv = am > 0.0f ? __fdiv_rn(am, 127.0f) : 0.0f;
+                                const float sv = am[r] > 0.0f ? __fdiv_rn(am[r], 127.0f) : 0.0f;
                                 a.sh[p0 + ii] = sv;
                                 if (a.tap_sh) a.tap_sh[ms[ii]] = sv;
                             }
                         }
                     }
                 }
-                asm volatile("bar.sync 3, 256;" ::: "memory");   // every read of the maxima and the scratch is done
-                if (ew < 4) s_amax[ew * 32 + lane] = 0u;       // (ordered before the next piece's maxima by bar 2)
+                asm volatile("bar.sync 3, 256;" ::: "memory");   // every read of the scratch is done
             }
             tcount++;
         }

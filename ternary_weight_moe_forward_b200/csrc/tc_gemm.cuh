@@ -96,8 +96,7 @@ struct TcSmem {
     static constexpr int kCodes = kB + C::kBS * kBBytes;           // [kCS] 2-bit codes
     static constexpr int kBars = kCodes + C::kCS * C::kCodeBytes;  // barriers, TMEM holder, abort word: 512 B
     static constexpr int kMeta = kBars + 512;                      // epilogue column metadata [2][2][128]
-    static constexpr int kTr = kMeta + 2 * 2 * kTcMaxN * 4;        // mode 1: per epilogue warp a 32 x 32 int16 tile
-    static constexpr int kTotal = kTr + (MODE == 1 ? kTcEpiWarps * 2048 : 0);
+    static constexpr int kTotal = kMeta + 2 * 2 * kTcMaxN * 4;
     static constexpr int kNumBars = 2 * (C::kCS + C::kBS + C::kAS) + 5;
     static_assert(C::kABytes % 1024 == 0 && kBBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(8 * kNumBars + 8 <= 512, "barrier area");
@@ -511,34 +510,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (MODE == 0) {
                     // h = SiLU(g) * u to the scratch; the slots' |h| maxima are taken
                     // when the piece is requantised (each slot's row is then in registers)
+                    // Sixteen columns at a time (register budget): the sixteen values are
+                    // computed with no branch between them, so their dependency chains
+                    // interleave, and stored afterwards (columns past the piece's end hold
+                    // no slot: computed, never stored).
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
-                        int g[16], u[16];   // sixteen columns at a time (register budget)
 #pragma unroll
-                        for (int j = 0; j < 32; j++) {
-                            const int col = c0 + j;
-                            if ((j & 15) == 0) {
-                                tmem_ld16(tb + c0 + j, g);
-                                tmem_ld16(tb + 128 + c0 + j, u);
-                                tmem_wait_ld();
+                        for (int jj = 0; jj < 32; jj += 16) {
+                            const int cb = c0 + jj;
+                            if (cb >= n) break;
+                            int g[16], u[16];
+                            tmem_ld16(tb + cb, g);
+                            tmem_ld16(tb + 128 + cb, u);
+                            tmem_wait_ld();
+                            float hv[16];
+#pragma unroll
+                            for (int j = 0; j < 16; j++) {
+                                const float sxt = mf[cb + j];
+                                const float gv = __fmul_rn((float)(g[j] >> 6), __fmul_rn(al0, sxt));
+                                const float uv = __fmul_rn((float)(u[j] >> 6), __fmul_rn(al1, sxt));
+                                hv[j] = swiglu(gv, uv);
                             }
-                            if (col < n) {
-                                const float sxt = mf[col];
-                                const int gi = g[j & 15] >> 6, ui = u[j & 15] >> 6;
-                                const float gv = __fmul_rn((float)gi, __fmul_rn(al0, sxt));
-                                const float uv = __fmul_rn((float)ui, __fmul_rn(al1, sxt));
-                                hs[(size_t)col * a.F + row] = swiglu(gv, uv);
-                                if (a.tap0) a.tap0[(size_t)ms[col] * a.F + row] = gi;
-                                if (a.tap1) a.tap1[(size_t)ms[col] * a.F + row] = ui;
+                            float *hd = hs + (size_t)cb * a.F + row;
+                            if (cb + 16 <= n) {
+#pragma unroll
+                                for (int j = 0; j < 16; j++) hd[(size_t)j * a.F] = hv[j];
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 16; j++)
+                                    if (cb + j < n) hd[(size_t)j * a.F] = hv[j];
+                            }
+                            if (a.tap0 || a.tap1) {
+                                // the raw accumulators, loaded again (checking runs only)
+                                tmem_ld16(tb + cb, g);
+                                tmem_ld16(tb + 128 + cb, u);
+                                tmem_wait_ld();
+                                for (int j = 0; j < 16 && cb + j < n; j++) {
+                                    if (a.tap0) a.tap0[(size_t)ms[cb + j] * a.F + row] = g[j] >> 6;
+                                    if (a.tap1) a.tap1[(size_t)ms[cb + j] * a.F + row] = u[j] >> 6;
+                                }
                             }
                         }
                     }
                 } else {
-                    // The warp's 32 channels x 32 slot columns, transposed through its
-                    // shared-memory tile (row = slot, 64 bytes of int16, 16-byte chunks
-                    // swizzled by (slot / 2) % 4 so that both sides are free of bank
-                    // conflicts), then written back per slot as four 16-byte stores of
-                    // acc >> 1 and one word of low bits (the column's ballot).
-                    uint8_t *tile = smem + L::kTr + ew * 2048;
+                    // The warp's 32 channels x 32 slot columns: per slot the 32 lanes
+                    // (consecutive channels) write acc >> 1 as one 64-byte run, and the
+                    // slot's low bits (the column's ballot) go out as one word from lane j.
                     const int row0 = rb * 128 + q * 32;   // this warp's first channel
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
                         int dd[32];
@@ -547,23 +564,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         uint32_t my_lo = 0;   // lane j: the low bits of column j
 #pragma unroll
                         for (int j = 0; j < 32; j++) {
-                            const int di = dd[j] >> 6;
-                            const int ck = (lane >> 3) ^ ((j >> 1) & 3);
-                            *reinterpret_cast<int16_t *>(tile + j * 64 + ck * 16 + (lane & 7) * 2) = (int16_t)(di >> 1);
-                            const uint32_t lo = __ballot_sync(FULL, di & 1);
-                            if (lane == j) my_lo = lo;
-                            if (a.tap0 && c0 + j < n) a.tap0[(size_t)ms[c0 + j] * a.D + row] = di;
+                            dd[j] >>= 6;
+                            const uint32_t lo = __ballot_sync(FULL, dd[j] & 1);
+                            my_lo = lane == j ? lo : my_lo;
                         }
-                        __syncwarp();
-                        if (c0 + lane < n) {
-                            const size_t p = (size_t)p0 + c0 + lane;
-                            uint4 *dst = reinterpret_cast<uint4 *>(a.acc_hi + p * a.D + row0);
+                        int16_t *dst = a.acc_hi + ((size_t)p0 + c0) * a.D + row0 + lane;
+                        if (c0 + 32 <= n) {
 #pragma unroll
-                            for (int k = 0; k < 4; k++)
-                                dst[k] = *reinterpret_cast<const uint4 *>(tile + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4));
-                            a.acc_lo[p * (a.D / 32) + (row0 >> 5)] = my_lo;
+                            for (int j = 0; j < 32; j++) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; j++)
+                                if (c0 + j < n) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
                         }
-                        __syncwarp();   // the tile is read before the next chunk overwrites it
+                        if (a.tap0)
+                            for (int j = 0; j < 32 && c0 + j < n; j++) a.tap0[(size_t)ms[c0 + j] * a.D + row] = dd[j];
+                        if (c0 + lane < n) a.acc_lo[((size_t)p0 + c0 + lane) * (a.D / 32) + (row0 >> 5)] = my_lo;
                     }
                     (void)al0;
                 }

@@ -417,6 +417,9 @@ def run_gpu(args, rank: int, world: int):
     stream = torch.cuda.current_stream(dev)
     xs = {T: bf16_from_bits(synth.activations(T, shape.d_model, seed=0, stream=rank), dev) for T in DECODE_T}
     ys = {T: torch.empty((T, shape.d_model), dtype=torch.float32, device=dev) for T in DECODE_T}
+    # the expert path of each batch size (the library decides: the fused kernel
+    # where all of a batch's expert clusters fit on the device at once)
+    fused = {T: tw.maple_moe_expert_path(layers[0].handle, T) == tw.MAPLE_PATH_DECODE_FUSED for T in DECODE_T}
     n_active = {T: [] for T in DECODE_T}   # experts touched, per layer
     for T in DECODE_T:
         for L in layers:
@@ -426,7 +429,7 @@ def run_gpu(args, rank: int, world: int):
     no_flush = torch.empty(0, dtype=torch.float32, device=dev)
 
     # The timed unit: per batch size one CUDA graph holding the forwards of all
-    # N_ROT layers in order (each forward is four kernels, each a programmatic
+    # N_ROT layers in order (each forward is two or four kernels, each a programmatic
     # dependent of the one before); one replay = N_ROT forwards, back to back,
     # timed with CUDA events on the stream.  Consecutive forwards read different
     # layers' weights.
@@ -479,8 +482,9 @@ def run_gpu(args, rank: int, world: int):
     fwd_T = {T: [t[1] / N_ROT for t in timed if t[0] == T] for T in DECODE_T}
     experts_ms = sum(x[2] - x[0] for T in DECODE_T for _, x in split[T])
     experts_alg = sum(experts_bytes(n_active[T][l], T) for T in DECODE_T for l, _ in split[T])
-    gu_ms = sum(x[1] - x[0] for T in DECODE_T for _, x in split[T])
-    gu_alg = sum(gate_up_bytes(n_active[T][l], T) for T in DECODE_T for l, _ in split[T])
+    # the gate/up kernel of the two-kernel path (the batches that take it)
+    gu_ms = sum(x[1] - x[0] for T in DECODE_T if not fused[T] for _, x in split[T])
+    gu_alg = sum(gate_up_bytes(n_active[T][l], T) for T in DECODE_T if not fused[T] for l, _ in split[T])
 
     # ---- end to end: pinned host x -> device, forward, y -> pinned host, all timed
     hx = {T: xs[T].cpu().pin_memory() for T in DECODE_T}
@@ -529,32 +533,24 @@ def run_gpu(args, rank: int, world: int):
         "experts_touched_mean": {str(T): statistics.mean(n_active[T]) for T in DECODE_T},
         "l2": f"inputs larger than L2: {N_ROT} independently seeded layers (6.4 GB of packed weights) "
               "in rotation, one per forward; no flush inside the timed region",
-        "per_T": {str(T): {"tokens_per_s": T / (statistics.mean(fwd_T[T]) * 1e-3),
-                           "us_per_forward": 1e3 * statistics.mean(fwd_T[T]),
-                           "us_per_forward_l2_flushed": 1e3 * statistics.mean(flushed[T]),
-                           "us_route": 1e3 * statistics.mean(x[0] for _, x in split[T]),
-                           "us_gate_up": 1e3 * statistics.mean(x[1] - x[0] for _, x in split[T]),
-                           "us_down_combine": 1e3 * statistics.mean(x[2] - x[1] for _, x in split[T]),
-                           "layer_hbm_frac": statistics.mean(decode_bytes(n, T) for n in n_active[T]) /
-                           (statistics.mean(fwd_T[T]) * 1e-3) / 1e9 / hbm,
-                           "experts_hbm_frac": statistics.mean(experts_bytes(n_active[T][l], T) / (
-                               (x[2] - x[0]) * 1e-3) / 1e9 / hbm for l, x in split[T]),
-                           "gate_up_hbm_frac": statistics.mean(gate_up_bytes(n_active[T][l], T) / (
-                               (x[1] - x[0]) * 1e-3) / 1e9 / hbm for l, x in split[T])}
-                  for T in DECODE_T},
+        "per_T": {str(T): per_T_entry(T, fused[T], fwd_T[T], flushed[T], split[T], n_active[T], hbm) for T in DECODE_T},
         "layer_roofline_frac": layer_bytes / (total_ms * 1e-3 / world) / 1e9 / hbm if world == 1 else None,
-        "roofline": {"kernel": "decode_stage_kernel<1> (gate/up: the dominant kernel)", "bound": "hbm",
+        "roofline": {"kernel": "decode_stage_kernel<1> (gate/up: the dominant kernel; batches of 32 and 64)",
+                     "bound": "hbm",
                      "achieved": gu_achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": gu_achieved / hbm, "traffic": measured_traffic(),
                      "traffic_launch": "T=64 (ncu, profiles/)",
                      "algorithmic_bytes_T64": gate_up_bytes(round(statistics.mean(n_active[64])), 64)},
-        "roofline_expert_stage": {"kernels": "decode_stage_kernel<1>, decode_stage_kernel<2>, dx_combine_kernel",
+        "roofline_expert_stage": {"kernels": "dx_fused_kernel (T in " + str([T for T in DECODE_T if fused[T]]) +
+                                             "); decode_stage_kernel<1>, decode_stage_kernel<2>, dx_combine_kernel "
+                                             "(the others)",
                                   "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                                   "frac": achieved / hbm},
         "e2e": {"value": whole_job_rate(tokens_rank, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(T * shape.d_model * 2 for T in DECODE_T),
                 "d2h_bytes_per_step": sum(T * shape.d_model * 4 for T in DECODE_T)},
-        "gpu_launches": 4 * len(DECODE_T) * N_ROT * args.steps,   # routing, gate/up, down, combine per forward
+        # per forward: routing + the fused expert kernel (T <= 8), or routing, gate/up, down, combine
+        "gpu_launches": sum(2 if fused[T] else 4 for T in DECODE_T) * N_ROT * args.steps,
         "cuda_graphs": True,
         "stage_split_from": stage_src,
         "clocks": clocks,
@@ -569,6 +565,27 @@ def run_gpu(args, rank: int, world: int):
         out["per_config"] = per
         out["roofline_prefill"] = per["prefill"]["roofline_gemms"]
     return out
+
+
+def per_T_entry(T, fused, fwd, flushed, split, n_active, hbm) -> dict:
+    """One decode batch size's line: times per forward and the stage split
+    (routing; experts: gate/up and down + combine, or the fused expert kernel)."""
+    ent = {"tokens_per_s": T / (statistics.mean(fwd) * 1e-3),
+           "us_per_forward": 1e3 * statistics.mean(fwd),
+           "us_per_forward_l2_flushed": 1e3 * statistics.mean(flushed),
+           "expert_path": "fused" if fused else "two-kernel",
+           "us_route": 1e3 * statistics.mean(x[0] for _, x in split),
+           "us_experts": 1e3 * statistics.mean(x[2] - x[0] for _, x in split),
+           "layer_hbm_frac": statistics.mean(decode_bytes(n, T) for n in n_active) /
+           (statistics.mean(fwd) * 1e-3) / 1e9 / hbm,
+           "experts_hbm_frac": statistics.mean(experts_bytes(n_active[l], T) / ((x[2] - x[0]) * 1e-3) / 1e9 / hbm
+                                               for l, x in split)}
+    if not fused:
+        ent["us_gate_up"] = 1e3 * statistics.mean(x[1] - x[0] for _, x in split)
+        ent["us_down_combine"] = 1e3 * statistics.mean(x[2] - x[1] for _, x in split)
+        ent["gate_up_hbm_frac"] = statistics.mean(gate_up_bytes(n_active[l], T) / ((x[1] - x[0]) * 1e-3) / 1e9 / hbm
+                                                  for l, x in split)
+    return ent
 
 
 def config_of(world: int) -> dict:

@@ -235,6 +235,9 @@ int maple_moe_device_flags(maple_moe_t layer, uint32_t *flags, int32_t clear);
 /* maple_moe_set_debug flags (testing the failure handling only) */
 #define MAPLE_DEBUG_STALL_DOWN 0x1u   /* the decode path's down kernel waits for a device word that
                                          nothing sets, so that its bounded wait expires */
+#define MAPLE_DEBUG_SPLIT_SMALL 0x2u  /* decode batches of at most 8 tokens take the two-kernel expert
+                                         path (gate/up kernel, down kernel, combine) instead of the
+                                         fused one-kernel path (one thread-block cluster per expert) */
 
 /*
  * Failure-handling knobs of a handle, for tests.  wait_limit_us: the limit of
@@ -243,6 +246,21 @@ int maple_moe_device_flags(maple_moe_t layer, uint32_t *flags, int32_t clear);
  * Takes effect for calls made after it returns.  Errors: INVALID_ARG.
  */
 int maple_moe_set_debug(maple_moe_t layer, int32_t wait_limit_us, uint32_t debug_flags);
+
+/* maple_moe_expert_path results */
+#define MAPLE_PATH_TC 0            /* tensor-core grouped GEMMs (gate/up + SwiGLU + requantisation, down), combine */
+#define MAPLE_PATH_DECODE 1        /* weight-streaming gate/up kernel, down kernel, combine kernel */
+#define MAPLE_PATH_DECODE_FUSED 2  /* one kernel: a thread-block cluster per active expert, combine included */
+
+/*
+ * Which expert path a forward of T tokens takes on this handle now (its
+ * configuration flags, debug flags and the device's cluster occupancy decide;
+ * the routing step is the same for all).  For measurement and tests: writes
+ * one of MAPLE_PATH_* to *path.  Launches nothing.  Errors: INVALID_ARG (path
+ * NULL, T < 1 or above the handle's max_tokens), UNSUPPORTED_SHAPE (a
+ * decode-only handle and T above its decode limit).
+ */
+int maple_moe_expert_path(maple_moe_t layer, int32_t T, int32_t *path);
 
 /* Synchronise all work of the layer and free everything it owns.  NULL is a no-op. */
 int maple_moe_destroy(maple_moe_t layer);

@@ -32,10 +32,15 @@ MAPLE_CFG_FORCE_TC = 0x2
 MAPLE_CFG_DECODE_ONLY = 0x4
 
 MAPLE_DEBUG_STALL_DOWN = 0x1
+MAPLE_DEBUG_SPLIT_SMALL = 0x2
+
+MAPLE_PATH_TC = 0
+MAPLE_PATH_DECODE = 1
+MAPLE_PATH_DECODE_FUSED = 2
 
 EXPORTED = ("maple_moe_status_string", "maple_moe_pack_ternary", "maple_moe_create", "maple_moe_route",
             "maple_moe_forward", "maple_moe_stack_forward", "maple_moe_set_stage_events", "maple_moe_device_flags",
-            "maple_moe_destroy", "maple_moe_route_noalloc", "maple_moe_set_debug")
+            "maple_moe_destroy", "maple_moe_route_noalloc", "maple_moe_set_debug", "maple_moe_expert_path")
 
 
 class MapleError(RuntimeError):
@@ -86,6 +91,7 @@ def lib():
         L.maple_moe_destroy.argtypes = [P]
         L.maple_moe_route_noalloc.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P, P]
         L.maple_moe_set_debug.argtypes = [P, I32, C.c_uint32]
+        L.maple_moe_expert_path.argtypes = [P, I32, C.POINTER(C.c_int32)]
         for name in EXPORTED:
             if name != "maple_moe_status_string":
                 getattr(L, name).restype = C.c_int
@@ -166,6 +172,13 @@ def maple_moe_route_noalloc(x, T: int, d_model: int, n_experts: int, top_k: int,
 def maple_moe_set_debug(handle, wait_limit_us: int = 0, debug_flags: int = 0) -> None:
     """Wait limit of the handle's bounded device waits (0 = 2 s) and test hooks."""
     _check(lib().maple_moe_set_debug(handle, wait_limit_us, debug_flags), "maple_moe_set_debug")
+
+
+def maple_moe_expert_path(handle, T: int) -> int:
+    """MAPLE_PATH_* of a forward of T tokens on this handle."""
+    p = C.c_int32(-1)
+    _check(lib().maple_moe_expert_path(handle, T, C.byref(p)), "maple_moe_expert_path")
+    return p.value
 
 
 def maple_moe_destroy(handle) -> None:

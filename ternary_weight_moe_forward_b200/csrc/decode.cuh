@@ -716,4 +716,373 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// Small decode batches (T <= 8): the whole expert stage in one kernel.
+// At T <= 8 an expert holds at most 8 slots, so every active expert is one
+// unit and one 8-token MMA n-tile.  One thread-block cluster of C CTAs per
+// unit; CTA r of the cluster takes the r-th slice of the expert's gate/up
+// outputs (F/C of them: F/8/C items) and of its down channels (D/C: F/16/C
+// items), so the expert's weights are in flight at once across C SMs and each
+// slice fits its CTA's shared memory (no slot is reused):
+//   1. each warp issues the bulk copies of its items (gate/up and down) at
+//      once; the unit's q_x rows come in as the gate/up B operand;
+//   2. gate/up items -> SwiGLU -> the slice of h in shared memory; each
+//      token's |h| maximum over the slice goes to every CTA of the cluster
+//      (distributed shared memory); cluster barrier;
+//   3. the maxima of all slices give each slot's s_h; every CTA requantises
+//      its slice and writes the codes into every CTA's down B operand (in
+//      fragment order), with the slice's code sums; cluster barrier;
+//   4. down items -> yE (position order) for the CTA's channels;
+//   5. combine: per (token, channel slice) a count of the token's K slots
+//      done; the CTA that completes it adds the K slots' yE in rank order
+//      (fmaf from 0, then the residual) into y, and sets the count back to 0.
+// The arithmetic of every value is that of the two-kernel path (the same
+// MMA planes, the same fp32 operations in the same order), so both give the
+// same bits.  Grid: (units at most) x C CTAs, launched as a programmatic
+// dependent of the routing kernel; clusters past the routing's unit count
+// return at once.  Every wait is bounded; after a failed wait the CTA still
+// takes the cluster barriers (doing no work), drains its copies and returns.
+// ---------------------------------------------------------------------------
+constexpr int kDfWarps = 16;
+constexpr int kDfThreads = kDfWarps * 32;
+
+struct DfArgs {
+    int T, D, E, K, F;
+    const float *sx;
+    const int *sumx;
+    const int8_t *qxp;        // [T][D] q_x rows in fragment order
+    const int *perm, *inv;    // position -> slot, slot -> position
+    const float *topk_w;      // [T][K]
+    const int4 *funits;       // {expert, first position | count << 16, tokens 0-3, tokens 4-7 (bytes)}
+    const int *n_units;
+    const uint8_t *w_gu, *w_dn;
+    float *ye;                // [T*K][D] position order
+    unsigned *ctr;            // [T][C] slots done per (token, channel slice), zero between launches
+    float *y;
+    const float *resid;       // optional
+    int *tap_acc_gate, *tap_acc_up, *tap_acc_down;
+    int8_t *tap_qh;
+    float *tap_sh;
+    unsigned *flag;
+    const unsigned *never;
+    uint64_t wait_ns;
+    int stall;                // test hook: the down phase waits for `never` to become 1
+};
+
+// shared-memory layout of dx_fused_kernel for a cluster of C CTAs
+struct DfSmem {
+    int ig, id, gu_bytes, dn_bytes, items, b1, b2, hl, amax, sums, side, comb, bars, total;
+    __host__ __device__ DfSmem(int D, int F, int C)
+    {
+        ig = mma_gu_items(F) / C;
+        id = mma_dn_items(F) / C;
+        gu_bytes = (int)mma_gu_item_bytes(D);
+        dn_bytes = (int)mma_dn_item_bytes(D, F);
+        items = 0;                                                   // ig gate/up items, then id down items
+        b1 = (items + ig * gu_bytes + id * dn_bytes + 1023) & ~1023;  // q_x B operand: D/128 blocks of 1 KB
+        b2 = b1 + (D / 128) * 1024;                                  // q_h B operand: F/128 blocks
+        hl = b2 + (F / 128) * 1024;                                  // [8][F/C] h of the slice
+        amax = hl + 8 * (F / C) * 4;                                 // [C][8] slice maxima (float)
+        sums = amax + C * 8 * 4;                                     // [C][8] slice code sums
+        side = sums + C * 8 * 4;                                     // per token: pos, slot, tok, s_x, sum_x, s_h, sum_h, last
+        comb = side + 8 * 8 * 4;                                     // per token and rank: combine weight, yE position [8][8] each
+        bars = (comb + 2 * 64 * 4 + 7) & ~7;                         // [ig + id] copy barriers, then the abort word
+        total = bars + 8 * (ig + id) + 16;
+    }
+};
+
+__global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
+{
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(1024) uint8_t dsm[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
+    const int c = blockIdx.x / C;
+    const int D = a.D, F = a.F, K = a.K;
+    const DfSmem L(D, F, C);
+    const int KB1 = D / 128, KB2 = F / 128, S2 = D / F;
+    const int IG = L.ig, NI = L.ig + L.id, FS = F / C, DS = D / C;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
+    uint8_t *b1 = dsm + L.b1;
+    uint8_t *b2 = dsm + L.b2;
+    float *hl = (float *)(dsm + L.hl);
+    float *s_amax = (float *)(dsm + L.amax);
+    int *s_sums = (int *)(dsm + L.sums);
+    int *s_pos = (int *)(dsm + L.side), *s_slot = s_pos + 8, *s_tok = s_slot + 8;
+    float *s_sx = (float *)(s_tok + 8);
+    int *s_sumx = (int *)(s_sx + 8);
+    float *s_sh = (float *)(s_sumx + 8);
+    int *s_sumh = (int *)(s_sh + 8), *s_last = s_sumh + 8;
+    float *s_cw = (float *)(dsm + L.comb);   // [8][8]: token n's rank-k weight
+    int *s_cinv = (int *)(s_cw + 64);        // [8][8]: the position of its rank-k slot
+    uint64_t *bars = (uint64_t *)(dsm + L.bars);
+    volatile uint32_t *abort = (volatile uint32_t *)(bars + NI);
+    const uint32_t bar0 = smem_addr(bars);
+    auto item_addr = [&](int i) {
+        return dsm + L.items + (i < IG ? i * L.gu_bytes : IG * L.gu_bytes + (i - IG) * L.dn_bytes);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NI; i++) mbar_init(bar0 + 8 * i, 1);
+        *abort = 0u;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the routing kernel's outputs: wait for its grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int n_units = __ldcg(a.n_units);
+    const int4 fu = __ldcg(a.funits + c);   // (read with the count: the array holds stale units past it)
+    if (c >= n_units) return;   // the whole cluster: n_units is the same for all its CTAs
+    // first cluster barrier, split: arriving says this CTA is running; its wait
+    // comes before the first access to another CTA's shared memory
+    cluster_arrive();
+    const int e = fu.x, p0 = fu.y & 0xffff;
+    int cnt = fu.y >> 16;
+    if (cnt > 8) {   // (at most T <= 8 slots per expert by construction)
+        if (threadIdx.x == 0) set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
+        cnt = 8;
+    }
+
+    // ---- 1. this warp's items, all copies at once (gate/up items r*IG.., down items r*ID..)
+    if (lane == 0)
+        for (int i = warp; i < NI; i += kDfWarps) {
+            const uint32_t bytes = i < IG ? L.gu_bytes : L.dn_bytes;
+            const uint8_t *src = i < IG ? a.w_gu + ((size_t)e * mma_gu_items(F) + r * IG + i) * L.gu_bytes
+                                        : a.w_dn + ((size_t)e * mma_dn_items(F) + r * L.id + (i - IG)) * L.dn_bytes;
+            mbar_expect_tx(bar0 + 8 * i, bytes);
+            bulk_g2s(smem_addr(item_addr(i)), src, bytes, bar0 + 8 * i);
+        }
+    // the unit's tokens, and their q_x rows into the B operand (fragment order,
+    // 128-byte swizzled); padding tokens of the n-tile are left as they are
+    const bool taps = a.tap_acc_gate || a.tap_acc_up || a.tap_qh || a.tap_sh || a.tap_acc_down;
+    auto tok = [&](int n) { return min((int)(((uint32_t)(n < 4 ? fu.z : fu.w) >> (8 * (n & 3))) & 0xffu), a.T - 1); };
+    if (threadIdx.x < cnt) {
+        const int n = threadIdx.x, t = tok(n);
+        s_pos[n] = p0 + n;
+        s_tok[n] = t;
+        s_slot[n] = taps ? __ldcg(a.perm + p0 + n) : 0;   // (slot order: for the taps only)
+        s_sx[n] = __ldcg(a.sx + t);
+        s_sumx[n] = __ldcg(a.sumx + t);
+    }
+    if (threadIdx.x >= 32 && threadIdx.x < 32 + 8 * K) {   // the combine's weights and yE positions, early
+        const int n = (threadIdx.x - 32) / K, k = threadIdx.x - 32 - n * K;
+        if (n < cnt) {
+            const int t = tok(n);
+            s_cw[n * 8 + k] = __ldcg(a.topk_w + t * K + k);
+            s_cinv[n * 8 + k] = __ldcg(a.inv + t * K + k);
+        }
+    }
+    const int cpr = D / 16;
+    for (int idx = threadIdx.x; idx < cnt * cpr; idx += kDfThreads) {
+        const int n = idx / cpr, cc = idx - n * cpr;
+        const int t = tok(n);
+        const uint32_t dst = smem_addr(b1 + (cc >> 3) * 1024 + dx_b_chunk(n, cc & 7));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                     "l"(reinterpret_cast<const uint4 *>(a.qxp + (size_t)t * D) + cc)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+
+    // ---- 2. gate/up items: item i of the slice is tile r*IG + i (outputs 8(r*IG+i) ..)
+    {
+        const uint32_t bb_lo = smem_addr(b1) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b1) + dx_b_chunk(g, 2 * tig + 1);
+        for (int i = warp; i < IG; i += kDfWarps) {
+            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
+            const uint8_t *ip = item_addr(i);
+            const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
+            int acc[2][4][4];
+            dx_tile<1>(smem_addr(ip) + lane * 16, bb_lo, bb_hi, KB1, 0, acc);
+            const int ol = 8 * i + g, o = r * FS + ol;
+            const float ag = alpha_s[g], au = alpha_s[8 + g];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; h2++) {
+                const int n = 2 * tig + h2;
+                if (n < cnt) {
+                    const int gd = dx_total(acc, 0, h2) - s_sumx[n];
+                    const int ud = dx_total(acc, 0, 2 + h2) - s_sumx[n];
+                    const float gv = __fmul_rn((float)gd, __fmul_rn(ag, s_sx[n]));
+                    const float uv = __fmul_rn((float)ud, __fmul_rn(au, s_sx[n]));
+                    hl[n * FS + ol] = swiglu(gv, uv);
+                    if (a.tap_acc_gate) a.tap_acc_gate[(size_t)s_slot[n] * F + o] = gd;
+                    if (a.tap_acc_up) a.tap_acc_up[(size_t)s_slot[n] * F + o] = ud;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const bool dead = *abort != 0;   // (no wait runs from here to the down phase: the same in every thread)
+    cluster_wait();   // every CTA of the cluster is running: distributed shared memory may be used
+    // each token's |h| maximum over the slice, to every CTA of the cluster
+    if (warp < cnt && !dead) {
+        float m = 0.0f;
+        for (int k = lane; k < FS; k += 32) m = fmaxf(m, fabsf(hl[warp * FS + k]));
+        m = warp_max(m);
+        if (lane < C) cluster.map_shared_rank(s_amax, lane)[r * 8 + warp] = m;
+    }
+    cluster.sync();
+
+    // ---- 3. s_h from the maxima of all slices; requantise the slice into every CTA's
+    // down B operand (word w = columns 4w .. 4w+3 of the slot's row), with the code sums
+    const int wps = FS / 4;   // words of the slice per token (a power of two <= 32)
+    if (threadIdx.x < cnt * wps && !dead) {
+        const int n = threadIdx.x / wps, wl = threadIdx.x - n * wps, w = r * wps + wl;
+        float amax = 0.0f;
+        for (int q = 0; q < C; q++) amax = fmaxf(amax, s_amax[q * 8 + n]);
+        const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+        const float4 hv = *reinterpret_cast<const float4 *>(hl + n * FS + 4 * wl);
+        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+        if (amax > 0.0f) {
+            q0 = quant_code(hv.x, inv);
+            q1 = quant_code(hv.y, inv);
+            q2 = quant_code(hv.z, inv);
+            q3 = quant_code(hv.w, inv);
+        }
+        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+                            ((uint32_t)(q3 & 0xff) << 24);
+        const int fp = frag_word_pos(w & 31);
+        const uint32_t off = (uint32_t)((w >> 5) * 1024) + dx_b_chunk(n, fp >> 2) + (fp & 3) * 4;
+        for (int q = 0; q < C; q++) *reinterpret_cast<uint32_t *>(cluster.map_shared_rank(b2, q) + off) = pk;
+        if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)s_slot[n] * F)[w] = pk;
+        int sum = q0 + q1 + q2 + q3;
+        const int live = cnt * wps - warp * 32;   // lanes of this warp in the mapping (whole groups of wps)
+        const unsigned mask = live >= 32 ? FULL : (1u << live) - 1u;
+        for (int o2 = wps / 2; o2 >= 1; o2 >>= 1) sum += __shfl_xor_sync(mask, sum, o2);
+        if (wl < C) cluster.map_shared_rank(s_sums, wl)[r * 8 + n] = sum;
+    }
+    cluster.sync();   // every code and sum is in place; no shared memory of another CTA is touched after this
+    if (threadIdx.x < cnt) {
+        const int n = threadIdx.x;
+        float amax = 0.0f;
+        int sum = 0;
+        for (int q = 0; q < C; q++) {
+            amax = fmaxf(amax, s_amax[q * 8 + n]);
+            sum += s_sums[q * 8 + n];
+        }
+        const float sv = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+        s_sh[n] = sv;
+        s_sumh[n] = sum;
+        if (a.tap_sh && r == 0) a.tap_sh[s_slot[n]] = sv;
+    }
+    if (a.stall && threadIdx.x == 0) {
+        // test hook: wait for a word nothing sets, so that the bounded wait expires
+        const uint64_t t0 = global_ns();
+        while (true) {
+            unsigned v;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a.never) : "memory");
+            if (v == 1u) break;
+            __nanosleep(256);
+            if (*abort || global_ns() - t0 > a.wait_ns) {
+                *abort = 1u;
+                set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
+                break;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- 4. down items: item i of the slice is item r*ID + i (tiles S2*(r*ID+i) ..)
+    if (!*abort) {   // (read after the barrier above: the same in every thread)
+        const uint32_t bb_lo = smem_addr(b2) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b2) + dx_b_chunk(g, 2 * tig + 1);
+        for (int i = IG + (kDfWarps - 1 - warp); i < NI; i += kDfWarps) {
+            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
+            const uint8_t *ip = item_addr(i);
+            const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
+            const int it = r * L.id + (i - IG);
+            const uint32_t aa = smem_addr(ip) + lane * 16;
+            auto store = [&](int dt, int dd, int d0, int d1) {   // channels 16dt + g and + 8, token dd
+                const int ch0 = 16 * dt + g, pos = s_pos[dd];
+                a.ye[(size_t)pos * D + ch0] = __fmul_rn((float)d0, __fmul_rn(alpha_s[16 * (dt - S2 * it) + g], s_sh[dd]));
+                a.ye[(size_t)pos * D + ch0 + 8] =
+                    __fmul_rn((float)d1, __fmul_rn(alpha_s[16 * (dt - S2 * it) + 8 + g], s_sh[dd]));
+                if (a.tap_acc_down) {
+                    a.tap_acc_down[(size_t)s_slot[dd] * D + ch0] = d0;
+                    a.tap_acc_down[(size_t)s_slot[dd] * D + ch0 + 8] = d1;
+                }
+            };
+            if (S2 == 4) {
+                int acc4[4][4][4];
+                dx_tile4(aa, KB2 * 512, bb_lo, bb_hi, KB2, acc4);
+#pragma unroll
+                for (int d = 0; d < 4; d++)
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        const int n = 2 * tig + h2;
+                        if (n < cnt)
+                            store(S2 * it + d, n,
+                                  acc4[d][0][h2] + (acc4[d][1][h2] >> 2) + (acc4[d][2][h2] >> 4) + (acc4[d][3][h2] >> 6) -
+                                      s_sumh[n],
+                                  acc4[d][0][2 + h2] + (acc4[d][1][2 + h2] >> 2) + (acc4[d][2][2 + h2] >> 4) +
+                                      (acc4[d][3][2 + h2] >> 6) - s_sumh[n]);
+                    }
+            } else {
+                for (int d = 0; d < S2; d++) {
+                    int acc[2][4][4];
+                    dx_tile<1>(aa + d * KB2 * 512, bb_lo, bb_hi, KB2, 0, acc);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        const int n = 2 * tig + h2;
+                        if (n < cnt)
+                            store(S2 * it + d, n, dx_total(acc, 0, h2) - s_sumh[n], dx_total(acc, 0, 2 + h2) - s_sumh[n]);
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- 5. combine: count this slice of each of the unit's tokens as done.  The
+    // count is an acquire-release atomic after the CTA barrier: it publishes every
+    // yE store of the CTA, and the CTA that completes a count sees every other
+    // CTA's (its readers are ordered after it by the next barrier).
+    __syncthreads();
+    if (threadIdx.x < cnt) {
+        int last = 0;
+        if (!*abort) {
+            const int t = s_tok[threadIdx.x];
+            unsigned prev;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.ctr + t * C + r) : "memory");
+            last = prev == (unsigned)(K - 1);
+            if (last) a.ctr[t * C + r] = 0u;   // every slot of (t, r) has arrived: nobody else touches it
+        }
+        s_last[threadIdx.x] = last;
+    }
+    __syncthreads();
+    for (int n = 0; n < cnt; n++) {
+        if (!s_last[n]) continue;
+        const int t = s_tok[n];
+        for (int c4 = threadIdx.x; c4 < DS / 4; c4 += kDfThreads) {
+            const int ch = r * DS + 4 * c4;
+            float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k < K; k++) {
+                const float wk = s_cw[n * 8 + k];
+                const float4 ev = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)s_cinv[n * 8 + k] * D + ch));
+                yv.x = __fmaf_rn(wk, ev.x, yv.x);
+                yv.y = __fmaf_rn(wk, ev.y, yv.y);
+                yv.z = __fmaf_rn(wk, ev.z, yv.z);
+                yv.w = __fmaf_rn(wk, ev.w, yv.w);
+            }
+            const size_t o = (size_t)t * D + ch;
+            if (a.resid) {
+                const float4 rv = *reinterpret_cast<const float4 *>(a.resid + o);
+                yv.x = __fadd_rn(rv.x, yv.x);
+                yv.y = __fadd_rn(rv.y, yv.y);
+                yv.z = __fadd_rn(rv.z, yv.z);
+                yv.w = __fadd_rn(rv.w, yv.w);
+            }
+            *reinterpret_cast<float4 *>(a.y + o) = yv;
+        }
+    }
+
+    // ---- exit: no copy may still be landing (after a failed wait: bounded waits)
+    if (threadIdx.x == 0 && *abort)
+        for (int i = 0; i < NI; i++) {
+            const uint64_t t0 = global_ns();
+            while (!mbar_test(bar0 + 8 * i, 0) && global_ns() - t0 < a.wait_ns) {
+            }
+        }
+}
+
 }  // namespace maple

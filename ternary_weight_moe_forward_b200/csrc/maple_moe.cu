@@ -40,6 +40,7 @@ struct maple_moe_s {
     int device;
     int optin;                     // shared memory a block may opt in to
     int route_clusters;            // decode batches route with route_cluster_kernel: clusters that fit at once (0: not used)
+    int df_fit[2];                 // dx_fused_kernel: clusters of 8 / of 4 CTAs that fit at once (0: not used)
     char *base;                    // one device allocation: weights + workspace
     // weights
     uint8_t *w_mma_gu, *w_mma_dn;  // decode layout (MMA tiles), null when not built
@@ -73,6 +74,8 @@ struct maple_moe_s {
     int2 *units;                   // decode kernels: units of <= 16 slots of one expert (routing kernel)
     int *n_units;
     const unsigned *dx_never;      // a word that stays 0 (the stall test hook)
+    unsigned *df_ctr;              // dx_fused_kernel: slots done per (token, channel slice) [8][8]
+    int4 *funits;                  // dx_fused_kernel: its units with their tokens [64]
     uint16_t *xn;                  // stack: normalised input of the current layer
     // flag word in host-mapped memory
     unsigned *flag_host;
@@ -254,6 +257,9 @@ static void route_cluster_config(maple_moe_t h, int T, int gt, cudaStream_t st, 
 // How many clusters of the cluster routing kernel run at once on this device
 // and shape (E <= 256, a multiple of 16; K <= 8; d_model <= 2048), 0 when it cannot run.
 // Sets the kernel's attributes; clears any CUDA error it causes.
+static void fused_setup(maple_moe_t h);
+static int fused_cluster(maple_moe_t h, int T);
+
 static int cluster_route_ok(maple_moe_t h)
 {
     if (h->E > kRcMaxExperts || h->E % kRcExperts || h->K > 8) return 0;   // (choices buffer: 8 per token)
@@ -368,7 +374,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     const size_t o_ahi = build_tc ? ar.take(S * D * 2) : 0, o_alo = build_tc ? ar.take(S * D / 8) : 0;
     const size_t o_ctr = ar.take(0);   // counters: zero between calls
     const size_t o_tg = ar.take(((Tm + kRouteTokens - 1) / kRouteTokens) * 4), o_gc = ar.take(4);
-    const size_t o_dx = ar.take((S64 + 1) * 4);
+    const size_t o_dx = ar.take((S64 + 1) * 4), o_dfc = ar.take(64 * 4), o_fu = ar.take(64 * 16);
     const size_t o_un = ar.take((E + (S64 + kUnitTokens - 1) / kUnitTokens + 1) * 8), o_nun = ar.take(4);
     const size_t o_ctr_end = ar.take(0);
     const size_t o_xn = ar.take(Tm * D * 2);
@@ -426,6 +432,8 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     h->glob_cnt = (unsigned *)(b + o_gc);
     h->dx_clear = (unsigned *)(b + o_dx);
     h->dx_never = h->dx_clear + S64;   // zeroed at create, written by nothing
+    h->df_ctr = (unsigned *)(b + o_dfc);
+    h->funits = (int4 *)(b + o_fu);
     h->units = (int2 *)(b + o_un);
     h->n_units = (int *)(b + o_nun);
     h->xn = (uint16_t *)(b + o_xn);
@@ -470,6 +478,7 @@ extern "C" int maple_moe_create(const maple_moe_config *config, const maple_moe_
     bool smem_ok = true;
     for (const void *k : kernels) smem_ok = allow_max_smem(k, h->device) && smem_ok;
     h->route_clusters = cluster_route_ok(h);
+    fused_setup(h);
     if (!maps_ok || !smem_ok || cudaGetLastError() != cudaSuccess) {
         cudaFree(h->base);
         cudaFreeHost(h->flag_host);
@@ -512,6 +521,7 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
     a.resid = norm_resid;   // (T <= 64 only) x = bf16(RMSNorm(resid)), computed by the routing kernel
     a.qxp = frag ? h->qxp : nullptr;   // the decode kernels' fragment-ordered q_x
     a.units = frag ? h->units : nullptr;   // and their units (built with the fused permutation)
+    a.funits = frag && fused_cluster(h, T) ? h->funits : nullptr;   // (the fused expert kernel's)
     a.n_units = h->n_units;
     a.T = T;
     a.D = h->D;
@@ -616,9 +626,130 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
 
 // the decode kernels: gate/up (+ SwiGLU, per-slot maxima), down (+
 // requantisation), combine; the first two persistent, one CTA per SM
+// dx_fused_kernel with clusters of C CTAs: the slices must split into whole
+// items, the requantisation's words of a slice (F/C/4 per token) must be a
+// power of two from C to 32, and the slices must fit shared memory
+static bool fused_shape_ok(maple_moe_t h, int C)
+{
+    const int F = h->F, wps = F / C / 4;
+    if (!h->w_mma_gu || h->K > 8 || h->F > h->D || h->D % h->F) return false;
+    if ((F / 8) % C || (F / 16) % C || wps < C || wps > 32 || (wps & (wps - 1))) return false;
+    return DfSmem(h->D, F, C).total <= h->optin;
+}
+
+static void fused_cluster_config(int C, int n_clusters, int smem, cudaStream_t st, cudaLaunchConfig_t *lc,
+                                 cudaLaunchAttribute *attr)
+{
+    memset(lc, 0, sizeof *lc);
+    lc->gridDim = dim3((unsigned)(n_clusters * C));
+    lc->blockDim = dim3(kDfThreads);
+    lc->dynamicSmemBytes = (size_t)smem;
+    lc->stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc->attrs = attr;
+    lc->numAttrs = 2;
+}
+
+// at create: which cluster sizes of dx_fused_kernel serve this shape, and how
+// many such clusters fit at once
+static void fused_setup(maple_moe_t h)
+{
+    h->df_fit[0] = h->df_fit[1] = 0;
+    int need = 0;
+    for (int C : {8, 4})
+        if (fused_shape_ok(h, C) && DfSmem(h->D, h->F, C).total > need) need = DfSmem(h->D, h->F, C).total;
+    if (!need) return;
+    if (cudaFuncSetAttribute((const void *)dx_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, need) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return;
+    }
+    for (int i = 0; i < 2; i++) {
+        const int C = i ? 4 : 8;
+        if (!fused_shape_ok(h, C)) continue;
+        cudaLaunchConfig_t lc;
+        cudaLaunchAttribute attr[2];
+        fused_cluster_config(C, 1, DfSmem(h->D, h->F, C).total, nullptr, &lc, attr);
+        lc.numAttrs = 1;   // (occupancy: the cluster shape only)
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, (const void *)dx_fused_kernel, &lc) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        h->df_fit[i] = n;
+    }
+}
+
+// cluster size of the fused expert kernel for a batch of T tokens (0: the
+// two-kernel path).  Its clusters (one per unit, at most min(T*K, E)) must all
+// fit at once: a second wave of clusters costs the whole kernel's latency
+// again, more than the two-kernel path takes.  Clusters of 8 where they all
+// fit, else of 4.
+static int fused_cluster(maple_moe_t h, int T)
+{
+    if (T > 8 || h->K > 8 || (h->debug_flags & MAPLE_DEBUG_SPLIT_SMALL)) return 0;
+    const int n = T * h->K < h->E ? T * h->K : h->E;
+    if (h->df_fit[0] >= n) return 8;
+    if (h->df_fit[1] >= n) return 4;
+    return 0;
+}
+
+static int run_experts_fused(maple_moe_t h, int T, int C, float *y, const float *resid, const maple_moe_taps *taps,
+                             cudaStream_t st)
+{
+    DfArgs d;
+    memset(&d, 0, sizeof d);
+    d.T = T;
+    d.D = h->D;
+    d.E = h->E;
+    d.K = h->K;
+    d.F = h->F;
+    d.sx = h->sx;
+    d.sumx = h->sumx;
+    d.qxp = h->qxp;
+    d.perm = h->perm;
+    d.inv = h->inv;
+    d.topk_w = h->topk_w;
+    d.funits = h->funits;
+    d.n_units = h->n_units;
+    d.w_gu = h->w_mma_gu;
+    d.w_dn = h->w_mma_dn;
+    d.ye = h->ye;
+    d.ctr = h->df_ctr;
+    d.y = y;
+    d.resid = resid;
+    if (taps) {
+        d.tap_acc_gate = taps->acc_gate;
+        d.tap_acc_up = taps->acc_up;
+        d.tap_acc_down = taps->acc_down;
+        d.tap_qh = taps->q_h;
+        d.tap_sh = taps->s_h;
+    }
+    d.flag = h->flag_dev;
+    d.never = h->dx_never;
+    d.wait_ns = h->wait_ns;
+    d.stall = (h->debug_flags & MAPLE_DEBUG_STALL_DOWN) ? 1 : 0;
+    // one cluster per unit: at most one unit per slot and per expert
+    const int n_clusters = T * h->K < h->E ? T * h->K : h->E;
+    cudaLaunchConfig_t lc;
+    cudaLaunchAttribute attr[2];
+    fused_cluster_config(C, n_clusters, DfSmem(h->D, h->F, C).total, st, &lc, attr);
+    if (cudaLaunchKernelEx(&lc, dx_fused_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
+    stage_event(h, 2, st);
+    stage_event(h, 3, st);
+    return launch_status();
+}
+
 static int run_experts_dec(maple_moe_t h, int T, float *y, const float *resid, const maple_moe_taps *taps,
                            cudaStream_t st)
 {
+    const int C = fused_cluster(h, T);
+    if (C) return run_experts_fused(h, T, C, y, resid, taps, st);
     const int n1 = dx_ring_slots(1, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
     const int n2 = dx_ring_slots(2, h->D, h->F, T, h->K, h->E, (size_t)h->optin);
     if (!n1 || !n2) return MAPLE_ERR_UNSUPPORTED_SHAPE;
@@ -879,9 +1010,20 @@ extern "C" int maple_moe_set_debug(maple_moe_t h, int32_t wait_limit_us, uint32_
 {
     int rc = check_handle(h);
     if (rc) return rc;
-    if (wait_limit_us < 0 || wait_limit_us > 60000000 || (debug_flags & ~MAPLE_DEBUG_STALL_DOWN)) return MAPLE_ERR_INVALID_ARG;
+    if (wait_limit_us < 0 || wait_limit_us > 60000000 || (debug_flags & ~(MAPLE_DEBUG_STALL_DOWN | MAPLE_DEBUG_SPLIT_SMALL))) return MAPLE_ERR_INVALID_ARG;
     h->wait_ns = wait_limit_us ? (uint64_t)wait_limit_us * 1000ull : kDefaultWaitNs;
     h->debug_flags = debug_flags;
+    return MAPLE_OK;
+}
+
+extern "C" int maple_moe_expert_path(maple_moe_t h, int32_t T, int32_t *path)
+{
+    int rc = check_handle(h);
+    if (rc) return rc;
+    if (!path || T < 1 || T > h->Tm) return MAPLE_ERR_INVALID_ARG;
+    const int nslot = (h->cfg_flags & MAPLE_CFG_FORCE_TC) ? 0 : dec_slots(h, T);
+    if (!nslot && !h->w_tc_gu) return MAPLE_ERR_UNSUPPORTED_SHAPE;
+    *path = !nslot ? MAPLE_PATH_TC : (fused_cluster(h, T) ? MAPLE_PATH_DECODE_FUSED : MAPLE_PATH_DECODE);
     return MAPLE_OK;
 }
 

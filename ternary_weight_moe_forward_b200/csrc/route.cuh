@@ -11,7 +11,7 @@ namespace maple {
 
 constexpr int kRouteTokens = 8;        // tokens per route CTA (one per warp)
 constexpr int kRouteExperts = 8;       // experts per route CTA (one per warp)
-constexpr int kFusedMarkBytes = 16384; // T*E bytes the fused single-CTA permutation can hold
+constexpr int kFusedMarkBytes = 16384; // largest T*E the fused one-warp permutation takes
 constexpr int kPermBlockTokens = 32;   // tokens per CTA of the multi-CTA permutation
 constexpr int kMaxExperts = 1024;
 constexpr int kRouteSmallT = 64;       // up to this many tokens the latency-oriented router runs
@@ -46,6 +46,9 @@ struct RouteArgs {
     int *n_units;
     unsigned *flag;
     int group_tokens;   // route_cluster_kernel: tokens per cluster (8 or 16)
+    // optional (with units, T <= 8 and K <= 8): per unit {expert, first position |
+    // count << 16, its tokens 0-3 and 4-7 as bytes}, for the fused expert kernel
+    int4 *funits;
 };
 
 constexpr int kUnitTokens = 16;   // slots of a decode unit (two 8-token MMA n-tiles)
@@ -59,6 +62,7 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pr
     const int n = pred ? 16 : 0;   // zero-fill when out of range
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem), "r"(n) : "memory");
 }
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -179,74 +183,69 @@ __device__ void quantize_token_warp(const RouteArgs &a, int t, const uint16_t *x
 // top-k (ties to the lower index) and softmax over the kept logits, one warp
 // per token; NPER = logits held per lane (E <= 32*NPER)
 // ---------------------------------------------------------------------------
-// A logit and its expert index as one 64-bit key whose unsigned order is the
-// rank order (larger logit first, equal logits by lower index): the float's
-// bits made order-preserving in the high word (-0 taken as +0, which compares
-// equal), the complement of the index in the low word.  No key is 0.
-__device__ __forceinline__ unsigned long long rank_key(float v, int e)
+// A logit as a 32-bit value whose unsigned order is the order of the logits:
+// the float's bits made order-preserving (-0 taken as +0, which compares
+// equal).  No finite or infinite logit maps to 0, which marks a taken entry.
+__device__ __forceinline__ uint32_t rank_value(float v)
 {
     uint32_t b = __float_as_uint(v);
     if (b == 0x80000000u) b = 0u;
-    const uint32_t o = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ((unsigned long long)o << 32) | (uint32_t)(0xffffffffu - (uint32_t)e);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ float rank_key_value(unsigned long long k)
+__device__ __forceinline__ float rank_value_float(uint32_t o)
 {
-    const uint32_t o = (uint32_t)(k >> 32);
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
-__device__ __forceinline__ int rank_key_index(unsigned long long k) { return (int)(0xffffffffu - (uint32_t)k); }
 
 // Top-k of one row of E logits (one warp); lane k < K ends with the k-th
-// choice (my_e) and its softmax weight (my_w).  A NaN logit ranks last and
-// raises the flag.
+// choice (my_e) and its softmax weight (my_w).  Ranking: larger logit first,
+// equal logits by lower index.  A NaN logit ranks last and raises the flag.
 template <int NPER, bool SMEM = false>
-__device__ __noinline__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
+__device__ __forceinline__ void topk_row_warp(const float *row, int E, int K, unsigned *flag, int &my_e, float &my_w)
 {
     const int lane = threadIdx.x & 31;
-    float lv[NPER];
+    uint32_t ov[NPER];
     bool nan_seen = false;
 #pragma unroll
     for (int j = 0; j < NPER; j++) {
-        int e = lane + 32 * j;
-        float v = -INFINITY;
+        const int e = lane + 32 * j;
+        ov[j] = 0u;
         if (e < E) {
-            v = SMEM ? row[e] : __ldcg(row + e);
+            float v = SMEM ? row[e] : __ldcg(row + e);
             if (isnan(v)) {
                 nan_seen = true;
                 v = -INFINITY;
             }
+            ov[j] = rank_value(v);
         }
-        lv[j] = v;
     }
     if (__any_sync(FULL, nan_seen) && lane == 0) set_flag(flag, MAPLE_DEVFLAG_NAN);
-    // K rounds of a warp-wide maximum of the keys not yet taken (a compact loop:
-    // this runs once per token group on an SM whose instruction cache is cold)
-    unsigned long long key[NPER];
-#pragma unroll
-    for (int j = 0; j < NPER; j++) key[j] = lane + 32 * j < E ? rank_key(lv[j], lane + 32 * j) : 0ull;
-    float my_v = 0.0f;
+    // K rounds: the warp's largest value not yet taken (one warp reduction),
+    // then the lowest index holding it (a second one); a compact loop, since
+    // this runs once per token group on an SM whose instruction cache is cold
+    uint32_t my_o = 0u;
     my_e = 0;
 #pragma unroll 1
     for (int k = 0; k < K; k++) {
-        unsigned long long best = 0ull;
+        uint32_t m = 0u;
 #pragma unroll
-        for (int j = 0; j < NPER; j++) best = key[j] > best ? key[j] : best;
+        for (int j = 0; j < NPER; j++) m = max(m, ov[j]);
+        const uint32_t best = __reduce_max_sync(FULL, m);
+        uint32_t ci = 0xffffffffu;
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(FULL, best, o);
-            best = other > best ? other : best;
-        }
-        const int be = rank_key_index(best);
+        for (int j = NPER - 1; j >= 0; j--)
+            if (ov[j] == best) ci = (uint32_t)(lane + 32 * j);
+        const int be = (int)__reduce_min_sync(FULL, ci);
 #pragma unroll
         for (int j = 0; j < NPER; j++)
-            if (lane + 32 * j == be) key[j] = 0ull;
+            if (lane + 32 * j == be) ov[j] = 0u;
         if (lane == k) {
-            my_v = rank_key_value(best);
+            my_o = best;
             my_e = be;
         }
     }
     // softmax over the kept logits: e_k = exp(l_k - l_0), S = e_0 + e_1 + ..., w_k = e_k / S
+    const float my_v = rank_value_float(my_o);
     const float l0 = __shfl_sync(FULL, my_v, 0);
     const float ek = exp_ref(__fsub_rn(my_v, l0));
     float S = 0.0f;
@@ -573,6 +572,11 @@ __device__ void route_perm_warp(const RouteArgs &a, const int *ch)
         if (cnt[i]) {
             a.active[act] = e;
             if (a.units) a.units[act] = make_int2(e, off | (cnt[i] << 16));
+            if (a.funits) {   // its tokens in order, one byte each
+                uint32_t m = (s_m8[e / 4] >> (8 * (e & 3))) & 0xffu, tk[2] = {0u, 0u};
+                for (int j = 0; m; j++, m &= m - 1u) tk[j >> 2] |= (uint32_t)(__ffs(m) - 1) << (8 * (j & 3));
+                a.funits[act] = make_int4(e, off | (cnt[i] << 16), (int)tk[0], (int)tk[1]);
+            }
             act++;
         }
         off += cnt[i];
@@ -619,6 +623,10 @@ __host__ __device__ inline size_t route_cluster_smem_bytes(int D, int E, int gt)
     return route_cluster_rows_bytes(D, E, gt) + (size_t)gt * E * 4 + (size_t)gt * 8 * 4;
 }
 
+// a cluster barrier in two halves (every thread of every CTA of the cluster)
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 template <int NI, int NPER>
 __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
 {
@@ -636,6 +644,9 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
     const int tg = blockIdx.y, t0 = tg * gt;
     const int nt = min(gt, a.T - t0);
     const int e = rank * kRcExperts + warp;
+    // first cluster barrier, split: arriving says this CTA is running; its wait
+    // comes before the first write into rank 0's shared memory
+    cluster_arrive();
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const float *wr = a.Wr + (size_t)e * a.D;
@@ -651,6 +662,7 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
     route_stage_tokens<NI>(a, xs, t0, nt);
 
     float *lg0 = cluster.map_shared_rank(lg, 0);   // rank 0's logit rows
+    cluster_wait();
     route_logits_warp<NI>(a, w0, w1, xs, nt, a.bias ? a.bias[e] : 0.0f, [&](int t, float v) {
         lg0[t * a.E + e] = v;
         if (a.tap_logits) a.tap_logits[(size_t)(t0 + t) * a.E + e] = v;
@@ -661,19 +673,20 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(RouteArgs a)
     // top-k by warps 0 .. nt-1 while warps 16-nt .. 15 quantise the tokens
     // (q_x feeds the expert kernels, not the router)
     int my_e = 0;
-    if (warp < nt) my_e = topk_token_warp<NPER, true>(a, t0 + warp, lg + warp * a.E);
+    if (warp < nt) {
+        my_e = topk_token_warp<NPER, true>(a, t0 + warp, lg + warp * a.E);
+    }
     if (warp >= kRcExperts - nt) quantize_token_warp<NI>(a, t0 + warp - (kRcExperts - nt), xs + (size_t)(warp - (kRcExperts - nt)) * a.D);
     if (!a.fuse_permute) return;
     if (gridDim.y == 1) {
-        // one token group: the choices are this CTA's own; one warp builds the
-        // permutation (T <= 8: no block-wide barrier)
-        if (warp < nt && lane < a.K) ch[warp * a.K + lane] = my_e;
-        __syncthreads();
-        if (a.T <= 8) {
-            if (warp == 0) route_perm_warp(a, ch);
-        } else {
-            route_fused_permutation(a, reinterpret_cast<unsigned long long *>(rsm), s_warp, [&](int sl) { return ch[sl]; });
-        }
+        // one token group: the choices are the top-k warps' own; once they are
+        // all in shared memory (a barrier of those warps alone: the quantising
+        // warps go on by themselves), warp 0 builds the permutation, its masks
+        // over the logit rows, which are no longer read
+        if (warp >= nt) return;
+        if (lane < a.K) ch[warp * a.K + lane] = my_e;
+        if (nt > 1) asm volatile("bar.sync 1, %0;" ::"r"(32 * nt) : "memory");
+        if (warp == 0) route_perm_warp(a, ch);   // (one group of 8 tokens: T <= 8)
         return;
     }
     // several token groups: the last to finish builds the permutation

@@ -60,6 +60,7 @@ def test_status_strings(lib):
 
 def test_argument_errors_before_any_cuda_call(lib):
     assert lib.maple_moe_destroy(None) == tw.MAPLE_OK
+    assert lib.maple_moe_expert_path(None, 1, C.byref(C.c_int32())) != tw.MAPLE_OK
     assert lib.maple_moe_create(None, None, None, None) == tw.MAPLE_ERR_INVALID_ARG
     w = tw.maple_moe_weights()
     h = C.c_void_p()

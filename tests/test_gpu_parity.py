@@ -234,3 +234,43 @@ def test_paths_agree_bitwise(big_weights, big):
     assert torch.equal(yt.view(torch.int32), yv.view(torch.int32))
     Lt.close()
     Lv.close()
+
+
+@pytest.mark.parametrize("T", [1, 2, 8])
+def test_small_batches_two_kernel_path(big_weights, big, T):
+    """Batches of at most 8 tokens normally take the fused one-kernel expert path;
+    the two-kernel path (gate/up kernel, down kernel, combine) stays exact too."""
+    L_orc, _ = big
+    Lg = Layer(BIG, big_weights, max_tokens=64)
+    tw.maple_moe_set_debug(Lg.handle, 0, tw.MAPLE_DEBUG_SPLIT_SMALL)
+    x = synth.activations(T, BIG.d_model, seed=500 + T)
+    _full_check(BIG, L_orc, Lg, x)
+    Lg.close()
+
+
+def test_small_batch_paths_agree_bitwise(big_weights):
+    """The fused small-batch expert kernel and the two-kernel path give identical bits."""
+    Lf = Layer(BIG, big_weights, max_tokens=64)
+    Ls = Layer(BIG, big_weights, max_tokens=64)
+    tw.maple_moe_set_debug(Ls.handle, 0, tw.MAPLE_DEBUG_SPLIT_SMALL)
+    for T in range(1, 9):
+        x = bf16_from_bits(synth.activations(T, BIG.d_model, seed=600 + T), "cuda")
+        yf, ys = Lf.forward(x), Ls.forward(x)
+        torch.cuda.synchronize()
+        assert torch.equal(yf.view(torch.int32), ys.view(torch.int32)), T
+    assert Lf.device_flags() == 0 and Ls.device_flags() == 0
+    Lf.close()
+    Ls.close()
+
+
+def test_expert_path_query(big_weights, big):
+    _, Lg = big
+    assert tw.maple_moe_expert_path(Lg.handle, 1) == tw.MAPLE_PATH_DECODE_FUSED
+    assert tw.maple_moe_expert_path(Lg.handle, 64) == tw.MAPLE_PATH_DECODE
+    assert tw.maple_moe_expert_path(Lg.handle, 4096) == tw.MAPLE_PATH_TC
+    Ls = Layer(BIG, big_weights, max_tokens=64)
+    tw.maple_moe_set_debug(Ls.handle, 0, tw.MAPLE_DEBUG_SPLIT_SMALL)
+    assert tw.maple_moe_expert_path(Ls.handle, 1) == tw.MAPLE_PATH_DECODE
+    with pytest.raises(tw.MapleError):
+        tw.maple_moe_expert_path(Ls.handle, 65)
+    Ls.close()

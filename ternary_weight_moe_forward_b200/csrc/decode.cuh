@@ -696,13 +696,29 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T * d4; i += gridDim.x * blockDim.x) {
         const int t = i / d4, c = 4 * (i - t * d4);
         float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < K; k++) {
-            const float wk = __ldcg(topk_w + t * K + k);
-            const float4 ev = __ldcg(reinterpret_cast<const float4 *>(ye + (size_t)__ldcg(inv + t * K + k) * D + c));
-            yv.x = __fmaf_rn(wk, ev.x, yv.x);
-            yv.y = __fmaf_rn(wk, ev.y, yv.y);
-            yv.z = __fmaf_rn(wk, ev.z, yv.z);
-            yv.w = __fmaf_rn(wk, ev.w, yv.w);
+        // eight ranks at a time: their positions and weights, then their yE rows, all
+        // loads in flight together; the sum still runs in rank order
+        for (int k0 = 0; k0 < K; k0 += 8) {
+            int pk[8];
+            float wk[8];
+            float4 ev[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (k0 + j < K) {
+                    pk[j] = __ldcg(inv + t * K + k0 + j);
+                    wk[j] = __ldcg(topk_w + t * K + k0 + j);
+                }
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (k0 + j < K) ev[j] = __ldcg(reinterpret_cast<const float4 *>(ye + (size_t)pk[j] * D + c));
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (k0 + j < K) {
+                    yv.x = __fmaf_rn(wk[j], ev[j].x, yv.x);
+                    yv.y = __fmaf_rn(wk[j], ev[j].y, yv.y);
+                    yv.z = __fmaf_rn(wk[j], ev[j].z, yv.z);
+                    yv.w = __fmaf_rn(wk[j], ev[j].w, yv.w);
+                }
         }
         const size_t o = (size_t)t * D + c;
         if (resid) {
@@ -723,10 +739,13 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
 // unit and one 8-token MMA n-tile.  One thread-block cluster of C CTAs per
 // unit; CTA r of the cluster takes the r-th slice of the expert's gate/up
 // outputs (F/C of them: F/8/C items) and of its down channels (D/C: F/16/C
-// items), so the expert's weights are in flight at once across C SMs and each
-// slice fits its CTA's shared memory (no slot is reused):
-//   1. each warp issues the bulk copies of its items (gate/up and down) at
-//      once; the unit's q_x rows come in as the gate/up B operand;
+// items), so the expert's weights are in flight at once across C SMs.  Where
+// the slice fits the CTA's shared memory every item has its own slot; else
+// (small C) the items go through a ring of ns >= F/16/C slots, refilled by
+// warp 0 as the gate/up items are consumed (so the down items never wait for a
+// slot that only the down phase frees):
+//   1. the bulk copies of the first ns items (gate/up, then down) are issued
+//      at once; the unit's q_x rows come in as the gate/up B operand;
 //   2. gate/up items -> SwiGLU -> the slice of h in shared memory; each
 //      token's |h| maximum over the slice goes to every CTA of the cluster
 //      (distributed shared memory); cluster barrier;
@@ -744,7 +763,8 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
 // return at once.  Every wait is bounded; after a failed wait the CTA still
 // takes the cluster barriers (doing no work), drains its copies and returns.
 // ---------------------------------------------------------------------------
-constexpr int kDfWarps = 16;
+constexpr int kDfWarps = 16;        // warp 0 refills the ring; warps 1-15 compute
+constexpr int kDfCompute = kDfWarps - 1;
 constexpr int kDfThreads = kDfWarps * 32;
 
 struct DfArgs {
@@ -768,27 +788,32 @@ struct DfArgs {
     const unsigned *never;
     uint64_t wait_ns;
     int stall;                // test hook: the down phase waits for `never` to become 1
+    int ns;                   // ring slots (0: every item of the slice has its own slot)
 };
 
-// shared-memory layout of dx_fused_kernel for a cluster of C CTAs
+// shared-memory layout of dx_fused_kernel for a cluster of C CTAs and ns ring
+// slots (0: one slot per item, of its exact size)
 struct DfSmem {
-    int ig, id, gu_bytes, dn_bytes, items, b1, b2, hl, amax, sums, side, comb, bars, total;
-    __host__ __device__ DfSmem(int D, int F, int C)
+    int ig, id, gu_bytes, dn_bytes, slot_bytes, nslot, items, b1, b2, hl, amax, sums, side, comb, bars, total;
+    __host__ __device__ DfSmem(int D, int F, int C, int ns)
     {
         ig = mma_gu_items(F) / C;
         id = mma_dn_items(F) / C;
         gu_bytes = (int)mma_gu_item_bytes(D);
         dn_bytes = (int)mma_dn_item_bytes(D, F);
-        items = 0;                                                   // ig gate/up items, then id down items
-        b1 = (items + ig * gu_bytes + id * dn_bytes + 1023) & ~1023;  // q_x B operand: D/128 blocks of 1 KB
+        slot_bytes = gu_bytes > dn_bytes ? gu_bytes : dn_bytes;
+        nslot = ns > 0 ? ns : ig + id;
+        items = 0;                                                   // the slots (ig gate/up items, then id down items)
+        const int ib = ns > 0 ? ns * slot_bytes : ig * gu_bytes + id * dn_bytes;
+        b1 = (items + ib + 1023) & ~1023;                            // q_x B operand: D/128 blocks of 1 KB
         b2 = b1 + (D / 128) * 1024;                                  // q_h B operand: F/128 blocks
         hl = b2 + (F / 128) * 1024;                                  // [8][F/C] h of the slice
         amax = hl + 8 * (F / C) * 4;                                 // [C][8] slice maxima (float)
         sums = amax + C * 8 * 4;                                     // [C][8] slice code sums
         side = sums + C * 8 * 4;                                     // per token: pos, slot, tok, s_x, sum_x, s_h, sum_h, last
         comb = side + 8 * 8 * 4;                                     // per token and rank: combine weight, yE position [8][8] each
-        bars = (comb + 2 * 64 * 4 + 7) & ~7;                         // [ig + id] copy barriers, then the abort word
-        total = bars + 8 * (ig + id) + 16;
+        bars = (comb + 2 * 64 * 4 + 7) & ~7;                         // full [nslot], empty [nslot], abort word,
+        total = bars + 16 * nslot + 16 + 8 * nslot;                  // then per slot: items consumed, copies issued
     }
 };
 
@@ -800,9 +825,11 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
     const int c = blockIdx.x / C;
     const int D = a.D, F = a.F, K = a.K;
-    const DfSmem L(D, F, C);
+    const DfSmem L(D, F, C, a.ns);
     const int KB1 = D / 128, KB2 = F / 128, S2 = D / F;
     const int IG = L.ig, NI = L.ig + L.id, FS = F / C, DS = D / C;
+    const bool ring = a.ns > 0;
+    const int NS = L.nslot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
     uint8_t *b1 = dsm + L.b1;
     uint8_t *b2 = dsm + L.b2;
@@ -817,14 +844,52 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     float *s_cw = (float *)(dsm + L.comb);   // [8][8]: token n's rank-k weight
     int *s_cinv = (int *)(s_cw + 64);        // [8][8]: the position of its rank-k slot
     uint64_t *bars = (uint64_t *)(dsm + L.bars);
-    volatile uint32_t *abort = (volatile uint32_t *)(bars + NI);
-    const uint32_t bar0 = smem_addr(bars);
+    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * NS);
+    volatile int *s_done = (volatile int *)(abort + 4);   // [NS] items consumed from each slot
+    volatile int *s_gen = s_done + NS;                    // [NS] copies issued into each slot
+    const uint32_t bar0 = smem_addr(bars), ebar0 = bar0 + 8 * NS;   // full, empty
     auto item_addr = [&](int i) {
-        return dsm + L.items + (i < IG ? i * L.gu_bytes : IG * L.gu_bytes + (i - IG) * L.dn_bytes);
+        return dsm + L.items +
+               (ring ? (i % NS) * L.slot_bytes : (i < IG ? i * L.gu_bytes : IG * L.gu_bytes + (i - IG) * L.dn_bytes));
+    };
+    auto item_src = [&](int i, int e_) {
+        return i < IG ? a.w_gu + ((size_t)e_ * mma_gu_items(F) + r * IG + i) * L.gu_bytes
+                      : a.w_dn + ((size_t)e_ * mma_dn_items(F) + r * L.id + (i - IG)) * L.dn_bytes;
+    };
+    // item i is in slot i % NS, round i / NS: wait for its copy (after the slot's
+    // previous round has been consumed, so that the parity wait cannot take the
+    // previous round's phase for this one); hand the slot back once it is read
+    auto take = [&](int i) -> bool {
+        const int sl = i % NS, rr = i / NS;
+        if (rr > 0 && lane == 0) {
+            const uint64_t t0 = global_ns();
+            while (s_done[sl] < rr) {
+                if (*abort || global_ns() - t0 > a.wait_ns) {
+                    *abort = 1u;
+                    set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+        return mbar_wait(bar0 + 8 * sl, rr & 1, abort, a.flag, a.wait_ns);
+    };
+    auto give = [&](int i) {
+        if (!ring) return;
+        __syncwarp();
+        if (lane == 0) {
+            s_done[i % NS] = i / NS + 1;
+            mbar_arrive(ebar0 + 8 * (i % NS));
+        }
     };
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NI; i++) mbar_init(bar0 + 8 * i, 1);
+        for (int i = 0; i < NS; i++) {
+            mbar_init(bar0 + 8 * i, 1);
+            mbar_init(ebar0 + 8 * i, 1);
+            s_done[i] = 0;
+            s_gen[i] = 0;
+        }
         *abort = 0u;
         fence_barrier_init();
     }
@@ -845,14 +910,14 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
         cnt = 8;
     }
 
-    // ---- 1. this warp's items, all copies at once (gate/up items r*IG.., down items r*ID..)
+    // ---- 1. the copies of the first NS items at once, spread over the warps (gate/up
+    // items r*IG.., down items r*ID..); the rest (ring) follow as slots free up
     if (lane == 0)
-        for (int i = warp; i < NI; i += kDfWarps) {
+        for (int i = warp; i < NS && i < NI; i += kDfWarps) {
             const uint32_t bytes = i < IG ? L.gu_bytes : L.dn_bytes;
-            const uint8_t *src = i < IG ? a.w_gu + ((size_t)e * mma_gu_items(F) + r * IG + i) * L.gu_bytes
-                                        : a.w_dn + ((size_t)e * mma_dn_items(F) + r * L.id + (i - IG)) * L.dn_bytes;
             mbar_expect_tx(bar0 + 8 * i, bytes);
-            bulk_g2s(smem_addr(item_addr(i)), src, bytes, bar0 + 8 * i);
+            bulk_g2s(smem_addr(item_addr(i)), item_src(i, e), bytes, bar0 + 8 * i);
+            s_gen[i] = 1;
         }
     // the unit's tokens, and their q_x rows into the B operand (fragment order,
     // 128-byte swizzled); padding tokens of the n-tile are left as they are
@@ -890,8 +955,21 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     // ---- 2. gate/up items: item i of the slice is tile r*IG + i (outputs 8(r*IG+i) ..)
     {
         const uint32_t bb_lo = smem_addr(b1) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b1) + dx_b_chunk(g, 2 * tig + 1);
-        for (int i = warp; i < IG; i += kDfWarps) {
-            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
+        if (warp == 0 && ring && lane == 0) {
+            // refill the ring: item i into slot i % NS once item i - NS has been
+            // consumed (a gate/up item: NS >= the down items, so no wait here
+            // depends on the down phase)
+            for (int i = NS; i < NI; i++) {
+                const int sl = i % NS, rr = i / NS;
+                if (!mbar_wait(ebar0 + 8 * sl, (rr - 1) & 1, abort, a.flag, a.wait_ns)) break;
+                const uint32_t bytes = i < IG ? L.gu_bytes : L.dn_bytes;
+                mbar_expect_tx(bar0 + 8 * sl, bytes);
+                bulk_g2s(smem_addr(item_addr(i)), item_src(i, e), bytes, bar0 + 8 * sl);
+                s_gen[sl] = rr + 1;
+            }
+        }
+        for (int i = warp - 1; warp > 0 && i < IG; i += kDfCompute) {
+            if (!take(i)) break;
             const uint8_t *ip = item_addr(i);
             const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
             int acc[2][4][4];
@@ -911,6 +989,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
                     if (a.tap_acc_up) a.tap_acc_up[(size_t)s_slot[n] * F + o] = ud;
                 }
             }
+            give(i);
         }
     }
     __syncthreads();
@@ -927,31 +1006,36 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
 
     // ---- 3. s_h from the maxima of all slices; requantise the slice into every CTA's
     // down B operand (word w = columns 4w .. 4w+3 of the slot's row), with the code sums
-    const int wps = FS / 4;   // words of the slice per token (a power of two <= 32)
-    if (threadIdx.x < cnt * wps && !dead) {
-        const int n = threadIdx.x / wps, wl = threadIdx.x - n * wps, w = r * wps + wl;
+    const int wps = FS / 4;              // words of the slice per token (a power of two >= C)
+    const int tpt = wps < 32 ? wps : 32; // threads per token, each taking wps / tpt words
+    if (threadIdx.x < cnt * tpt && !dead) {
+        const int n = threadIdx.x / tpt, wl0 = threadIdx.x - n * tpt;
         float amax = 0.0f;
         for (int q = 0; q < C; q++) amax = fmaxf(amax, s_amax[q * 8 + n]);
         const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-        const float4 hv = *reinterpret_cast<const float4 *>(hl + n * FS + 4 * wl);
-        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
-        if (amax > 0.0f) {
-            q0 = quant_code(hv.x, inv);
-            q1 = quant_code(hv.y, inv);
-            q2 = quant_code(hv.z, inv);
-            q3 = quant_code(hv.w, inv);
+        int sum = 0;
+        for (int wl = wl0; wl < wps; wl += tpt) {
+            const int w = r * wps + wl;
+            const float4 hv = *reinterpret_cast<const float4 *>(hl + n * FS + 4 * wl);
+            int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+            if (amax > 0.0f) {
+                q0 = quant_code(hv.x, inv);
+                q1 = quant_code(hv.y, inv);
+                q2 = quant_code(hv.z, inv);
+                q3 = quant_code(hv.w, inv);
+            }
+            const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+                                ((uint32_t)(q3 & 0xff) << 24);
+            const int fp = frag_word_pos(w & 31);
+            const uint32_t off = (uint32_t)((w >> 5) * 1024) + dx_b_chunk(n, fp >> 2) + (fp & 3) * 4;
+            for (int q = 0; q < C; q++) *reinterpret_cast<uint32_t *>(cluster.map_shared_rank(b2, q) + off) = pk;
+            if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)s_slot[n] * F)[w] = pk;
+            sum += q0 + q1 + q2 + q3;
         }
-        const uint32_t pk = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
-                            ((uint32_t)(q3 & 0xff) << 24);
-        const int fp = frag_word_pos(w & 31);
-        const uint32_t off = (uint32_t)((w >> 5) * 1024) + dx_b_chunk(n, fp >> 2) + (fp & 3) * 4;
-        for (int q = 0; q < C; q++) *reinterpret_cast<uint32_t *>(cluster.map_shared_rank(b2, q) + off) = pk;
-        if (a.tap_qh) reinterpret_cast<uint32_t *>(a.tap_qh + (size_t)s_slot[n] * F)[w] = pk;
-        int sum = q0 + q1 + q2 + q3;
-        const int live = cnt * wps - warp * 32;   // lanes of this warp in the mapping (whole groups of wps)
+        const int live = cnt * tpt - warp * 32;   // lanes of this warp in the mapping (whole groups of tpt)
         const unsigned mask = live >= 32 ? FULL : (1u << live) - 1u;
-        for (int o2 = wps / 2; o2 >= 1; o2 >>= 1) sum += __shfl_xor_sync(mask, sum, o2);
-        if (wl < C) cluster.map_shared_rank(s_sums, wl)[r * 8 + n] = sum;
+        for (int o2 = tpt / 2; o2 >= 1; o2 >>= 1) sum += __shfl_xor_sync(mask, sum, o2);
+        if (wl0 < C) cluster.map_shared_rank(s_sums, wl0)[r * 8 + n] = sum;
     }
     cluster.sync();   // every code and sum is in place; no shared memory of another CTA is touched after this
     if (threadIdx.x < cnt) {
@@ -987,8 +1071,8 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     // ---- 4. down items: item i of the slice is item r*ID + i (tiles S2*(r*ID+i) ..)
     if (!*abort) {   // (read after the barrier above: the same in every thread)
         const uint32_t bb_lo = smem_addr(b2) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b2) + dx_b_chunk(g, 2 * tig + 1);
-        for (int i = IG + (kDfWarps - 1 - warp); i < NI; i += kDfWarps) {
-            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
+        for (int i = IG + (warp - 1); warp > 0 && i < NI; i += kDfCompute) {
+            if (!take(i)) break;
             const uint8_t *ip = item_addr(i);
             const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
             const int it = r * L.id + (i - IG);
@@ -1030,6 +1114,7 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
                     }
                 }
             }
+            give(i);
         }
     }
 
@@ -1056,14 +1141,19 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
         for (int c4 = threadIdx.x; c4 < DS / 4; c4 += kDfThreads) {
             const int ch = r * DS + 4 * c4;
             float4 yv = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < K; k++) {
-                const float wk = s_cw[n * 8 + k];
-                const float4 ev = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)s_cinv[n * 8 + k] * D + ch));
-                yv.x = __fmaf_rn(wk, ev.x, yv.x);
-                yv.y = __fmaf_rn(wk, ev.y, yv.y);
-                yv.z = __fmaf_rn(wk, ev.z, yv.z);
-                yv.w = __fmaf_rn(wk, ev.w, yv.w);
-            }
+            float4 ev[8];   // (K <= 8) every rank's row in flight at once, summed in rank order
+#pragma unroll
+            for (int k = 0; k < 8; k++)
+                if (k < K) ev[k] = __ldcg(reinterpret_cast<const float4 *>(a.ye + (size_t)s_cinv[n * 8 + k] * D + ch));
+#pragma unroll
+            for (int k = 0; k < 8; k++)
+                if (k < K) {
+                    const float wk = s_cw[n * 8 + k];
+                    yv.x = __fmaf_rn(wk, ev[k].x, yv.x);
+                    yv.y = __fmaf_rn(wk, ev[k].y, yv.y);
+                    yv.z = __fmaf_rn(wk, ev[k].z, yv.z);
+                    yv.w = __fmaf_rn(wk, ev[k].w, yv.w);
+                }
             const size_t o = (size_t)t * D + ch;
             if (a.resid) {
                 const float4 rv = *reinterpret_cast<const float4 *>(a.resid + o);
@@ -1077,10 +1167,13 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     }
 
     // ---- exit: no copy may still be landing (after a failed wait: bounded waits)
+    __syncthreads();
     if (threadIdx.x == 0 && *abort)
-        for (int i = 0; i < NI; i++) {
+        for (int sl = 0; sl < NS; sl++) {
+            const int gen = s_gen[sl];   // copies issued into the slot; the last has phase gen - 1
+            if (!gen) continue;
             const uint64_t t0 = global_ns();
-            while (!mbar_test(bar0 + 8 * i, 0) && global_ns() - t0 < a.wait_ns) {
+            while (!mbar_test(bar0 + 8 * sl, (gen - 1) & 1) && global_ns() - t0 < a.wait_ns) {
             }
         }
 }

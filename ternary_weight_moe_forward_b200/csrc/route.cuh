@@ -52,6 +52,7 @@ struct RouteArgs {
 };
 
 constexpr int kUnitTokens = 16;   // slots of a decode unit (two 8-token MMA n-tiles)
+constexpr int kPermCacheSlots = 512;   // route_fused_permutation: slots whose expert it keeps in shared memory
 constexpr int kRcExperts = 16;    // route_cluster_kernel: experts per CTA (one per warp)
 constexpr int kRcMaxExperts = 256;
 constexpr int kRcMaxGroup = 16;   // route_cluster_kernel: tokens per cluster at most (one top-k warp each)
@@ -404,10 +405,12 @@ __device__ void route_fused_permutation(const RouteArgs &a, unsigned long long *
 {
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_off[kMaxExperts + 1];
+    __shared__ short s_ev[kPermCacheSlots];   // the first slots' experts, read once
     for (int ee = threadIdx.x; ee < a.E; ee += blockDim.x) s_mask[ee] = 0ull;
     __syncthreads();
     for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
         const int ee = expert_of(sl);
+        if (sl < kPermCacheSlots) s_ev[sl] = (short)(ee < 0 || ee >= a.E ? -1 : ee);
         if (ee < 0 || ee >= a.E) {
             set_flag(a.flag, MAPLE_DEVFLAG_BAD_INDEX);
             continue;
@@ -427,7 +430,7 @@ __device__ void route_fused_permutation(const RouteArgs &a, unsigned long long *
         }
     }
     for (int sl = threadIdx.x; sl < a.T * a.K; sl += blockDim.x) {
-        const int ee = expert_of(sl);
+        const int ee = sl < kPermCacheSlots ? (int)s_ev[sl] : expert_of(sl);
         if (ee < 0 || ee >= a.E) continue;
         const int t = sl / a.K;
         const int p = s_off[ee] + __popcll(s_mask[ee] & ((1ull << t) - 1ull));

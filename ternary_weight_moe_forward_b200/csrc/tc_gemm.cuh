@@ -510,10 +510,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                 if (MODE == 0) {
                     // h = SiLU(g) * u to the scratch; the slots' |h| maxima are taken
                     // when the piece is requantised (each slot's row is then in registers)
-                    // Sixteen columns at a time (register budget): the sixteen values are
-                    // computed with no branch between them, so their dependency chains
-                    // interleave, and stored afterwards (columns past the piece's end hold
-                    // no slot: computed, never stored).
+                    // Sixteen columns per TMEM load, eight values at a time computed with
+                    // no branch between them, so that their dependency chains interleave,
+                    // and stored afterwards (columns past the piece's end hold no slot:
+                    // computed, never stored).
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
 #pragma unroll
                         for (int jj = 0; jj < 32; jj += 16) {
@@ -523,22 +523,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                             tmem_ld16(tb + cb, g);
                             tmem_ld16(tb + 128 + cb, u);
                             tmem_wait_ld();
-                            float hv[16];
-#pragma unroll
-                            for (int j = 0; j < 16; j++) {
-                                const float sxt = mf[cb + j];
-                                const float gv = __fmul_rn((float)(g[j] >> 6), __fmul_rn(al0, sxt));
-                                const float uv = __fmul_rn((float)(u[j] >> 6), __fmul_rn(al1, sxt));
-                                hv[j] = swiglu(gv, uv);
-                            }
                             float *hd = hs + (size_t)cb * a.F + row;
-                            if (cb + 16 <= n) {
 #pragma unroll
-                                for (int j = 0; j < 16; j++) hd[(size_t)j * a.F] = hv[j];
-                            } else {
+                            for (int j0 = 0; j0 < 16; j0 += 8) {   // eight chains at a time (register budget)
+                                float hv[8];
 #pragma unroll
-                                for (int j = 0; j < 16; j++)
-                                    if (cb + j < n) hd[(size_t)j * a.F] = hv[j];
+                                for (int j = 0; j < 8; j++) {
+                                    const float sxt = mf[cb + j0 + j];
+                                    const float gv = __fmul_rn((float)(g[j0 + j] >> 6), __fmul_rn(al0, sxt));
+                                    const float uv = __fmul_rn((float)(u[j0 + j] >> 6), __fmul_rn(al1, sxt));
+                                    hv[j] = swiglu(gv, uv);
+                                }
+                                if (cb + j0 + 8 <= n) {
+#pragma unroll
+                                    for (int j = 0; j < 8; j++) hd[(size_t)(j0 + j) * a.F] = hv[j];
+                                } else {
+#pragma unroll
+                                    for (int j = 0; j < 8; j++)
+                                        if (cb + j0 + j < n) hd[(size_t)(j0 + j) * a.F] = hv[j];
+                                }
                             }
                             if (a.tap0 || a.tap1) {
                                 // the raw accumulators, loaded again (checking runs only)
@@ -558,27 +561,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                     // slot's low bits (the column's ballot) go out as one word from lane j.
                     const int row0 = rb * 128 + q * 32;   // this warp's first channel
                     for (int c0 = 32 * hf; c0 < n; c0 += 64) {
-                        int dd[32];
-                        tmem_ld32(tb + c0, dd);
-                        tmem_wait_ld();
                         uint32_t my_lo = 0;   // lane j: the low bits of column j
 #pragma unroll
-                        for (int j = 0; j < 32; j++) {
-                            dd[j] >>= 6;
-                            const uint32_t lo = __ballot_sync(FULL, dd[j] & 1);
-                            my_lo = lane == j ? lo : my_lo;
-                        }
-                        int16_t *dst = a.acc_hi + ((size_t)p0 + c0) * a.D + row0 + lane;
-                        if (c0 + 32 <= n) {
+                        for (int hh = 0; hh < 32; hh += 16) {   // sixteen columns at a time (register budget)
+                            const int cb = c0 + hh;
+                            int dd[16];
+                            tmem_ld16(tb + cb, dd);
+                            tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 32; j++) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
-                        } else {
+                            for (int j = 0; j < 16; j++) {
+                                dd[j] >>= 6;
+                                const uint32_t lo = __ballot_sync(FULL, dd[j] & 1);
+                                my_lo = lane == hh + j ? lo : my_lo;
+                            }
+                            int16_t *dst = a.acc_hi + ((size_t)p0 + cb) * a.D + row0 + lane;
+                            if (cb + 16 <= n) {
 #pragma unroll
-                            for (int j = 0; j < 32; j++)
-                                if (c0 + j < n) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
+                                for (int j = 0; j < 16; j++) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 16; j++)
+                                    if (cb + j < n) dst[(size_t)j * a.D] = (int16_t)(dd[j] >> 1);
+                            }
+                            if (a.tap0)
+                                for (int j = 0; j < 16 && cb + j < n; j++) a.tap0[(size_t)ms[cb + j] * a.D + row] = dd[j];
                         }
-                        if (a.tap0)
-                            for (int j = 0; j < 32 && c0 + j < n; j++) a.tap0[(size_t)ms[c0 + j] * a.D + row] = dd[j];
                         if (c0 + lane < n) a.acc_lo[((size_t)p0 + c0 + lane) * (a.D / 32) + (row0 >> 5)] = my_lo;
                     }
                     (void)al0;
@@ -742,20 +749,42 @@ __global__ void combine_kernel(const int16_t *acc_hi, const uint32_t *acc_lo, co
         const int t = (int)(i / (D / 4));
         const int c = 4 * (int)(i % (D / 4));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < K; k++) {
-            const int sl = t * K + k, p = __ldg(inv + sl), e = __ldg(topk_idx + sl);
-            const float w = __ldg(topk_w + sl), s = __ldg(sh + p);
-            const uint2 hv = __ldcs(reinterpret_cast<const uint2 *>(acc_hi + (size_t)p * D + c));
-            const uint32_t lo = __ldg(acc_lo + (size_t)p * (D / 32) + (c >> 5)) >> (c & 31);
-            const float4 al = __ldg(reinterpret_cast<const float4 *>(alpha_down + (size_t)e * D + c));
-            const int a0 = 2 * (int)(int16_t)(hv.x & 0xffffu) + (int)(lo & 1u);
-            const int a1 = 2 * (int)(int16_t)(hv.x >> 16) + (int)((lo >> 1) & 1u);
-            const int a2 = 2 * (int)(int16_t)(hv.y & 0xffffu) + (int)((lo >> 2) & 1u);
-            const int a3 = 2 * (int)(int16_t)(hv.y >> 16) + (int)((lo >> 3) & 1u);
-            acc.x = __fmaf_rn(w, __fmul_rn((float)a0, __fmul_rn(al.x, s)), acc.x);
-            acc.y = __fmaf_rn(w, __fmul_rn((float)a1, __fmul_rn(al.y, s)), acc.y);
-            acc.z = __fmaf_rn(w, __fmul_rn((float)a2, __fmul_rn(al.z, s)), acc.z);
-            acc.w = __fmaf_rn(w, __fmul_rn((float)a3, __fmul_rn(al.w, s)), acc.w);
+        // four ranks at a time: their indices, then their rows, all loads in flight
+        // together; the sum still runs in rank order
+        for (int k0 = 0; k0 < K; k0 += 4) {
+            int p[4], e[4];
+            float w[4], s[4];
+            uint2 hv[4];
+            uint32_t lo[4];
+            float4 al[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (k0 + j < K) {
+                    const int sl = t * K + k0 + j;
+                    p[j] = __ldg(inv + sl);
+                    e[j] = __ldg(topk_idx + sl);
+                    w[j] = __ldg(topk_w + sl);
+                }
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (k0 + j < K) {
+                    s[j] = __ldg(sh + p[j]);
+                    hv[j] = __ldcs(reinterpret_cast<const uint2 *>(acc_hi + (size_t)p[j] * D + c));
+                    lo[j] = __ldg(acc_lo + (size_t)p[j] * (D / 32) + (c >> 5)) >> (c & 31);
+                    al[j] = __ldg(reinterpret_cast<const float4 *>(alpha_down + (size_t)e[j] * D + c));
+                }
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+                if (k0 + j < K) {
+                    const int a0 = 2 * (int)(int16_t)(hv[j].x & 0xffffu) + (int)(lo[j] & 1u);
+                    const int a1 = 2 * (int)(int16_t)(hv[j].x >> 16) + (int)((lo[j] >> 1) & 1u);
+                    const int a2 = 2 * (int)(int16_t)(hv[j].y & 0xffffu) + (int)((lo[j] >> 2) & 1u);
+                    const int a3 = 2 * (int)(int16_t)(hv[j].y >> 16) + (int)((lo[j] >> 3) & 1u);
+                    acc.x = __fmaf_rn(w[j], __fmul_rn((float)a0, __fmul_rn(al[j].x, s[j])), acc.x);
+                    acc.y = __fmaf_rn(w[j], __fmul_rn((float)a1, __fmul_rn(al[j].y, s[j])), acc.y);
+                    acc.z = __fmaf_rn(w[j], __fmul_rn((float)a2, __fmul_rn(al[j].z, s[j])), acc.z);
+                    acc.w = __fmaf_rn(w[j], __fmul_rn((float)a3, __fmul_rn(al[j].w, s[j])), acc.w);
+                }
         }
         if (resid) {
             const float4 r = reinterpret_cast<const float4 *>(resid)[i];

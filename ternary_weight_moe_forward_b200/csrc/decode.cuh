@@ -541,22 +541,31 @@ __global__ void __launch_bounds__(kDxThreads, 1)
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++) {
                         if (nt >= ntiles) break;
+                        // both tokens' SwiGLU chains with no branch between them (a padding
+                        // token's side data repeat the unit's last token: finite, never stored)
+                        float hv[2];
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; h2++) {
+                            const int n = 8 * nt + 2 * tig + h2;
+                            const int gd = dx_total(acc, nt, h2) - sd->sum[n];
+                            const int ud = dx_total(acc, nt, 2 + h2) - sd->sum[n];
+                            hv[h2] = swiglu(__fmul_rn((float)gd, __fmul_rn(ag, sd->s[n])),
+                                            __fmul_rn((float)ud, __fmul_rn(au, sd->s[n])));
+                        }
                         float hm[2];
 #pragma unroll
                         for (int h2 = 0; h2 < 2; h2++) {
                             const int n = 8 * nt + 2 * tig + h2;
                             hm[h2] = 0.0f;
                             if (n < cnt) {
-                                const int pos = sd->pos[n], slot_t = t_perm[pos];
-                                const int gd = dx_total(acc, nt, h2) - sd->sum[n];
-                                const int ud = dx_total(acc, nt, 2 + h2) - sd->sum[n];
-                                const float gv = __fmul_rn((float)gd, __fmul_rn(ag, sd->s[n]));
-                                const float uv = __fmul_rn((float)ud, __fmul_rn(au, sd->s[n]));
-                                const float hv = swiglu(gv, uv);
-                                a.h[(size_t)pos * F + o] = hv;
-                                hm[h2] = fabsf(hv);
-                                if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot_t * F + o] = gd;
-                                if (a.tap_acc_up) a.tap_acc_up[(size_t)slot_t * F + o] = ud;
+                                const int pos = sd->pos[n];
+                                a.h[(size_t)pos * F + o] = hv[h2];
+                                hm[h2] = fabsf(hv[h2]);
+                                if (a.tap_acc_gate || a.tap_acc_up) {
+                                    const int slot_t = t_perm[pos];
+                                    if (a.tap_acc_gate) a.tap_acc_gate[(size_t)slot_t * F + o] = dx_total(acc, nt, h2) - sd->sum[n];
+                                    if (a.tap_acc_up) a.tap_acc_up[(size_t)slot_t * F + o] = dx_total(acc, nt, 2 + h2) - sd->sum[n];
+                                }
                             }
                         }
                         // maxima over the tile's 8 outputs (lanes of equal tig), then over the unit
@@ -739,13 +748,10 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
 // unit and one 8-token MMA n-tile.  One thread-block cluster of C CTAs per
 // unit; CTA r of the cluster takes the r-th slice of the expert's gate/up
 // outputs (F/C of them: F/8/C items) and of its down channels (D/C: F/16/C
-// items), so the expert's weights are in flight at once across C SMs.  Where
-// the slice fits the CTA's shared memory every item has its own slot; else
-// (small C) the items go through a ring of ns >= F/16/C slots, refilled by
-// warp 0 as the gate/up items are consumed (so the down items never wait for a
-// slot that only the down phase frees):
-//   1. the bulk copies of the first ns items (gate/up, then down) are issued
-//      at once; the unit's q_x rows come in as the gate/up B operand;
+// items), so the expert's weights are in flight at once across C SMs and each
+// slice fits its CTA's shared memory (no slot is reused):
+//   1. each warp issues the bulk copies of its items (gate/up and down) at
+//      once; the unit's q_x rows come in as the gate/up B operand;
 //   2. gate/up items -> SwiGLU -> the slice of h in shared memory; each
 //      token's |h| maximum over the slice goes to every CTA of the cluster
 //      (distributed shared memory); cluster barrier;
@@ -763,8 +769,7 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *ye, const 
 // return at once.  Every wait is bounded; after a failed wait the CTA still
 // takes the cluster barriers (doing no work), drains its copies and returns.
 // ---------------------------------------------------------------------------
-constexpr int kDfWarps = 16;        // warp 0 refills the ring; warps 1-15 compute
-constexpr int kDfCompute = kDfWarps - 1;
+constexpr int kDfWarps = 16;
 constexpr int kDfThreads = kDfWarps * 32;
 
 struct DfArgs {
@@ -788,32 +793,27 @@ struct DfArgs {
     const unsigned *never;
     uint64_t wait_ns;
     int stall;                // test hook: the down phase waits for `never` to become 1
-    int ns;                   // ring slots (0: every item of the slice has its own slot)
 };
 
-// shared-memory layout of dx_fused_kernel for a cluster of C CTAs and ns ring
-// slots (0: one slot per item, of its exact size)
+// shared-memory layout of dx_fused_kernel for a cluster of C CTAs
 struct DfSmem {
-    int ig, id, gu_bytes, dn_bytes, slot_bytes, nslot, items, b1, b2, hl, amax, sums, side, comb, bars, total;
-    __host__ __device__ DfSmem(int D, int F, int C, int ns)
+    int ig, id, gu_bytes, dn_bytes, items, b1, b2, hl, amax, sums, side, comb, bars, total;
+    __host__ __device__ DfSmem(int D, int F, int C)
     {
         ig = mma_gu_items(F) / C;
         id = mma_dn_items(F) / C;
         gu_bytes = (int)mma_gu_item_bytes(D);
         dn_bytes = (int)mma_dn_item_bytes(D, F);
-        slot_bytes = gu_bytes > dn_bytes ? gu_bytes : dn_bytes;
-        nslot = ns > 0 ? ns : ig + id;
-        items = 0;                                                   // the slots (ig gate/up items, then id down items)
-        const int ib = ns > 0 ? ns * slot_bytes : ig * gu_bytes + id * dn_bytes;
-        b1 = (items + ib + 1023) & ~1023;                            // q_x B operand: D/128 blocks of 1 KB
+        items = 0;                                                   // ig gate/up items, then id down items
+        b1 = (items + ig * gu_bytes + id * dn_bytes + 1023) & ~1023;  // q_x B operand: D/128 blocks of 1 KB
         b2 = b1 + (D / 128) * 1024;                                  // q_h B operand: F/128 blocks
         hl = b2 + (F / 128) * 1024;                                  // [8][F/C] h of the slice
         amax = hl + 8 * (F / C) * 4;                                 // [C][8] slice maxima (float)
         sums = amax + C * 8 * 4;                                     // [C][8] slice code sums
         side = sums + C * 8 * 4;                                     // per token: pos, slot, tok, s_x, sum_x, s_h, sum_h, last
         comb = side + 8 * 8 * 4;                                     // per token and rank: combine weight, yE position [8][8] each
-        bars = (comb + 2 * 64 * 4 + 7) & ~7;                         // full [nslot], empty [nslot], abort word,
-        total = bars + 16 * nslot + 16 + 8 * nslot;                  // then per slot: items consumed, copies issued
+        bars = (comb + 2 * 64 * 4 + 7) & ~7;                         // [ig + id] copy barriers, then the abort word
+        total = bars + 8 * (ig + id) + 16;
     }
 };
 
@@ -825,11 +825,9 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     const int C = (int)cluster.num_blocks(), r = (int)cluster.block_rank();
     const int c = blockIdx.x / C;
     const int D = a.D, F = a.F, K = a.K;
-    const DfSmem L(D, F, C, a.ns);
+    const DfSmem L(D, F, C);
     const int KB1 = D / 128, KB2 = F / 128, S2 = D / F;
     const int IG = L.ig, NI = L.ig + L.id, FS = F / C, DS = D / C;
-    const bool ring = a.ns > 0;
-    const int NS = L.nslot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tig = lane & 3;
     uint8_t *b1 = dsm + L.b1;
     uint8_t *b2 = dsm + L.b2;
@@ -844,52 +842,14 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     float *s_cw = (float *)(dsm + L.comb);   // [8][8]: token n's rank-k weight
     int *s_cinv = (int *)(s_cw + 64);        // [8][8]: the position of its rank-k slot
     uint64_t *bars = (uint64_t *)(dsm + L.bars);
-    volatile uint32_t *abort = (volatile uint32_t *)(bars + 2 * NS);
-    volatile int *s_done = (volatile int *)(abort + 4);   // [NS] items consumed from each slot
-    volatile int *s_gen = s_done + NS;                    // [NS] copies issued into each slot
-    const uint32_t bar0 = smem_addr(bars), ebar0 = bar0 + 8 * NS;   // full, empty
+    volatile uint32_t *abort = (volatile uint32_t *)(bars + NI);
+    const uint32_t bar0 = smem_addr(bars);
     auto item_addr = [&](int i) {
-        return dsm + L.items +
-               (ring ? (i % NS) * L.slot_bytes : (i < IG ? i * L.gu_bytes : IG * L.gu_bytes + (i - IG) * L.dn_bytes));
-    };
-    auto item_src = [&](int i, int e_) {
-        return i < IG ? a.w_gu + ((size_t)e_ * mma_gu_items(F) + r * IG + i) * L.gu_bytes
-                      : a.w_dn + ((size_t)e_ * mma_dn_items(F) + r * L.id + (i - IG)) * L.dn_bytes;
-    };
-    // item i is in slot i % NS, round i / NS: wait for its copy (after the slot's
-    // previous round has been consumed, so that the parity wait cannot take the
-    // previous round's phase for this one); hand the slot back once it is read
-    auto take = [&](int i) -> bool {
-        const int sl = i % NS, rr = i / NS;
-        if (rr > 0 && lane == 0) {
-            const uint64_t t0 = global_ns();
-            while (s_done[sl] < rr) {
-                if (*abort || global_ns() - t0 > a.wait_ns) {
-                    *abort = 1u;
-                    set_flag(a.flag, MAPLE_DEVFLAG_TIMEOUT);
-                    break;
-                }
-            }
-        }
-        __syncwarp();
-        return mbar_wait(bar0 + 8 * sl, rr & 1, abort, a.flag, a.wait_ns);
-    };
-    auto give = [&](int i) {
-        if (!ring) return;
-        __syncwarp();
-        if (lane == 0) {
-            s_done[i % NS] = i / NS + 1;
-            mbar_arrive(ebar0 + 8 * (i % NS));
-        }
+        return dsm + L.items + (i < IG ? i * L.gu_bytes : IG * L.gu_bytes + (i - IG) * L.dn_bytes);
     };
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; i++) {
-            mbar_init(bar0 + 8 * i, 1);
-            mbar_init(ebar0 + 8 * i, 1);
-            s_done[i] = 0;
-            s_gen[i] = 0;
-        }
+        for (int i = 0; i < NI; i++) mbar_init(bar0 + 8 * i, 1);
         *abort = 0u;
         fence_barrier_init();
     }
@@ -910,14 +870,14 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
         cnt = 8;
     }
 
-    // ---- 1. the copies of the first NS items at once, spread over the warps (gate/up
-    // items r*IG.., down items r*ID..); the rest (ring) follow as slots free up
+    // ---- 1. this warp's items, all copies at once (gate/up items r*IG.., down items r*ID..)
     if (lane == 0)
-        for (int i = warp; i < NS && i < NI; i += kDfWarps) {
+        for (int i = warp; i < NI; i += kDfWarps) {
             const uint32_t bytes = i < IG ? L.gu_bytes : L.dn_bytes;
+            const uint8_t *src = i < IG ? a.w_gu + ((size_t)e * mma_gu_items(F) + r * IG + i) * L.gu_bytes
+                                        : a.w_dn + ((size_t)e * mma_dn_items(F) + r * L.id + (i - IG)) * L.dn_bytes;
             mbar_expect_tx(bar0 + 8 * i, bytes);
-            bulk_g2s(smem_addr(item_addr(i)), item_src(i, e), bytes, bar0 + 8 * i);
-            s_gen[i] = 1;
+            bulk_g2s(smem_addr(item_addr(i)), src, bytes, bar0 + 8 * i);
         }
     // the unit's tokens, and their q_x rows into the B operand (fragment order,
     // 128-byte swizzled); padding tokens of the n-tile are left as they are
@@ -955,21 +915,8 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     // ---- 2. gate/up items: item i of the slice is tile r*IG + i (outputs 8(r*IG+i) ..)
     {
         const uint32_t bb_lo = smem_addr(b1) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b1) + dx_b_chunk(g, 2 * tig + 1);
-        if (warp == 0 && ring && lane == 0) {
-            // refill the ring: item i into slot i % NS once item i - NS has been
-            // consumed (a gate/up item: NS >= the down items, so no wait here
-            // depends on the down phase)
-            for (int i = NS; i < NI; i++) {
-                const int sl = i % NS, rr = i / NS;
-                if (!mbar_wait(ebar0 + 8 * sl, (rr - 1) & 1, abort, a.flag, a.wait_ns)) break;
-                const uint32_t bytes = i < IG ? L.gu_bytes : L.dn_bytes;
-                mbar_expect_tx(bar0 + 8 * sl, bytes);
-                bulk_g2s(smem_addr(item_addr(i)), item_src(i, e), bytes, bar0 + 8 * sl);
-                s_gen[sl] = rr + 1;
-            }
-        }
-        for (int i = warp - 1; warp > 0 && i < IG; i += kDfCompute) {
-            if (!take(i)) break;
+        for (int i = warp; i < IG; i += kDfWarps) {
+            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
             const uint8_t *ip = item_addr(i);
             const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
             int acc[2][4][4];
@@ -989,7 +936,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
                     if (a.tap_acc_up) a.tap_acc_up[(size_t)s_slot[n] * F + o] = ud;
                 }
             }
-            give(i);
         }
     }
     __syncthreads();
@@ -1071,8 +1017,8 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     // ---- 4. down items: item i of the slice is item r*ID + i (tiles S2*(r*ID+i) ..)
     if (!*abort) {   // (read after the barrier above: the same in every thread)
         const uint32_t bb_lo = smem_addr(b2) + dx_b_chunk(g, 2 * tig), bb_hi = smem_addr(b2) + dx_b_chunk(g, 2 * tig + 1);
-        for (int i = IG + (warp - 1); warp > 0 && i < NI; i += kDfCompute) {
-            if (!take(i)) break;
+        for (int i = IG + (kDfWarps - 1 - warp); i < NI; i += kDfWarps) {
+            if (!mbar_wait(bar0 + 8 * i, 0, abort, a.flag, a.wait_ns)) break;
             const uint8_t *ip = item_addr(i);
             const float *alpha_s = reinterpret_cast<const float *>(ip + 4 * D);
             const int it = r * L.id + (i - IG);
@@ -1114,7 +1060,6 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
                     }
                 }
             }
-            give(i);
         }
     }
 
@@ -1167,13 +1112,10 @@ __global__ void __launch_bounds__(kDfThreads, 1) dx_fused_kernel(DfArgs a)
     }
 
     // ---- exit: no copy may still be landing (after a failed wait: bounded waits)
-    __syncthreads();
     if (threadIdx.x == 0 && *abort)
-        for (int sl = 0; sl < NS; sl++) {
-            const int gen = s_gen[sl];   // copies issued into the slot; the last has phase gen - 1
-            if (!gen) continue;
+        for (int i = 0; i < NI; i++) {
             const uint64_t t0 = global_ns();
-            while (!mbar_test(bar0 + 8 * sl, (gen - 1) & 1) && global_ns() - t0 < a.wait_ns) {
+            while (!mbar_test(bar0 + 8 * i, 0) && global_ns() - t0 < a.wait_ns) {
             }
         }
 }

@@ -40,8 +40,7 @@ struct maple_moe_s {
     int device;
     int optin;                     // shared memory a block may opt in to
     int route_clusters;            // decode batches route with route_cluster_kernel: clusters that fit at once (0: not used)
-    int df_fit[3];                 // dx_fused_kernel: clusters of 8 / 4 / 2 CTAs that fit at once (0: not used)
-    int df_ns[3];                  // and their ring slots (0: one slot per item)
+    int df_fit[2];                 // dx_fused_kernel: clusters of 8 / 4 CTAs that fit at once (0: not used)
     char *base;                    // one device allocation: weights + workspace
     // weights
     uint8_t *w_mma_gu, *w_mma_dn;  // decode layout (MMA tiles), null when not built
@@ -628,21 +627,14 @@ static int run_route(maple_moe_t h, const uint16_t *x, int T, const maple_moe_ta
 // the decode kernels: gate/up (+ SwiGLU, per-slot maxima), down (+
 // requantisation), combine; the first two persistent, one CTA per SM
 // dx_fused_kernel with clusters of C CTAs: the slices must split into whole
-// items and the requantisation's words of a slice (F/C/4 per token) must be a
-// power of two of at least C.  Returns the ring slots (0: every item of the
-// slice has its own slot), or -1 when the slice does not fit shared memory even
-// with the smallest ring (as many slots as down items, so that no refill waits
-// for the down phase).
-static int fused_shape_ns(maple_moe_t h, int C)
+// items, the requantisation's words of a slice (F/C/4 per token) must be a
+// power of two of at least C, and the slices must fit shared memory
+static bool fused_shape_ok(maple_moe_t h, int C)
 {
     const int F = h->F, wps = F / C / 4;
-    if (!h->w_mma_gu || h->K > 8 || h->F > h->D || h->D % h->F) return -1;
-    if ((F / 8) % C || (F / 16) % C || wps < C || (wps & (wps - 1))) return -1;
-    if (DfSmem(h->D, F, C, 0).total <= h->optin) return 0;
-    const int ig = mma_gu_items(F) / C, id = mma_dn_items(F) / C;
-    for (int ns = ig + id - 1; ns >= id && ns >= 1; ns--)
-        if (DfSmem(h->D, F, C, ns).total <= h->optin) return ns;
-    return -1;
+    if (!h->w_mma_gu || h->K > 8 || h->F > h->D || h->D % h->F) return false;
+    if ((F / 8) % C || (F / 16) % C || wps < C || (wps & (wps - 1))) return false;
+    return DfSmem(h->D, F, C).total <= h->optin;
 }
 
 static void fused_cluster_config(int C, int n_clusters, int smem, cudaStream_t st, cudaLaunchConfig_t *lc,
@@ -665,16 +657,15 @@ static void fused_cluster_config(int C, int n_clusters, int smem, cudaStream_t s
 
 // at create: which cluster sizes of dx_fused_kernel serve this shape, and how
 // many such clusters fit at once
-static const int kDfSizes[3] = {8, 4, 2};   // cluster sizes of dx_fused_kernel, in order of preference
+static const int kDfSizes[2] = {8, 4};   // cluster sizes of dx_fused_kernel, in order of preference
 
 static void fused_setup(maple_moe_t h)
 {
     int need = 0;
-    for (int i = 0; i < 3; i++) {
+    for (int i = 0; i < 2; i++) {
         h->df_fit[i] = 0;
-        h->df_ns[i] = fused_shape_ns(h, kDfSizes[i]);
-        if (h->df_ns[i] >= 0 && DfSmem(h->D, h->F, kDfSizes[i], h->df_ns[i]).total > need)
-            need = DfSmem(h->D, h->F, kDfSizes[i], h->df_ns[i]).total;
+        if (fused_shape_ok(h, kDfSizes[i]) && DfSmem(h->D, h->F, kDfSizes[i]).total > need)
+            need = DfSmem(h->D, h->F, kDfSizes[i]).total;
     }
     if (!need) return;
     if (cudaFuncSetAttribute((const void *)dx_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, need) !=
@@ -682,12 +673,12 @@ static void fused_setup(maple_moe_t h)
         cudaGetLastError();
         return;
     }
-    for (int i = 0; i < 3; i++) {
+    for (int i = 0; i < 2; i++) {
         const int C = kDfSizes[i];
-        if (h->df_ns[i] < 0) continue;
+        if (!fused_shape_ok(h, C)) continue;
         cudaLaunchConfig_t lc;
         cudaLaunchAttribute attr[2];
-        fused_cluster_config(C, 1, DfSmem(h->D, h->F, C, h->df_ns[i]).total, nullptr, &lc, attr);
+        fused_cluster_config(C, 1, DfSmem(h->D, h->F, C).total, nullptr, &lc, attr);
         lc.numAttrs = 1;   // (occupancy: the cluster shape only)
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, (const void *)dx_fused_kernel, &lc) != cudaSuccess) {
@@ -701,21 +692,16 @@ static void fused_setup(maple_moe_t h)
 // cluster size of the fused expert kernel for a batch of T tokens (0: the
 // two-kernel path).  Its clusters (one per unit, at most min(T*K, E)) must all
 // fit at once: a second wave of clusters costs the whole kernel's latency
-// again, more than the two-kernel path takes.  The largest size (8, 4, 2)
-// whose clusters all fit.
+// again, more than the two-kernel path takes.  The larger size (8, 4) whose
+// clusters all fit.  (Two-CTA clusters with a ring of slots, so that T = 8 fits
+// in one wave, measured no faster than the two-kernel path: the slowest
+// cluster's combine and the weight stream of 400 KB per CTA set its pace.)
 static int fused_cluster(maple_moe_t h, int T)
 {
     if (T > 8 || h->K > 8 || (h->debug_flags & MAPLE_DEBUG_SPLIT_SMALL)) return 0;
     const int n = T * h->K < h->E ? T * h->K : h->E;
-    for (int i = 0; i < 3; i++)
+    for (int i = 0; i < 2; i++)
         if (h->df_fit[i] >= n) return kDfSizes[i];
-    return 0;
-}
-
-static int fused_ns(maple_moe_t h, int C)
-{
-    for (int i = 0; i < 3; i++)
-        if (kDfSizes[i] == C) return h->df_ns[i];
     return 0;
 }
 
@@ -754,12 +740,11 @@ static int run_experts_fused(maple_moe_t h, int T, int C, float *y, const float 
     d.never = h->dx_never;
     d.wait_ns = h->wait_ns;
     d.stall = (h->debug_flags & MAPLE_DEBUG_STALL_DOWN) ? 1 : 0;
-    d.ns = fused_ns(h, C);
     // one cluster per unit: at most one unit per slot and per expert
     const int n_clusters = T * h->K < h->E ? T * h->K : h->E;
     cudaLaunchConfig_t lc;
     cudaLaunchAttribute attr[2];
-    fused_cluster_config(C, n_clusters, DfSmem(h->D, h->F, C, d.ns).total, st, &lc, attr);
+    fused_cluster_config(C, n_clusters, DfSmem(h->D, h->F, C).total, st, &lc, attr);
     if (cudaLaunchKernelEx(&lc, dx_fused_kernel, d) != cudaSuccess) return MAPLE_ERR_CUDA;
     stage_event(h, 2, st);
     stage_event(h, 3, st);

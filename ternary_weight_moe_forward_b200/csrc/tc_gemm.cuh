@@ -178,6 +178,30 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
+// L2 cache policies: the weight codes are read once (evict first), the
+// gate/up kernel's h scratch is read back once by the same CTA (evict last)
+__device__ __forceinline__ uint64_t l2_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar, uint64_t pol)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_f32_hint(float *p, float v, uint64_t pol)
+{
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
 // 2-D tiled TMA load (box given by the tensor map) into 128B-swizzled shared memory
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
 {
@@ -356,6 +380,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
     if (warp == 0) {
         // ---------------- bulk copies of the 2-bit codes, up to CS stages ahead
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first();
             uint32_t it = 0;
             bool ok = true;
             int pc, rb;
@@ -369,8 +394,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                         break;
                     }
                     mbar_expect_tx(b_codes_full + 8 * s, Cfg::kCodeBytes);
-                    bulk_g2s(smem_addr(smem + L::kCodes + s * Cfg::kCodeBytes), src + (size_t)ks * Cfg::kCodeBytes,
-                             Cfg::kCodeBytes, b_codes_full + 8 * s);
+                    bulk_g2s_hint(smem_addr(smem + L::kCodes + s * Cfg::kCodeBytes), src + (size_t)ks * Cfg::kCodeBytes,
+                             Cfg::kCodeBytes, b_codes_full + 8 * s, pol);
                 }
             }
             if (!ok) {
@@ -471,6 +496,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
         const int ldo = MODE == 0 ? a.F : a.D;
         const float *scale_src = MODE == 0 ? a.pscale : a.sh;
         float *hs = MODE == 0 ? a.out + (size_t)blockIdx.x * kTcMaxN * a.F : nullptr;   // [128 slots][F]
+        const uint64_t pol_h = l2_evict_last();   // (the scratch is read back by this CTA)
         auto fetch = [&](int buf, const int4 &P, int rbk, float &al0, float &al1) {
             const int row = rbk * 128 + r;
             al0 = a.alpha0[(size_t)P.x * ldo + row];
@@ -536,11 +562,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_gemm_kernel(const __grid_con
                                 }
                                 if (cb + j0 + 8 <= n) {
 #pragma unroll
-                                    for (int j = 0; j < 8; j++) hd[(size_t)(j0 + j) * a.F] = hv[j];
+                                    for (int j = 0; j < 8; j++) st_f32_hint(hd + (size_t)(j0 + j) * a.F, hv[j], pol_h);
                                 } else {
 #pragma unroll
                                     for (int j = 0; j < 8; j++)
-                                        if (cb + j0 + j < n) hd[(size_t)(j0 + j) * a.F] = hv[j];
+                                        if (cb + j0 + j < n) st_f32_hint(hd + (size_t)(j0 + j) * a.F, hv[j], pol_h);
                                 }
                             }
                             if (a.tap0 || a.tap1) {
@@ -749,42 +775,20 @@ __global__ void combine_kernel(const int16_t *acc_hi, const uint32_t *acc_lo, co
         const int t = (int)(i / (D / 4));
         const int c = 4 * (int)(i % (D / 4));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        // four ranks at a time: their indices, then their rows, all loads in flight
-        // together; the sum still runs in rank order
-        for (int k0 = 0; k0 < K; k0 += 4) {
-            int p[4], e[4];
-            float w[4], s[4];
-            uint2 hv[4];
-            uint32_t lo[4];
-            float4 al[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                if (k0 + j < K) {
-                    const int sl = t * K + k0 + j;
-                    p[j] = __ldg(inv + sl);
-                    e[j] = __ldg(topk_idx + sl);
-                    w[j] = __ldg(topk_w + sl);
-                }
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                if (k0 + j < K) {
-                    s[j] = __ldg(sh + p[j]);
-                    hv[j] = __ldcs(reinterpret_cast<const uint2 *>(acc_hi + (size_t)p[j] * D + c));
-                    lo[j] = __ldg(acc_lo + (size_t)p[j] * (D / 32) + (c >> 5)) >> (c & 31);
-                    al[j] = __ldg(reinterpret_cast<const float4 *>(alpha_down + (size_t)e[j] * D + c));
-                }
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-                if (k0 + j < K) {
-                    const int a0 = 2 * (int)(int16_t)(hv[j].x & 0xffffu) + (int)(lo[j] & 1u);
-                    const int a1 = 2 * (int)(int16_t)(hv[j].x >> 16) + (int)((lo[j] >> 1) & 1u);
-                    const int a2 = 2 * (int)(int16_t)(hv[j].y & 0xffffu) + (int)((lo[j] >> 2) & 1u);
-                    const int a3 = 2 * (int)(int16_t)(hv[j].y >> 16) + (int)((lo[j] >> 3) & 1u);
-                    acc.x = __fmaf_rn(w[j], __fmul_rn((float)a0, __fmul_rn(al[j].x, s[j])), acc.x);
-                    acc.y = __fmaf_rn(w[j], __fmul_rn((float)a1, __fmul_rn(al[j].y, s[j])), acc.y);
-                    acc.z = __fmaf_rn(w[j], __fmul_rn((float)a2, __fmul_rn(al[j].z, s[j])), acc.z);
-                    acc.w = __fmaf_rn(w[j], __fmul_rn((float)a3, __fmul_rn(al[j].w, s[j])), acc.w);
-                }
+        for (int k = 0; k < K; k++) {
+            const int sl = t * K + k, p = __ldg(inv + sl), e = __ldg(topk_idx + sl);
+            const float w = __ldg(topk_w + sl), s = __ldg(sh + p);
+            const uint2 hv = __ldcs(reinterpret_cast<const uint2 *>(acc_hi + (size_t)p * D + c));
+            const uint32_t lo = __ldg(acc_lo + (size_t)p * (D / 32) + (c >> 5)) >> (c & 31);
+            const float4 al = __ldg(reinterpret_cast<const float4 *>(alpha_down + (size_t)e * D + c));
+            const int a0 = 2 * (int)(int16_t)(hv.x & 0xffffu) + (int)(lo & 1u);
+            const int a1 = 2 * (int)(int16_t)(hv.x >> 16) + (int)((lo >> 1) & 1u);
+            const int a2 = 2 * (int)(int16_t)(hv.y & 0xffffu) + (int)((lo >> 2) & 1u);
+            const int a3 = 2 * (int)(int16_t)(hv.y >> 16) + (int)((lo >> 3) & 1u);
+            acc.x = __fmaf_rn(w, __fmul_rn((float)a0, __fmul_rn(al.x, s)), acc.x);
+            acc.y = __fmaf_rn(w, __fmul_rn((float)a1, __fmul_rn(al.y, s)), acc.y);
+            acc.z = __fmaf_rn(w, __fmul_rn((float)a2, __fmul_rn(al.z, s)), acc.z);
+            acc.w = __fmaf_rn(w, __fmul_rn((float)a3, __fmul_rn(al.w, s)), acc.w);
         }
         if (resid) {
             const float4 r = reinterpret_cast<const float4 *>(resid)[i];

@@ -60,3 +60,23 @@ def test_reference_arm_line():
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_committed_profile_matches_the_sources():
+    """The committed ncu summary of the dominant kernel belongs to the sources in
+    the tree, so the bench line carries its measured DRAM traffic."""
+    assert bench.measured_traffic() is not None
+
+
+def test_per_batch_entry_by_expert_path():
+    # split: (route, after gate/up, end) in ms, per layer
+    split = [(0, (0.010, 0.020, 0.030)), (1, (0.012, 0.022, 0.031))]
+    fused = bench.per_T_entry(1, True, [0.02, 0.02], [0.025], split, [8, 8], 6650.0)
+    assert fused["expert_path"] == "fused"
+    assert "us_gate_up" not in fused and "gate_up_hbm_frac" not in fused
+    assert abs(fused["us_experts"] - 1e3 * (0.020 + 0.019) / 2) < 1e-9
+    two = bench.per_T_entry(64, False, [0.07], [0.08], split, [222, 222], 6650.0)
+    assert two["expert_path"] == "two-kernel"
+    assert abs(two["us_gate_up"] - 1e3 * (0.010 + 0.010) / 2) < 1e-9
+    assert abs(two["us_down_combine"] - 1e3 * (0.010 + 0.009) / 2) < 1e-9
+    assert abs(two["tokens_per_s"] - 64 / 0.07e-3) < 1e-6 * two["tokens_per_s"]

@@ -11,7 +11,7 @@ namespace maple {
 
 constexpr int kRouteTokens = 8;        // tokens per route CTA (one per warp)
 constexpr int kRouteExperts = 8;       // experts per route CTA (one per warp)
-constexpr int kFusedMarkBytes = 16384; // largest T*E the fused one-warp permutation takes
+constexpr int kFusedMarkBytes = 16384; // largest T*E the routing kernel builds the permutation for itself
 constexpr int kPermBlockTokens = 32;   // tokens per CTA of the multi-CTA permutation
 constexpr int kMaxExperts = 1024;
 constexpr int kRouteSmallT = 64;       // up to this many tokens the latency-oriented router runs

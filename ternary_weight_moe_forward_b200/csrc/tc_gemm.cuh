@@ -32,7 +32,8 @@
 // warp issuing for most of the kernel.)  A CTA takes whole pieces (all F/128 row blocks of one piece in a
 // row, pieces dealt out in a snake order over the size-sorted list), so that
 // it holds every h value of its slots: the epilogue writes h = SiLU(g) * u
-// (fp32) to a per-CTA scratch area that stays in L2; after the piece's last
+// (fp32) to a per-CTA scratch area, stored with an L2 evict-last policy (and
+// the codes copied evict-first) so that it stays in L2; after the piece's last
 // row block the epilogue warps requantise the slots, a slot's row at a time
 // in registers (its |h| maximum by a warp reduction, then the int8 absmax
 // codes q_h and the scale s_h), so no fp32 h leaves the chip.
